@@ -1,0 +1,207 @@
+"""MoE expert-parallel token routing on one B200: Python binding of libmep.
+
+Every function here is argument marshalling around the C ABI declared in
+``include/mep.h`` (same names): it checks dtypes and devices of torch tensors, passes
+their device pointers and the current CUDA stream, and raises ``MepError`` on a
+non-OK status. All computation runs in the library's CUDA kernels; there is no CPU or
+PyTorch fallback. If ``libmep.so`` has not been built, importing the binding's
+functions raises immediately.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmep.so")
+
+MEP_PLAN_BALANCED = 0
+MEP_PLAN_GROUPED = 1
+MEP_MAX_KEYS = 4096
+MEP_MAX_K = 32
+
+DERR_KEY_RANGE = 0x1
+DERR_ROW_RANGE = 0x2
+DERR_TABLE = 0x4
+DERR_MASK = 0x8
+
+STATUS = {0: "MEP_OK", 1: "MEP_ERR_NULLPTR", 2: "MEP_ERR_DTYPE", 3: "MEP_ERR_SHAPE",
+          4: "MEP_ERR_VALUE", 5: "MEP_ERR_WORKSPACE", 6: "MEP_ERR_CUDA"}
+
+
+class MepError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        name = STATUS.get(status, str(status))
+        extra = ""
+        if status == 6:
+            extra = f" (cudaError {lib().mep_last_cuda_error()})"
+        super().__init__(f"{what}: {name}{extra}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmep.so (built in-tree by ``dispatch_combine_topk_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libmep.so not found at {LIB_PATH}; build it with "
+                              "`python -m dispatch_combine_topk_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+        L.mep_version.restype = i32
+        L.mep_status_string.argtypes = [ctypes.c_int]
+        L.mep_status_string.restype = ctypes.c_char_p
+        L.mep_last_cuda_error.restype = i32
+        L.mep_get_error.argtypes = [P, i32]
+        L.mep_histogram.argtypes = [P, i64, i32, P, P]
+        L.mep_plan_workspace_size.argtypes = [i32, i32, i32, i32]
+        L.mep_plan_workspace_size.restype = ctypes.c_size_t
+        L.mep_plan.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P,
+                               ctypes.c_size_t, P]
+        L.mep_update_expert.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i64, i64, P, P, P]
+        L.mep_dispatch.argtypes = [P, P, i64, i32, i64, i32, P, P, i64, P]
+        L.mep_dequantize.argtypes = [P, P, i64, i64, P, P]
+        L.mep_combine.argtypes = [P, i64, P, P, i64, i32, i64, P, P]
+        for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
+                  "mep_dispatch", "mep_dequantize", "mep_combine"]:
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ok(rc: int, what: str):
+    if rc != 0:
+        raise MepError(rc, what)
+
+
+def mep_get_error(clear: bool = True) -> int:
+    """Sticky device error word of the current device (synchronises the device)."""
+    code = ctypes.c_int32(0)
+    _ok(lib().mep_get_error(ctypes.byref(code), int(clear)), "mep_get_error")
+    return code.value
+
+
+def mep_histogram(ids: torch.Tensor, n_keys: int, hist: torch.Tensor, stream=None):
+    _ok(lib().mep_histogram(_ptr(ids, torch.int32, "ids"), ids.numel(), n_keys,
+                            _ptr(hist, torch.int32, "hist"), _stream(stream)), "mep_histogram")
+    return hist
+
+
+def mep_plan_workspace_size(R: int, n_keys: int, S: int, K: int) -> int:
+    return int(lib().mep_plan_workspace_size(R, n_keys, S, K))
+
+
+@dataclasses.dataclass
+class PlanBuffers:
+    """Device outputs of mep_plan (see include/mep.h for their layout)."""
+
+    pos: torch.Tensor        # int32 [N]
+    hist: torch.Tensor       # int32 [n_keys]
+    rank_off: torch.Tensor   # int32 [R+1]
+    load: torch.Tensor       # int32 [R]
+    rep_count: torch.Tensor  # int32 [R]
+    rep_key: torch.Tensor    # int32 [R, n_keys]
+    rep_cu: torch.Tensor     # int32 [R, n_keys+1]
+    stats: torch.Tensor      # int32 [8] (mep_plan_stats_t)
+    workspace: torch.Tensor  # uint8, 256-byte aligned
+
+    @staticmethod
+    def allocate(R: int, n_keys: int, S: int, K: int, device=None) -> "PlanBuffers":
+        dev = device or torch.device("cuda", torch.cuda.current_device())
+        z = lambda *s: torch.empty(s, dtype=torch.int32, device=dev)
+        ws = torch.empty(max(256, mep_plan_workspace_size(R, n_keys, S, K)), dtype=torch.uint8,
+                         device=dev)
+        return PlanBuffers(z(R * S * K), z(n_keys), z(R + 1), z(R), z(R), z(R, n_keys),
+                           z(R, n_keys + 1), z(8), ws)
+
+    def stats_dict(self) -> dict:
+        s = self.stats.tolist()
+        return dict(max_load=s[0], max_chunk=s[1], redundant=s[2], prefetched=s[3], n_kept=s[4],
+                    max_hist=s[5], n_ranks_used=s[6])
+
+
+def mep_plan(ids: torch.Tensor, R: int, n_keys: int, S: int, K: int, out: PlanBuffers,
+             mode: int = MEP_PLAN_BALANCED, keys_per_rank: int = 0,
+             keep: Optional[torch.Tensor] = None, stream=None) -> PlanBuffers:
+    if ids.numel() != R * S * K:
+        raise ValueError("ids must hold R*S*K slots")
+    rc = lib().mep_plan(_ptr(ids, torch.int32, "ids"), _ptr(keep, torch.uint8, "keep"), R, n_keys,
+                        S, K, mode, keys_per_rank, _ptr(out.pos), _ptr(out.hist),
+                        _ptr(out.rank_off), _ptr(out.load), _ptr(out.rep_count),
+                        _ptr(out.rep_key), _ptr(out.rep_cu), _ptr(out.stats),
+                        _ptr(out.workspace), out.workspace.numel(), _stream(stream))
+    _ok(rc, "mep_plan")
+    return out
+
+
+def mep_update_expert(expert_ids: torch.Tensor, eplb_table: torch.Tensor,
+                      expert_scales: Optional[torch.Tensor], pruning_threshold: Optional[torch.Tensor],
+                      active_mask: Optional[torch.Tensor], local_rank_id: int, world_size: int,
+                      balance_mode: int, balanced_expert_ids: torch.Tensor,
+                      balanced_active_mask: torch.Tensor, stream=None):
+    BS, K = expert_ids.shape
+    E, F = eplb_table.shape
+    rc = lib().mep_update_expert(_ptr(expert_ids, torch.int32, "expert_ids"),
+                                 _ptr(eplb_table, torch.int32, "eplb_table"),
+                                 _ptr(expert_scales, torch.float32, "expert_scales"),
+                                 _ptr(pruning_threshold, torch.float32, "pruning_threshold"),
+                                 _ptr(active_mask, torch.uint8, "active_mask"), BS, K, E, F,
+                                 local_rank_id, world_size, balance_mode,
+                                 _ptr(balanced_expert_ids, torch.int32, "balanced_expert_ids"),
+                                 _ptr(balanced_active_mask, torch.uint8, "balanced_active_mask"),
+                                 _stream(stream))
+    _ok(rc, "mep_update_expert")
+    return balanced_expert_ids, balanced_active_mask
+
+
+def mep_dispatch(x: torch.Tensor, pos: torch.Tensor, K: int, recv: torch.Tensor,
+                 recv_scale: Optional[torch.Tensor] = None, quant: int = 0, stream=None):
+    T, H = x.shape
+    want = torch.int8 if quant == 1 else torch.bfloat16
+    rows = recv.shape[0]
+    rc = lib().mep_dispatch(_ptr(x, torch.bfloat16, "x"), _ptr(pos, torch.int32, "pos"), T, K, H,
+                            quant, _ptr(recv, want, "recv"),
+                            _ptr(recv_scale, torch.float32, "recv_scale"), rows, _stream(stream))
+    _ok(rc, "mep_dispatch")
+    return recv
+
+
+def mep_dequantize(q: torch.Tensor, scale: torch.Tensor, y: torch.Tensor, stream=None):
+    rows, H = q.shape
+    _ok(lib().mep_dequantize(_ptr(q, torch.int8, "q"), _ptr(scale, torch.float32, "scale"), rows, H,
+                             _ptr(y, torch.bfloat16, "y"), _stream(stream)), "mep_dequantize")
+    return y
+
+
+def mep_combine(y: torch.Tensor, pos: torch.Tensor, gates: torch.Tensor, K: int,
+                out: torch.Tensor, stream=None):
+    T, H = out.shape
+    rc = lib().mep_combine(_ptr(y, torch.bfloat16, "y"), y.shape[0], _ptr(pos, torch.int32, "pos"),
+                           _ptr(gates, torch.float32, "gates"), T, K, H,
+                           _ptr(out, torch.bfloat16, "out"), _stream(stream))
+    _ok(rc, "mep_combine")
+    return out

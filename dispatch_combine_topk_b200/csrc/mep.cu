@@ -1,0 +1,282 @@
+// libmep — C ABI of MoE expert-parallel token routing on one B200 (sm_100a).
+// Entry points, argument checks and launch configuration. The declarations, with the
+// meaning, layout, ownership and error behaviour of every argument, are in mep.h.
+//
+// One translation unit on purpose: the device error word lives here and every kernel
+// reaches it without relocatable device code.
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "mep.h"
+#include "common.cuh"
+#include "plan_kernels.cuh"
+#include "route_kernels.cuh"
+
+namespace {
+
+thread_local int32_t t_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];
+bool g_attrs_set[kMaxDevices];
+
+// SM count of the current device (cached), and one-time kernel attributes.
+int sm_count()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (g_sm_count[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        g_sm_count[dev] = n > 0 ? n : 148;
+    }
+    if (!g_attrs_set[dev]) {
+        const int big = 200 * 1024;
+        cudaFuncSetAttribute(mep::k_rank, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(mep::k_tile_count, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(mep::k_histogram, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(mep::k_plan_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        g_attrs_set[dev] = true;
+    }
+    return g_sm_count[dev];
+}
+
+mep_status_t launched()
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        t_last_cuda_error = (int32_t)e;
+        return MEP_ERR_CUDA;
+    }
+    return MEP_OK;
+}
+
+inline bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+inline size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// Token-parallel grid: a multiple of the SM count, never more CTAs than tokens.
+inline int token_grid(int64_t T, int per_sm)
+{
+    int64_t g = (int64_t)sm_count() * per_sm;
+    if (T < g) g = T;
+    return (int)(g > 0 ? g : 1);
+}
+
+inline int elem_grid(int64_t total, int threads)
+{
+    int64_t g = (total + threads - 1) / threads;
+    int64_t cap = (int64_t)sm_count() * 8;
+    if (g > cap) g = cap;
+    return (int)(g > 0 ? g : 1);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t mep_version(void) { return (1 << 16) | 0; }
+
+const char *mep_status_string(mep_status_t s)
+{
+    switch (s) {
+    case MEP_OK: return "MEP_OK";
+    case MEP_ERR_NULLPTR: return "MEP_ERR_NULLPTR: a required pointer is NULL";
+    case MEP_ERR_DTYPE: return "MEP_ERR_DTYPE: unsupported element type or quantisation mode";
+    case MEP_ERR_SHAPE: return "MEP_ERR_SHAPE: a size is outside the supported range";
+    case MEP_ERR_VALUE: return "MEP_ERR_VALUE: an argument value is outside its range";
+    case MEP_ERR_WORKSPACE: return "MEP_ERR_WORKSPACE: workspace NULL, too small or misaligned";
+    case MEP_ERR_CUDA: return "MEP_ERR_CUDA: a CUDA call failed";
+    }
+    return "unknown mep_status_t";
+}
+
+int32_t mep_last_cuda_error(void) { return t_last_cuda_error; }
+
+mep_status_t mep_get_error(int32_t *code, int32_t clear)
+{
+    if (!code) return MEP_ERR_NULLPTR;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(code, mep::g_error_word, sizeof(int32_t));
+    if (e == cudaSuccess && clear) {
+        const int32_t zero = 0;
+        e = cudaMemcpyToSymbol(mep::g_error_word, &zero, sizeof(int32_t));
+    }
+    if (e != cudaSuccess) {
+        t_last_cuda_error = (int32_t)e;
+        return MEP_ERR_CUDA;
+    }
+    return MEP_OK;
+}
+
+mep_status_t mep_histogram(const int32_t *ids, int64_t n, int32_t n_keys, int32_t *hist,
+                           mep_stream_t stream)
+{
+    if ((!ids && n > 0) || !hist) return MEP_ERR_NULLPTR;
+    if (n < 0 || n >= ((int64_t)1 << 31) || n_keys < 1 || n_keys > MEP_MAX_KEYS) return MEP_ERR_SHAPE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int sms = sm_count();
+    if (cudaMemsetAsync(hist, 0, sizeof(int32_t) * n_keys, s) != cudaSuccess) return launched();
+    if (n == 0) return launched();
+    int64_t tiles = mep::ceil_div(n, mep::kPlanTile);
+    int grid = (int)(tiles < 2 * sms ? tiles : 2 * sms);
+    mep::k_histogram<<<grid, mep::kPlanWarps * 32, sizeof(int32_t) * n_keys, s>>>(ids, n, n_keys, hist);
+    return launched();
+}
+
+size_t mep_plan_workspace_size(int32_t R, int32_t n_keys, int32_t S, int32_t K)
+{
+    if (R < 1 || S < 1 || K < 1 || n_keys < 1) return 0;
+    const int64_t N = (int64_t)R * S * K;
+    const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
+    return align256(sizeof(int32_t) * (size_t)tiles * n_keys) + align256(sizeof(int32_t) * (size_t)(n_keys + 1));
+}
+
+mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_t n_keys,
+                      int32_t S, int32_t K, int32_t mode, int32_t keys_per_rank,
+                      int32_t *pos, int32_t *hist, int32_t *rank_off, int32_t *load,
+                      int32_t *rep_count, int32_t *rep_key, int32_t *rep_cu,
+                      mep_plan_stats_t *stats, void *workspace, size_t workspace_bytes,
+                      mep_stream_t stream)
+{
+    if (!ids || !pos || !hist || !rank_off || !rep_count || !rep_key || !rep_cu || !stats)
+        return MEP_ERR_NULLPTR;
+    if (R < 1 || S < 1 || K < 1 || K > MEP_MAX_K || n_keys < 1 || n_keys > MEP_MAX_KEYS ||
+        R > MEP_MAX_KEYS)
+        return MEP_ERR_SHAPE;
+    const int64_t N = (int64_t)R * S * K;
+    if (N >= ((int64_t)1 << 31)) return MEP_ERR_SHAPE;
+    if (mode == MEP_PLAN_BALANCED) {
+        if (n_keys % R != 0 || keep) return MEP_ERR_VALUE;
+    } else if (mode == MEP_PLAN_GROUPED) {
+        if (keys_per_rank < 1 || (int64_t)keys_per_rank * R != n_keys) return MEP_ERR_VALUE;
+    } else {
+        return MEP_ERR_VALUE;
+    }
+    const size_t need = mep_plan_workspace_size(R, n_keys, S, K);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return MEP_ERR_WORKSPACE;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    sm_count();
+    const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
+    int32_t *tile_cnt = (int32_t *)workspace;
+    int32_t *key_off = (int32_t *)((char *)workspace + align256(sizeof(int32_t) * (size_t)tiles * n_keys));
+    const int threads = mep::kPlanWarps * 32;
+
+    mep::k_tile_count<<<(unsigned)tiles, threads, sizeof(int32_t) * n_keys, s>>>(ids, keep, N, n_keys, tile_cnt);
+    mep::k_scan<<<1, 1024, 0, s>>>(tile_cnt, (int32_t)tiles, n_keys, hist, key_off);
+    mep::k_rank<<<(unsigned)tiles, threads, sizeof(int32_t) * mep::kPlanWarps * n_keys, s>>>(
+        ids, keep, N, n_keys, tile_cnt, key_off, pos);
+    const size_t meta_smem = sizeof(int32_t) * (size_t)(2 * (n_keys + 1) + (R + 1) + R);
+    mep::k_plan_meta<<<1, 1024, meta_smem, s>>>(hist, key_off, R, n_keys, (int64_t)S * K, mode,
+                                                keys_per_rank, rank_off, load, rep_count, rep_key,
+                                                rep_cu, (int32_t *)stats);
+    return launched();
+}
+
+mep_status_t mep_update_expert(const int32_t *expert_ids, const int32_t *eplb_table,
+                               const float *expert_scales, const float *pruning_threshold,
+                               const uint8_t *active_mask, int64_t BS, int32_t K,
+                               int32_t n_experts, int32_t F, int64_t local_rank_id,
+                               int64_t world_size, int64_t balance_mode,
+                               int32_t *balanced_expert_ids, uint8_t *balanced_active_mask,
+                               mep_stream_t stream)
+{
+    if (!expert_ids || !eplb_table || !balanced_expert_ids || !balanced_active_mask)
+        return MEP_ERR_NULLPTR;
+    if ((expert_scales == nullptr) != (pruning_threshold == nullptr)) return MEP_ERR_NULLPTR;
+    if (active_mask && !expert_scales) return MEP_ERR_NULLPTR;
+    if (BS < 1 || K < 1 || K > 16 || n_experts < 1 || n_experts > 1024 || K > n_experts)
+        return MEP_ERR_SHAPE;
+    if (world_size < 1 || F < 2 || F > world_size + 1) return MEP_ERR_SHAPE;
+    if (balance_mode != 0 && balance_mode != 1) return MEP_ERR_VALUE;
+    if (balance_mode == 0 && (world_size < 2 || world_size > 768)) return MEP_ERR_VALUE;
+    if (balance_mode == 0 && (local_rank_id < 0 || local_rank_id >= world_size)) return MEP_ERR_VALUE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int threads = 128;
+    int64_t g = (BS + threads - 1) / threads;
+    int cap = sm_count() * 4;
+    mep::k_update_expert<<<(unsigned)(g < cap ? g : cap), threads, 0, s>>>(
+        expert_ids, eplb_table, expert_scales, pruning_threshold, active_mask, BS, K, n_experts, F,
+        local_rank_id, world_size, balance_mode, balanced_expert_ids, balanced_active_mask);
+    return launched();
+}
+
+mep_status_t mep_dispatch(const uint16_t *x, const int32_t *pos, int64_t T, int32_t K,
+                          int64_t H, int32_t quant, void *recv, float *recv_scale,
+                          int64_t rows, mep_stream_t stream)
+{
+    if (quant != 0 && quant != 1) return MEP_ERR_DTYPE;
+    if (T > 0 && (!x || !pos || (!recv && rows > 0) || (quant == 1 && !recv_scale && rows > 0)))
+        return MEP_ERR_NULLPTR;
+    if (T < 0 || K < 1 || K > MEP_MAX_K || H < 1 || rows < 0 || T * K >= ((int64_t)1 << 31))
+        return MEP_ERR_SHAPE;
+    if (T == 0) return MEP_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int grid = token_grid(T, 8);
+    if (quant == 0) {
+        if (H % 8 == 0 && aligned(x, 16) && aligned(recv, 16)) {
+            mep::k_dispatch_copy<uint4><<<grid, 256, 0, s>>>((const uint4 *)x, pos, T, K, H / 8, rows,
+                                                             (uint4 *)recv);
+        } else {
+            mep::k_dispatch_copy<uint16_t><<<grid, 256, 0, s>>>(x, pos, T, K, H, rows, (uint16_t *)recv);
+        }
+    } else {
+        if (H % 8 == 0 && aligned(x, 16) && aligned(recv, 8)) {
+            mep::k_dispatch_int8<<<grid, 256, 0, s>>>((const uint4 *)x, pos, T, K, H / 8, rows,
+                                                      (uint2 *)recv, recv_scale);
+        } else {
+            mep::k_dispatch_int8_scalar<<<grid, 256, 0, s>>>(x, pos, T, K, H, rows, (int8_t *)recv,
+                                                             recv_scale);
+        }
+    }
+    return launched();
+}
+
+mep_status_t mep_dequantize(const int8_t *q, const float *scale, int64_t rows, int64_t H,
+                            uint16_t *y, mep_stream_t stream)
+{
+    if (rows > 0 && (!q || !scale || !y)) return MEP_ERR_NULLPTR;
+    if (rows < 0 || H < 1) return MEP_ERR_SHAPE;
+    if (rows == 0) return MEP_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (H % 8 == 0 && aligned(q, 8) && aligned(y, 16)) {
+        const int64_t total = rows * (H / 8);
+        mep::k_dequant8<<<elem_grid(total, 256), 256, 0, s>>>((const uint2 *)q, scale, rows, H / 8, (uint4 *)y);
+    } else {
+        mep::k_dequant_scalar<<<elem_grid(rows * H, 256), 256, 0, s>>>(q, scale, rows, H, y);
+    }
+    return launched();
+}
+
+mep_status_t mep_combine(const uint16_t *y, int64_t rows, const int32_t *pos,
+                         const float *gates, int64_t T, int32_t K, int64_t H, uint16_t *out,
+                         mep_stream_t stream)
+{
+    if (T > 0 && (!pos || !gates || !out || (!y && rows > 0))) return MEP_ERR_NULLPTR;
+    if (T < 0 || K < 1 || K > MEP_MAX_K || H < 1 || rows < 0 || T * K >= ((int64_t)1 << 31))
+        return MEP_ERR_SHAPE;
+    if (T == 0) return MEP_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int grid = token_grid(T, 8);
+    if (H % 8 == 0 && aligned(y, 16) && aligned(out, 16)) {
+        const uint4 *yv = (const uint4 *)y;
+        uint4 *ov = (uint4 *)out;
+        const int64_t H8 = H / 8;
+        switch (K) {
+        case 1: mep::k_combine_v8<1><<<grid, 256, 0, s>>>(yv, pos, gates, T, K, H8, rows, ov); break;
+        case 2: mep::k_combine_v8<2><<<grid, 256, 0, s>>>(yv, pos, gates, T, K, H8, rows, ov); break;
+        case 4: mep::k_combine_v8<4><<<grid, 256, 0, s>>>(yv, pos, gates, T, K, H8, rows, ov); break;
+        case 6: mep::k_combine_v8<6><<<grid, 256, 0, s>>>(yv, pos, gates, T, K, H8, rows, ov); break;
+        case 8: mep::k_combine_v8<8><<<grid, 256, 0, s>>>(yv, pos, gates, T, K, H8, rows, ov); break;
+        default: mep::k_combine_v8<0><<<grid, 256, 0, s>>>(yv, pos, gates, T, K, H8, rows, ov); break;
+        }
+    } else {
+        mep::k_combine_scalar<<<grid, 256, 0, s>>>(y, pos, gates, T, K, H, rows, out);
+    }
+    return launched();
+}
+
+}  // extern "C"

@@ -1,0 +1,337 @@
+// Histogram and placement-plan kernels (sm_100a).
+//
+// The balanced plan of MoonEP (every rank receives exactly S*K token-slots, hot experts
+// spill onto temporary redundant replicas on the next ranks; twodots.gr article on
+// MoonEP) orders slots by (home(e), e, src, t, k). home(e) is monotone in e and the
+// flat slot index orders (src, t, k), so the order is a stable counting sort by key:
+//   row(n) = off[key] + #{m < n : key(m) == key(n)}.
+// The grouped plan over physical instance ids is the same sort with dropped slots
+// removed. Both are done in three passes over the ids (4 bytes per slot each):
+//   k_tile_count  per-tile key counts              (warp-aggregated with match.any)
+//   k_scan        per-key prefix over tiles + exclusive prefix over keys
+//   k_rank        per-slot stable rank inside its tile, written as the final row
+// and one single-CTA pass over the keys, k_plan_meta, that writes the per-rank replica
+// tables (cu_seqlens) and the summary counts.
+#pragma once
+
+#include "common.cuh"
+
+namespace mep {
+
+constexpr int kPlanWarps = 8;                    // warps per tile CTA
+constexpr int kPlanTile = kPlanWarps * 32 * 8;   // 2048 slots per tile, 256 per warp
+
+// Key of slot n: the id, or -1 when the slot is dropped or its id is out of range.
+__device__ __forceinline__ int32_t slot_key(const int32_t *ids, const uint8_t *keep, int64_t n,
+                                            int64_t N, int32_t n_keys)
+{
+    if (n >= N) return -1;
+    if (keep && !keep[n]) return -1;
+    int32_t e = ids[n];
+    if (e < 0 || e >= n_keys) {
+        flag_error(0x1);
+        return -1;
+    }
+    return e;
+}
+
+// hist[key] += count of key in this CTA's tile (global atomics, one per distinct key
+// per CTA). Used by mep_histogram.
+__global__ void __launch_bounds__(kPlanWarps * 32)
+k_histogram(const int32_t *__restrict__ ids, int64_t N, int32_t n_keys, int32_t *__restrict__ hist)
+{
+    extern __shared__ int32_t sh[];
+    for (int i = threadIdx.x; i < n_keys; i += blockDim.x) sh[i] = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    for (int64_t n0 = (int64_t)blockIdx.x * kPlanTile; n0 < N; n0 += (int64_t)gridDim.x * kPlanTile) {
+        for (int64_t n = n0 + threadIdx.x - lane; n < n0 + kPlanTile; n += blockDim.x) {
+            int32_t key = slot_key(ids, nullptr, n + lane, N, n_keys);
+            uint32_t peers = __match_any_sync(0xffffffffu, key);
+            if (key >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sh[key], __popc(peers));
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_keys; i += blockDim.x)
+        if (sh[i]) atomicAdd(&hist[i], sh[i]);
+}
+
+// tile_cnt[tile, key] = slots of `key` in tile `blockIdx.x`.
+__global__ void __launch_bounds__(kPlanWarps * 32)
+k_tile_count(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, int64_t N,
+             int32_t n_keys, int32_t *__restrict__ tile_cnt)
+{
+    extern __shared__ int32_t sh[];
+    for (int i = threadIdx.x; i < n_keys; i += blockDim.x) sh[i] = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t base = (int64_t)blockIdx.x * kPlanTile;
+    for (int64_t n = base + threadIdx.x - lane; n < base + kPlanTile; n += blockDim.x) {
+        int32_t key = slot_key(ids, keep, n + lane, N, n_keys);
+        uint32_t peers = __match_any_sync(0xffffffffu, key);
+        if (key >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sh[key], __popc(peers));
+    }
+    __syncthreads();
+    int32_t *out = tile_cnt + (int64_t)blockIdx.x * n_keys;
+    for (int i = threadIdx.x; i < n_keys; i += blockDim.x) out[i] = sh[i];
+}
+
+// One CTA of 1024 threads. In place: tile_cnt[t, key] <- sum_{t' < t} tile_cnt[t', key].
+// hist[key] = sum over tiles; key_off = exclusive prefix of hist over keys, with
+// key_off[n_keys] = total.
+__global__ void __launch_bounds__(1024)
+k_scan(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys, int32_t *__restrict__ hist,
+       int32_t *__restrict__ key_off)
+{
+    __shared__ int32_t part[32][33];
+    __shared__ int32_t wsum[32];
+    __shared__ int32_t carry;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int seg = (n_tiles + 31) / 32;
+    const int t0 = min(n_tiles, warp * seg), t1 = min(n_tiles, t0 + seg);
+    for (int e0 = 0; e0 < n_keys; e0 += 32) {
+        const int e = e0 + lane;
+        const bool ok = e < n_keys;
+        int32_t s = 0;
+        if (ok)
+            for (int t = t0; t < t1; t++) s += tile_cnt[(int64_t)t * n_keys + e];
+        part[warp][lane] = s;
+        __syncthreads();
+        if (warp == 0) {
+            int32_t run = 0;
+            for (int w = 0; w < 32; w++) {
+                int32_t v = part[w][lane];
+                part[w][lane] = run;
+                run += v;
+            }
+            if (ok) hist[e] = run;
+        }
+        __syncthreads();
+        if (ok) {
+            int32_t run = part[warp][lane];
+            for (int t = t0; t < t1; t++) {
+                int64_t i = (int64_t)t * n_keys + e;
+                int32_t v = tile_cnt[i];
+                tile_cnt[i] = run;
+                run += v;
+            }
+        }
+        __syncthreads();
+    }
+    // exclusive scan of hist over keys, 1024 keys per round
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    for (int e0 = 0; e0 < n_keys; e0 += 1024) {
+        const int e = e0 + threadIdx.x;
+        int32_t v = e < n_keys ? hist[e] : 0;
+        int32_t inc = v;
+        for (int d = 1; d < 32; d <<= 1) {
+            int32_t u = __shfl_up_sync(0xffffffffu, inc, d);
+            if (lane >= d) inc += u;
+        }
+        if (lane == 31) wsum[warp] = inc;
+        __syncthreads();
+        if (warp == 0) {
+            int32_t w = wsum[lane], wi = w;
+            for (int d = 1; d < 32; d <<= 1) {
+                int32_t u = __shfl_up_sync(0xffffffffu, wi, d);
+                if (lane >= d) wi += u;
+            }
+            wsum[lane] = wi - w;  // exclusive prefix of warp totals
+        }
+        __syncthreads();
+        const int32_t c = carry;
+        if (e < n_keys) key_off[e] = c + wsum[warp] + inc - v;
+        __syncthreads();
+        if (threadIdx.x == 1023) carry = c + wsum[31] + inc;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) key_off[n_keys] = carry;
+}
+
+// pos[n] = key_off[key] + (slots of key in earlier tiles) + (earlier slots of key in this
+// tile). Each warp owns a contiguous quarter... an eighth of the tile: it counts its
+// sub-range per key, the CTA turns those counts into per-warp bases, then each warp
+// walks its sub-range again in order, ranking equal keys with match.any.
+__global__ void __launch_bounds__(kPlanWarps * 32)
+k_rank(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, int64_t N, int32_t n_keys,
+       const int32_t *__restrict__ tile_base, const int32_t *__restrict__ key_off,
+       int32_t *__restrict__ pos)
+{
+    extern __shared__ int32_t cnt[];  // [kPlanWarps][n_keys]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < kPlanWarps * n_keys; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+    constexpr int kSub = kPlanTile / kPlanWarps;
+    const int64_t lo = (int64_t)blockIdx.x * kPlanTile + warp * kSub;
+    int32_t *mine = cnt + warp * n_keys;
+    for (int64_t n0 = lo; n0 < lo + kSub; n0 += 32) {
+        int32_t key = slot_key(ids, keep, n0 + lane, N, n_keys);
+        uint32_t peers = __match_any_sync(0xffffffffu, key);
+        if (key >= 0 && lane == __ffs(peers) - 1) mine[key] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    const int32_t *tb = tile_base + (int64_t)blockIdx.x * n_keys;
+    for (int e = threadIdx.x; e < n_keys; e += blockDim.x) {
+        int32_t run = key_off[e] + tb[e];
+        for (int w = 0; w < kPlanWarps; w++) {
+            int32_t v = cnt[w * n_keys + e];
+            cnt[w * n_keys + e] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    const uint32_t lt = lanemask_lt();
+    for (int64_t n0 = lo; n0 < lo + kSub; n0 += 32) {
+        const int64_t n = n0 + lane;
+        // slot_key flags out-of-range ids once more here; the bit is idempotent
+        int32_t key = slot_key(ids, keep, n, N, n_keys);
+        uint32_t peers = __match_any_sync(0xffffffffu, key);
+        int32_t p = -1;
+        if (key >= 0) p = mine[key] + __popc(peers & lt);
+        __syncwarp();
+        if (key >= 0 && lane == __ffs(peers) - 1) mine[key] += __popc(peers);
+        __syncwarp();
+        if (n < N) pos[n] = p;
+    }
+}
+
+// Rank that receives row `row` (row < total rows).
+__device__ __forceinline__ int32_t row_rank_balanced(int64_t row, int64_t SK) { return (int32_t)(row / SK); }
+
+// Smallest index i in [0, n] with a[i] > x (a ascending), for a in shared memory.
+__device__ __forceinline__ int32_t upper_bound_sh(const int32_t *a, int32_t n, int64_t x)
+{
+    int32_t lo = 0, hi = n + 1;
+    while (lo < hi) {
+        int32_t mid = (lo + hi) >> 1;
+        if (a[mid] > x) hi = mid;
+        else lo = mid + 1;
+    }
+    return lo;
+}
+
+// One CTA of 1024 threads: per-rank replica tables and the summary counts.
+// Dynamic shared memory: key_off (n_keys+1) + nz (n_keys+1) + rank_off (R+1) + e_lo (R).
+__global__ void __launch_bounds__(1024)
+k_plan_meta(const int32_t *__restrict__ hist, const int32_t *__restrict__ key_off_g, int32_t R,
+            int32_t n_keys, int64_t SK, int32_t mode, int32_t keys_per_rank,
+            int32_t *__restrict__ rank_off_out, int32_t *__restrict__ load_out,
+            int32_t *__restrict__ rep_count, int32_t *__restrict__ rep_key,
+            int32_t *__restrict__ rep_cu, int32_t *__restrict__ stats)
+{
+    extern __shared__ int32_t smem[];
+    int32_t *koff = smem;                    // n_keys + 1
+    int32_t *nz = koff + (n_keys + 1);       // n_keys + 1: exclusive count of non-empty keys
+    int32_t *roff = nz + (n_keys + 1);       // R + 1
+    int32_t *elo = roff + (R + 1);           // R: first key on each rank
+    __shared__ int32_t s_red[8];
+    __shared__ int32_t wsum[32];
+    __shared__ int32_t carry;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int32_t cap = n_keys;
+    const int32_t per_rank = (mode == 0) ? n_keys / R : keys_per_rank;
+
+    for (int i = threadIdx.x; i <= n_keys; i += blockDim.x) koff[i] = key_off_g[i];
+    if (threadIdx.x < 8) s_red[threadIdx.x] = 0;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    // nz = exclusive prefix count of keys with hist > 0
+    for (int e0 = 0; e0 <= n_keys; e0 += 1024) {
+        const int e = e0 + threadIdx.x;
+        int32_t v = (e < n_keys && koff[e + 1] > koff[e]) ? 1 : 0;
+        int32_t inc = v;
+        for (int d = 1; d < 32; d <<= 1) {
+            int32_t u = __shfl_up_sync(0xffffffffu, inc, d);
+            if (lane >= d) inc += u;
+        }
+        if (lane == 31) wsum[warp] = inc;
+        __syncthreads();
+        if (warp == 0) {
+            int32_t w = wsum[lane], wi = w;
+            for (int d = 1; d < 32; d <<= 1) {
+                int32_t u = __shfl_up_sync(0xffffffffu, wi, d);
+                if (lane >= d) wi += u;
+            }
+            wsum[lane] = wi - w;
+        }
+        __syncthreads();
+        const int32_t c = carry;
+        if (e <= n_keys) nz[e] = c + wsum[warp] + inc - v;
+        __syncthreads();
+        if (threadIdx.x == 1023) carry = c + wsum[31] + inc;
+        __syncthreads();
+    }
+    // rank offsets
+    for (int r = threadIdx.x; r <= R; r += blockDim.x) {
+        int64_t ro = (mode == 0) ? (int64_t)r * SK : (int64_t)koff[min(n_keys, r * keys_per_rank)];
+        roff[r] = (int32_t)ro;
+        rank_off_out[r] = (int32_t)ro;
+    }
+    __syncthreads();
+    // first key of each non-empty rank; replica counts; clear the tables
+    for (int r = threadIdx.x; r < R; r += blockDim.x) {
+        int32_t cnt = 0, first = 0;
+        if (roff[r + 1] > roff[r]) {
+            first = upper_bound_sh(koff, n_keys, roff[r]) - 1;
+            int32_t last = upper_bound_sh(koff, n_keys, (int64_t)roff[r + 1] - 1) - 1;
+            cnt = nz[last + 1] - nz[first];
+            atomicAdd(&s_red[6], 1);
+        }
+        elo[r] = first;
+        rep_count[r] = cnt;
+        atomicMax(&s_red[1], roff[r + 1] - roff[r]);
+        if (load_out) {
+            int32_t l;
+            if (mode == 0) l = koff[min(n_keys, (r + 1) * per_rank)] - koff[r * per_rank];
+            else l = roff[r + 1] - roff[r];
+            load_out[r] = l;
+        }
+    }
+    for (int64_t i = threadIdx.x; i < (int64_t)R * cap; i += blockDim.x) rep_key[i] = -1;
+    for (int64_t i = threadIdx.x; i < (int64_t)R * (cap + 1); i += blockDim.x) rep_cu[i] = 0;
+    __syncthreads();
+    // one thread per key: write its replica entries on every rank it spans
+    for (int e = threadIdx.x; e < n_keys; e += blockDim.x) {
+        const int32_t b = koff[e], en = koff[e + 1];
+        atomicMax(&s_red[5], en - b);
+        if (mode == 0 && e % per_rank == 0) {
+            int32_t l = koff[min(n_keys, e + per_rank)] - b;   // home load of rank e/per_rank
+            atomicMax(&s_red[0], l);
+        }
+        if (en <= b) continue;
+        int32_t r0, r1;
+        if (mode == 0) {
+            r0 = row_rank_balanced(b, SK);
+            r1 = row_rank_balanced((int64_t)en - 1, SK);
+        } else {
+            r0 = r1 = e / keys_per_rank;
+        }
+        const int32_t home = e / per_rank;
+        int32_t pf = 0;
+        for (int32_t r = r0; r <= r1; r++) {
+            const int32_t j = nz[e] - nz[elo[r]];
+            rep_key[(int64_t)r * cap + j] = e;
+            rep_cu[(int64_t)r * (cap + 1) + j] = max(b, roff[r]) - roff[r];
+            if (mode == 0 && r != home) pf++;
+        }
+        if (r1 > r0) atomicAdd(&s_red[2], r1 - r0);
+        if (pf) atomicAdd(&s_red[3], pf);
+    }
+    __syncthreads();
+    for (int r = threadIdx.x; r < R; r += blockDim.x)
+        rep_cu[(int64_t)r * (cap + 1) + rep_count[r]] = roff[r + 1] - roff[r];
+    if (threadIdx.x == 0) {
+        stats[0] = (mode == 0) ? s_red[0] : s_red[1];
+        stats[1] = s_red[1];
+        stats[2] = s_red[2];
+        stats[3] = s_red[3];
+        stats[4] = koff[n_keys];
+        stats[5] = s_red[5];
+        stats[6] = s_red[6];
+        stats[7] = 0;
+    }
+}
+
+}  // namespace mep

@@ -1,0 +1,257 @@
+/*
+ * mep.h — C ABI of libmep: MoE expert-parallel token routing on one B200 (sm_100a).
+ *
+ * The path: a per-expert histogram of the top-K expert ids, a perfectly balanced
+ * placement plan (every one of R ranks receives exactly S*K token-slots; experts that
+ * straddle a rank boundary get temporary redundant replicas), the logical->physical
+ * expert mapping with score-threshold pruning, and dispatch / combine of bf16 hidden
+ * rows. The R expert-parallel ranks are R partitions of one GPU's memory: rank r's
+ * receive buffer is rows [rank_off[r], rank_off[r+1]) of one [rows, H] array.
+ *
+ * Conventions for every call
+ *  - Pointers named in a signature are DEVICE pointers owned by the caller unless the
+ *    comment says otherwise; the library keeps no reference after the call returns
+ *    and allocates no device memory. Scratch memory comes from the caller through a
+ *    workspace argument whose size a *_workspace_size query returns (the two-phase
+ *    "query the workspace size, then execute on a stream" pattern of the aclnn
+ *    interfaces, gitcode ops-transformer aclnnMoeUpdateExpert doc, 函数原型).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream) and never synchronise the host, so a chain plan -> dispatch -> combine
+ *    needs no host round trip (MoonEP's static shapes remove per-layer host syncs:
+ *    twodots.gr article on MoonEP, static-shapes paragraph). All of them can be
+ *    issued into a CUDA graph capture, except mep_get_error.
+ *  - A call first checks its arguments on the host and returns a status without
+ *    launching anything when one is wrong: MEP_ERR_NULLPTR / MEP_ERR_DTYPE /
+ *    MEP_ERR_SHAPE / MEP_ERR_VALUE mirror the aclnn codes 161001 (null tensor),
+ *    161002 (unsupported data type) and 561002 (shape or value out of range) of the
+ *    aclnnMoeUpdateExpert doc (返回值).
+ *  - Errors that depend on the data (an expert id out of range, a malformed
+ *    eplb_table row, an active mask with a true after a false, a row index outside
+ *    the receive buffer) cannot be seen on the host. The kernels then skip the
+ *    offending element (never touching memory outside the buffers) and set a bit in a
+ *    sticky per-device error word that mep_get_error reads. Nothing traps.
+ *  - bf16 data is passed as its 16-bit patterns (uint16_t); int8 codes as int8_t.
+ *  - Receive buffers are overwritten by the next dispatch; views into them must not
+ *    outlive it (the zero-copy lifetime rule of MoonEP, twodots.gr article on
+ *    MoonEP, zero-copy views paragraph).
+ *
+ * Notation: global token g = src*S + t, slot n = g*K + k, N = R*S*K, T = R*S;
+ * home(e) = e / (E/R).
+ */
+#ifndef MEP_H
+#define MEP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *mep_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    MEP_OK = 0,
+    MEP_ERR_NULLPTR = 1,   /* a required pointer is NULL (cf. aclnn 161001) */
+    MEP_ERR_DTYPE = 2,     /* unsupported element type or quantisation mode (cf. 161002) */
+    MEP_ERR_SHAPE = 3,     /* a size outside the supported range (cf. 561002) */
+    MEP_ERR_VALUE = 4,     /* an argument value outside its range (cf. 561002) */
+    MEP_ERR_WORKSPACE = 5, /* workspace NULL, too small or not 256-byte aligned */
+    MEP_ERR_CUDA = 6       /* a CUDA call failed; the CUDA error is in mep_last_cuda_error() */
+} mep_status_t;
+
+/* Bits of the device error word (see mep_get_error). */
+#define MEP_DERR_KEY_RANGE 0x1  /* an expert / instance id outside [0, n_keys) */
+#define MEP_DERR_ROW_RANGE 0x2  /* a slot row outside [-1, rows) */
+#define MEP_DERR_TABLE     0x4  /* eplb_table: count outside [1, F-1] or instance id outside [0, 1024) */
+#define MEP_DERR_MASK      0x8  /* active_mask has a true after a false */
+
+/* Plan modes. */
+#define MEP_PLAN_BALANCED 0
+#define MEP_PLAN_GROUPED  1
+
+/* Limits. */
+#define MEP_MAX_KEYS 4096   /* experts (balanced) or physical instances (grouped) */
+#define MEP_MAX_K    32     /* experts per token in dispatch / combine / plan */
+
+/* Plan summary, written by mep_plan to device memory. All counts are exact integers;
+ * maxvio = max_load / (S*K) - 1 (before planning) and max_chunk / (S*K) - 1 (after)
+ * are left to the caller so that they are computed once, in double precision. */
+typedef struct {
+    int32_t max_load;   /* max over ranks of the rows its home experts would receive */
+    int32_t max_chunk;  /* max over ranks of the rows it receives under the plan */
+    int32_t redundant;  /* sum over experts of (#ranks holding a replica - 1) */
+    int32_t prefetched; /* #(rank, expert) replicas placed on a rank other than home(e) */
+    int32_t n_kept;     /* slots placed (N minus dropped slots) */
+    int32_t max_hist;   /* max over keys of hist (expert-level load) */
+    int32_t n_ranks_used; /* ranks that receive at least one row */
+    int32_t reserved;
+} mep_plan_stats_t;
+
+/* Library version, (major << 16) | minor. */
+int32_t mep_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char *mep_status_string(mep_status_t status);
+
+/* The cudaError_t of the last call that returned MEP_ERR_CUDA on this host thread. */
+int32_t mep_last_cuda_error(void);
+
+/*
+ * Reads the sticky device error word of the CURRENT device into *code (a host
+ * pointer; 0 = no data error since the last clear), after synchronising the device.
+ * With clear != 0 the word is reset to 0. Returns MEP_ERR_NULLPTR if code is NULL.
+ * This is the only call that synchronises.
+ */
+mep_status_t mep_get_error(int32_t *code, int32_t clear);
+
+/*
+ * a1 — per-expert histogram (tokens per expert: twodots.gr article on MoonEP, "six
+ * checks before trying MoonEP": measure tokens per expert and maxvio).
+ *   hist[e] = #{ i in [0,n) : ids[i] == e },  e in [0, n_keys).
+ * ids: int32 [n]; hist: int32 [n_keys] (overwritten). Ids outside [0, n_keys) are not
+ * counted and set MEP_DERR_KEY_RANGE.
+ * Errors: NULL pointer (MEP_ERR_NULLPTR); n < 0, n >= 2^31, n_keys outside
+ * [1, MEP_MAX_KEYS] (MEP_ERR_SHAPE).
+ */
+mep_status_t mep_histogram(const int32_t *ids, int64_t n, int32_t n_keys, int32_t *hist,
+                           mep_stream_t stream);
+
+/* Bytes of workspace mep_plan needs for N = R*S*K slots and n_keys keys. */
+size_t mep_plan_workspace_size(int32_t R, int32_t n_keys, int32_t S, int32_t K);
+
+/*
+ * a2 — placement plan: the row of every slot in the R ranks' receive buffers.
+ *
+ * MEP_PLAN_BALANCED (keys = logical experts, n_keys = E, E % R == 0, keep == NULL):
+ *   the perfectly balanced plan of MoonEP (twodots.gr article on MoonEP: every rank
+ *   processes exactly S*K token-slots; a few temporary redundant replicas of hot
+ *   experts absorb the skew). Slots are ordered by (home(e), e, src, t, k) and the
+ *   ordered list is cut into R chunks of S*K rows; rank r receives rows
+ *   [r*S*K, (r+1)*S*K). An expert whose rows straddle a cut has a replica on every
+ *   rank it reaches. Because home(e) is monotone in e and the slot index orders
+ *   (src, t, k), the row of slot n is  off[e] + #{m < n : ids[m] == e}  with off the
+ *   exclusive prefix sum of hist: a stable counting sort.
+ * MEP_PLAN_GROUPED (keys = physical instance ids after mep_update_expert,
+ *   n_keys = R * keys_per_rank, keep optional): every kept slot goes to the rank that
+ *   hosts its instance, rank = key / keys_per_rank; rows are ordered by (key, slot)
+ *   and packed, rank r owning rows [rank_off[r], rank_off[r+1]); dropped slots
+ *   (keep[n] == 0) get pos = -1. (Receive layout of aclnnMoeDistributeDispatch after
+ *   the aclnnMoeUpdateExpert mapping, gitcode ops-transformer doc, 调用示例.)
+ *
+ * Inputs:  ids int32 [N] (slot n = (src*S + t)*K + k); keep uint8 [N] or NULL.
+ * Outputs (all device, overwritten):
+ *   pos       int32 [N]           row of every slot, -1 = dropped
+ *   hist      int32 [n_keys]      slots per key (kept slots only)
+ *   rank_off  int32 [R+1]         first row of every rank, rank_off[R] = n_kept
+ *   load      int32 [R] or NULL   rows rank r would receive if no expert moved:
+ *                                 sum of hist over its home keys
+ *   rep_count int32 [R]           replicas (distinct keys) on each rank
+ *   rep_key   int32 [R, n_keys]   the keys of rank r's replicas, ascending; -1 after
+ *                                 rep_count[r]
+ *   rep_cu    int32 [R, n_keys+1] cu_seqlens of rank r's replicas relative to
+ *                                 rank_off[r] (the grouped-GEMM offsets MoonEP's
+ *                                 planner produces); 0 after rep_count[r]
+ *   stats     mep_plan_stats_t [1]
+ * Workspace: at least mep_plan_workspace_size(R, n_keys, S, K) bytes, 256-byte aligned.
+ * Errors: NULL pointer; R, S, K < 1, K > MEP_MAX_K, N >= 2^31, n_keys outside
+ * [1, MEP_MAX_KEYS] (MEP_ERR_SHAPE); mode unknown, E % R != 0, keep given in
+ * balanced mode, keys_per_rank * R != n_keys in grouped mode (MEP_ERR_VALUE);
+ * workspace too small (MEP_ERR_WORKSPACE). Ids outside [0, n_keys) are dropped
+ * (pos = -1) and set MEP_DERR_KEY_RANGE.
+ */
+mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_t n_keys,
+                      int32_t S, int32_t K, int32_t mode, int32_t keys_per_rank,
+                      int32_t *pos, int32_t *hist, int32_t *rank_off, int32_t *load,
+                      int32_t *rep_count, int32_t *rep_key, int32_t *rep_cu,
+                      mep_plan_stats_t *stats, void *workspace, size_t workspace_bytes,
+                      mep_stream_t stream);
+
+/*
+ * a3 — logical->physical expert mapping and score-threshold pruning
+ * (aclnnMoeUpdateExpert, gitcode ops-transformer doc, 功能说明 / 参数说明).
+ *
+ * For slot (i, k), e = expert_ids[i,k], c = eplb_table[e, 0] (instances of e):
+ *   c == 1            -> balanced_expert_ids[i,k] = eplb_table[e, 1]
+ *   balance_mode 0    -> eplb_table[e, local_rank_id / ceil(world_size / c) + 1]  (by rank)
+ *   balance_mode 1    -> eplb_table[e, (i mod c) + 1]                             (by token)
+ * (ceil is a true ceiling; i is the token index.)
+ * Pruning: v_i = sum_k fl(expert_scales[i,k] * pruning_threshold[k]) accumulated in
+ * fp32 in ascending k; balanced_active_mask[i,k] = active_mask[i] &&
+ * !(expert_scales[i,k] < v_i). Without scales and threshold the mask is
+ * active_mask[i] broadcast over k (all 1 when active_mask is NULL too).
+ *
+ * expert_ids int32 [BS, K]; eplb_table int32 [n_experts, F] (column 0 = count in
+ * [1, F-1], columns 1..count = distinct instance ids in [0, 1024)); expert_scales fp32
+ * [BS, K] (descending within a token) or NULL; pruning_threshold fp32 [K] or NULL;
+ * active_mask uint8 [BS] (every 1 before every 0) or NULL.
+ * Outputs: balanced_expert_ids int32 [BS, K]; balanced_active_mask uint8 [BS, K].
+ * Errors: NULL required pointer; scales without threshold or the reverse; a mask
+ * without scales and threshold (MEP_ERR_NULLPTR, the doc's pairing rules);
+ * BS < 1, K outside [1, 16], K > n_experts, n_experts outside [1, 1024], F outside
+ * [2, world_size + 1] (MEP_ERR_SHAPE); balance_mode outside {0,1}, world_size outside
+ * [2, 768] or local_rank_id outside [0, world_size) in mode 0 (MEP_ERR_VALUE).
+ * The doc's BS <= 512 is a limit of the Ascend part and is not enforced.
+ * Data errors: id out of range (MEP_DERR_KEY_RANGE, output -1), bad table row
+ * (MEP_DERR_TABLE, output -1), mask order (MEP_DERR_MASK).
+ */
+mep_status_t mep_update_expert(const int32_t *expert_ids, const int32_t *eplb_table,
+                               const float *expert_scales, const float *pruning_threshold,
+                               const uint8_t *active_mask, int64_t BS, int32_t K,
+                               int32_t n_experts, int32_t F, int64_t local_rank_id,
+                               int64_t world_size, int64_t balance_mode,
+                               int32_t *balanced_expert_ids, uint8_t *balanced_active_mask,
+                               mep_stream_t stream);
+
+/*
+ * a4 — dispatch: every kept slot's token row written straight to its final row of the
+ * receive buffer (MoonEP zero-copy dispatch: tokens land in their final,
+ * expert-grouped positions; twodots.gr article on MoonEP, zero-copy paragraph).
+ *   quant == 0:  recv[pos[n], :] = x[n / K, :]                  (bf16 copy)
+ *   quant == 1:  per-token dynamic symmetric int8 (one fp32 scale per token, the
+ *                dynamicScales output of aclnnMoeDistributeDispatch):
+ *                amax = max_h |x[g,h]|, scale = amax / 127 (fp32 division),
+ *                q = clamp(round_half_even(x / scale), -127, 127), q = 0 if amax == 0;
+ *                recv[pos[n], :] = q (int8), recv_scale[pos[n]] = scale.
+ * x bf16 [T, H]; pos int32 [T*K] (-1 = dropped); recv bf16 or int8 [rows, H];
+ * recv_scale fp32 [rows] (quant == 1 only, else ignored). Rows no slot points at are
+ * left untouched.
+ * Errors: NULL pointer; T < 0, K outside [1, MEP_MAX_K], H < 1, rows < 0,
+ * T*K >= 2^31 (MEP_ERR_SHAPE); quant outside {0,1} (MEP_ERR_DTYPE). A pos outside
+ * [-1, rows) is skipped and sets MEP_DERR_ROW_RANGE.
+ */
+mep_status_t mep_dispatch(const uint16_t *x, const int32_t *pos, int64_t T, int32_t K,
+                          int64_t H, int32_t quant, void *recv, float *recv_scale,
+                          int64_t rows, mep_stream_t stream);
+
+/*
+ * Identity expert on int8 rows: y[r, h] = bf16_rne(fl(float(q[r,h]) * scale[r])).
+ * Turns an int8 dispatch result back into bf16 rows for combine.
+ * q int8 [rows, H]; scale fp32 [rows]; y bf16 [rows, H].
+ * Errors: NULL pointer; rows < 0, H < 1 (MEP_ERR_SHAPE).
+ */
+mep_status_t mep_dequantize(const int8_t *q, const float *scale, int64_t rows, int64_t H,
+                            uint16_t *y, mep_stream_t stream);
+
+/*
+ * a5 — combine: the K returned rows of every token weighted by its gates and summed
+ * back in token order (aclnnMoeDistributeCombine: expandX rows weighted by
+ * expertScales; gitcode ops-transformer aclnnMoeUpdateExpert doc, 调用示例).
+ *   out[g, h] = bf16_rne( sum over k = 0..K-1 with pos[g*K+k] >= 0, in ascending k,
+ *                         of fl(gates[g*K+k] * float(y[pos[g*K+k], h])) )
+ * accumulated in fp32 starting from +0, each product and sum rounded on its own (no
+ * fused multiply-add). A token with no kept slot gives a zero row.
+ * y bf16 [rows, H]; pos int32 [T*K]; gates fp32 [T*K]; out bf16 [T, H].
+ * Errors: NULL pointer; T < 0, K outside [1, MEP_MAX_K], H < 1, rows < 0,
+ * T*K >= 2^31 (MEP_ERR_SHAPE). A pos outside [-1, rows) is treated as dropped and
+ * sets MEP_DERR_ROW_RANGE.
+ */
+mep_status_t mep_combine(const uint16_t *y, int64_t rows, const int32_t *pos,
+                         const float *gates, int64_t T, int32_t K, int64_t H, uint16_t *out,
+                         mep_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MEP_H */

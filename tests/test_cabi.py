@@ -1,0 +1,101 @@
+"""The C-ABI library on a machine without a GPU: it builds, loads, exports every
+function include/mep.h declares, and rejects bad arguments with the documented status
+before touching the GPU (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "mep.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mep_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from dispatch_combine_topk_b200 import build
+    build.build()
+    import dispatch_combine_topk_b200 as mep
+    return mep.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert {"mep_plan", "mep_update_expert", "mep_dispatch", "mep_combine", "mep_histogram",
+            "mep_plan_workspace_size", "mep_get_error", "mep_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version(L):
+    assert L.mep_version() >> 16 == 1
+    for code in range(7):
+        assert L.mep_status_string(code)
+    assert b"unknown" in L.mep_status_string(99)
+
+
+FAKE = ctypes.c_void_p(0x1000)   # never dereferenced: every call below fails its checks
+
+
+def test_plan_argument_checks(L):
+    P = FAKE
+    args = lambda **kw: dict(dict(ids=P, keep=None, R=2, E=4, S=2, K=2, mode=0, kpr=0,
+                                  ws=P, wsb=1 << 20), **kw)
+
+    def call(a):
+        return L.mep_plan(a["ids"], a["keep"], a["R"], a["E"], a["S"], a["K"], a["mode"], a["kpr"],
+                          P, P, P, None, P, P, P, P, a["ws"], a["wsb"], None)
+    assert call(args(ids=None)) == 1                      # NULLPTR
+    assert call(args(R=0)) == 3                           # SHAPE
+    assert call(args(K=33)) == 3
+    assert call(args(E=5000)) == 3
+    assert call(args(R=1 << 16, S=1 << 16)) == 3          # N >= 2^31
+    assert call(args(E=5)) == 4                           # VALUE: E % R != 0
+    assert call(args(keep=P)) == 4                        # VALUE: mask in balanced mode
+    assert call(args(mode=7)) == 4
+    assert call(args(mode=1, kpr=3)) == 4                 # kpr * R != n_keys
+    assert call(args(ws=None)) == 5                       # WORKSPACE
+    assert call(args(wsb=8)) == 5
+    assert call(args(ws=ctypes.c_void_p(0x1008))) == 5    # not 256-byte aligned
+    assert L.mep_plan_workspace_size(8, 64, 4096, 8) >= 128 * 64 * 4
+
+
+def test_update_expert_argument_checks(L):
+    P = FAKE
+
+    def call(scales=None, thr=None, act=None, BS=4, K=2, E=8, F=2, rank=0, ws=2, mode=0):
+        return L.mep_update_expert(P, P, scales, thr, act, BS, K, E, F, rank, ws, mode, P, P, None)
+    assert call(scales=P) == 1
+    assert call(thr=P) == 1
+    assert call(act=P) == 1
+    assert call(K=17) == 3
+    assert call(E=1025) == 3
+    assert call(K=3, E=2) == 3
+    assert call(F=4) == 3            # F > world_size + 1
+    assert call(mode=2) == 4
+    assert call(ws=769) == 4
+    assert call(rank=2) == 4
+    assert call(ws=1) == 4           # F=2 <= ws+1 is fine; ws < 2 in mode 0 -> VALUE
+
+
+def test_dispatch_combine_argument_checks(L):
+    P = FAKE
+    assert L.mep_dispatch(P, P, 4, 2, 64, 2, P, P, 8, None) == 2         # DTYPE
+    assert L.mep_dispatch(None, P, 4, 2, 64, 0, P, None, 8, None) == 1   # NULLPTR
+    assert L.mep_dispatch(P, P, 4, 2, 64, 1, P, None, 8, None) == 1      # int8 without scales
+    assert L.mep_dispatch(P, P, 4, 0, 64, 0, P, None, 8, None) == 3
+    assert L.mep_dispatch(P, P, 4, 2, 0, 0, P, None, 8, None) == 3
+    assert L.mep_dispatch(P, P, 0, 2, 64, 0, P, None, 8, None) == 0      # empty: no launch
+    assert L.mep_combine(P, 8, None, P, 4, 2, 64, P, None) == 1
+    assert L.mep_combine(P, 8, P, P, 4, 33, 64, P, None) == 3
+    assert L.mep_combine(P, -1, P, P, 4, 2, 64, P, None) == 3
+    assert L.mep_combine(P, 8, P, P, 0, 2, 64, P, None) == 0
+    assert L.mep_histogram(P, 10, 0, P, None) == 3
+    assert L.mep_histogram(P, 10, 4, None, None) == 1
+    assert L.mep_dequantize(None, P, 4, 8, P, None) == 1
+    assert L.mep_get_error(None, 0) == 1

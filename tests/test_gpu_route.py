@@ -1,0 +1,258 @@
+"""GPU parity of dispatch (bf16 and int8), dequantisation and combine against the
+oracle: element by element at small sizes (several CTAs, ragged rows), and at the full
+workload sizes on sampled tokens the oracle routes one by one plus properties checked
+on every row."""
+import numpy as np
+import pytest
+import torch
+
+import dispatch_combine_topk_b200 as mep
+import oracle
+import synth
+from gpu_helpers import bits, dev, gpu_plan_balanced, gpu_plan_grouped
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clear_error_word():
+    torch.cuda.set_device(0)
+    mep.mep_get_error(clear=True)
+    yield
+
+
+def _rand_bf16(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * scale).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("T,K,H", [(1, 1, 8), (37, 3, 256), (64, 8, 4096), (5, 32, 72),
+                                   (33, 2, 7), (12, 4, 130), (300, 6, 7168)])
+@pytest.mark.parametrize("quant", [0, 1])
+def test_dispatch_combine_small_exact(T, K, H, quant):
+    rng = np.random.default_rng(T * 100 + K * 10 + H + quant)
+    rows = T * K + 3
+    pos = rng.permutation(rows)[: T * K].astype(np.int32)
+    pos[rng.random(T * K) < 0.15] = -1
+    x = _rand_bf16((T, H), T + H, scale=float(rng.uniform(0.01, 50)))
+    gates = rng.random(T * K).astype(np.float32)
+    xb = bits(x)
+    x_d, pos_d = x.to(dev()), torch.from_numpy(pos).to(dev())
+    if quant == 0:
+        recv = torch.zeros((rows, H), dtype=torch.bfloat16, device=dev())
+        mep.mep_dispatch(x_d, pos_d, K, recv)
+        ref = oracle.dispatch(xb, pos, K, rows)
+        assert np.array_equal(bits(recv), ref)
+        y_d, y_ref = recv, ref
+    else:
+        recv = torch.zeros((rows, H), dtype=torch.int8, device=dev())
+        sc = torch.zeros(rows, dtype=torch.float32, device=dev())
+        mep.mep_dispatch(x_d, pos_d, K, recv, sc, quant=1)
+        q_ref, s_ref = oracle.dispatch_int8(xb, pos, K, rows)
+        assert np.array_equal(recv.cpu().numpy(), q_ref)
+        assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+        y_d = torch.empty((rows, H), dtype=torch.bfloat16, device=dev())
+        mep.mep_dequantize(recv, sc, y_d)
+        y_ref = oracle.dequantize(q_ref, s_ref)
+        assert np.array_equal(bits(y_d), y_ref)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev())
+    mep.mep_combine(y_d, pos_d, torch.from_numpy(gates).to(dev()), K, out)
+    assert np.array_equal(bits(out), oracle.combine(y_ref, pos, gates, K))
+    assert mep.mep_get_error() == 0
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 4, 5, 6, 8, 16, 32])
+def test_combine_random_rows_every_k(K):
+    """Arbitrary expert rows (not copies of the token) and every K: catches a slot that
+    reads the wrong row or sums in another order."""
+    rng = np.random.default_rng(K)
+    T, H, rows = 97, 1024, 500
+    y = _rand_bf16((rows, H), 100 + K)
+    pos = rng.integers(0, rows, T * K).astype(np.int32)
+    pos[rng.random(T * K) < 0.1] = -1
+    gates = (rng.standard_normal(T * K) * 3).astype(np.float32)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev())
+    mep.mep_combine(y.to(dev()), torch.from_numpy(pos).to(dev()), torch.from_numpy(gates).to(dev()), K, out)
+    assert np.array_equal(bits(out), oracle.combine(bits(y), pos, gates, K))
+
+
+def test_quant_edge_rows():
+    """Zero rows (scale 0), exact ties (scale 1), outliers, denormal-range values."""
+    H, K = 64, 2
+    x = torch.zeros((4, H), dtype=torch.float32)
+    x[1, :12] = torch.tensor([127.0, 2.5, 3.5, -2.5, -3.5, 0.5, 1.5, -0.5, 0.0, 126.5, -127.0, 0.25])
+    x[2] = torch.linspace(-3000, 3000, H)
+    x[3] = torch.linspace(-1e-37, 1e-37, H)
+    xb16 = x.to(torch.bfloat16)
+    pos = np.arange(4 * K, dtype=np.int32)
+    recv = torch.zeros((4 * K, H), dtype=torch.int8, device=dev())
+    sc = torch.zeros(4 * K, dtype=torch.float32, device=dev())
+    mep.mep_dispatch(xb16.to(dev()), torch.from_numpy(pos).to(dev()), K, recv, sc, quant=1)
+    q_ref, s_ref = oracle.dispatch_int8(bits(xb16), pos, K, 4 * K)
+    assert np.array_equal(recv.cpu().numpy(), q_ref)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert recv[2:4].abs().max().item() == 0 and sc[0].item() == 0.0
+
+
+def test_row_out_of_range_is_skipped_and_flagged():
+    T, K, H = 4, 2, 64
+    x = _rand_bf16((T, H), 1).to(dev())
+    pos = torch.tensor([0, 1, 2, 3, 4, 5, 6, 99], dtype=torch.int32, device=dev())
+    recv = torch.zeros((T * K + 4, H), dtype=torch.bfloat16, device=dev())
+    mep.mep_dispatch(x, pos, K, recv[: T * K])
+    assert mep.mep_get_error() & mep.DERR_ROW_RANGE
+    assert recv[T * K:].abs().max().item() == 0   # guard rows untouched
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev())
+    mep.mep_combine(recv[: T * K], pos, torch.ones(T * K, device=dev()), K, out)
+    assert mep.mep_get_error() & mep.DERR_ROW_RANGE
+
+
+def test_empty_inputs():
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device=dev())
+    pos = torch.empty(0, dtype=torch.int32, device=dev())
+    recv = torch.empty((0, 64), dtype=torch.bfloat16, device=dev())
+    mep.mep_dispatch(x, pos, 4, recv)
+    out = torch.empty((0, 64), dtype=torch.bfloat16, device=dev())
+    mep.mep_combine(recv, pos, torch.empty(0, device=dev()), 4, out)
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- full workloads
+
+def _route_full(name):
+    """Plan + dispatch (+ dequant) + combine of a whole workload on the GPU, exactly as
+    bench.py launches it."""
+    w = synth.get(name)
+    ids, gates = synth.router(w)
+    x = synth.hidden(w)
+    pb = gpu_plan_balanced(ids, w.R, w.E, w.S, w.K)
+    x_d = x.to(dev())
+    g_d = torch.from_numpy(gates).to(dev())
+    if w.quant:
+        recv = torch.empty((w.N, w.H), dtype=torch.int8, device=dev())
+        sc = torch.empty(w.N, dtype=torch.float32, device=dev())
+        mep.mep_dispatch(x_d, pb.pos, w.K, recv, sc, quant=1)
+        y = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev())
+        mep.mep_dequantize(recv, sc, y)
+    else:
+        recv, sc = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev()), None
+        mep.mep_dispatch(x_d, pb.pos, w.K, recv)
+        y = recv
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev())
+    mep.mep_combine(y, pb.pos, g_d, w.K, out)
+    torch.cuda.synchronize()
+    return w, ids, gates, x, x_d, pb, recv, sc, y, out
+
+
+def _row_checksum(t, chunk=32768):
+    """Per-row sum of the raw 16-bit (or 8-bit) patterns, on the device, in row chunks
+    (int32 is exact: |sum| <= 32768 * H)."""
+    if t.dtype == torch.bfloat16:
+        t = t.view(torch.int16)
+    out = torch.empty(t.shape[0], dtype=torch.int32, device=t.device)
+    for i in range(0, t.shape[0], chunk):
+        out[i:i + chunk] = t[i:i + chunk].to(torch.int32).sum(1, dtype=torch.int32)
+    return out
+
+
+@pytest.mark.parametrize("name", ["r8", "skew", "int8"])
+def test_full_workload_sampled_and_properties(name):
+    w, ids, gates, x, x_d, pb, recv, sc, y, out = _route_full(name)
+    assert mep.mep_get_error() == 0
+    p = oracle.plan_balanced(ids, w.R, w.E, w.S, w.K)
+    assert np.array_equal(pb.pos.cpu().numpy(), p.pos)
+    pos_d = pb.pos.long()
+    g_of_slot = torch.arange(w.N, device=dev()) // w.K
+    # every row: the row a slot landed on carries that slot's token (checksums)
+    if not w.quant:
+        assert torch.equal(_row_checksum(recv)[pos_d], _row_checksum(x_d)[g_of_slot])
+    # every token: identity expert with softmax gates gives back the expert row exactly
+    if not w.quant:
+        assert torch.equal(out.view(torch.int16), x_d.view(torch.int16))
+    else:
+        first = pos_d.view(w.T, w.K)[:, 0]
+        assert torch.equal(out.view(torch.int16), y[first].view(torch.int16))
+        # all K copies of a token carry the same codes and scale
+        cs = _row_checksum(recv)
+        assert torch.equal(cs[pos_d].view(w.T, w.K), cs[first][:, None].expand(w.T, w.K))
+        assert torch.equal(sc[pos_d].view(w.T, w.K), sc[first][:, None].expand(w.T, w.K))
+    # sampled tokens, routed one by one by the oracle (first and last tokens of every
+    # rank, plus random ones)
+    rng = np.random.default_rng(11)
+    toks = np.unique(np.concatenate([np.arange(w.R) * w.S, np.arange(1, w.R + 1) * w.S - 1,
+                                     rng.integers(0, w.T, 200)]))
+    xb = bits(x[toks])
+    kept = np.ones((toks.size, w.K), bool)
+    ref = oracle.route_tokens(xb, kept, gates[toks], w.K, w.quant)
+    assert np.array_equal(bits(out[torch.from_numpy(toks).to(dev())]), ref)
+    slots = (toks[:, None] * w.K + np.arange(w.K)[None, :]).ravel()
+    rows = torch.from_numpy(p.pos[slots].astype(np.int64)).to(dev())
+    for i, t in enumerate(toks):
+        pos_small = np.arange(w.K, dtype=np.int32)
+        if w.quant:
+            q_ref, s_ref = oracle.dispatch_int8(xb[i:i + 1], pos_small, w.K, w.K)
+            got_q = recv[rows[i * w.K:(i + 1) * w.K]].cpu().numpy()
+            got_s = sc[rows[i * w.K:(i + 1) * w.K]].cpu().numpy()
+            assert np.array_equal(got_q, q_ref) and np.array_equal(got_s, s_ref)
+        else:
+            ref_rows = oracle.dispatch(xb[i:i + 1], pos_small, w.K, w.K)
+            assert np.array_equal(bits(recv[rows[i * w.K:(i + 1) * w.K]]), ref_rows)
+
+
+def test_full_r8_combine_random_expert_rows():
+    """Full-size combine on arbitrary expert rows, sampled tokens checked by the oracle."""
+    w = synth.get("r8")
+    ids, gates = synth.router(w)
+    pb = gpu_plan_balanced(ids, w.R, w.E, w.S, w.K)
+    y = synth.expert_outputs(w, w.N)
+    y_d = y.to(dev())
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev())
+    mep.mep_combine(y_d, pb.pos, torch.from_numpy(gates).to(dev()), w.K, out)
+    pos = pb.pos.cpu().numpy()
+    toks = np.random.default_rng(12).integers(0, w.T, 300)
+    for t in toks:
+        rows = pos[t * w.K:(t + 1) * w.K]
+        ys = bits(y[torch.from_numpy(rows.astype(np.int64))])
+        ref = oracle.combine(ys, np.arange(w.K, dtype=np.int32), gates[t], w.K)
+        assert np.array_equal(bits(out[int(t)]), ref[0])
+
+
+def test_mapping_workload_dispatch_combine_exact():
+    """The page-4 op end to end: mapping + pruning on every rank, grouped plan over the
+    272 physical instances, dispatch H=4096, combine; every element compared."""
+    w = synth.get("map")
+    ids, gates = synth.router(w)
+    table, thr, active = synth.mapping_inputs(w)
+    n_keys = w.R * w.place_per_rank
+    for mode in (0, 1):
+        bi = torch.empty((w.T, w.K), dtype=torch.int32, device=dev())
+        bm = torch.empty((w.T, w.K), dtype=torch.uint8, device=dev())
+        oi = np.empty_like(ids)
+        om = np.empty(ids.shape, bool)
+        for r in range(w.R):
+            sl = slice(r * w.S, (r + 1) * w.S)
+            mep.mep_update_expert(torch.from_numpy(ids[sl].copy()).to(dev()),
+                                  torch.from_numpy(table).to(dev()),
+                                  torch.from_numpy(gates[sl].copy()).to(dev()),
+                                  torch.from_numpy(thr).to(dev()),
+                                  torch.from_numpy(active[sl].astype(np.uint8)).to(dev()),
+                                  r, w.R, mode, bi[sl], bm[sl])
+            oi[sl], om[sl] = oracle.update_expert(ids[sl], table, gates[sl], thr, active[sl], r, w.R, mode)
+        pb = mep.PlanBuffers.allocate(w.R, n_keys, w.S, w.K, dev())
+        mep.mep_plan(bi.view(-1), w.R, n_keys, w.S, w.K, pb, mode=mep.MEP_PLAN_GROUPED,
+                     keys_per_rank=w.place_per_rank, keep=bm.view(-1))
+        p = oracle.plan_grouped(oi, om, w.R, n_keys, w.place_per_rank, w.S, w.K)
+        assert np.array_equal(pb.pos.cpu().numpy(), p.pos)
+        x = synth.hidden(w)
+        rows = p.n_kept
+        recv = torch.zeros((rows, w.H), dtype=torch.bfloat16, device=dev())
+        mep.mep_dispatch(x.to(dev()), pb.pos, w.K, recv)
+        y_ref = oracle.dispatch(bits(x), p.pos, w.K, rows)
+        assert np.array_equal(bits(recv), y_ref)
+        out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev())
+        mep.mep_combine(recv, pb.pos, torch.from_numpy(gates).to(dev()), w.K, out)
+        assert np.array_equal(bits(out), oracle.combine(y_ref, p.pos, gates, w.K))
+        # inactive tokens come back as zero rows
+        inactive = np.flatnonzero(~active)
+        assert not bits(out[torch.from_numpy(inactive).to(dev())]).any()
+    assert mep.mep_get_error() == 0
