@@ -91,7 +91,7 @@ def test_quant_edge_rows():
     q_ref, s_ref = oracle.dispatch_int8(bits(xb16), pos, K, 4 * K)
     assert np.array_equal(recv.cpu().numpy(), q_ref)
     assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
-    assert recv[2:4].abs().max().item() == 0 and sc[0].item() == 0.0
+    assert recv[0:2].abs().max().item() == 0 and sc[0].item() == 0.0   # token 0: zero row
 
 
 def test_row_out_of_range_is_skipped_and_flagged():
@@ -167,11 +167,12 @@ def test_full_workload_sampled_and_properties(name):
     if not w.quant:
         assert torch.equal(_row_checksum(recv)[pos_d], _row_checksum(x_d)[g_of_slot])
     # every token: identity expert with softmax gates gives back the expert row exactly
+    # (as values: a -0 input comes back as +0, since 0 + -0 = +0)
     if not w.quant:
-        assert torch.equal(out.view(torch.int16), x_d.view(torch.int16))
+        assert torch.equal(out.float(), x_d.float())
     else:
         first = pos_d.view(w.T, w.K)[:, 0]
-        assert torch.equal(out.view(torch.int16), y[first].view(torch.int16))
+        assert torch.equal(out.float(), y[first].float())
         # all K copies of a token carry the same codes and scale
         cs = _row_checksum(recv)
         assert torch.equal(cs[pos_d].view(w.T, w.K), cs[first][:, None].expand(w.T, w.K))

@@ -1,0 +1,56 @@
+"""The multi-rank host logic of bench.py on CPU with gloo, world_size 2: every rank
+routes its own independent batch, the job time is the max over ranks, and the
+reference arm prints from rank 0 only."""
+import io
+import os
+import contextlib
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    import synth
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = synth.scaled(synth.get("tiny"), S=16)
+        wr = bench.rank_workload(w, rank)
+        ids, _ = synth.router(wr)
+        t = torch.from_numpy(ids.astype(np.int64)).view(-1)
+        gathered = [torch.empty_like(t) for _ in range(world)]
+        dist.all_gather(gathered, t)
+        differ = not torch.equal(gathered[0], gathered[1])
+        m = bench.max_over_ranks(1.5 + rank * 2.0, dist, torch.device("cpu"))
+        buf = io.StringIO()
+        with contextlib.redirect_stdout(buf):
+            args = type("A", (), dict(steps=1, warmup=0, gpus=world, ref_div=4))()
+            bench.run_reference(args, w)
+        q.put((rank, differ, m, buf.getvalue(), wr.seed))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29000 + os.getpid() % 1000
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=240) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, d0, m0, out0, s0), (r1, d1, m1, out1, s1) = res
+    assert d0 and d1                      # independent batches
+    assert s0 != s1
+    assert m0 == m1 == 3.5                # max over ranks
+    assert '"impl": "reference"' in out0 and out1 == ""
