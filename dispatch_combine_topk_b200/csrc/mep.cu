@@ -19,6 +19,8 @@ namespace {
 thread_local int32_t t_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
+// Shared memory the bulk dispatch may use per CTA (one CTA per SM).
+constexpr int kBulkSmemMax = 200 * 1024;
 int g_sm_count[kMaxDevices];
 bool g_attrs_set[kMaxDevices];
 
@@ -38,6 +40,8 @@ int sm_count()
         cudaFuncSetAttribute(mep::k_tile_count, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(mep::k_histogram, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(mep::k_plan_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+        cudaFuncSetAttribute(mep::k_dispatch_bulk<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBulkSmemMax);
+        cudaFuncSetAttribute(mep::k_dispatch_bulk<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBulkSmemMax);
         g_attrs_set[dev] = true;
     }
     return g_sm_count[dev];
@@ -217,7 +221,16 @@ mep_status_t mep_dispatch(const uint16_t *x, const int32_t *pos, int64_t T, int3
     cudaStream_t s = (cudaStream_t)stream;
     const int grid = token_grid(T, 8);
     if (quant == 0) {
-        if (H % 8 == 0 && aligned(x, 16) && aligned(recv, 16)) {
+        const size_t row_bytes = (size_t)H * 2;
+        const bool vec_ok = H % 8 == 0 && aligned(x, 16) && aligned(recv, 16);
+        const size_t head = mep::kDispatchSmemHead;
+        if (vec_ok && head + 4 * row_bytes <= (size_t)kBulkSmemMax) {
+            const int g = (int)(T < sm_count() ? T : sm_count());
+            mep::k_dispatch_bulk<4><<<g, 32, head + 4 * row_bytes, s>>>(x, pos, T, K, H, rows, (uint16_t *)recv);
+        } else if (vec_ok && head + 2 * row_bytes <= (size_t)kBulkSmemMax) {
+            const int g = (int)(T < sm_count() ? T : sm_count());
+            mep::k_dispatch_bulk<2><<<g, 32, head + 2 * row_bytes, s>>>(x, pos, T, K, H, rows, (uint16_t *)recv);
+        } else if (vec_ok) {
             mep::k_dispatch_copy<uint4><<<grid, 256, 0, s>>>((const uint4 *)x, pos, T, K, H / 8, rows,
                                                              (uint4 *)recv);
         } else {

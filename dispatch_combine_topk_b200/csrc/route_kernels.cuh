@@ -9,6 +9,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "tma.cuh"
 
 namespace mep {
 
@@ -112,6 +113,85 @@ k_dispatch_copy(const V *__restrict__ x, const int32_t *__restrict__ pos, int64_
         }
         __syncthreads();
     }
+}
+
+// bf16 copy through shared memory with bulk copies (the default path).
+//
+// One CTA of one warp per SM, tokens strided over the CTAs. A ring of kStages row
+// buffers in shared memory: lane 0 bulk-loads token rows ahead into the ring (each
+// completion tracked by an mbarrier), lanes k < K each bulk-store the staged row to the
+// row of slot k and wait until their stores have finished reading the stage, then the
+// stage is refilled with the token kStages ahead. The row bytes travel HBM -> smem once
+// and smem -> HBM K times with no register traffic; the bulk engine keeps the K stores
+// of every SM in flight.
+//
+// Dynamic shared memory: 8*kStages (barriers) + 128*kStages (row indices), padded to
+// kDispatchSmemHead, then kStages rows of row_bytes. Requires row_bytes % 16 == 0 and
+// 16-byte aligned x and recv.
+constexpr int kDispatchSmemHead = 2048;
+
+template <int kStages>
+__global__ void __launch_bounds__(32)
+k_dispatch_bulk(const uint16_t *__restrict__ x, const int32_t *__restrict__ pos, int64_t T, int K, int64_t H,
+                int64_t rows, uint16_t *__restrict__ recv)
+{
+    extern __shared__ __align__(128) int32_t smem_i32[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(smem_i32);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
+    int32_t *srow = reinterpret_cast<int32_t *>(smem + 8 * kStages);   // [kStages][32]
+    unsigned char *stage = smem + kDispatchSmemHead;
+    const uint32_t row_bytes = (uint32_t)(H * 2);
+    const int lane = threadIdx.x;
+    if (lane == 0) {
+        for (int s = 0; s < kStages; s++) mbar_init(&bar[s], 1);
+        mbar_fence_init();
+    }
+    __syncwarp();
+    const int64_t n = blockIdx.x < T ? (T - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    auto token = [&](int64_t i) { return (int64_t)blockIdx.x + i * gridDim.x; };
+    auto fetch = [&](int64_t i) {
+        const int s = (int)(i % kStages);
+        const int64_t t = token(i);
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&bar[s], row_bytes);
+            bulk_load_g2s(stage + (size_t)s * row_bytes, x + t * H, row_bytes, &bar[s]);
+        }
+        if (lane < K) {
+            int32_t p = pos[t * K + lane];
+            if (p < -1 || (int64_t)p >= rows) {
+                flag_error(0x2);
+                p = -1;
+            }
+            srow[s * 32 + lane] = p;
+        }
+    };
+    for (int64_t i = 0; i < n && i < kStages; i++) fetch(i);
+    __syncwarp();
+    for (int64_t i = 0; i < n; i++) {
+        const int s = (int)(i % kStages);
+        const bool ok = mbar_wait_bounded(&bar[s], (uint32_t)((i / kStages) & 1));
+        if (!__all_sync(0xffffffffu, ok)) {
+            // A load never completed: record it, wait (bounded) for the other loads
+            // still in flight into this CTA's ring, and leave.
+            if (lane == 0) {
+                flag_error(0x10);
+                for (int64_t j = i + 1; j < n && j < i + kStages; j++)
+                    mbar_wait_bounded(&bar[j % kStages], (uint32_t)((j / kStages) & 1));
+            }
+            break;
+        }
+        if (lane < K) {
+            const int32_t p = srow[s * 32 + lane];
+            if (p >= 0) bulk_store_s2g(recv + (int64_t)p * H, stage + (size_t)s * row_bytes, row_bytes);
+            bulk_commit();
+            bulk_wait_read_all();
+        }
+        __syncwarp();
+        if (i + kStages < n) fetch(i + kStages);
+        __syncwarp();
+    }
+    if (lane < K) bulk_wait_all();
+    __syncwarp();
 }
 
 // Quantise 8 fp32 values to int8 with the per-token scale; packed little-endian.

@@ -65,6 +65,7 @@ typedef enum {
 #define MEP_DERR_ROW_RANGE 0x2  /* a slot row outside [-1, rows) */
 #define MEP_DERR_TABLE     0x4  /* eplb_table: count outside [1, F-1] or instance id outside [0, 1024) */
 #define MEP_DERR_MASK      0x8  /* active_mask has a true after a false */
+#define MEP_DERR_TIMEOUT   0x10 /* a bounded wait inside a kernel ran out; that kernel stopped early */
 
 /* Plan modes. */
 #define MEP_PLAN_BALANCED 0

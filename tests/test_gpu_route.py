@@ -257,3 +257,37 @@ def test_mapping_workload_dispatch_combine_exact():
         inactive = np.flatnonzero(~active)
         assert not bits(out[torch.from_numpy(inactive).to(dev())]).any()
     assert mep.mep_get_error() == 0
+
+
+@pytest.mark.parametrize("case", ["huge_row", "misaligned"])
+def test_dispatch_fallback_paths(case):
+    """Rows too large to stage twice in shared memory take the 16-byte register path;
+    buffers that are not 16-byte aligned take the element path. Both must agree with
+    the oracle like the staged path does."""
+    rng = np.random.default_rng(31)
+    if case == "huge_row":
+        T, K, H = 6, 3, 51200
+        x = _rand_bf16((T, H), 5)
+        x_d = x.to(dev())
+        rows = T * K
+        recv = torch.zeros((rows, H), dtype=torch.bfloat16, device=dev())
+    else:
+        T, K, H = 9, 4, 64
+        x = _rand_bf16((T, H), 6)
+        flat = torch.zeros(T * H + 4, dtype=torch.bfloat16, device=dev())
+        x_d = flat[4:].view(T, H)                      # 8 bytes off a 16-byte boundary
+        x_d.copy_(x.to(dev()))
+        rows = T * K
+        rflat = torch.zeros(rows * H + 4, dtype=torch.bfloat16, device=dev())
+        recv = rflat[4:].view(rows, H)
+    pos = rng.permutation(rows).astype(np.int32)
+    pos[rng.random(T * K) < 0.2] = -1
+    pos_d = torch.from_numpy(pos).to(dev())
+    mep.mep_dispatch(x_d, pos_d, K, recv)
+    ref = oracle.dispatch(bits(x), pos, K, rows)
+    assert np.array_equal(bits(recv), ref)
+    gates = rng.random(T * K).astype(np.float32)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev())
+    mep.mep_combine(recv, pos_d, torch.from_numpy(gates).to(dev()), K, out)
+    assert np.array_equal(bits(out), oracle.combine(ref, pos, gates, K))
+    assert mep.mep_get_error() == 0
