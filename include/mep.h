@@ -18,8 +18,8 @@
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
  *    stream) and never synchronise the host, so a chain plan -> dispatch -> combine
  *    needs no host round trip (MoonEP's static shapes remove per-layer host syncs:
- *    twodots.gr article on MoonEP, static-shapes paragraph). All of them can be
- *    issued into a CUDA graph capture, except mep_get_error.
+ *    twodots.gr article on MoonEP, static-shapes paragraph). Only mep_get_error
+ *    synchronises.
  *  - A call first checks its arguments on the host and returns a status without
  *    launching anything when one is wrong: MEP_ERR_NULLPTR / MEP_ERR_DTYPE /
  *    MEP_ERR_SHAPE / MEP_ERR_VALUE mirror the aclnn codes 161001 (null tensor),
