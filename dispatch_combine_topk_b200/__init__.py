@@ -205,3 +205,27 @@ def mep_combine(y: torch.Tensor, pos: torch.Tensor, gates: torch.Tensor, K: int,
                            _ptr(out, torch.bfloat16, "out"), _stream(stream))
     _ok(rc, "mep_combine")
     return out
+
+
+MEP_PLAN_STATIC_WS_BYTES = 4 << 20
+
+
+def mep_plan_static_ws(ids: torch.Tensor, R: int, n_keys: int, S: int, K: int, out: PlanBuffers,
+                       mode: int = MEP_PLAN_BALANCED, keys_per_rank: int = 0,
+                       keep: Optional[torch.Tensor] = None, stream=None) -> PlanBuffers:
+    """mep_plan for callers that cannot allocate device memory: the scratch is a 4 MiB
+    array inside libmep (``out.workspace`` is not used). See include/mep.h."""
+    f = lib().mep_plan_static_ws
+    if f.argtypes is None:
+        P, i32 = ctypes.c_void_p, ctypes.c_int32
+        f.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P]
+        f.restype = ctypes.c_int
+    if ids.numel() != R * S * K:
+        raise ValueError("ids must hold R*S*K slots")
+    rc = f(_ptr(ids, torch.int32, "ids"), _ptr(keep, torch.uint8, "keep"), R, n_keys, S, K, mode,
+           keys_per_rank, _ptr(out.pos), _ptr(out.hist), _ptr(out.rank_off), _ptr(out.load),
+           _ptr(out.rep_count), _ptr(out.rep_key), _ptr(out.rep_cu), _ptr(out.stats),
+           _stream(stream))
+    _ok(rc, "mep_plan_static_ws")
+    return out
+

@@ -293,3 +293,49 @@ mep_status_t mep_combine(const uint16_t *y, int64_t rows, const int32_t *pos,
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------
+// mep_plan with scratch compiled into the library, for callers that cannot allocate.
+
+// The scratch: one copy on every device that loads this library, for the life of the
+// process. In host code this name is only a stand-in for the symbol; the device address
+// comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_plan_static_ws[MEP_PLAN_STATIC_WS_BYTES];
+
+namespace {
+void *g_plan_static_ws_addr[kMaxDevices];   // device address of g_plan_static_ws, per device
+}
+
+extern "C" mep_status_t mep_plan_static_ws(const int32_t *ids, const uint8_t *keep, int32_t R,
+                                           int32_t n_keys, int32_t S, int32_t K, int32_t mode,
+                                           int32_t keys_per_rank, int32_t *pos, int32_t *hist,
+                                           int32_t *rank_off, int32_t *load, int32_t *rep_count,
+                                           int32_t *rep_key, int32_t *rep_cu,
+                                           mep_plan_stats_t *stats, mep_stream_t stream)
+{
+    if (!ids || !pos || !hist || !rank_off || !rep_count || !rep_key || !rep_cu || !stats)
+        return MEP_ERR_NULLPTR;
+    const size_t need = mep_plan_workspace_size(R, n_keys, S, K);
+    if (need == 0) return MEP_ERR_SHAPE;
+    if (need > (size_t)MEP_PLAN_STATIC_WS_BYTES) return MEP_ERR_WORKSPACE;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        t_last_cuda_error = (int32_t)e;
+        return MEP_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return MEP_ERR_VALUE;
+    void *ws = g_plan_static_ws_addr[dev];
+    if (!ws) {
+        // once per device, with that device current
+        e = cudaGetSymbolAddress(&ws, g_plan_static_ws);
+        if (e != cudaSuccess || !ws) {
+            t_last_cuda_error = (int32_t)(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+            return MEP_ERR_CUDA;
+        }
+        g_plan_static_ws_addr[dev] = ws;
+    }
+    return mep_plan(ids, keep, R, n_keys, S, K, mode, keys_per_rank, pos, hist, rank_off, load,
+                    rep_count, rep_key, rep_cu, stats, ws, (size_t)MEP_PLAN_STATIC_WS_BYTES, stream);
+}
+

@@ -168,6 +168,44 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
                       mep_plan_stats_t *stats, void *workspace, size_t workspace_bytes,
                       mep_stream_t stream);
 
+/* Size of the scratch array compiled into libmep for mep_plan_static_ws: 4 MiB. */
+#define MEP_PLAN_STATIC_WS_BYTES (4u << 20)
+
+/*
+ * mep_plan for callers that cannot allocate device memory. The paper has no
+ * counterpart to this entry point; it exists for users of this library.
+ *
+ * Who needs it: code that must not call cudaMalloc at the point where it plans, such
+ * as a program whose device memory is all owned by another allocator (a caching
+ * allocator or a fixed pool that a stray cudaMalloc would overdraw or fragment), a
+ * serving loop in which cudaMalloc / cudaFree could stall the device, or a plain C
+ * program that links libmep and has no allocator of its own for scratch.
+ *
+ * Arguments, outputs and results are exactly those of mep_plan, minus the workspace:
+ * the scratch is a file-scope device array of MEP_PLAN_STATIC_WS_BYTES inside libmep,
+ * which every GPU that loads the library holds until the process exits. Inputs and
+ * outputs are still the caller's. This call allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ *
+ * Set-up: the first call on each device looks up the array's device address with
+ * cudaGetSymbolAddress (for the device current at that call) and keeps it; make that
+ * first call on a device before any stream capture.
+ * Sharing: all calls on a device use the same array, which keeps the contents of the
+ * last call. The plan kernels write every scratch word before they read it, so nothing
+ * has to be cleared between calls. Calls that overlap on the GPU (unordered streams)
+ * race on the array and produce wrong plans: order them.
+ * Limit: plans whose mep_plan_workspace_size(R, n_keys, S, K) is at most
+ * MEP_PLAN_STATIC_WS_BYTES, for instance up to 2,097,152 slots with up to 1023 keys.
+ * Errors: those of mep_plan; MEP_ERR_WORKSPACE for a plan larger than the array;
+ * MEP_ERR_CUDA if the address lookup fails.
+ */
+mep_status_t mep_plan_static_ws(const int32_t *ids, const uint8_t *keep, int32_t R,
+                                int32_t n_keys, int32_t S, int32_t K, int32_t mode,
+                                int32_t keys_per_rank, int32_t *pos, int32_t *hist,
+                                int32_t *rank_off, int32_t *load, int32_t *rep_count,
+                                int32_t *rep_key, int32_t *rep_cu, mep_plan_stats_t *stats,
+                                mep_stream_t stream);
+
 /*
  * a3 — logical->physical expert mapping and score-threshold pruning
  * (aclnnMoeUpdateExpert, gitcode ops-transformer doc, 功能说明 / 参数说明).
