@@ -33,6 +33,7 @@ import torch
 import synth
 
 METRIC = "dispatch+combine token-slots/s and achieved HBM GB/s (% of peak), 1 B200"
+L2_BYTES = 126 << 20
 UNIT = "token-slots/s"
 
 
@@ -42,6 +43,52 @@ def load_peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------- captured traffic
+
+CSRC = os.path.join(ROOT, "dispatch_combine_topk_b200", "csrc")
+
+
+def kernel_source_hash(name: str) -> str:
+    """sha256 of a kernel's own source text (from its declaration to its closing brace)
+    plus the shared helpers, so that a captured traffic figure is only reported for the
+    kernel it was measured on."""
+    import hashlib
+    import re
+
+    h = hashlib.sha256()
+    for fn in ("route_kernels.cuh", "plan_kernels.cuh"):
+        src = open(os.path.join(CSRC, fn)).read()
+        m = re.search(r"\n(?:template <[^>]*>\n)?__global__[^\n]*\n?" + re.escape(name) + r"\(", src)
+        if m:
+            end = src.index("\n}\n", m.start())
+            h.update(src[m.start():end + 3].encode())
+            break
+    else:
+        return ""
+    h.update(open(os.path.join(CSRC, "common.cuh")).read().encode())
+    return h.hexdigest()[:16]
+
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch, from the ncu captures
+# summarised in profiles/, scaled to the full workload by the rows routed (a capture on
+# S=1024 of the r8 workload routes a quarter of its rows).
+TRAFFIC = {
+    ("k_dispatch_warp", "r8_e64_s4096_k8_h7168"): {
+        "bytes": 4 * 998.09e6, "src": "0a17c397b27cf663",
+        "note": "profiles/k_dispatch_warp_r8_s1024.md: 998.1 MB at S=1024, x4"},
+    ("k_combine_v8", "r8_e64_s4096_k8_h7168"): {
+        "bytes": 4 * 1009.43e6, "src": "a9d5f41e42e115fa",
+        "note": "profiles/k_combine_v8_r8_s1024.md: 1009.4 MB at S=1024, x4"},
+}
+
+
+def captured_traffic(kernel: str, workload: str):
+    t = TRAFFIC.get((kernel, workload))
+    if not t or kernel_source_hash(kernel) != t["src"]:
+        return None, None
+    return t["bytes"], t["note"]
 
 
 # ------------------------------------------------------------------ clock sampler
@@ -102,47 +149,68 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-# ---------------------------------------------------------------- byte accounting
-
-def algorithmic_bytes(w):
-    """Minimum bytes each kernel must move per launch (per step)."""
-    row = 2 * w.H
-    disp = w.T * row + w.N * row + 4 * w.N                 # read x once, write K copies, read pos
-    comb = w.N * row + w.T * row + 8 * w.N                 # read K rows, write x, read pos+gates
-    plan = 3 * 4 * w.N + 4 * w.N                           # 3 passes over ids, write pos
-    return {"plan": plan, "dispatch": disp, "combine": comb}
-
-
 # ------------------------------------------------------------------- oracle timing
 
 def oracle_sample(w, S_sample):
     """Time the oracle (as it stands) on a bounded sample: the same workload with S
-    reduced to S_sample tokens per rank. Returns (token-slots/s, description)."""
+    reduced to S_sample tokens per rank. The timed steps are those of the GPU step
+    (mapping and grouped plan, or the balanced plan; dispatch, bf16 or int8; combine);
+    the int8 identity expert (dequantisation) is not timed, as on the GPU.
+    Returns (token-slots/s, description, seconds)."""
     import oracle
 
     ws = synth.scaled(w, S=S_sample)
     ids, gates = synth.router(ws)
     x = synth.hidden(ws).view(torch.int16).numpy().view(np.uint16)
     oracle.lib()
+    parts = {}
     t0 = time.perf_counter()
-    p = oracle.plan_balanced(ids, ws.R, ws.E, ws.S, ws.K)
+    if ws.mapping:
+        table, thr, active = synth.mapping_inputs(ws)
+        bi = np.empty_like(ids)
+        bm = np.empty(ids.shape, bool)
+        for r in range(ws.R):
+            sl = slice(r * ws.S, (r + 1) * ws.S)
+            bi[sl], bm[sl] = oracle.update_expert(ids[sl], table, gates[sl], thr, active[sl], r, ws.R, 0)
+        p = oracle.plan_grouped(bi, bm, ws.R, ws.R * ws.place_per_rank, ws.place_per_rank, ws.S, ws.K)
+    else:
+        p = oracle.plan_balanced(ids, ws.R, ws.E, ws.S, ws.K)
     t1 = time.perf_counter()
-    y = oracle.dispatch(x, p.pos, ws.K, ws.N)
-    t2 = time.perf_counter()
+    parts["plan"] = t1 - t0
+    rows = p.n_kept
+    if ws.quant:
+        q, sc = oracle.dispatch_int8(x, p.pos, ws.K, rows)
+        t2 = time.perf_counter()
+        y = oracle.dequantize(q, sc)
+        del q
+        t2b = time.perf_counter()
+    else:
+        y = oracle.dispatch(x, p.pos, ws.K, rows)
+        t2 = t2b = time.perf_counter()
+    parts["dispatch"] = t2 - t1
     oracle.combine(y, p.pos, gates, ws.K)
     t3 = time.perf_counter()
-    dt = t3 - t0
-    desc = (f"oracle plan+dispatch+combine on R={ws.R} E={ws.E} S={ws.S} K={ws.K} H={ws.H} "
-            f"({ws.N} token-slots; S reduced from {w.S}); plan {t1 - t0:.3f}s dispatch "
-            f"{t2 - t1:.3f}s combine {t3 - t2:.3f}s")
+    parts["combine"] = t3 - t2b
+    dt = parts["plan"] + parts["dispatch"] + parts["combine"]
+    desc = (f"oracle {'mapping+grouped plan' if ws.mapping else 'plan'}+"
+            f"{'int8 ' if ws.quant else ''}dispatch+combine on R={ws.R} E={ws.E} S={ws.S} K={ws.K} "
+            f"H={ws.H} ({ws.N} token-slots; S reduced from {w.S}); "
+            + " ".join(f"{k} {v:.3f}s" for k, v in parts.items()))
     return ws.N / dt, desc, dt
+
+
+def cpu_sample_S(w, div: int) -> int:
+    """Tokens per rank of the CPU sample: S/div, and small enough that the host copy of
+    the receive rows stays under 2^31 elements."""
+    cap = max(1, -(-w.N * w.H // (1 << 31)))
+    return max(1, w.S // max(div, cap))
 
 
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    S_sample = max(1, w.S // args.ref_div)
+    S_sample = cpu_sample_S(w, args.ref_div)
     for _ in range(args.warmup):
         oracle_sample(w, S_sample)
     vals, tot = [], 0.0
@@ -185,6 +253,133 @@ def max_over_ranks(value: float, pg, device) -> float:
 
 # --------------------------------------------------------------------- GPU bench
 
+class Route:
+    """Device buffers and the launch sequence of one routing step for one workload.
+
+    Balanced workloads: plan (mep_plan) -> dispatch (bf16, or int8 for the int8
+    workload) -> combine. The identity expert returns the dispatched rows; for int8 it is
+    mep_dequantize, run once before timing (its output is the same at every step, since
+    the inputs are fixed) and not part of the timed step.
+    Mapping workload: mep_update_expert for every rank -> grouped plan over the physical
+    instances -> dispatch -> combine.
+    """
+
+    def __init__(self, mep, w, dev):
+        self.mep, self.w, self.dev = mep, w, dev
+        ids, gates = synth.router(w)
+        x = synth.hidden(w)
+        self.host = dict(ids=torch.from_numpy(ids).view(-1), gates=torch.from_numpy(gates).view(-1), x=x)
+        self.ids = self.host["ids"].to(dev)
+        self.gates = self.host["gates"].to(dev)
+        self.x = x.to(dev)
+        self.out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
+        self.launches = 0
+        if w.mapping:
+            table, thr, active = synth.mapping_inputs(w)
+            self.table = torch.from_numpy(table).to(dev)
+            self.thr = torch.from_numpy(thr).to(dev)
+            self.active = torch.from_numpy(active.astype(np.uint8)).to(dev)
+            self.bids = torch.empty((w.T, w.K), dtype=torch.int32, device=dev)
+            self.bmask = torch.empty((w.T, w.K), dtype=torch.uint8, device=dev)
+            self.n_keys = w.R * w.place_per_rank
+            self.pb = mep.PlanBuffers.allocate(w.R, self.n_keys, w.S, w.K, dev)
+            self.recv = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
+            self.y = self.recv
+        else:
+            self.pb = mep.PlanBuffers.allocate(w.R, w.E, w.S, w.K, dev)
+            if w.quant:
+                self.recv = torch.empty((w.N, w.H), dtype=torch.int8, device=dev)
+                self.scale = torch.empty(w.N, dtype=torch.float32, device=dev)
+                self.y = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
+            else:
+                self.recv = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
+                self.y = self.recv
+        torch.cuda.synchronize()
+
+    def plan(self, s):
+        w, mep = self.w, self.mep
+        if w.mapping:
+            g2 = self.gates.view(w.T, w.K)
+            ids2 = self.ids.view(w.T, w.K)
+            for r in range(w.R):
+                sl = slice(r * w.S, (r + 1) * w.S)
+                mep.mep_update_expert(ids2[sl], self.table, g2[sl], self.thr, self.active[sl], r, w.R,
+                                      0, self.bids[sl], self.bmask[sl], stream=s)
+            mep.mep_plan(self.bids.view(-1), w.R, self.n_keys, w.S, w.K, self.pb,
+                         mode=mep.MEP_PLAN_GROUPED, keys_per_rank=w.place_per_rank,
+                         keep=self.bmask.view(-1), stream=s)
+            return w.R + 4
+        mep.mep_plan(self.ids, w.R, w.E, w.S, w.K, self.pb, stream=s)
+        return 4
+
+    def dispatch(self, s):
+        w = self.w
+        if w.quant:
+            self.mep.mep_dispatch(self.x, self.pb.pos, w.K, self.recv, self.scale, quant=1, stream=s)
+        else:
+            self.mep.mep_dispatch(self.x, self.pb.pos, w.K, self.recv, stream=s)
+        return 1
+
+    def expert(self, s):
+        if self.w.quant:
+            self.mep.mep_dequantize(self.recv, self.scale, self.y, stream=s)
+
+    def combine(self, s):
+        self.mep.mep_combine(self.y, self.pb.pos, self.gates, self.w.K, self.out, stream=s)
+        return 1
+
+    def step(self, s, ev=None):
+        if ev is not None:
+            ev[0].record(s)
+        n = self.plan(s)
+        if ev is not None:
+            ev[1].record(s)
+        n += self.dispatch(s)
+        if ev is not None:
+            ev[2].record(s)
+        n += self.combine(s)
+        if ev is not None:
+            ev[3].record(s)
+        return n
+
+    def result_ok(self) -> bool:
+        """Closed form of the identity expert with gates summing to 1: every token whose
+        K slots are all kept comes back as its expert row (compared as values)."""
+        w = self.w
+        if w.mapping:
+            return bool(torch.isfinite(self.out.float()).all())
+        if w.quant:
+            first = self.pb.pos.view(w.T, w.K)[:, 0].long()
+            return torch.equal(self.out.float(), self.y[first].float())
+        return torch.equal(self.out.float(), self.x.float())
+
+    def kernel_name(self, step: str) -> str:
+        """The library kernel that runs a step on this workload's shapes."""
+        w = self.w
+        if step == "combine":
+            return "k_combine_v8" if w.H % 8 == 0 else "k_combine_scalar"
+        if w.quant:
+            return "k_dispatch_int8_staged" if w.H % 16 == 0 else "k_dispatch_int8"
+        return "k_dispatch_warp" if w.H % 8 == 0 else "k_dispatch_copy"
+
+    def working_set_bytes(self) -> int:
+        return (self.x.numel() * 2 + self.recv.numel() * self.recv.element_size() +
+                self.out.numel() * 2 + self.ids.numel() * 8)
+
+    def bytes(self):
+        """Algorithmic bytes per launch of dispatch and combine, and of the plan."""
+        w = self.w
+        row = 2 * w.H
+        n_rows = int(self.pb.stats_dict()["n_kept"])
+        if w.quant:
+            disp = w.T * row + n_rows * w.H + 4 * n_rows + 4 * w.N
+        else:
+            disp = w.T * row + n_rows * row + 4 * w.N
+        comb = n_rows * row + w.T * row + 8 * w.N
+        plan = 16 * w.N
+        return {"plan": plan, "dispatch": disp, "combine": comb}
+
+
 def run_gpu(args, w):
     import dispatch_combine_topk_b200 as mep
 
@@ -201,53 +396,43 @@ def run_gpu(args, w):
                                 device_id=dev)
         pg = dist
     # every rank routes its own independent batch (different seed)
-    wr = rank_workload(w, rank)
-    ids, gates = synth.router(wr)
-    x = synth.hidden(wr)
+    rt = Route(mep, rank_workload(w, rank), dev)
     stream = torch.cuda.Stream(dev)
-    ids_d = torch.from_numpy(ids).to(dev).view(-1)
-    g_d = torch.from_numpy(gates).to(dev).view(-1)
-    x_d = x.to(dev)
-    pb = mep.PlanBuffers.allocate(w.R, w.E, w.S, w.K, dev)
-    recv = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
-    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
-    torch.cuda.synchronize()
-
-    def step(s, ev=None):
-        if ev is not None:
-            ev[0].record(s)
-        mep.mep_plan(ids_d, w.R, w.E, w.S, w.K, pb, stream=s)
-        if ev is not None:
-            ev[1].record(s)
-        mep.mep_dispatch(x_d, pb.pos, w.K, recv, stream=s)
-        if ev is not None:
-            ev[2].record(s)
-        mep.mep_combine(recv, pb.pos, g_d, w.K, out, stream=s)
-        if ev is not None:
-            ev[3].record(s)
-
     with torch.cuda.stream(stream):
+        rt.step(stream)
+        rt.expert(stream)
         for _ in range(args.warmup):
-            step(stream)
+            rt.step(stream)
     stream.synchronize()
     mep.mep_get_error(clear=True)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # A working set that fits in L2 is flushed between steps (a 256 MB write, outside
+    # the step's events); larger ones are not.
+    flush = None
+    if rt.working_set_bytes() < 2 * L2_BYTES:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
+    launches = 0
     with ClockSampler(local) as clk:
         with torch.cuda.stream(stream):
             start.record(stream)
             for i in range(args.steps):
-                step(stream, evs[i])
+                if flush is not None:
+                    flush.fill_(i & 0xff)
+                launches += rt.step(stream, evs[i])
             end.record(stream)
         stream.synchronize()
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
-    ms = start.elapsed_time(end)
+    if flush is None:
+        ms = start.elapsed_time(end)
+    else:
+        ms = float(sum(e[0].elapsed_time(e[3]) for e in evs))
     err = mep.mep_get_error(clear=True)
     if err:
         raise RuntimeError(f"device error word {err:#x} after the timed steps")
@@ -256,20 +441,19 @@ def run_gpu(args, w):
     t_comb = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
     ms_max = max_over_ranks(ms, pg, dev)
     ms_step = ms_max / args.steps
+    ok_device = rt.result_ok()
 
     # end to end: pinned host inputs -> device -> step -> result back to the host
-    x_h = x.pin_memory()
-    ids_h = torch.from_numpy(ids).view(-1).pin_memory()
-    g_h = torch.from_numpy(gates).view(-1).pin_memory()
+    h = {k: v.pin_memory() for k, v in rt.host.items()}
     out_h = torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
 
     def e2e_step(s):
-        ids_d.copy_(ids_h, non_blocking=True)
-        g_d.copy_(g_h, non_blocking=True)
-        x_d.copy_(x_h, non_blocking=True)
-        step(s)
-        out_h.copy_(out, non_blocking=True)
+        rt.ids.copy_(h["ids"], non_blocking=True)
+        rt.gates.copy_(h["gates"], non_blocking=True)
+        rt.x.copy_(h["x"], non_blocking=True)
+        rt.step(s)
+        out_h.copy_(rt.out, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for _ in range(2):
@@ -285,21 +469,22 @@ def run_gpu(args, w):
         e1.record(stream)
     stream.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, pg, dev)
-    # identity expert + gates summing to 1: the result equals the input (as values)
-    ok = torch.equal(out.float(), x_d.float())
-    h2d = x_h.numel() * 2 + ids_h.numel() * 4 + g_h.numel() * 4
+    ok_e2e = rt.result_ok()
+    h2d = sum(v.numel() * v.element_size() for v in h.values())
     d2h = out_h.numel() * 2
 
     if rank == 0:
         peak, peak_kind = load_peaks()
-        ab = algorithmic_bytes(w)
+        ab = rt.bytes()
         dom = "dispatch" if t_disp >= t_comb else "combine"
         t_dom = t_disp if dom == "dispatch" else t_comb
         achieved = ab[dom] / (t_dom * 1e-3) / 1e9
+        kname = rt.kernel_name(dom)
+        traffic, traffic_note = captured_traffic(kname, w.name)
         dc_gbs = (ab["dispatch"] + ab["combine"]) / ((t_disp + t_comb) * 1e-3) / 1e9
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            v, desc, _ = oracle_sample(w, w.S)
+            v, desc, _ = oracle_sample(w, cpu_sample_S(w, args.cpu_div))
             cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
         line = {
             "metric": METRIC,
@@ -308,25 +493,28 @@ def run_gpu(args, w):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic",
+            "dtype": "int8" if w.quant else "bf16", "data": "synthetic",
             "config": {"workload": w.name, "R": w.R, "E": w.E, "S": w.S, "K": w.K, "H": w.H,
                        "token_slots_per_gpu": w.N, "seed": w.seed, "parallelism": f"replicas{world}",
-                       "l2": f"inputs larger than L2 (x {w.T * w.H * 2 / 1e6:.0f} MB, recv "
-                             f"{w.N * w.H * 2 / 1e9:.2f} GB; L2 126 MB): no flush"},
+                       "l2": (f"working set {rt.working_set_bytes() / 1e6:.0f} MB "
+                              + ("< 2x L2 (126 MB): L2 flushed between steps (256 MB write, "
+                                 "not timed)" if flush is not None else
+                                 "> 2x L2 (126 MB): inputs larger than L2, no flush"))},
             "breakdown_ms": {"plan": t_plan, "dispatch": t_disp, "combine": t_comb},
             "dispatch_combine": {"token_slots_per_s": w.N / ((t_disp + t_comb) * 1e-3),
                                  "hbm_gbs": dc_gbs, "frac_of_peak": dc_gbs / peak,
                                  "frac_of_8tbs_nominal": dc_gbs / 8000.0},
-            "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
+            "roofline": {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "algorithmic_bytes": ab[dom], "traffic": None},
+                         "algorithmic_bytes": ab[dom], "traffic": traffic,
+                         "traffic_source": traffic_note},
             "cpu_baseline": cpu,
             "e2e": {"value": world * w.N / (e2e_ms * 1e-3), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "result_matches_input": bool(ok)},
-            "gpu_launches": 6 * args.steps,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "result_check": {"device": ok_device, "e2e": ok_e2e},
+            "gpu_launches": launches,
             "clocks": clk.summary(),
-            "plan_stats": pb.stats_dict(),
+            "plan_stats": rt.pb.stats_dict(),
         }
         print(json.dumps(line), flush=True)
     if pg:
@@ -342,7 +530,9 @@ def main():
     ap.add_argument("--impl", default="mep", choices=["mep", "reference"])
     ap.add_argument("--workload", default="r8")
     ap.add_argument("--ref-div", type=int, default=8,
-                    help="the oracle routes S/ref_div tokens per rank per step")
+                    help="--impl reference: the oracle routes S/ref_div tokens per rank per step")
+    ap.add_argument("--cpu-div", type=int, default=1,
+                    help="cpu_baseline: the oracle routes S/cpu_div tokens per rank once")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens-per-rank", type=int, default=0,
                     help="override S (a smaller case of the same workload, e.g. for profiling)")

@@ -19,7 +19,7 @@ namespace {
 thread_local int32_t t_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
-// Shared memory the bulk dispatch may use per CTA (one CTA per SM).
+// Shared memory the staged int8 dispatch may use per CTA.
 constexpr int kBulkSmemMax = 200 * 1024;
 int g_sm_count[kMaxDevices];
 bool g_attrs_set[kMaxDevices];
@@ -40,8 +40,8 @@ int sm_count()
         cudaFuncSetAttribute(mep::k_tile_count, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(mep::k_histogram, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(mep::k_plan_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(mep::k_dispatch_bulk<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBulkSmemMax);
-        cudaFuncSetAttribute(mep::k_dispatch_bulk<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBulkSmemMax);
+        cudaFuncSetAttribute(mep::k_dispatch_int8_staged<4, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kBulkSmemMax);
         g_attrs_set[dev] = true;
     }
     return g_sm_count[dev];
@@ -135,7 +135,7 @@ size_t mep_plan_workspace_size(int32_t R, int32_t n_keys, int32_t S, int32_t K)
     if (R < 1 || S < 1 || K < 1 || n_keys < 1) return 0;
     const int64_t N = (int64_t)R * S * K;
     const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
-    return align256(sizeof(int32_t) * (size_t)tiles * n_keys) + align256(sizeof(int32_t) * (size_t)(n_keys + 1));
+    return align256(sizeof(int32_t) * (size_t)tiles * n_keys);
 }
 
 mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_t n_keys,
@@ -166,15 +166,14 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
     sm_count();
     const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
     int32_t *tile_cnt = (int32_t *)workspace;
-    int32_t *key_off = (int32_t *)((char *)workspace + align256(sizeof(int32_t) * (size_t)tiles * n_keys));
     const int threads = mep::kPlanWarps * 32;
 
     mep::k_tile_count<<<(unsigned)tiles, threads, sizeof(int32_t) * n_keys, s>>>(ids, keep, N, n_keys, tile_cnt);
-    mep::k_scan<<<1, 1024, 0, s>>>(tile_cnt, (int32_t)tiles, n_keys, hist, key_off);
-    mep::k_rank<<<(unsigned)tiles, threads, sizeof(int32_t) * mep::kPlanWarps * n_keys, s>>>(
-        ids, keep, N, n_keys, tile_cnt, key_off, pos);
+    mep::k_scan_cols<<<(unsigned)mep::ceil_div(n_keys, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, n_keys, hist);
+    const size_t rank_smem = sizeof(int32_t) * ((size_t)mep::kPlanWarps * n_keys + n_keys + 1 + 33);
+    mep::k_rank<<<(unsigned)tiles, threads, rank_smem, s>>>(ids, keep, N, n_keys, tile_cnt, hist, pos);
     const size_t meta_smem = sizeof(int32_t) * (size_t)(2 * (n_keys + 1) + (R + 1) + R);
-    mep::k_plan_meta<<<1, 1024, meta_smem, s>>>(hist, key_off, R, n_keys, (int64_t)S * K, mode,
+    mep::k_plan_meta<<<1, 1024, meta_smem, s>>>(hist, R, n_keys, (int64_t)S * K, mode,
                                                 keys_per_rank, rank_off, load, rep_count, rep_key,
                                                 rep_cu, (int32_t *)stats);
     return launched();
@@ -221,23 +220,25 @@ mep_status_t mep_dispatch(const uint16_t *x, const int32_t *pos, int64_t T, int3
     cudaStream_t s = (cudaStream_t)stream;
     const int grid = token_grid(T, 8);
     if (quant == 0) {
-        const size_t row_bytes = (size_t)H * 2;
-        const bool vec_ok = H % 8 == 0 && aligned(x, 16) && aligned(recv, 16);
-        const size_t head = mep::kDispatchSmemHead;
-        if (vec_ok && head + 4 * row_bytes <= (size_t)kBulkSmemMax) {
-            const int g = (int)(T < sm_count() ? T : sm_count());
-            mep::k_dispatch_bulk<4><<<g, 32, head + 4 * row_bytes, s>>>(x, pos, T, K, H, rows, (uint16_t *)recv);
-        } else if (vec_ok && head + 2 * row_bytes <= (size_t)kBulkSmemMax) {
-            const int g = (int)(T < sm_count() ? T : sm_count());
-            mep::k_dispatch_bulk<2><<<g, 32, head + 2 * row_bytes, s>>>(x, pos, T, K, H, rows, (uint16_t *)recv);
-        } else if (vec_ok) {
-            mep::k_dispatch_copy<uint4><<<grid, 256, 0, s>>>((const uint4 *)x, pos, T, K, H / 8, rows,
-                                                             (uint4 *)recv);
+        if (H % 8 == 0 && aligned(x, 16) && aligned(recv, 16)) {
+            // one warp per token, 8 warps per CTA, up to 64 CTAs per SM in waves
+            const int64_t ctas = mep::ceil_div(T, 8);
+            const int64_t cap = (int64_t)sm_count() * 64;
+            mep::k_dispatch_warp<<<(int)(ctas < cap ? ctas : cap), 256, 0, s>>>((const uint4 *)x, pos, T, K, H / 8,
+                                                                              rows, (uint4 *)recv);
         } else {
             mep::k_dispatch_copy<uint16_t><<<grid, 256, 0, s>>>(x, pos, T, K, H, rows, (uint16_t *)recv);
         }
     } else {
-        if (H % 8 == 0 && aligned(x, 16) && aligned(recv, 8)) {
+        const size_t staged_smem = (size_t)mep::kDispatchSmemHead + 4 * (size_t)H * 2 + 2 * (size_t)H;
+        if (H % 16 == 0 && aligned(x, 16) && aligned(recv, 16) && staged_smem <= (size_t)kBulkSmemMax) {
+            int per_sm = 0;
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mep::k_dispatch_int8_staged<4, 128>, 128,
+                                                          staged_smem);
+            per_sm = per_sm < 1 ? 1 : (per_sm > 3 ? 3 : per_sm);
+            mep::k_dispatch_int8_staged<4, 128><<<token_grid(T, per_sm), 128, staged_smem, s>>>(
+                x, pos, T, K, H, rows, (int8_t *)recv, recv_scale);
+        } else if (H % 8 == 0 && aligned(x, 16) && aligned(recv, 8)) {
             mep::k_dispatch_int8<<<grid, 256, 0, s>>>((const uint4 *)x, pos, T, K, H / 8, rows,
                                                       (uint2 *)recv, recv_scale);
         } else {

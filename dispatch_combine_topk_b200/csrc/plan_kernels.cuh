@@ -8,10 +8,12 @@
 // The grouped plan over physical instance ids is the same sort with dropped slots
 // removed. Both are done in three passes over the ids (4 bytes per slot each):
 //   k_tile_count  per-tile key counts              (warp-aggregated with match.any)
-//   k_scan        per-key prefix over tiles + exclusive prefix over keys
+//   k_scan_cols   per-key prefix over tiles and hist, one CTA per 32 keys
 //   k_rank        per-slot stable rank inside its tile, written as the final row
 // and one single-CTA pass over the keys, k_plan_meta, that writes the per-rank replica
-// tables (cu_seqlens) and the summary counts.
+// tables (cu_seqlens) and the summary counts. The exclusive prefix of hist over keys
+// (off) is small (at most 4096 keys) and is recomputed in shared memory by each CTA that
+// needs it.
 #pragma once
 
 #include "common.cuh"
@@ -76,92 +78,99 @@ k_tile_count(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, 
     for (int i = threadIdx.x; i < n_keys; i += blockDim.x) out[i] = sh[i];
 }
 
-// One CTA of 1024 threads. In place: tile_cnt[t, key] <- sum_{t' < t} tile_cnt[t', key].
-// hist[key] = sum over tiles; key_off = exclusive prefix of hist over keys, with
-// key_off[n_keys] = total.
+// Exclusive prefix sum of in[0..n) into out[0..n], with out[n] = the total. Called by
+// every thread of the block; `scratch` holds 33 ints of shared memory. Ends with a
+// block barrier.
+__device__ __forceinline__ void block_exclusive_scan(const int32_t *__restrict__ in, int n, int32_t *out,
+                                                     int32_t *scratch)
+{
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+    const int per = (n + nt - 1) / nt;
+    const int lo = min(n, tid * per), hi = min(n, lo + per);
+    int32_t sum = 0;
+    for (int i = lo; i < hi; i++) sum += in[i];
+    int32_t inc = sum;
+    for (int d = 1; d < 32; d <<= 1) {
+        const int32_t u = __shfl_up_sync(0xffffffffu, inc, d);
+        if (lane >= d) inc += u;
+    }
+    if (lane == 31) scratch[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const int32_t w = lane < nw ? scratch[lane] : 0;
+        int32_t wi = w;
+        for (int d = 1; d < 32; d <<= 1) {
+            const int32_t u = __shfl_up_sync(0xffffffffu, wi, d);
+            if (lane >= d) wi += u;
+        }
+        scratch[lane] = wi - w;
+        if (lane == 31) scratch[32] = wi;
+    }
+    __syncthreads();
+    int32_t run = scratch[warp] + inc - sum;
+    for (int i = lo; i < hi; i++) {
+        out[i] = run;
+        run += in[i];
+    }
+    if (tid == 0) out[n] = scratch[32];
+    __syncthreads();
+}
+
+// CTA c owns keys [32c, 32c + 32), one per lane; its 32 warps split the tiles. In place:
+// tile_cnt[t, key] <- sum_{t' < t} tile_cnt[t', key], and hist[key] = sum over tiles.
 __global__ void __launch_bounds__(1024)
-k_scan(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys, int32_t *__restrict__ hist,
-       int32_t *__restrict__ key_off)
+k_scan_cols(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys, int32_t *__restrict__ hist)
 {
     __shared__ int32_t part[32][33];
-    __shared__ int32_t wsum[32];
-    __shared__ int32_t carry;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int seg = (n_tiles + 31) / 32;
     const int t0 = min(n_tiles, warp * seg), t1 = min(n_tiles, t0 + seg);
-    for (int e0 = 0; e0 < n_keys; e0 += 32) {
-        const int e = e0 + lane;
-        const bool ok = e < n_keys;
-        int32_t s = 0;
-        if (ok)
-            for (int t = t0; t < t1; t++) s += tile_cnt[(int64_t)t * n_keys + e];
-        part[warp][lane] = s;
-        __syncthreads();
-        if (warp == 0) {
-            int32_t run = 0;
-            for (int w = 0; w < 32; w++) {
-                int32_t v = part[w][lane];
-                part[w][lane] = run;
-                run += v;
-            }
-            if (ok) hist[e] = run;
-        }
-        __syncthreads();
-        if (ok) {
-            int32_t run = part[warp][lane];
-            for (int t = t0; t < t1; t++) {
-                int64_t i = (int64_t)t * n_keys + e;
-                int32_t v = tile_cnt[i];
-                tile_cnt[i] = run;
-                run += v;
-            }
-        }
-        __syncthreads();
+    const int e = blockIdx.x * 32 + lane;
+    const bool ok = e < n_keys;
+    int32_t s = 0;
+    if (ok) {
+#pragma unroll 4
+        for (int t = t0; t < t1; t++) s += tile_cnt[(int64_t)t * n_keys + e];
     }
-    // exclusive scan of hist over keys, 1024 keys per round
-    if (threadIdx.x == 0) carry = 0;
+    part[warp][lane] = s;
     __syncthreads();
-    for (int e0 = 0; e0 < n_keys; e0 += 1024) {
-        const int e = e0 + threadIdx.x;
-        int32_t v = e < n_keys ? hist[e] : 0;
-        int32_t inc = v;
-        for (int d = 1; d < 32; d <<= 1) {
-            int32_t u = __shfl_up_sync(0xffffffffu, inc, d);
-            if (lane >= d) inc += u;
+    if (warp == 0) {
+        int32_t run = 0;
+        for (int w = 0; w < 32; w++) {
+            const int32_t v = part[w][lane];
+            part[w][lane] = run;
+            run += v;
         }
-        if (lane == 31) wsum[warp] = inc;
-        __syncthreads();
-        if (warp == 0) {
-            int32_t w = wsum[lane], wi = w;
-            for (int d = 1; d < 32; d <<= 1) {
-                int32_t u = __shfl_up_sync(0xffffffffu, wi, d);
-                if (lane >= d) wi += u;
-            }
-            wsum[lane] = wi - w;  // exclusive prefix of warp totals
-        }
-        __syncthreads();
-        const int32_t c = carry;
-        if (e < n_keys) key_off[e] = c + wsum[warp] + inc - v;
-        __syncthreads();
-        if (threadIdx.x == 1023) carry = c + wsum[31] + inc;
-        __syncthreads();
+        if (ok) hist[e] = run;
     }
-    if (threadIdx.x == 0) key_off[n_keys] = carry;
+    __syncthreads();
+    if (ok) {
+        int32_t run = part[warp][lane];
+        for (int t = t0; t < t1; t++) {
+            const int64_t i = (int64_t)t * n_keys + e;
+            const int32_t v = tile_cnt[i];
+            tile_cnt[i] = run;
+            run += v;
+        }
+    }
 }
 
-// pos[n] = key_off[key] + (slots of key in earlier tiles) + (earlier slots of key in this
-// tile). Each warp owns a contiguous quarter... an eighth of the tile: it counts its
-// sub-range per key, the CTA turns those counts into per-warp bases, then each warp
-// walks its sub-range again in order, ranking equal keys with match.any.
+// pos[n] = off[key] + (slots of key in earlier tiles) + (earlier slots of key in this
+// tile), off = exclusive prefix of hist over keys. Each warp owns an eighth of the
+// tile: it counts its sub-range per key, the CTA turns those counts into per-warp bases,
+// then each warp walks its sub-range again in order, ranking equal keys with match.any.
+// Dynamic shared memory: cnt [kPlanWarps][n_keys], off [n_keys + 1], scratch [33].
 __global__ void __launch_bounds__(kPlanWarps * 32)
 k_rank(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, int64_t N, int32_t n_keys,
-       const int32_t *__restrict__ tile_base, const int32_t *__restrict__ key_off,
+       const int32_t *__restrict__ tile_base, const int32_t *__restrict__ hist,
        int32_t *__restrict__ pos)
 {
-    extern __shared__ int32_t cnt[];  // [kPlanWarps][n_keys]
+    extern __shared__ int32_t cnt[];
+    int32_t *key_off = cnt + kPlanWarps * n_keys;
+    int32_t *scan_scratch = key_off + n_keys + 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < kPlanWarps * n_keys; i += blockDim.x) cnt[i] = 0;
-    __syncthreads();
+    block_exclusive_scan(hist, n_keys, key_off, scan_scratch);
     constexpr int kSub = kPlanTile / kPlanWarps;
     const int64_t lo = (int64_t)blockIdx.x * kPlanTile + warp * kSub;
     int32_t *mine = cnt + warp * n_keys;
@@ -215,7 +224,7 @@ __device__ __forceinline__ int32_t upper_bound_sh(const int32_t *a, int32_t n, i
 // One CTA of 1024 threads: per-rank replica tables and the summary counts.
 // Dynamic shared memory: key_off (n_keys+1) + nz (n_keys+1) + rank_off (R+1) + e_lo (R).
 __global__ void __launch_bounds__(1024)
-k_plan_meta(const int32_t *__restrict__ hist, const int32_t *__restrict__ key_off_g, int32_t R,
+k_plan_meta(const int32_t *__restrict__ hist, int32_t R,
             int32_t n_keys, int64_t SK, int32_t mode, int32_t keys_per_rank,
             int32_t *__restrict__ rank_off_out, int32_t *__restrict__ load_out,
             int32_t *__restrict__ rep_count, int32_t *__restrict__ rep_key,
@@ -233,7 +242,8 @@ k_plan_meta(const int32_t *__restrict__ hist, const int32_t *__restrict__ key_of
     const int32_t cap = n_keys;
     const int32_t per_rank = (mode == 0) ? n_keys / R : keys_per_rank;
 
-    for (int i = threadIdx.x; i <= n_keys; i += blockDim.x) koff[i] = key_off_g[i];
+    __shared__ int32_t scan_scratch[33];
+    block_exclusive_scan(hist, n_keys, koff, scan_scratch);
     if (threadIdx.x < 8) s_red[threadIdx.x] = 0;
     if (threadIdx.x == 0) carry = 0;
     __syncthreads();

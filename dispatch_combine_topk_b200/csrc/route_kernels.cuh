@@ -1,11 +1,9 @@
 // Mapping, dispatch, dequantisation and combine kernels (sm_100a).
 //
 // Dispatch and combine are HBM-bound permute-copies: dispatch reads each token row
-// once and writes it K times, combine reads K rows per token and writes one. One CTA
-// works on one token at a time (grid-stride over tokens, grid = a multiple of the SM
-// count); its threads stride over the row in 16-byte chunks so that every warp access
-// is 512 contiguous bytes. The K row indices of the token are read once into shared
-// memory.
+// once and writes it K times, combine reads K rows per token and writes one. Rows are
+// moved in 16-byte chunks so that every warp access is 512 contiguous bytes, and the K
+// row indices of a token are read once per token.
 #pragma once
 
 #include "common.cuh"
@@ -87,8 +85,8 @@ __device__ __forceinline__ void load_token_rows(const int32_t *__restrict__ pos,
 
 // ------------------------------------------------------------------ dispatch (a4)
 
-// bf16 copy: recv[pos[t*K+k], :] = x[t, :]. V = uint4 (8 bf16 per access) when H % 8 ==
-// 0 and both pointers are 16-byte aligned, else uint16_t.
+// bf16 copy for unaligned buffers or H % 8 != 0: recv[pos[t*K+k], :] = x[t, :], one CTA
+// per token, one element per access.
 template <typename V>
 __global__ void __launch_bounds__(256)
 k_dispatch_copy(const V *__restrict__ x, const int32_t *__restrict__ pos, int64_t T, int K,
@@ -115,83 +113,52 @@ k_dispatch_copy(const V *__restrict__ x, const int32_t *__restrict__ pos, int64_
     }
 }
 
-// bf16 copy through shared memory with bulk copies (the default path).
+// bf16 copy, one warp per token (the default path).
 //
-// One CTA of one warp per SM, tokens strided over the CTAs. A ring of kStages row
-// buffers in shared memory: lane 0 bulk-loads token rows ahead into the ring (each
-// completion tracked by an mbarrier), lanes k < K each bulk-store the staged row to the
-// row of slot k and wait until their stores have finished reading the stage, then the
-// stage is refilled with the token kStages ahead. The row bytes travel HBM -> smem once
-// and smem -> HBM K times with no register traffic; the bulk engine keeps the K stores
-// of every SM in flight.
-//
-// Dynamic shared memory: 8*kStages (barriers) + 128*kStages (row indices), padded to
-// kDispatchSmemHead, then kStages rows of row_bytes. Requires row_bytes % 16 == 0 and
-// 16-byte aligned x and recv.
-constexpr int kDispatchSmemHead = 2048;
+// A warp reads its token's K row indices once (lane k holds slot k, broadcast with
+// shuffles), then walks the row in 16-byte chunks, kUnroll chunks per lane in flight,
+// storing each loaded chunk K times. No block barriers: a warp moves on to its next
+// token as soon as its stores are issued. Launched with many more warps than fit on
+// the GPU at once, so the last tokens spread over the whole machine. Measured against
+// bulk copies staged through shared memory (one issuing warp per SM) this path moves
+// more bytes per second on both 8 KB and 14 KB rows, since 64 warps per SM keep more
+// stores in flight than one bulk-copy issuer.
+// Requires H % 8 == 0 and 16-byte aligned x and recv.
+constexpr int kDispatchUnroll = 4;
 
-template <int kStages>
-__global__ void __launch_bounds__(32)
-k_dispatch_bulk(const uint16_t *__restrict__ x, const int32_t *__restrict__ pos, int64_t T, int K, int64_t H,
-                int64_t rows, uint16_t *__restrict__ recv)
+__global__ void __launch_bounds__(256)
+k_dispatch_warp(const uint4 *__restrict__ x, const int32_t *__restrict__ pos, int64_t T, int K, int64_t H8,
+                int64_t rows, uint4 *__restrict__ recv)
 {
-    extern __shared__ __align__(128) int32_t smem_i32[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>(smem_i32);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
-    int32_t *srow = reinterpret_cast<int32_t *>(smem + 8 * kStages);   // [kStages][32]
-    unsigned char *stage = smem + kDispatchSmemHead;
-    const uint32_t row_bytes = (uint32_t)(H * 2);
-    const int lane = threadIdx.x;
-    if (lane == 0) {
-        for (int s = 0; s < kStages; s++) mbar_init(&bar[s], 1);
-        mbar_fence_init();
-    }
-    __syncwarp();
-    const int64_t n = blockIdx.x < T ? (T - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-    auto token = [&](int64_t i) { return (int64_t)blockIdx.x + i * gridDim.x; };
-    auto fetch = [&](int64_t i) {
-        const int s = (int)(i % kStages);
-        const int64_t t = token(i);
-        if (lane == 0) {
-            mbar_arrive_expect_tx(&bar[s], row_bytes);
-            bulk_load_g2s(stage + (size_t)s * row_bytes, x + t * H, row_bytes, &bar[s]);
-        }
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+        int32_t mine = -1;
         if (lane < K) {
-            int32_t p = pos[t * K + lane];
-            if (p < -1 || (int64_t)p >= rows) {
+            mine = pos[t * K + lane];
+            if (mine < -1 || (int64_t)mine >= rows) {
                 flag_error(0x2);
-                p = -1;
+                mine = -1;
             }
-            srow[s * 32 + lane] = p;
         }
-    };
-    for (int64_t i = 0; i < n && i < kStages; i++) fetch(i);
-    __syncwarp();
-    for (int64_t i = 0; i < n; i++) {
-        const int s = (int)(i % kStages);
-        const bool ok = mbar_wait_bounded(&bar[s], (uint32_t)((i / kStages) & 1));
-        if (!__all_sync(0xffffffffu, ok)) {
-            // A load never completed: record it, wait (bounded) for the other loads
-            // still in flight into this CTA's ring, and leave.
-            if (lane == 0) {
-                flag_error(0x10);
-                for (int64_t j = i + 1; j < n && j < i + kStages; j++)
-                    mbar_wait_bounded(&bar[j % kStages], (uint32_t)((j / kStages) & 1));
+        const uint4 *src = x + t * H8;
+        // warp-uniform trip count: every lane reaches the shuffles below
+        for (int64_t base = 0; base < H8; base += 32 * kDispatchUnroll) {
+            const int64_t c0 = base + lane;
+            uint4 v[kDispatchUnroll];
+#pragma unroll
+            for (int u = 0; u < kDispatchUnroll; u++)
+                if (c0 + 32 * u < H8) v[u] = ld_stream(src + c0 + 32 * u);
+            for (int k = 0; k < K; k++) {
+                const int32_t p = __shfl_sync(0xffffffffu, mine, k);
+                if (p < 0) continue;
+                uint4 *dst = recv + (int64_t)p * H8;
+#pragma unroll
+                for (int u = 0; u < kDispatchUnroll; u++)
+                    if (c0 + 32 * u < H8) st_v4(dst + c0 + 32 * u, v[u]);
             }
-            break;
         }
-        if (lane < K) {
-            const int32_t p = srow[s * 32 + lane];
-            if (p >= 0) bulk_store_s2g(recv + (int64_t)p * H, stage + (size_t)s * row_bytes, row_bytes);
-            bulk_commit();
-            bulk_wait_read_all();
-        }
-        __syncwarp();
-        if (i + kStages < n) fetch(i + kStages);
-        __syncwarp();
     }
-    if (lane < K) bulk_wait_all();
-    __syncwarp();
 }
 
 // Quantise 8 fp32 values to int8 with the per-token scale; packed little-endian.
@@ -252,6 +219,118 @@ k_dispatch_int8(const uint4 *__restrict__ x, const int32_t *__restrict__ pos, in
         }
         __syncthreads();
     }
+}
+
+// Bytes before the row stages in the staged kernels' shared memory (barriers, row
+// indices, a reduction buffer).
+constexpr int kDispatchSmemHead = 2048;
+
+// Per-token dynamic int8 staged through shared memory (the default int8 path).
+//
+// kThreads threads per CTA, several CTAs per SM, tokens strided over CTAs. Warp 0 keeps
+// a ring of kStages bf16 rows filled by bulk loads (mbarrier completion) ahead of the
+// token being quantised. For each token all threads reduce amax over the staged row,
+// quantise it into one of two int8 row buffers, and lanes k < K of warp 0 bulk-store
+// the codes to the row of slot k and write the scale. The int8 buffer of token i is
+// reused at token i+2, after its stores have finished reading it.
+//
+// Dynamic shared memory: head (barriers, row indices, reduction) kDispatchSmemHead,
+// then kStages bf16 rows (2H bytes each), then 2 int8 rows (H bytes each).
+// Requires H % 16 == 0 and 16-byte aligned x and recv.
+template <int kStages, int kThreads>
+__global__ void __launch_bounds__(kThreads)
+k_dispatch_int8_staged(const uint16_t *__restrict__ x, const int32_t *__restrict__ pos, int64_t T, int K,
+                       int64_t H, int64_t rows, int8_t *__restrict__ recv, float *__restrict__ recv_scale)
+{
+    extern __shared__ __align__(128) int32_t smem_i32[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(smem_i32);
+    const uint32_t row_bytes = (uint32_t)(H * 2), q_bytes = (uint32_t)H;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
+    int32_t *srow = reinterpret_cast<int32_t *>(smem + 8 * kStages);              // [kStages][32]
+    float *red = reinterpret_cast<float *>(smem + 8 * kStages + 128 * kStages);   // [kThreads / 32]
+    unsigned char *stage = smem + kDispatchSmemHead;
+    unsigned char *qbuf = stage + (size_t)kStages * row_bytes;                    // [2][H]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        for (int s = 0; s < kStages; s++) mbar_init(&bar[s], 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    const int64_t n = blockIdx.x < T ? (T - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    auto token = [&](int64_t i) { return (int64_t)blockIdx.x + i * gridDim.x; };
+    auto fetch = [&](int64_t i) {   // warp 0 only
+        const int s = (int)(i % kStages);
+        const int64_t t = token(i);
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&bar[s], row_bytes);
+            bulk_load_g2s(stage + (size_t)s * row_bytes, x + t * H, row_bytes, &bar[s]);
+        }
+        if (lane < K) {
+            int32_t p = pos[t * K + lane];
+            if (p < -1 || (int64_t)p >= rows) {
+                flag_error(0x2);
+                p = -1;
+            }
+            srow[s * 32 + lane] = p;
+        }
+    };
+    if (warp == 0)
+        for (int64_t i = 0; i < n && i < kStages; i++) fetch(i);
+    __syncthreads();
+    const int64_t H8 = H / 8;
+    for (int64_t i = 0; i < n; i++) {
+        const int s = (int)(i % kStages);
+        const bool ok = mbar_wait_bounded(&bar[s], (uint32_t)((i / kStages) & 1));
+        if (!__syncthreads_and(ok)) {
+            if (tid == 0) {
+                flag_error(0x10);
+                for (int64_t j = i + 1; j < n && j < i + kStages; j++)
+                    mbar_wait_bounded(&bar[j % kStages], (uint32_t)((j / kStages) & 1));
+            }
+            break;
+        }
+        const uint4 *row = reinterpret_cast<const uint4 *>(stage + (size_t)s * row_bytes);
+        float amax = 0.0f;
+        for (int64_t c = tid; c < H8; c += kThreads) {
+            const uint4 v = row[c];
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16lo(v.x)), fabsf(bf16hi(v.x))),
+                                     fmaxf(fabsf(bf16lo(v.y)), fabsf(bf16hi(v.y)))));
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16lo(v.z)), fabsf(bf16hi(v.z))),
+                                     fmaxf(fabsf(bf16lo(v.w)), fabsf(bf16hi(v.w)))));
+        }
+        for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+        if (lane == 0) red[warp] = amax;
+        // the int8 buffer filled below was last stored two tokens ago
+        if (warp == 0 && lane < K) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        __syncthreads();
+        float m = red[0];
+        for (int w = 1; w < kThreads / 32; w++) m = fmaxf(m, red[w]);
+        const float scale = __fdiv_rn(m, 127.0f);
+        uint2 *q = reinterpret_cast<uint2 *>(qbuf + (size_t)(i & 1) * q_bytes);
+        for (int64_t c = tid; c < H8; c += kThreads) {
+            const uint4 v = row[c];
+            uint2 o;
+            o.x = q8x4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y), scale);
+            o.y = q8x4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w), scale);
+            q[c] = o;
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (warp == 0) {
+            if (lane < K) {
+                const int32_t p = srow[s * 32 + lane];
+                if (p >= 0) {
+                    bulk_store_s2g(recv + (int64_t)p * H, q, q_bytes);
+                    recv_scale[p] = scale;
+                }
+                bulk_commit();
+            }
+            __syncwarp();
+            if (i + kStages < n) fetch(i + kStages);   // every thread is done with stage s
+        }
+    }
+    if (warp == 0 && lane < K) bulk_wait_all();
+    __syncthreads();
 }
 
 // Scalar fallback of the int8 dispatch for any H and alignment.

@@ -195,7 +195,7 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
  * has to be cleared between calls. Calls that overlap on the GPU (unordered streams)
  * race on the array and produce wrong plans: order them.
  * Limit: plans whose mep_plan_workspace_size(R, n_keys, S, K) is at most
- * MEP_PLAN_STATIC_WS_BYTES, for instance up to 2,097,152 slots with up to 1023 keys.
+ * MEP_PLAN_STATIC_WS_BYTES, for instance up to 2,097,152 slots with up to 1024 keys.
  * Errors: those of mep_plan; MEP_ERR_WORKSPACE for a plan larger than the array;
  * MEP_ERR_CUDA if the address lookup fails.
  */

@@ -290,4 +290,12 @@ def test_dispatch_fallback_paths(case):
     out = torch.empty((T, H), dtype=torch.bfloat16, device=dev())
     mep.mep_combine(recv, pos_d, torch.from_numpy(gates).to(dev()), K, out)
     assert np.array_equal(bits(out), oracle.combine(ref, pos, gates, K))
+    # the int8 dispatch on the same buffers (its fallbacks for large or unaligned rows)
+    q = torch.zeros((rows, H), dtype=torch.int8, device=dev())
+    q_view = q if case == "huge_row" else torch.zeros(rows * H + 8, dtype=torch.int8, device=dev())[8:].view(rows, H)
+    sc = torch.zeros(rows, dtype=torch.float32, device=dev())
+    mep.mep_dispatch(x_d, pos_d, K, q_view, sc, quant=1)
+    q_ref, s_ref = oracle.dispatch_int8(bits(x), pos, K, rows)
+    assert np.array_equal(q_view.cpu().numpy(), q_ref)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
     assert mep.mep_get_error() == 0
