@@ -439,8 +439,46 @@ def run_gpu(args, w):
     t_plan = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     t_disp = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     t_comb = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
-    ms_max = max_over_ranks(ms, pg, dev)
-    ms_step = ms_max / args.steps
+    ms_eager = max_over_ranks(ms, pg, dev) / args.steps
+
+    # The same step captured once into a CUDA graph and replayed: the launches of a step
+    # go to the GPU as one unit (this matters most for small, launch-bound workloads).
+    graph_ms = None
+    if args.graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            rt.step(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g.replay()
+        stream.synchronize()
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            if flush is None:
+                g0.record(stream)
+                for _ in range(args.steps):
+                    g.replay()
+                g1.record(stream)
+                stream.synchronize()
+                gms = g0.elapsed_time(g1)
+            else:
+                gms = 0.0
+                for i in range(args.steps):
+                    flush.fill_(i & 0xff)
+                    g0.record(stream)
+                    g.replay()
+                    g1.record(stream)
+                    stream.synchronize()
+                    gms += g0.elapsed_time(g1)
+        graph_ms = max_over_ranks(gms, pg, dev) / args.steps
+        err = mep.mep_get_error(clear=True)
+        if err:
+            raise RuntimeError(f"device error word {err:#x} after the graph replays")
+        del g
+    ms_step = graph_ms if graph_ms is not None else ms_eager
     ok_device = rt.result_ok()
 
     # end to end: pinned host inputs -> device -> step -> result back to the host
@@ -492,6 +530,8 @@ def run_gpu(args, w):
             "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step,
+            "timing": {"mode": "cuda_graph_replay" if graph_ms is not None else "eager",
+                       "graph_ms_per_step": graph_ms, "eager_ms_per_step": ms_eager},
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int8" if w.quant else "bf16", "data": "synthetic",
             "config": {"workload": w.name, "R": w.R, "E": w.E, "S": w.S, "K": w.K, "H": w.H,
@@ -534,6 +574,9 @@ def main():
     ap.add_argument("--cpu-div", type=int, default=1,
                     help="cpu_baseline: the oracle routes S/cpu_div tokens per rank once")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", type=int, default=1,
+                    help="1: time the step as a replayed CUDA graph (per-kernel breakdown "
+                         "still comes from the eager steps); 0: eager only")
     ap.add_argument("--tokens-per-rank", type=int, default=0,
                     help="override S (a smaller case of the same workload, e.g. for profiling)")
     args = ap.parse_args()

@@ -293,7 +293,16 @@ mep_status_t mep_combine(const uint16_t *y, int64_t rows, const int32_t *pos,
     return launched();
 }
 
+mep_status_t mep_selftest_bounded_wait(int32_t max_polls, int32_t *timed_out, mep_stream_t stream)
+{
+    if (!timed_out) return MEP_ERR_NULLPTR;
+    if (max_polls < 1 || max_polls > mep::kWaitPolls) return MEP_ERR_VALUE;
+    mep::k_selftest_wait<<<1, 32, 0, (cudaStream_t)stream>>>(max_polls, timed_out);
+    return launched();
+}
+
 }  // extern "C"
+
 
 // ------------------------------------------------------------------------------------
 // mep_plan with scratch compiled into the library, for callers that cannot allocate.

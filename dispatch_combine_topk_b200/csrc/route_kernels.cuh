@@ -497,4 +497,25 @@ k_combine_scalar(const uint16_t *__restrict__ y, const int32_t *__restrict__ pos
     }
 }
 
+// --------------------------------------------------------------- wait self-test
+
+// Waits, with the library's bounded wait, on an mbarrier that nothing ever completes:
+// the wait runs out after max_polls polls, the kernel records MEP_DERR_TIMEOUT and
+// returns, exactly as a routing kernel whose bulk load never landed would.
+__global__ void k_selftest_wait(int max_polls, int32_t *timed_out)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);     // one arrival expected, none ever made
+        mbar_fence_init();
+    }
+    __syncthreads();
+    const bool ok = mbar_wait_bounded(&bar, 0, max_polls);
+    if (threadIdx.x == 0) {
+        if (!ok) flag_error(0x10);
+        *timed_out = ok ? 0 : 1;
+    }
+}
+
 }  // namespace mep
+

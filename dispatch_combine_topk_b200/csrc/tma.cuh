@@ -26,12 +26,14 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
 }
 
 // Wait for the phase with the given parity to complete. Non-blocking test with a
-// nanosleep back-off, at most ~2^22 polls (well under a second). Returns false if the
-// phase did not complete in that time.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity)
+// nanosleep back-off, at most max_polls polls (the default, 2^22, is well under a
+// second). Returns false if the phase did not complete in that time.
+constexpr int kWaitPolls = 1 << 22;
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int max_polls = kWaitPolls)
 {
     const uint32_t addr = smem_addr(bar);
-    for (int it = 0; it < (1 << 22); it++) {
+    for (int it = 0; it < max_polls; it++) {
         uint32_t done;
         asm volatile("{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
                      " selp.u32 %0, 1, 0, p;\n}\n"

@@ -19,7 +19,9 @@
  *    stream) and never synchronise the host, so a chain plan -> dispatch -> combine
  *    needs no host round trip (MoonEP's static shapes remove per-layer host syncs:
  *    twodots.gr article on MoonEP, static-shapes paragraph). Only mep_get_error
- *    synchronises.
+ *    synchronises. mep_plan, mep_update_expert, mep_dispatch, mep_dequantize and
+ *    mep_combine can be captured into a CUDA graph and replayed on new inputs, once each
+ *    has been called eagerly on the device (the first call sets kernel attributes).
  *  - A call first checks its arguments on the host and returns a status without
  *    launching anything when one is wrong: MEP_ERR_NULLPTR / MEP_ERR_DTYPE /
  *    MEP_ERR_SHAPE / MEP_ERR_VALUE mirror the aclnn codes 161001 (null tensor),
@@ -167,6 +169,18 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
                       int32_t *rep_count, int32_t *rep_key, int32_t *rep_cu,
                       mep_plan_stats_t *stats, void *workspace, size_t workspace_bytes,
                       mep_stream_t stream);
+
+/*
+ * Diagnostic: checks the failure path of the kernels' bounded waits on this GPU.
+ * Launches one CTA that waits, with the same bounded mbarrier wait the staged int8
+ * dispatch uses, on a barrier that nothing ever completes. After max_polls polls
+ * (1 .. 2^22; each poll backs off ~64 ns) the wait gives up, the kernel sets
+ * MEP_DERR_TIMEOUT in the device error word, writes 1 to *timed_out (a device int32)
+ * and returns; the context stays usable. Nothing waits without a bound, so this call
+ * cannot hang. Errors: NULL timed_out (MEP_ERR_NULLPTR), max_polls out of range
+ * (MEP_ERR_VALUE).
+ */
+mep_status_t mep_selftest_bounded_wait(int32_t max_polls, int32_t *timed_out, mep_stream_t stream);
 
 /* Size of the scratch array compiled into libmep for mep_plan_static_ws: 4 MiB. */
 #define MEP_PLAN_STATIC_WS_BYTES (4u << 20)

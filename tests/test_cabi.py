@@ -99,3 +99,7 @@ def test_dispatch_combine_argument_checks(L):
     assert L.mep_histogram(P, 10, 4, None, None) == 1
     assert L.mep_dequantize(None, P, 4, 8, P, None) == 1
     assert L.mep_get_error(None, 0) == 1
+    L.mep_selftest_bounded_wait.argtypes = [ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
+    assert L.mep_selftest_bounded_wait(10, None, None) == 1
+    assert L.mep_selftest_bounded_wait(0, P, None) == 4
+    assert L.mep_selftest_bounded_wait(1 << 23, P, None) == 4
