@@ -18,32 +18,35 @@ from . import build as _build
 _lib = None
 
 
+def _configure(L):
+    """Declare the C signatures on a loaded oracle library."""
+    P = ctypes.c_void_p
+    i32, i64 = ctypes.c_int32, ctypes.c_int64
+    L.orc_float_to_bf16.argtypes = [ctypes.c_float]
+    L.orc_float_to_bf16.restype = ctypes.c_uint16
+    L.orc_bf16_to_float.argtypes = [ctypes.c_uint16]
+    L.orc_bf16_to_float.restype = ctypes.c_float
+    L.orc_histogram.argtypes = [P, i64, i32, P]
+    L.orc_plan_balanced.argtypes = [P, i32, i32, i32, i32, P, P, P, i32, P, P, P, P]
+    L.orc_plan_grouped.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, P, i32, P, P, P, P]
+    L.orc_update_expert.argtypes = [P, i64, i32, P, i32, i32, P, P, P, i64, i64, i64, P, P]
+    L.orc_dispatch.argtypes = [P, P, i64, i32, i64, i64, P]
+    L.orc_quantize_row.argtypes = [P, i64, P, P]
+    L.orc_quantize_row.restype = None
+    L.orc_dispatch_int8.argtypes = [P, P, i64, i32, i64, i64, P, P]
+    L.orc_dequantize.argtypes = [P, P, i64, i64, P]
+    L.orc_dequantize.restype = None
+    L.orc_combine.argtypes = [P, i64, P, P, i64, i32, i64, P]
+    for name in ["orc_histogram", "orc_plan_balanced", "orc_plan_grouped",
+                 "orc_update_expert", "orc_dispatch", "orc_dispatch_int8", "orc_combine"]:
+        getattr(L, name).restype = ctypes.c_int
+    return L
+
+
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
-        L = ctypes.CDLL(path)
-        P = ctypes.c_void_p
-        i32, i64 = ctypes.c_int32, ctypes.c_int64
-        L.orc_float_to_bf16.argtypes = [ctypes.c_float]
-        L.orc_float_to_bf16.restype = ctypes.c_uint16
-        L.orc_bf16_to_float.argtypes = [ctypes.c_uint16]
-        L.orc_bf16_to_float.restype = ctypes.c_float
-        L.orc_histogram.argtypes = [P, i64, i32, P]
-        L.orc_plan_balanced.argtypes = [P, i32, i32, i32, i32, P, P, P, i32, P, P, P, P]
-        L.orc_plan_grouped.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, P, i32, P, P, P, P]
-        L.orc_update_expert.argtypes = [P, i64, i32, P, i32, i32, P, P, P, i64, i64, i64, P, P]
-        L.orc_dispatch.argtypes = [P, P, i64, i32, i64, i64, P]
-        L.orc_quantize_row.argtypes = [P, i64, P, P]
-        L.orc_quantize_row.restype = None
-        L.orc_dispatch_int8.argtypes = [P, P, i64, i32, i64, i64, P, P]
-        L.orc_dequantize.argtypes = [P, P, i64, i64, P]
-        L.orc_dequantize.restype = None
-        L.orc_combine.argtypes = [P, i64, P, P, i64, i32, i64, P]
-        for name in ["orc_histogram", "orc_plan_balanced", "orc_plan_grouped",
-                     "orc_update_expert", "orc_dispatch", "orc_dispatch_int8", "orc_combine"]:
-            getattr(L, name).restype = ctypes.c_int
-        _lib = L
+        _lib = _configure(ctypes.CDLL(_build.build()))
     return _lib
 
 

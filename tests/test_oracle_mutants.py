@@ -1,0 +1,116 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of the oracle's C source, builds the copy into
+a temporary library on the CPU, swaps it in for the oracle, and requires that at least
+one of the pins named for that case fails. A pin that cannot tell the planted mistake
+from the correct oracle would leave the oracle unpinned where that mistake could hide.
+"""
+import ctypes
+import importlib
+import inspect
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle import build as oracle_build
+
+# (what the mistake is, text replaced, replacement, pins expected to catch it)
+MUTANTS = [
+    ("plan order ignores the source rank",
+     "    if (a->src != b->src) return a->src < b->src ? -1 : 1;\n", "",
+     ["test_oracle_plan.test_plan_hand_example", "test_oracle_plan.test_plan_exhaustive_tiny"]),
+    ("home rank by modulo instead of division",
+     "sl[n].rank = e / per_rank;", "sl[n].rank = e % R;",
+     ["test_oracle_plan.test_plan_hand_example", "test_oracle_plan.test_plan_exhaustive_tiny"]),
+    ("cut at S*K-1 rows",
+     "row_rank[i] = (int32_t)(i / SK);", "row_rank[i] = (int32_t)(i / (SK - 1 > 0 ? SK - 1 : 1)) % R;",
+     ["test_oracle_plan.test_plan_hand_example", "test_oracle_plan.test_plan_exhaustive_tiny"]),
+    ("redundant counts every instance",
+     "if (inst[e] > 1) redundant += inst[e] - 1;", "redundant += inst[e];",
+     ["test_oracle_plan.test_plan_hand_example", "test_oracle_plan.test_plan_single_hot_expert_spans_every_rank"]),
+    ("prefetched counts home replicas",
+     "if (r != e / per_rank) prefetched += 1;", "prefetched += 1;",
+     ["test_oracle_plan.test_plan_hand_example", "test_oracle_plan.test_plan_balanced_input_keeps_experts_home"]),
+    ("histogram double-counts",
+     "        hist[e] += 1;\n    }\n    return ORC_OK;", "        hist[e] += (e == 0) ? 2 : 1;\n    }\n    return ORC_OK;",
+     ["test_oracle_plan.test_histogram_matches_bincount_and_sums_to_n"]),
+    ("grouped plan keeps dropped slots",
+     "                if (keep && !keep[n]) continue;\n", "",
+     ["test_oracle_plan.test_grouped_plan_packs_kept_slots_by_instance"]),
+    ("mapping mode 0 with a floor instead of a ceiling",
+     "(world_size + c - 1) / c;", "world_size / c;",
+     ["test_oracle_update_expert.test_mode0_column_never_exceeds_count",
+      "test_oracle_update_expert.test_mapping_hand_example"]),
+    ("mapping mode 1 by flat slot index",
+     "col = (i % c) + 1;", "col = ((i * K + k) % c) + 1;",
+     ["test_oracle_update_expert.test_mapping_hand_example", "test_oracle_update_expert.test_mode1_round_robin_by_token"]),
+    ("mapping mode 1 without the +1",
+     "col = (i % c) + 1;", "col = (i % c);",
+     ["test_oracle_update_expert.test_mapping_hand_example", "test_oracle_update_expert.test_mode1_round_robin_by_token"]),
+    ("pruning keeps the low scores (the literal line)",
+     "!(scales[i * K + k] < v)", "(scales[i * K + k] < v)",
+     ["test_oracle_update_expert.test_pruning_hand_example"]),
+    ("threshold value is the last product only",
+     "                v = v + prod;", "                v = prod;",
+     ["test_oracle_update_expert.test_pruning_hand_example"]),
+    ("quantisation rounds half away from zero",
+     "float r = nearbyintf(v);", "float r = roundf(v);",
+     ["test_oracle_numerics.test_quant_half_even_golden"]),
+    ("quantisation scale over 128",
+     "float scale = amax / 127.0f;", "float scale = amax / 128.0f;",
+     ["test_oracle_numerics.test_quant_half_even_golden", "test_oracle_numerics.test_quant_properties"]),
+    ("bf16 conversion truncates",
+     "u = u + 0x7fffu + keep_lsb;", "u = u;",
+     ["test_oracle_numerics.test_float_to_bf16_matches_torch"]),
+    ("dispatch copies the wrong token",
+     "const uint16_t *src = x + (n / K) * H;", "const uint16_t *src = x + (n % K) * H;",
+     ["test_oracle_numerics.test_dispatch_copies_rows_to_their_positions"]),
+    ("combine weights every slot by the first gate",
+     "float prod = gates[g * K + k] * bf16_bits_to_float(y[p * H + h]);",
+     "float prod = gates[g * K] * bf16_bits_to_float(y[p * H + h]);",
+     ["test_oracle_numerics.test_combine_softmax_gates_identity_expert_returns_x",
+      "test_oracle_numerics.test_combine_random_rows_within_error_bound"]),
+    ("combine skips the last slot",
+     "                acc = acc + prod;", "                if (k + 1 < K) acc = acc + prod;",
+     ["test_oracle_numerics.test_combine_k1_is_one_rounded_product",
+      ("test_oracle_numerics.test_combine_equal_power_of_two_gates_is_exact", {"K": 4})]),
+]
+
+
+def _run_pin(pin, golden_dir):
+    """Run one pin: a 'module.function' name, or (name, arguments of a parametrized pin)."""
+    pin, kwargs = (pin, {}) if isinstance(pin, str) else (pin[0], dict(pin[1]))
+    mod, fn = pin.split(".")
+    f = getattr(importlib.import_module(mod), fn)
+    if "golden_dir" in inspect.signature(f).parameters:
+        kwargs["golden_dir"] = golden_dir
+    f(**kwargs)
+
+
+@pytest.fixture(scope="module")
+def oracle_source():
+    return open(oracle_build.SRC).read()
+
+
+@pytest.mark.parametrize("what,find,repl,pins", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(what, find, repl, pins, oracle_source, tmp_path, golden_dir,
+                                   monkeypatch):
+    assert oracle_source.count(find) == 1, f"mutation target not unique: {what}"
+    # the correct oracle passes these pins
+    for pin in pins:
+        _run_pin(pin, golden_dir)
+    src = tmp_path / "mutant.c"
+    src.write_text(oracle_source.replace(find, repl))
+    so = tmp_path / "mutant.so"
+    subprocess.run(["gcc", *oracle_build.CFLAGS, str(src), "-o", str(so), "-lm"], check=True,
+                   capture_output=True)
+    monkeypatch.setattr(oracle, "_lib", oracle._configure(ctypes.CDLL(os.fspath(so))))
+    caught = []
+    for pin in pins:
+        try:
+            _run_pin(pin, golden_dir)
+        except (AssertionError, oracle.OracleError):
+            caught.append(pin)
+    assert caught, f"no pin caught the planted mistake: {what}"
