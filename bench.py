@@ -154,8 +154,8 @@ class ClockSampler:
 def oracle_sample(w, S_sample):
     """Time the oracle (as it stands) on a bounded sample: the same workload with S
     reduced to S_sample tokens per rank. The timed steps are those of the GPU step
-    (mapping and grouped plan, or the balanced plan; dispatch, bf16 or int8; combine);
-    the int8 identity expert (dequantisation) is not timed, as on the GPU.
+    (mapping and grouped plan, or the balanced plan; dispatch, bf16 or int8; combine,
+    of the int8 rows on the int8 workload).
     Returns (token-slots/s, description, seconds)."""
     import oracle
 
@@ -181,16 +181,14 @@ def oracle_sample(w, S_sample):
     if ws.quant:
         q, sc = oracle.dispatch_int8(x, p.pos, ws.K, rows)
         t2 = time.perf_counter()
-        y = oracle.dequantize(q, sc)
-        del q
-        t2b = time.perf_counter()
+        oracle.combine_int8(q, sc, p.pos, gates, ws.K)
     else:
         y = oracle.dispatch(x, p.pos, ws.K, rows)
-        t2 = t2b = time.perf_counter()
-    parts["dispatch"] = t2 - t1
-    oracle.combine(y, p.pos, gates, ws.K)
+        t2 = time.perf_counter()
+        oracle.combine(y, p.pos, gates, ws.K)
     t3 = time.perf_counter()
-    parts["combine"] = t3 - t2b
+    parts["dispatch"] = t2 - t1
+    parts["combine"] = t3 - t2
     dt = parts["plan"] + parts["dispatch"] + parts["combine"]
     desc = (f"oracle {'mapping+grouped plan' if ws.mapping else 'plan'}+"
             f"{'int8 ' if ws.quant else ''}dispatch+combine on R={ws.R} E={ws.E} S={ws.S} K={ws.K} "
@@ -257,9 +255,9 @@ class Route:
     """Device buffers and the launch sequence of one routing step for one workload.
 
     Balanced workloads: plan (mep_plan) -> dispatch (bf16, or int8 for the int8
-    workload) -> combine. The identity expert returns the dispatched rows; for int8 it is
-    mep_dequantize, run once before timing (its output is the same at every step, since
-    the inputs are fixed) and not part of the timed step.
+    workload) -> combine. The identity expert returns the dispatched rows; on the int8
+    workload they stay int8 and the combine reads the codes and scales
+    (mep_combine_int8, the same result as dequantising first).
     Mapping workload: mep_update_expert for every rank -> grouped plan over the physical
     instances -> dispatch -> combine.
     """
@@ -290,7 +288,6 @@ class Route:
             if w.quant:
                 self.recv = torch.empty((w.N, w.H), dtype=torch.int8, device=dev)
                 self.scale = torch.empty(w.N, dtype=torch.float32, device=dev)
-                self.y = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
             else:
                 self.recv = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
                 self.y = self.recv
@@ -320,12 +317,13 @@ class Route:
             self.mep.mep_dispatch(self.x, self.pb.pos, w.K, self.recv, stream=s)
         return 1
 
-    def expert(self, s):
-        if self.w.quant:
-            self.mep.mep_dequantize(self.recv, self.scale, self.y, stream=s)
-
     def combine(self, s):
-        self.mep.mep_combine(self.y, self.pb.pos, self.gates, self.w.K, self.out, stream=s)
+        if self.w.quant:
+            # the identity expert on int8 rows: the combine reads the codes and scales
+            self.mep.mep_combine_int8(self.recv, self.scale, self.pb.pos, self.gates, self.w.K,
+                                      self.out, stream=s)
+        else:
+            self.mep.mep_combine(self.y, self.pb.pos, self.gates, self.w.K, self.out, stream=s)
         return 1
 
     def step(self, s, ev=None):
@@ -350,13 +348,19 @@ class Route:
             return bool(torch.isfinite(self.out.float()).all())
         if w.quant:
             first = self.pb.pos.view(w.T, w.K)[:, 0].long()
-            return torch.equal(self.out.float(), self.y[first].float())
+            y_first = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=self.dev)
+            self.mep.mep_dequantize(self.recv[first], self.scale[first], y_first)
+            return torch.equal(self.out.float(), y_first.float())
         return torch.equal(self.out.float(), self.x.float())
 
     def kernel_name(self, step: str) -> str:
         """The library kernel that runs a step on this workload's shapes."""
         w = self.w
         if step == "combine":
+            if w.quant:
+                if w.H % 16 == 0:
+                    return "k_combine_int8_v16"
+                return "k_combine_int8_v8" if w.H % 8 == 0 else "k_combine_int8_scalar"
             return "k_combine_v8" if w.H % 8 == 0 else "k_combine_scalar"
         if w.quant:
             return "k_dispatch_int8_staged" if w.H % 16 == 0 else "k_dispatch_int8"
@@ -373,9 +377,10 @@ class Route:
         n_rows = int(self.pb.stats_dict()["n_kept"])
         if w.quant:
             disp = w.T * row + n_rows * w.H + 4 * n_rows + 4 * w.N
+            comb = n_rows * w.H + 4 * n_rows + w.T * row + 8 * w.N
         else:
             disp = w.T * row + n_rows * row + 4 * w.N
-        comb = n_rows * row + w.T * row + 8 * w.N
+            comb = n_rows * row + w.T * row + 8 * w.N
         plan = 16 * w.N
         return {"plan": plan, "dispatch": disp, "combine": comb}
 
@@ -399,8 +404,6 @@ def run_gpu(args, w):
     rt = Route(mep, rank_workload(w, rank), dev)
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
-        rt.step(stream)
-        rt.expert(stream)
         for _ in range(args.warmup):
             rt.step(stream)
     stream.synchronize()

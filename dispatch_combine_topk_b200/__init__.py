@@ -69,8 +69,9 @@ def lib() -> ctypes.CDLL:
         L.mep_dispatch.argtypes = [P, P, i64, i32, i64, i32, P, P, i64, P]
         L.mep_dequantize.argtypes = [P, P, i64, i64, P, P]
         L.mep_combine.argtypes = [P, i64, P, P, i64, i32, i64, P, P]
+        L.mep_combine_int8.argtypes = [P, P, i64, P, P, i64, i32, i64, P, P]
         for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
-                  "mep_dispatch", "mep_dequantize", "mep_combine"]:
+                  "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8"]:
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -204,6 +205,18 @@ def mep_combine(y: torch.Tensor, pos: torch.Tensor, gates: torch.Tensor, K: int,
                            _ptr(gates, torch.float32, "gates"), T, K, H,
                            _ptr(out, torch.bfloat16, "out"), _stream(stream))
     _ok(rc, "mep_combine")
+    return out
+
+
+def mep_combine_int8(yq: torch.Tensor, y_scale: torch.Tensor, pos: torch.Tensor, gates: torch.Tensor,
+                     K: int, out: torch.Tensor, stream=None):
+    """Combine of int8 rows with per-row scales (dequantisation fused into the sum)."""
+    T, H = out.shape
+    rc = lib().mep_combine_int8(_ptr(yq, torch.int8, "yq"), _ptr(y_scale, torch.float32, "y_scale"),
+                                yq.shape[0], _ptr(pos, torch.int32, "pos"),
+                                _ptr(gates, torch.float32, "gates"), T, K, H,
+                                _ptr(out, torch.bfloat16, "out"), _stream(stream))
+    _ok(rc, "mep_combine_int8")
     return out
 
 

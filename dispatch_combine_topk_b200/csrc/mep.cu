@@ -293,6 +293,47 @@ mep_status_t mep_combine(const uint16_t *y, int64_t rows, const int32_t *pos,
     return launched();
 }
 
+mep_status_t mep_combine_int8(const int8_t *yq, const float *y_scale, int64_t rows, const int32_t *pos,
+                              const float *gates, int64_t T, int32_t K, int64_t H, uint16_t *out,
+                              mep_stream_t stream)
+{
+    if (T > 0 && (!pos || !gates || !out || ((!yq || !y_scale) && rows > 0))) return MEP_ERR_NULLPTR;
+    if (T < 0 || K < 1 || K > MEP_MAX_K || H < 1 || rows < 0 || T * K >= ((int64_t)1 << 31))
+        return MEP_ERR_SHAPE;
+    if (T == 0) return MEP_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int grid = token_grid(T, 8);
+    if (H % 16 == 0 && aligned(yq, 16) && aligned(out, 16)) {
+        const uint4 *yv = (const uint4 *)yq;
+        uint4 *ov = (uint4 *)out;
+        const int64_t H16 = H / 16;
+        const int g16 = token_grid(T, 16);
+        switch (K) {
+        case 1: mep::k_combine_int8_v16<1><<<g16, 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16, rows, ov); break;
+        case 2: mep::k_combine_int8_v16<2><<<g16, 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16, rows, ov); break;
+        case 4: mep::k_combine_int8_v16<4><<<g16, 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16, rows, ov); break;
+        case 6: mep::k_combine_int8_v16<6><<<g16, 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16, rows, ov); break;
+        case 8: mep::k_combine_int8_v16<8><<<g16, 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16, rows, ov); break;
+        default: mep::k_combine_int8_v16<0><<<g16, 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16, rows, ov); break;
+        }
+    } else if (H % 8 == 0 && aligned(yq, 8) && aligned(out, 16)) {
+        const uint2 *yv = (const uint2 *)yq;
+        uint4 *ov = (uint4 *)out;
+        const int64_t H8 = H / 8;
+        switch (K) {
+        case 1: mep::k_combine_int8_v8<1><<<grid, 256, 0, s>>>(yv, y_scale, pos, gates, T, K, H8, rows, ov); break;
+        case 2: mep::k_combine_int8_v8<2><<<grid, 256, 0, s>>>(yv, y_scale, pos, gates, T, K, H8, rows, ov); break;
+        case 4: mep::k_combine_int8_v8<4><<<grid, 256, 0, s>>>(yv, y_scale, pos, gates, T, K, H8, rows, ov); break;
+        case 6: mep::k_combine_int8_v8<6><<<grid, 256, 0, s>>>(yv, y_scale, pos, gates, T, K, H8, rows, ov); break;
+        case 8: mep::k_combine_int8_v8<8><<<grid, 256, 0, s>>>(yv, y_scale, pos, gates, T, K, H8, rows, ov); break;
+        default: mep::k_combine_int8_v8<0><<<grid, 256, 0, s>>>(yv, y_scale, pos, gates, T, K, H8, rows, ov); break;
+        }
+    } else {
+        mep::k_combine_int8_scalar<<<grid, 256, 0, s>>>(yq, y_scale, pos, gates, T, K, H, rows, out);
+    }
+    return launched();
+}
+
 mep_status_t mep_selftest_bounded_wait(int32_t max_polls, int32_t *timed_out, mep_stream_t stream)
 {
     if (!timed_out) return MEP_ERR_NULLPTR;

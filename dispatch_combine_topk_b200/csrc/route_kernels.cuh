@@ -497,6 +497,201 @@ k_combine_scalar(const uint16_t *__restrict__ y, const int32_t *__restrict__ pos
     }
 }
 
+// --------------------------------------------------- combine of int8 rows (f1)
+
+// bf16 value of one dequantised code, as a float: bf16_rne(fl(q * scale)).
+__device__ __forceinline__ float dequant_bf16(int32_t q, float scale)
+{
+    return __bfloat162float(__float2bfloat16_rn(__fmul_rn((float)q, scale)));
+}
+
+// out[t, :] = bf16( sum_k fl(gate[t,k] * bf16(fl(q[pos[t,k], :] * scale[pos[t,k]]))) ):
+// exactly mep_dequantize followed by mep_combine, without writing the bf16 rows. One
+// CTA per token; each thread owns 8 columns (one 8-byte load of codes per slot), all K
+// loads of a chunk in flight before the first add.
+template <int KC>
+__global__ void __launch_bounds__(256)
+k_combine_int8_v8(const uint2 *__restrict__ yq, const float *__restrict__ yscale, const int32_t *__restrict__ pos,
+                  const float *__restrict__ gates, int64_t T, int Krt, int64_t H8, int64_t rows,
+                  uint4 *__restrict__ out)
+{
+    constexpr bool kFixed = KC > 0;
+    __shared__ int32_t sp[kMaxK];
+    __shared__ float sg[kMaxK];
+    __shared__ float ss[kMaxK];
+    const int K = kFixed ? KC : Krt;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        load_token_rows(pos, t, K, rows, sp);
+        if (threadIdx.x < K) sg[threadIdx.x] = gates[t * K + threadIdx.x];
+        __syncthreads();
+        if (threadIdx.x < K) ss[threadIdx.x] = sp[threadIdx.x] >= 0 ? yscale[sp[threadIdx.x]] : 0.0f;
+        __syncthreads();
+        for (int64_t c = threadIdx.x; c < H8; c += blockDim.x) {
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) acc[j] = 0.0f;
+            // Codes to floats without the conversion unit: with the sign bit flipped a
+            // code q is the byte q + 128, which a byte permute places in the mantissa of
+            // 1.5 * 2^23; subtracting 1.5 * 2^23 + 128 gives q exactly. The bf16
+            // rounding of fl(q * scale) is one packed round-to-nearest-even conversion
+            // per two values.
+            auto add = [&](const uint2 &v, float g, float sc) {
+                const uint32_t w[2] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u};
+#pragma unroll
+                for (int h = 0; h < 2; h++) {
+                    float p[4];
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const float qf = __uint_as_float(__byte_perm(w[h], 0x4B400000u, 0x7650u + j)) - 12583040.0f;
+                        p[j] = __fmul_rn(qf, sc);
+                    }
+                    const uint32_t b01 = pack_bf16x2(p[0], p[1]);
+                    const uint32_t b23 = pack_bf16x2(p[2], p[3]);
+                    acc[4 * h + 0] = __fadd_rn(acc[4 * h + 0], __fmul_rn(g, bf16lo(b01)));
+                    acc[4 * h + 1] = __fadd_rn(acc[4 * h + 1], __fmul_rn(g, bf16hi(b01)));
+                    acc[4 * h + 2] = __fadd_rn(acc[4 * h + 2], __fmul_rn(g, bf16lo(b23)));
+                    acc[4 * h + 3] = __fadd_rn(acc[4 * h + 3], __fmul_rn(g, bf16hi(b23)));
+                }
+            };
+            if constexpr (kFixed) {
+                uint2 v[KC];
+#pragma unroll
+                for (int k = 0; k < KC; k++) {
+                    const int32_t p = sp[k];
+                    v[k] = p >= 0 ? yq[(int64_t)p * H8 + c] : make_uint2(0, 0);
+                }
+#pragma unroll
+                for (int k = 0; k < KC; k++)
+                    if (sp[k] >= 0) add(v[k], sg[k], ss[k]);
+            } else {
+                for (int k = 0; k < K; k++) {
+                    const int32_t p = sp[k];
+                    if (p < 0) continue;
+                    add(yq[(int64_t)p * H8 + c], sg[k], ss[k]);
+                }
+            }
+            uint4 o;
+            o.x = pack_bf16x2(acc[0], acc[1]);
+            o.y = pack_bf16x2(acc[2], acc[3]);
+            o.z = pack_bf16x2(acc[4], acc[5]);
+            o.w = pack_bf16x2(acc[6], acc[7]);
+            st_v4(out + t * H8 + c, o);
+        }
+        __syncthreads();
+    }
+}
+
+// Same sum with 16 codes per slot per thread (one 16-byte load per slot, K of them in
+// flight per chunk): the path for H % 16 == 0 and 16-byte aligned buffers.
+template <int KC>
+__global__ void __launch_bounds__(128)
+k_combine_int8_v16(const uint4 *__restrict__ yq, const float *__restrict__ yscale, const int32_t *__restrict__ pos,
+                   const float *__restrict__ gates, int64_t T, int Krt, int64_t H16, int64_t rows,
+                   uint4 *__restrict__ out)
+{
+    constexpr bool kFixed = KC > 0;
+    __shared__ int32_t sp[kMaxK];
+    __shared__ float sg[kMaxK];
+    __shared__ float ss[kMaxK];
+    const int K = kFixed ? KC : Krt;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        load_token_rows(pos, t, K, rows, sp);
+        if (threadIdx.x < K) sg[threadIdx.x] = gates[t * K + threadIdx.x];
+        __syncthreads();
+        if (threadIdx.x < K) ss[threadIdx.x] = sp[threadIdx.x] >= 0 ? yscale[sp[threadIdx.x]] : 0.0f;
+        __syncthreads();
+        for (int64_t c = threadIdx.x; c < H16; c += blockDim.x) {
+            float2 acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) acc[j] = make_float2(0.0f, 0.0f);
+            // codes -> floats as in k_combine_int8_v8 (byte permute into 1.5 * 2^23); the
+            // exact bias subtraction and the code * scale product run on pairs of columns
+            // (packed f32x2, each half rounded on its own)
+            const float2 bias = make_float2(12583040.0f, 12583040.0f);
+            auto add = [&](const uint4 &v, float g, float sc) {
+                const uint32_t w[4] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u, v.z ^ 0x80808080u,
+                                       v.w ^ 0x80808080u};
+                const float2 g2 = make_float2(g, g), s2 = make_float2(sc, sc);
+#pragma unroll
+                for (int h = 0; h < 4; h++) {
+#pragma unroll
+                    for (int j = 0; j < 4; j += 2) {
+                        const float2 qb = make_float2(__uint_as_float(__byte_perm(w[h], 0x4B400000u, 0x7650u + j)),
+                                                      __uint_as_float(__byte_perm(w[h], 0x4B400000u, 0x7651u + j)));
+                        const float2 qf = add2_rn(qb, make_float2(-bias.x, -bias.y));
+                        const float2 p = mul2_rn(qf, s2);
+                        const uint32_t bb = pack_bf16x2(p.x, p.y);
+                        // gate product and sum stay scalar: a packed multiply feeding a
+                        // packed add may be fused into one rounding, which the sum's
+                        // definition (two roundings) does not allow
+                        float2 &a = acc[2 * h + j / 2];
+                        a.x = __fadd_rn(a.x, __fmul_rn(g2.x, bf16lo(bb)));
+                        a.y = __fadd_rn(a.y, __fmul_rn(g2.y, bf16hi(bb)));
+                    }
+                }
+            };
+            if constexpr (kFixed) {
+                uint4 v[KC];
+#pragma unroll
+                for (int k = 0; k < KC; k++) {
+                    const int32_t p = sp[k];
+                    v[k] = p >= 0 ? ld_stream(yq + (int64_t)p * H16 + c) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int k = 0; k < KC; k++)
+                    if (sp[k] >= 0) add(v[k], sg[k], ss[k]);
+            } else {
+                for (int k = 0; k < K; k++) {
+                    const int32_t p = sp[k];
+                    if (p < 0) continue;
+                    add(ld_stream(yq + (int64_t)p * H16 + c), sg[k], ss[k]);
+                }
+            }
+            uint4 o0, o1;
+            o0.x = pack_bf16x2(acc[0].x, acc[0].y);
+            o0.y = pack_bf16x2(acc[1].x, acc[1].y);
+            o0.z = pack_bf16x2(acc[2].x, acc[2].y);
+            o0.w = pack_bf16x2(acc[3].x, acc[3].y);
+            o1.x = pack_bf16x2(acc[4].x, acc[4].y);
+            o1.y = pack_bf16x2(acc[5].x, acc[5].y);
+            o1.z = pack_bf16x2(acc[6].x, acc[6].y);
+            o1.w = pack_bf16x2(acc[7].x, acc[7].y);
+            st_v4(out + t * 2 * H16 + 2 * c, o0);
+            st_v4(out + t * 2 * H16 + 2 * c + 1, o1);
+        }
+        __syncthreads();
+    }
+}
+
+// Element version for any H and alignment.
+__global__ void __launch_bounds__(256)
+k_combine_int8_scalar(const int8_t *__restrict__ yq, const float *__restrict__ yscale,
+                      const int32_t *__restrict__ pos, const float *__restrict__ gates, int64_t T, int K,
+                      int64_t H, int64_t rows, uint16_t *__restrict__ out)
+{
+    __shared__ int32_t sp[kMaxK];
+    __shared__ float sg[kMaxK];
+    __shared__ float ss[kMaxK];
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        load_token_rows(pos, t, K, rows, sp);
+        if (threadIdx.x < K) sg[threadIdx.x] = gates[t * K + threadIdx.x];
+        __syncthreads();
+        if (threadIdx.x < K) ss[threadIdx.x] = sp[threadIdx.x] >= 0 ? yscale[sp[threadIdx.x]] : 0.0f;
+        __syncthreads();
+        for (int64_t h = threadIdx.x; h < H; h += blockDim.x) {
+            float acc = 0.0f;
+            for (int k = 0; k < K; k++) {
+                const int32_t p = sp[k];
+                if (p < 0) continue;
+                acc = __fadd_rn(acc, __fmul_rn(sg[k], dequant_bf16(yq[(int64_t)p * H + h], ss[k])));
+            }
+            __nv_bfloat16 b = __float2bfloat16_rn(acc);
+            out[t * H + h] = *reinterpret_cast<uint16_t *>(&b);
+        }
+        __syncthreads();
+    }
+}
+
 // --------------------------------------------------------------- wait self-test
 
 // Waits, with the library's bounded wait, on an mbarrier that nothing ever completes:

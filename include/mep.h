@@ -171,6 +171,23 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
                       mep_stream_t stream);
 
 /*
+ * a5 with int8 rows (quantised return path) — combine of per-row int8 codes with one
+ * fp32 scale per row, as when the rows coming back to the token's rank are quantised
+ * for the exchange (commQuantMode of aclnnMoeDistributeCombineV2, gitcode
+ * ops-transformer aclnnMoeUpdateExpert doc, 调用示例):
+ *   out[g, h] = bf16_rne( sum over kept k, ascending, of
+ *                         fl(gates[g*K+k] * bf16_rne(fl(float(yq[p, h]) * y_scale[p]))) ),
+ *   p = pos[g*K+k]
+ * i.e. exactly mep_dequantize followed by mep_combine, without writing the bf16 rows:
+ * it reads H bytes per kept slot instead of 2H.
+ * yq int8 [rows, H]; y_scale fp32 [rows]; pos int32 [T*K]; gates fp32 [T*K];
+ * out bf16 [T, H]. Errors and data errors as mep_combine.
+ */
+mep_status_t mep_combine_int8(const int8_t *yq, const float *y_scale, int64_t rows,
+                              const int32_t *pos, const float *gates, int64_t T, int32_t K,
+                              int64_t H, uint16_t *out, mep_stream_t stream);
+
+/*
  * Diagnostic: checks the failure path of the kernels' bounded waits on this GPU.
  * Launches one CTA that waits, with the same bounded mbarrier wait the staged int8
  * dispatch uses, on a barrier that nothing ever completes. After max_polls polls

@@ -219,6 +219,12 @@ def combine(y_bits, pos, gates, K: int) -> np.ndarray:
     return out
 
 
+def combine_int8(q, scale, pos, gates, K: int) -> np.ndarray:
+    """Combine of int8 rows with per-row scales: by definition the combine of the
+    dequantised rows, y = bf16(fl(q * scale)) (the two oracle steps, composed)."""
+    return combine(dequantize(q, scale), pos, gates, K)
+
+
 def route_tokens(x_bits, kept, gates, K: int, quant: int = 0) -> np.ndarray:
     """Dispatch -> identity expert -> combine for a few tokens, one token at a time.
 

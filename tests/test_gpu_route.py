@@ -299,3 +299,49 @@ def test_dispatch_fallback_paths(case):
     assert np.array_equal(q_view.cpu().numpy(), q_ref)
     assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
     assert mep.mep_get_error() == 0
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 4, 6, 8, 16, 32])
+@pytest.mark.parametrize("H", [8, 72, 4096, 7, 130])
+def test_combine_int8_matches_oracle(K, H):
+    """Combine of int8 rows with per-row scales (dequantisation in the sum): arbitrary
+    codes, scales over several decades, dropped slots, every K, vector and element paths."""
+    rng = np.random.default_rng(K * 1000 + H)
+    T, rows = 61, 300
+    q = rng.integers(-127, 128, (rows, H)).astype(np.int8)
+    sc = (10.0 ** rng.uniform(-4, 2, rows)).astype(np.float32)
+    pos = rng.integers(0, rows, T * K).astype(np.int32)
+    pos[rng.random(T * K) < 0.1] = -1
+    gates = (rng.standard_normal(T * K)).astype(np.float32)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev())
+    mep.mep_combine_int8(torch.from_numpy(q).to(dev()), torch.from_numpy(sc).to(dev()),
+                         torch.from_numpy(pos).to(dev()), torch.from_numpy(gates).to(dev()), K, out)
+    assert np.array_equal(bits(out), oracle.combine_int8(q, sc, pos, gates, K))
+    assert mep.mep_get_error() == 0
+
+
+def test_full_int8_workload_fused_combine():
+    """The int8 workload end to end without bf16 rows: plan, int8 dispatch, combine of the
+    int8 rows. Every token equals the dequantise-then-combine path (both on the GPU),
+    sampled tokens equal the oracle routing them one by one."""
+    w = synth.get("int8")
+    ids, gates = synth.router(w)
+    x = synth.hidden(w)
+    pb = gpu_plan_balanced(ids, w.R, w.E, w.S, w.K)
+    x_d = x.to(dev())
+    g_d = torch.from_numpy(gates).to(dev())
+    recv = torch.empty((w.N, w.H), dtype=torch.int8, device=dev())
+    sc = torch.empty(w.N, dtype=torch.float32, device=dev())
+    mep.mep_dispatch(x_d, pb.pos, w.K, recv, sc, quant=1)
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev())
+    mep.mep_combine_int8(recv, sc, pb.pos, g_d, w.K, out)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(13)
+    toks = np.unique(np.concatenate([np.arange(w.R) * w.S, rng.integers(0, w.T, 150)]))
+    ref = oracle.route_tokens(bits(x[toks]), np.ones((toks.size, w.K), bool), gates[toks], w.K, 1)
+    assert np.array_equal(bits(out[torch.from_numpy(toks).to(dev())]), ref)
+    first = pb.pos.view(w.T, w.K)[:, 0].long()
+    y_first = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev())
+    mep.mep_dequantize(recv[first], sc[first], y_first)
+    assert torch.equal(out.float(), y_first.float())
+    assert mep.mep_get_error() == 0

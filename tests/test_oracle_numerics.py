@@ -180,3 +180,33 @@ def test_route_tokens_matches_whole_pipeline():
         full = oracle.combine(y, pos, g, K)
         one = oracle.route_tokens(x, (pos >= 0).reshape(T, K), g.reshape(T, K), K, quant)
         assert np.array_equal(full, one)
+
+
+def test_combine_int8_identity_rows_return_the_dequantised_row():
+    """int8 round trip with gates summing to 1: every token's K rows are the same codes
+    and scale, so the combine gives back bf16(q*scale) of its row (as values)."""
+    rng = np.random.default_rng(9)
+    T, K, H = 12, 8, 96
+    x = _bits((torch.randn(T, H, generator=torch.Generator().manual_seed(9)) * 7).to(torch.bfloat16))
+    z = rng.standard_normal((T, K))
+    g = (np.exp(z) / np.exp(z).sum(1, keepdims=True)).astype(np.float32)
+    pos = rng.permutation(T * K).astype(np.int32)
+    q, sc = oracle.dispatch_int8(x, pos, K, T * K)
+    out = oracle.combine_int8(q, sc, pos, g, K)
+    for t in range(T):
+        q0, s0 = oracle.quantize_row(x[t])
+        row = oracle.bf16_to_float(oracle.dequantize(q0[None, :], np.array([s0], np.float32))[0])
+        assert np.array_equal(oracle.bf16_to_float(out[t]), row)
+
+
+def test_combine_int8_k1_is_rounded_product_of_rounded_dequant():
+    rng = np.random.default_rng(10)
+    T, H = 7, 40
+    q = rng.integers(-127, 128, (T, H)).astype(np.int8)
+    sc = rng.random(T).astype(np.float32)
+    g = rng.random(T).astype(np.float32)
+    pos = np.arange(T, dtype=np.int32)
+    out = oracle.combine_int8(q, sc, pos, g, 1)
+    y = (torch.from_numpy(q.astype(np.float32)) * torch.from_numpy(sc)[:, None]).to(torch.bfloat16).float()
+    ref = _bits((torch.from_numpy(g)[:, None] * y).to(torch.bfloat16))
+    assert np.array_equal(out, ref)
