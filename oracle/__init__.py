@@ -37,6 +37,11 @@ def _configure(L):
     L.orc_dequantize.argtypes = [P, P, i64, i64, P]
     L.orc_dequantize.restype = None
     L.orc_combine.argtypes = [P, i64, P, P, i64, i32, i64, P]
+    L.orc_double_to_bf16.argtypes = [ctypes.c_double]
+    L.orc_double_to_bf16.restype = ctypes.c_uint16
+    L.orc_combine_add_rmsnorm.argtypes = [P, i64, P, P, i64, i32, i64, P, P, ctypes.c_double,
+                                          P, P, P, P]
+    L.orc_combine_add_rmsnorm.restype = ctypes.c_int
     for name in ["orc_histogram", "orc_plan_balanced", "orc_plan_grouped",
                  "orc_update_expert", "orc_dispatch", "orc_dispatch_int8", "orc_combine"]:
         getattr(L, name).restype = ctypes.c_int
@@ -245,3 +250,30 @@ def route_tokens(x_bits, kept, gates, K: int, quant: int = 0) -> np.ndarray:
             y = dispatch(x[i:i + 1], pos, K, K)
         out[i] = combine(y, pos, np.asarray(gates[i], np.float32), K)[0]
     return out
+
+
+def double_to_bf16(values) -> np.ndarray:
+    """binary64 -> bf16 bits, round to nearest even, in one rounding (element by element)."""
+    v = np.asarray(values, np.float64).ravel()
+    L = lib()
+    return np.array([L.orc_double_to_bf16(float(x)) for x in v], np.uint16).reshape(np.shape(values))
+
+
+def combine_add_rmsnorm(y_bits, pos, gates, K: int, residual_bits, gamma_bits, eps: float):
+    """Combine, residual add and RMSNorm. Returns (x_out bits, y_out bits, y_exact
+    float64 [T,H], rstd float64 [T])."""
+    y = _c(y_bits, np.uint16)
+    rows, H = y.shape
+    pos = _c(pos, np.int32).ravel()
+    gates = _c(gates, np.float32).ravel()
+    T = pos.size // K
+    res = _c(residual_bits, np.uint16)
+    gam = _c(gamma_bits, np.uint16).ravel()
+    x_out = np.empty((T, H), np.uint16)
+    y_out = np.empty((T, H), np.uint16)
+    y_exact = np.empty((T, H), np.float64)
+    rstd = np.empty(T, np.float64)
+    rc = lib().orc_combine_add_rmsnorm(_p(y), rows, _p(pos), _p(gates), T, K, H, _p(res), _p(gam),
+                                       float(eps), _p(x_out), _p(y_out), _p(y_exact), _p(rstd))
+    _check(rc, "combine_add_rmsnorm")
+    return x_out, y_out, y_exact, rstd

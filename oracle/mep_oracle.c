@@ -477,3 +477,74 @@ int orc_combine(const uint16_t *y, int64_t rows, const int32_t *pos, const float
     }
     return ORC_OK;
 }
+
+/* ------------------------------------------- f4: combine + residual + RMSNorm */
+
+/* binary64 -> bf16 bits, round to nearest, ties to even, directly (no intermediate
+ * binary32 rounding): the value with 8 significant bits nearest to v; below 2^-126 the
+ * bf16 grid is the fixed step 2^-133. */
+uint16_t orc_double_to_bf16(double v)
+{
+    if (v != v) return 0x7fc0u;
+    if (v == 0.0) return signbit(v) ? 0x8000u : 0x0000u;
+    int e;
+    double m = frexp(v, &e);               /* v = m * 2^e, 0.5 <= |m| < 1 */
+    double r;
+    if (e - 1 >= -126) {
+        r = ldexp(nearbyint(ldexp(m, 8)), e - 8);   /* 8 significant bits */
+    } else {
+        r = ldexp(nearbyint(ldexp(v, 133)), -133);  /* subnormal grid */
+    }
+    float f = (float)r;                    /* exact: r has at most 8 significant bits */
+    if (fabs(r) > 3.3895313892515355e38) f = (float)(v > 0 ? INFINITY : -INFINITY);
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+/*
+ * Combine followed by residual add and RMSNorm (aclnnMoeDistributeCombineAddRmsNorm:
+ * residualX, gamma, yOut, rstdOut, xOut; gitcode ops-transformer aclnnMoeUpdateExpert
+ * doc, 调用示例). For token g, with c = the combine output row (bf16, as orc_combine):
+ *   x_h      = c_h + residual_h                      (exact, binary64)
+ *   x_out_h  = bf16(x_h)
+ *   rstd     = 1 / sqrt( (1/H) sum_h x_h^2 + eps )   (binary64)
+ *   y_h      = x_h * rstd * gamma_h                  (binary64; y_exact)
+ *   y_out_h  = bf16(y_h)
+ * Outputs x_out and y_out as bf16 bits, y_exact [T,H] and rstd [T] as binary64.
+ */
+int orc_combine_add_rmsnorm(const uint16_t *y, int64_t rows, const int32_t *pos, const float *gates,
+                            int64_t T, int32_t K, int64_t H, const uint16_t *residual,
+                            const uint16_t *gamma, double eps, uint16_t *x_out, uint16_t *y_out,
+                            double *y_exact, double *rstd)
+{
+    if (T < 0 || K <= 0 || H <= 0 || rows < 0 || eps < 0) return ORC_EARG;
+    uint16_t *c = (uint16_t *)malloc((size_t)(T > 0 ? T : 1) * (size_t)H * sizeof(uint16_t));
+    double *x = (double *)malloc((size_t)H * sizeof(double));
+    if (!c || !x) {
+        free(c); free(x);
+        return ORC_EARG;
+    }
+    int rc = orc_combine(y, rows, pos, gates, T, K, H, c);
+    if (rc != ORC_OK) {
+        free(c); free(x);
+        return rc;
+    }
+    for (int64_t g = 0; g < T; g++) {
+        double ss = 0.0;
+        for (int64_t h = 0; h < H; h++) {
+            x[h] = (double)bf16_bits_to_float(c[g * H + h]) + (double)bf16_bits_to_float(residual[g * H + h]);
+            x_out[g * H + h] = orc_double_to_bf16(x[h]);
+            ss += x[h] * x[h];
+        }
+        double r = 1.0 / sqrt(ss / (double)H + eps);
+        rstd[g] = r;
+        for (int64_t h = 0; h < H; h++) {
+            double v = x[h] * r * (double)bf16_bits_to_float(gamma[h]);
+            y_exact[g * H + h] = v;
+            y_out[g * H + h] = orc_double_to_bf16(v);
+        }
+    }
+    free(c); free(x);
+    return ORC_OK;
+}
