@@ -262,8 +262,9 @@ class Route:
     instances -> dispatch -> combine.
     """
 
-    def __init__(self, mep, w, dev):
+    def __init__(self, mep, w, dev, epilogue: str = "none"):
         self.mep, self.w, self.dev = mep, w, dev
+        self.epilogue = epilogue
         ids, gates = synth.router(w)
         x = synth.hidden(w)
         self.host = dict(ids=torch.from_numpy(ids).view(-1), gates=torch.from_numpy(gates).view(-1), x=x)
@@ -272,6 +273,12 @@ class Route:
         self.x = x.to(dev)
         self.out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
         self.launches = 0
+        if epilogue == "add_rmsnorm":
+            # combine fused with residual add + RMSNorm: residual rows and gamma as inputs
+            self.residual = synth.expert_outputs(w, w.T).to(dev)
+            self.gamma = torch.ones(w.H, dtype=torch.bfloat16, device=dev)
+            self.y_norm = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
+            self.rstd = torch.empty(w.T, dtype=torch.float32, device=dev)
         if w.mapping:
             table, thr, active = synth.mapping_inputs(w)
             self.table = torch.from_numpy(table).to(dev)
@@ -318,6 +325,11 @@ class Route:
         return 1
 
     def combine(self, s):
+        if self.epilogue == "add_rmsnorm":
+            self.mep.mep_combine_add_rmsnorm(self.y, self.pb.pos, self.gates, self.w.K, self.residual,
+                                             self.gamma, 1e-6, self.out, self.y_norm, self.rstd,
+                                             stream=s)
+            return 1
         if self.w.quant:
             # the identity expert on int8 rows: the combine reads the codes and scales
             self.mep.mep_combine_int8(self.recv, self.scale, self.pb.pos, self.gates, self.w.K,
@@ -344,6 +356,9 @@ class Route:
         """Closed form of the identity expert with gates summing to 1: every token whose
         K slots are all kept comes back as its expert row (compared as values)."""
         w = self.w
+        if self.epilogue == "add_rmsnorm":
+            ref = (self.x.float() + self.residual.float()).to(torch.bfloat16).float()
+            return torch.equal(self.out.float(), ref) and bool(torch.isfinite(self.y_norm.float()).all())
         if w.mapping:
             return bool(torch.isfinite(self.out.float()).all())
         if w.quant:
@@ -357,6 +372,8 @@ class Route:
         """The library kernel that runs a step on this workload's shapes."""
         w = self.w
         if step == "combine":
+            if self.epilogue == "add_rmsnorm":
+                return "k_combine_add_rmsnorm_v8" if w.H % 8 == 0 else "k_combine_add_rmsnorm_scalar"
             if w.quant:
                 if w.H % 16 == 0:
                     return "k_combine_int8_v16"
@@ -381,6 +398,8 @@ class Route:
         else:
             disp = w.T * row + n_rows * row + 4 * w.N
             comb = n_rows * row + w.T * row + 8 * w.N
+        if self.epilogue == "add_rmsnorm":
+            comb += 2 * w.T * row + 4 * w.T + row   # residual in, normalised rows out, rstd, gamma
         plan = 16 * w.N
         return {"plan": plan, "dispatch": disp, "combine": comb}
 
@@ -401,7 +420,9 @@ def run_gpu(args, w):
                                 device_id=dev)
         pg = dist
     # every rank routes its own independent batch (different seed)
-    rt = Route(mep, rank_workload(w, rank), dev)
+    if args.epilogue != "none" and (w.quant or w.mapping):
+        raise SystemExit("--epilogue applies to the balanced bf16 workloads")
+    rt = Route(mep, rank_workload(w, rank), dev, args.epilogue)
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -538,6 +559,7 @@ def run_gpu(args, w):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int8" if w.quant else "bf16", "data": "synthetic",
             "config": {"workload": w.name, "R": w.R, "E": w.E, "S": w.S, "K": w.K, "H": w.H,
+                       "epilogue": args.epilogue,
                        "token_slots_per_gpu": w.N, "seed": w.seed, "parallelism": f"replicas{world}",
                        "l2": (f"working set {rt.working_set_bytes() / 1e6:.0f} MB "
                               + ("< 2x L2 (126 MB): L2 flushed between steps (256 MB write, "
@@ -580,6 +602,8 @@ def main():
     ap.add_argument("--graph", type=int, default=1,
                     help="1: time the step as a replayed CUDA graph (per-kernel breakdown "
                          "still comes from the eager steps); 0: eager only")
+    ap.add_argument("--epilogue", default="none", choices=["none", "add_rmsnorm"],
+                    help="add_rmsnorm: combine fused with residual add + RMSNorm")
     ap.add_argument("--tokens-per-rank", type=int, default=0,
                     help="override S (a smaller case of the same workload, e.g. for profiling)")
     args = ap.parse_args()

@@ -70,8 +70,11 @@ def lib() -> ctypes.CDLL:
         L.mep_dequantize.argtypes = [P, P, i64, i64, P, P]
         L.mep_combine.argtypes = [P, i64, P, P, i64, i32, i64, P, P]
         L.mep_combine_int8.argtypes = [P, P, i64, P, P, i64, i32, i64, P, P]
+        L.mep_combine_add_rmsnorm.argtypes = [P, i64, P, P, i64, i32, i64, P, P, ctypes.c_float,
+                                              P, P, P, P]
         for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
-                  "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8"]:
+                  "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8",
+                  "mep_combine_add_rmsnorm"]:
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -218,6 +221,22 @@ def mep_combine_int8(yq: torch.Tensor, y_scale: torch.Tensor, pos: torch.Tensor,
                                 _ptr(out, torch.bfloat16, "out"), _stream(stream))
     _ok(rc, "mep_combine_int8")
     return out
+
+
+def mep_combine_add_rmsnorm(y: torch.Tensor, pos: torch.Tensor, gates: torch.Tensor, K: int,
+                            residual: torch.Tensor, gamma: torch.Tensor, eps: float,
+                            x_out: torch.Tensor, y_out: torch.Tensor, rstd_out: torch.Tensor,
+                            stream=None):
+    """Combine, residual add and RMSNorm in one kernel (see include/mep.h)."""
+    T, H = x_out.shape
+    rc = lib().mep_combine_add_rmsnorm(
+        _ptr(y, torch.bfloat16, "y"), y.shape[0], _ptr(pos, torch.int32, "pos"),
+        _ptr(gates, torch.float32, "gates"), T, K, H, _ptr(residual, torch.bfloat16, "residual"),
+        _ptr(gamma, torch.bfloat16, "gamma"), float(eps), _ptr(x_out, torch.bfloat16, "x_out"),
+        _ptr(y_out, torch.bfloat16, "y_out"), _ptr(rstd_out, torch.float32, "rstd_out"),
+        _stream(stream))
+    _ok(rc, "mep_combine_add_rmsnorm")
+    return x_out, y_out, rstd_out
 
 
 MEP_PLAN_STATIC_WS_BYTES = 4 << 20

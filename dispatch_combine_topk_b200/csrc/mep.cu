@@ -42,6 +42,13 @@ int sm_count()
         cudaFuncSetAttribute(mep::k_plan_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(mep::k_dispatch_int8_staged<4, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kBulkSmemMax);
+        const int norm_smem = (int)(sizeof(float) * MEP_RMSNORM_MAX_H);
+        cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
+        cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<6>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
+        cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
+        cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
+        cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
+        cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_scalar, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
         g_attrs_set[dev] = true;
     }
     return g_sm_count[dev];
@@ -330,6 +337,40 @@ mep_status_t mep_combine_int8(const int8_t *yq, const float *y_scale, int64_t ro
         }
     } else {
         mep::k_combine_int8_scalar<<<grid, 256, 0, s>>>(yq, y_scale, pos, gates, T, K, H, rows, out);
+    }
+    return launched();
+}
+
+mep_status_t mep_combine_add_rmsnorm(const uint16_t *y, int64_t rows, const int32_t *pos, const float *gates,
+                                     int64_t T, int32_t K, int64_t H, const uint16_t *residual,
+                                     const uint16_t *gamma, float eps, uint16_t *x_out, uint16_t *y_out,
+                                     float *rstd_out, mep_stream_t stream)
+{
+    if (T > 0 && (!pos || !gates || !residual || !gamma || !x_out || !y_out || !rstd_out || (!y && rows > 0)))
+        return MEP_ERR_NULLPTR;
+    if (T < 0 || K < 1 || K > MEP_MAX_K || H < 1 || H > MEP_RMSNORM_MAX_H || rows < 0 ||
+        T * K >= ((int64_t)1 << 31))
+        return MEP_ERR_SHAPE;
+    if (!(eps >= 0.0f) || eps > 1.0e30f) return MEP_ERR_VALUE;
+    if (T == 0) return MEP_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int grid = token_grid(T, 8);
+    const size_t smem = sizeof(float) * (size_t)H;
+    if (H % 8 == 0 && aligned(y, 16) && aligned(residual, 16) && aligned(gamma, 16) && aligned(x_out, 16) &&
+        aligned(y_out, 16)) {
+        const uint4 *yv = (const uint4 *)y, *rv = (const uint4 *)residual, *gv = (const uint4 *)gamma;
+        uint4 *xo = (uint4 *)x_out, *yo = (uint4 *)y_out;
+        const int64_t H8 = H / 8;
+        switch (K) {
+        case 8: mep::k_combine_add_rmsnorm_v8<8><<<grid, 256, smem, s>>>(yv, pos, gates, T, K, H8, rows, rv, gv, eps, xo, yo, rstd_out); break;
+        case 6: mep::k_combine_add_rmsnorm_v8<6><<<grid, 256, smem, s>>>(yv, pos, gates, T, K, H8, rows, rv, gv, eps, xo, yo, rstd_out); break;
+        case 4: mep::k_combine_add_rmsnorm_v8<4><<<grid, 256, smem, s>>>(yv, pos, gates, T, K, H8, rows, rv, gv, eps, xo, yo, rstd_out); break;
+        case 2: mep::k_combine_add_rmsnorm_v8<2><<<grid, 256, smem, s>>>(yv, pos, gates, T, K, H8, rows, rv, gv, eps, xo, yo, rstd_out); break;
+        default: mep::k_combine_add_rmsnorm_v8<0><<<grid, 256, smem, s>>>(yv, pos, gates, T, K, H8, rows, rv, gv, eps, xo, yo, rstd_out); break;
+        }
+    } else {
+        mep::k_combine_add_rmsnorm_scalar<<<grid, 256, smem, s>>>(y, pos, gates, T, K, H, rows, residual, gamma, eps,
+                                                                x_out, y_out, rstd_out);
     }
     return launched();
 }

@@ -692,6 +692,161 @@ k_combine_int8_scalar(const int8_t *__restrict__ yq, const float *__restrict__ y
     }
 }
 
+// ------------------------------------------- combine + residual add + RMSNorm (f4)
+
+// Block-wide sum of one float per thread (blockDim.x a multiple of 32, at most 1024);
+// red holds 33 floats of shared memory. Every thread gets the sum. Ends with a barrier.
+__device__ __forceinline__ float block_sum(float v, float *red)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        float t = lane < nw ? red[lane] : 0.0f;
+        for (int d = 16; d > 0; d >>= 1) t += __shfl_xor_sync(0xffffffffu, t, d);
+        if (lane == 0) red[32] = t;
+    }
+    __syncthreads();
+    return red[32];
+}
+
+// For every token: c = the combine output row (bf16, as k_combine_v8), x = fl(c + r)
+// with r the residual row, x_out = bf16(x), rstd = rsqrt_rn(fl(sum x^2 / H) + eps),
+// y_out = bf16(fl(fl(x * rstd) * gamma)). The fp32 row x is kept in shared memory
+// (H floats) between the reduction and the second pass.
+template <int KC>
+__global__ void __launch_bounds__(256)
+k_combine_add_rmsnorm_v8(const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
+                         const float *__restrict__ gates, int64_t T, int Krt, int64_t H8, int64_t rows,
+                         const uint4 *__restrict__ residual, const uint4 *__restrict__ gamma, float eps,
+                         uint4 *__restrict__ x_out, uint4 *__restrict__ y_out, float *__restrict__ rstd_out)
+{
+    constexpr bool kFixed = KC > 0;
+    extern __shared__ float xs[];    // [H]
+    __shared__ int32_t sp[kMaxK];
+    __shared__ float sg[kMaxK];
+    __shared__ float red[33];
+    const int K = kFixed ? KC : Krt;
+    const float inv_h = 1.0f / (float)(H8 * 8);
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        load_token_rows(pos, t, K, rows, sp);
+        if (threadIdx.x < K) sg[threadIdx.x] = gates[t * K + threadIdx.x];
+        __syncthreads();
+        float ss = 0.0f;
+        for (int64_t c = threadIdx.x; c < H8; c += blockDim.x) {
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) acc[j] = 0.0f;
+            if constexpr (kFixed) {
+                uint4 v[KC];
+#pragma unroll
+                for (int k = 0; k < KC; k++) {
+                    const int32_t p = sp[k];
+                    v[k] = p >= 0 ? ld_stream(y + (int64_t)p * H8 + c) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int k = 0; k < KC; k++) {
+                    if (sp[k] < 0) continue;
+                    const float g = sg[k];
+                    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        acc[2 * j] = __fadd_rn(acc[2 * j], __fmul_rn(g, bf16lo(w[j])));
+                        acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], __fmul_rn(g, bf16hi(w[j])));
+                    }
+                }
+            } else {
+                for (int k = 0; k < K; k++) {
+                    const int32_t p = sp[k];
+                    if (p < 0) continue;
+                    const uint4 vv = ld_stream(y + (int64_t)p * H8 + c);
+                    const float g = sg[k];
+                    const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        acc[2 * j] = __fadd_rn(acc[2 * j], __fmul_rn(g, bf16lo(w[j])));
+                        acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], __fmul_rn(g, bf16hi(w[j])));
+                    }
+                }
+            }
+            const uint4 r = ld_stream(residual + t * H8 + c);
+            const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+            uint32_t xo[4];
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const uint32_t cb = pack_bf16x2(acc[2 * j], acc[2 * j + 1]);   // the combine output
+                const float x0 = __fadd_rn(bf16lo(cb), bf16lo(rw[j]));
+                const float x1 = __fadd_rn(bf16hi(cb), bf16hi(rw[j]));
+                xs[8 * c + 2 * j] = x0;
+                xs[8 * c + 2 * j + 1] = x1;
+                ss = fmaf(x0, x0, ss);
+                ss = fmaf(x1, x1, ss);
+                xo[j] = pack_bf16x2(x0, x1);
+            }
+            st_v4(x_out + t * H8 + c, make_uint4(xo[0], xo[1], xo[2], xo[3]));
+        }
+        const float total = block_sum(ss, red);
+        const float rstd = __frsqrt_rn(__fadd_rn(__fmul_rn(total, inv_h), eps));
+        if (threadIdx.x == 0) rstd_out[t] = rstd;
+        for (int64_t c = threadIdx.x; c < H8; c += blockDim.x) {
+            const uint4 gm = gamma[c];
+            const uint32_t gw[4] = {gm.x, gm.y, gm.z, gm.w};
+            uint32_t yo[4];
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const float y0 = __fmul_rn(__fmul_rn(xs[8 * c + 2 * j], rstd), bf16lo(gw[j]));
+                const float y1 = __fmul_rn(__fmul_rn(xs[8 * c + 2 * j + 1], rstd), bf16hi(gw[j]));
+                yo[j] = pack_bf16x2(y0, y1);
+            }
+            st_v4(y_out + t * H8 + c, make_uint4(yo[0], yo[1], yo[2], yo[3]));
+        }
+        __syncthreads();
+    }
+}
+
+// Element version for any H and alignment (same arithmetic).
+__global__ void __launch_bounds__(256)
+k_combine_add_rmsnorm_scalar(const uint16_t *__restrict__ y, const int32_t *__restrict__ pos,
+                             const float *__restrict__ gates, int64_t T, int K, int64_t H, int64_t rows,
+                             const uint16_t *__restrict__ residual, const uint16_t *__restrict__ gamma,
+                             float eps, uint16_t *__restrict__ x_out, uint16_t *__restrict__ y_out,
+                             float *__restrict__ rstd_out)
+{
+    extern __shared__ float xs[];    // [H]
+    __shared__ int32_t sp[kMaxK];
+    __shared__ float sg[kMaxK];
+    __shared__ float red[33];
+    const float inv_h = 1.0f / (float)H;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        load_token_rows(pos, t, K, rows, sp);
+        if (threadIdx.x < K) sg[threadIdx.x] = gates[t * K + threadIdx.x];
+        __syncthreads();
+        float ss = 0.0f;
+        for (int64_t h = threadIdx.x; h < H; h += blockDim.x) {
+            float acc = 0.0f;
+            for (int k = 0; k < K; k++) {
+                const int32_t p = sp[k];
+                if (p < 0) continue;
+                acc = __fadd_rn(acc, __fmul_rn(sg[k], bf16lo(y[(int64_t)p * H + h])));
+            }
+            const float cval = bf16lo(pack_bf16x2(acc, 0.0f) & 0xffffu);
+            const float x = __fadd_rn(cval, bf16lo(residual[t * H + h]));
+            xs[h] = x;
+            ss = fmaf(x, x, ss);
+            x_out[t * H + h] = (uint16_t)(pack_bf16x2(x, 0.0f) & 0xffffu);
+        }
+        const float total = block_sum(ss, red);
+        const float rstd = __frsqrt_rn(__fadd_rn(__fmul_rn(total, inv_h), eps));
+        if (threadIdx.x == 0) rstd_out[t] = rstd;
+        for (int64_t h = threadIdx.x; h < H; h += blockDim.x) {
+            const float v = __fmul_rn(__fmul_rn(xs[h], rstd), bf16lo(gamma[h]));
+            y_out[t * H + h] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xffffu);
+        }
+        __syncthreads();
+    }
+}
+
 // --------------------------------------------------------------- wait self-test
 
 // Waits, with the library's bounded wait, on an mbarrier that nothing ever completes:

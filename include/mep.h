@@ -187,6 +187,35 @@ mep_status_t mep_combine_int8(const int8_t *yq, const float *y_scale, int64_t ro
                               const int32_t *pos, const float *gates, int64_t T, int32_t K,
                               int64_t H, uint16_t *out, mep_stream_t stream);
 
+/* Largest hidden size of mep_combine_add_rmsnorm (one fp32 row in shared memory). */
+#define MEP_RMSNORM_MAX_H 49152
+
+/*
+ * f4 — combine fused with residual add and RMSNorm (aclnnMoeDistributeCombineAddRmsNorm:
+ * residualX (BS,1,H), gamma (H,), yOut (BS,1,H), rstdOut (BS,1,1), xOut (BS,1,H);
+ * gitcode ops-transformer aclnnMoeUpdateExpert doc, 调用示例). The page names the
+ * arguments but not the formula; this is the plain add-then-RMSNorm reading. For every
+ * token g, with c_h = the combine output of mep_combine (bf16):
+ *   x_h      = fl(c_h + residual_h)                      (fp32)
+ *   x_out_h  = bf16_rne(x_h)
+ *   rstd     = rsqrt_rn(fl(fl(sum_h x_h^2) / H) + eps)   (fp32; the sum's order is the
+ *                                                          kernel's, not fixed)
+ *   y_out_h  = bf16_rne(fl(fl(x_h * rstd) * gamma_h))
+ * x_out is exact (the sum c + residual rounded once to bf16); y_out and rstd carry the
+ * rounding of an fp32 sum of H squares: within 1 bf16 ulp (y_out) and a relative
+ * ((H+3)/2 + 2) * 2^-24 (rstd) of the exact values.
+ * y bf16 [rows, H]; pos int32 [T*K]; gates fp32 [T*K]; residual bf16 [T, H]; gamma bf16
+ * [H]; x_out, y_out bf16 [T, H]; rstd_out fp32 [T].
+ * Errors: NULL pointer; T < 0, K outside [1, MEP_MAX_K], H outside [1, MEP_RMSNORM_MAX_H],
+ * rows < 0 (MEP_ERR_SHAPE); eps negative or not finite (MEP_ERR_VALUE). Data errors as
+ * mep_combine.
+ */
+mep_status_t mep_combine_add_rmsnorm(const uint16_t *y, int64_t rows, const int32_t *pos,
+                                     const float *gates, int64_t T, int32_t K, int64_t H,
+                                     const uint16_t *residual, const uint16_t *gamma, float eps,
+                                     uint16_t *x_out, uint16_t *y_out, float *rstd_out,
+                                     mep_stream_t stream);
+
 /*
  * Diagnostic: checks the failure path of the kernels' bounded waits on this GPU.
  * Launches one CTA that waits, with the same bounded mbarrier wait the staged int8
