@@ -42,6 +42,11 @@ def _configure(L):
     L.orc_combine_add_rmsnorm.argtypes = [P, i64, P, P, i64, i32, i64, P, P, ctypes.c_double,
                                           P, P, P, P]
     L.orc_combine_add_rmsnorm.restype = ctypes.c_int
+    L.orc_prefetch_plan.argtypes = [P, P, i32, i32, i32, i32, P, P]
+    L.orc_prefetch_weights.argtypes = [P, P, i32, i32, i32, i64, P]
+    L.orc_grad_reduce.argtypes = [P, P, P, i32, i32, i32, i64]
+    for name in ["orc_prefetch_plan", "orc_prefetch_weights", "orc_grad_reduce"]:
+        getattr(L, name).restype = ctypes.c_int
     for name in ["orc_histogram", "orc_plan_balanced", "orc_plan_grouped",
                  "orc_update_expert", "orc_dispatch", "orc_dispatch_int8", "orc_combine"]:
         getattr(L, name).restype = ctypes.c_int
@@ -277,3 +282,40 @@ def combine_add_rmsnorm(y_bits, pos, gates, K: int, residual_bits, gamma_bits, e
                                        float(eps), _p(x_out), _p(y_out), _p(y_exact), _p(rstd))
     _check(rc, "combine_add_rmsnorm")
     return x_out, y_out, y_exact, rstd
+
+
+# --------------------------------------------------------------------- f2 / f3
+
+def prefetch_plan(rep_count, rep_key, R: int, E: int, B: int):
+    """Slot of every prefetched replica and the weight row every replica reads.
+    Returns (slot_expert int32 [R, B], rep_weight int32 [R, cap])."""
+    rep_count = _c(rep_count, np.int32).ravel()
+    rep_key = _c(rep_key, np.int32)
+    cap = rep_key.shape[1]
+    slot_expert = np.empty((R, B), np.int32)
+    rep_weight = np.empty((R, cap), np.int32)
+    _check(lib().orc_prefetch_plan(_p(rep_count), _p(rep_key), R, E, cap, B, _p(slot_expert),
+                                   _p(rep_weight)), "prefetch_plan")
+    return slot_expert, rep_weight
+
+
+def prefetch_weights(w_home_bits, slot_expert, R: int, B: int, w_slots_bits=None):
+    w_home = _c(w_home_bits, np.uint16)
+    E = w_home.shape[0]
+    D = int(np.prod(w_home.shape[1:]))
+    se = _c(slot_expert, np.int32).ravel()
+    out = (np.zeros((R * B,) + w_home.shape[1:], np.uint16) if w_slots_bits is None
+           else np.array(w_slots_bits, np.uint16, copy=True))
+    _check(lib().orc_prefetch_weights(_p(w_home), _p(se), E, R, B, D, _p(out)), "prefetch_weights")
+    return out
+
+
+def grad_reduce(grad_home, grad_slots, slot_expert, R: int, B: int):
+    """Returns (new grad_home, new grad_slots) as float32 copies."""
+    gh = np.array(grad_home, np.float32, copy=True, order="C")
+    gs = np.array(grad_slots, np.float32, copy=True, order="C")
+    E = gh.shape[0]
+    D = int(np.prod(gh.shape[1:]))
+    se = _c(slot_expert, np.int32).ravel()
+    _check(lib().orc_grad_reduce(_p(gh), _p(gs), _p(se), E, R, B, D), "grad_reduce")
+    return gh, gs

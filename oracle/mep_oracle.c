@@ -548,3 +548,91 @@ int orc_combine_add_rmsnorm(const uint16_t *y, int64_t rows, const int32_t *pos,
     free(c); free(x);
     return ORC_OK;
 }
+
+/* ------------------------------- f2 / f3: replica weight prefetch and grad reduce */
+
+/*
+ * Prefetch slots (MoonEP memory contract; twodots.gr article on MoonEP: weights
+ * [E+B, H, H'], rows 0..E-1 the ranks' own experts, rows E..E+B-1 per-rank prefetch
+ * slots; B = E/R for training, 3-4 for inference; when a rank needs more remote experts
+ * than it has slots, it reads them from the home rank).
+ * Simulated layout: one weight array of E + R*B rows, rows [0, E) the home experts
+ * (expert e at row e, on rank e / (E/R)), rows E + r*B + b the slots of rank r.
+ * For every rank r, walk its replicas in order; a replica of an expert whose home is
+ * another rank takes the next free slot (slot_expert[r][b] = e, weight row E + r*B + b)
+ * while slots remain, else it reads the home row e. Home replicas read row e.
+ * Outputs slot_expert [R, B] (-1 = unused) and rep_weight [R, cap] (-1 past rep_count).
+ */
+int orc_prefetch_plan(const int32_t *rep_count, const int32_t *rep_key, int32_t R, int32_t E, int32_t cap,
+                      int32_t B, int32_t *slot_expert, int32_t *rep_weight)
+{
+    if (R <= 0 || E <= 0 || E % R != 0 || cap < 0 || B < 0) return ORC_EARG;
+    const int32_t per_rank = E / R;
+    for (int32_t r = 0; r < R; r++) {
+        for (int32_t b = 0; b < B; b++) slot_expert[(int64_t)r * B + b] = -1;
+        for (int32_t j = 0; j < cap; j++) rep_weight[(int64_t)r * cap + j] = -1;
+        if (rep_count[r] < 0 || rep_count[r] > cap) return ORC_EDATA;
+        int32_t used = 0;
+        for (int32_t j = 0; j < rep_count[r]; j++) {
+            int32_t e = rep_key[(int64_t)r * cap + j];
+            if (e < 0 || e >= E) return ORC_EDATA;
+            int32_t row;
+            if (e / per_rank == r) {
+                row = e;
+            } else if (used < B) {
+                slot_expert[(int64_t)r * B + used] = e;
+                row = E + r * B + used;
+                used++;
+            } else {
+                row = e;                    /* no slot left: read from the home rank */
+            }
+            rep_weight[(int64_t)r * cap + j] = row;
+        }
+    }
+    return ORC_OK;
+}
+
+/* w_slots[r*B + b, :] = w_home[slot_expert[r][b], :] for every used slot; D elements
+ * (bf16 bits) per expert. Unused slots are left as they are. */
+int orc_prefetch_weights(const uint16_t *w_home, const int32_t *slot_expert, int32_t E, int32_t R, int32_t B,
+                         int64_t D, uint16_t *w_slots)
+{
+    if (E <= 0 || R <= 0 || B < 0 || D <= 0) return ORC_EARG;
+    for (int64_t s = 0; s < (int64_t)R * B; s++) {
+        int32_t e = slot_expert[s];
+        if (e < 0) continue;
+        if (e >= E) return ORC_EDATA;
+        for (int64_t i = 0; i < D; i++) w_slots[s * D + i] = w_home[(int64_t)e * D + i];
+    }
+    return ORC_OK;
+}
+
+/*
+ * Replica gradient reduce (MoonEP: the gradients of a prefetched copy go to a separate
+ * reduce buffer [R, B, H, H']; the home rank reads the slots that hold its experts, adds
+ * them into its parameter gradient and clears them). For every expert e and element i,
+ * in binary32, slots taken in ascending (rank, slot) order:
+ *   grad_home[e][i] = (...(grad_home[e][i] + grad_slots[s0][i]) + grad_slots[s1][i]) ...
+ * over the slots s with slot_expert[s] == e; then those slots are set to zero.
+ */
+int orc_grad_reduce(float *grad_home, float *grad_slots, const int32_t *slot_expert, int32_t E, int32_t R,
+                    int32_t B, int64_t D)
+{
+    if (E <= 0 || R <= 0 || B < 0 || D <= 0) return ORC_EARG;
+    for (int64_t s = 0; s < (int64_t)R * B; s++)
+        if (slot_expert[s] >= E || slot_expert[s] < -1) return ORC_EDATA;
+    for (int32_t e = 0; e < E; e++) {
+        for (int64_t s = 0; s < (int64_t)R * B; s++) {
+            if (slot_expert[s] != e) continue;
+            for (int64_t i = 0; i < D; i++) {
+                float v = grad_home[(int64_t)e * D + i] + grad_slots[s * D + i];
+                grad_home[(int64_t)e * D + i] = v;
+            }
+        }
+    }
+    for (int64_t s = 0; s < (int64_t)R * B; s++) {
+        if (slot_expert[s] < 0) continue;
+        for (int64_t i = 0; i < D; i++) grad_slots[s * D + i] = 0.0f;
+    }
+    return ORC_OK;
+}

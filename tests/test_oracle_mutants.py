@@ -72,6 +72,17 @@ MUTANTS = [
      "float prod = gates[g * K] * bf16_bits_to_float(y[p * H + h]);",
      ["test_oracle_numerics.test_combine_softmax_gates_identity_expert_returns_x",
       "test_oracle_numerics.test_combine_random_rows_within_error_bound"]),
+    ("prefetch gives home replicas a slot",
+     "            if (e / per_rank == r) {\n                row = e;", "            if (0) {\n                row = e;",
+     ["test_oracle_prefetch.test_prefetch_hand_example",
+      ("test_oracle_prefetch.test_prefetch_properties", {"name": "tiny", "B": 4})]),
+    ("grad reduce adds in descending rank order",
+     "        for (int64_t s = 0; s < (int64_t)R * B; s++) {\n            if (slot_expert[s] != e) continue;",
+     "        for (int64_t s = (int64_t)R * B - 1; s >= 0; s--) {\n            if (slot_expert[s] != e) continue;",
+     ["test_oracle_prefetch.test_grad_reduce_adds_in_ascending_rank_order"]),
+    ("grad reduce leaves the slots uncleared",
+     "        for (int64_t i = 0; i < D; i++) grad_slots[s * D + i] = 0.0f;\n", "",
+     ["test_oracle_prefetch.test_grad_reduce_conserves_integer_gradients"]),
     ("combine skips the last slot",
      "                acc = acc + prod;", "                if (k + 1 < K) acc = acc + prod;",
      ["test_oracle_numerics.test_combine_k1_is_one_rounded_product",
