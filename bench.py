@@ -404,6 +404,57 @@ class Route:
         return {"plan": plan, "dispatch": disp, "combine": comb}
 
 
+def weight_side(mep, rt, args, dev, stream):
+    """The replica weight prefetch and the replica gradient reduce of the step's plan,
+    with B = E/R slots per rank (MoonEP's training setting) and experts of H x ffn_dim.
+    Timed separately from the routing step, with CUDA events over `steps` repetitions."""
+    w = rt.w
+    B = w.E // w.R
+    D = w.H * args.ffn_dim
+    cap = rt.pb.rep_key.shape[1]
+    g = torch.Generator(device=dev).manual_seed(1)
+    se = torch.empty((w.R, B), dtype=torch.int32, device=dev)
+    rw = torch.empty((w.R, cap), dtype=torch.int32, device=dev)
+    w_home = torch.randn((w.E, D), generator=g, device=dev).to(torch.bfloat16)
+    w_slots = torch.empty((w.R * B, D), dtype=torch.bfloat16, device=dev)
+    grad_home = torch.randn((w.E, D), generator=g, device=dev)
+    grad_slots = torch.randn((w.R * B, D), generator=g, device=dev)
+    reps = max(3, min(args.steps, 20))
+
+    def prefetch():
+        mep.mep_prefetch_plan(rt.pb, w.R, w.E, B, se, rw, stream=stream)
+        mep.mep_prefetch_weights(w_home, se, w.R, B, w_slots, stream=stream)
+
+    def reduce():
+        mep.mep_grad_reduce(grad_home, grad_slots, se, w.R, B, stream=stream)
+
+    out = {"B": B, "ffn_dim": args.ffn_dim, "bytes_per_expert_bf16": 2 * D}
+    with torch.cuda.stream(stream):
+        prefetch()
+    stream.synchronize()
+    used = int((se >= 0).sum().item())
+    for name, fn, nbytes in [("prefetch", prefetch, 2 * 2 * D * used),
+                             ("grad_reduce", reduce, None)]:
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+        stream.synchronize()
+        t = e0.elapsed_time(e1) / reps
+        if nbytes is None:
+            experts = int(torch.unique(se[se >= 0]).numel())
+            nbytes = 4 * D * (2 * experts + 2 * used)     # read+write home rows and slots
+        out[name] = {"ms": t, "gbs": nbytes / (t * 1e-3) / 1e9, "bytes": nbytes}
+    out["slots_used"] = used
+    del w_home, w_slots, grad_home, grad_slots
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_gpu(args, w):
     import dispatch_combine_topk_b200 as mep
 
@@ -464,6 +515,7 @@ def run_gpu(args, w):
     t_disp = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     t_comb = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
     ms_eager = max_over_ranks(ms, pg, dev) / args.steps
+    weights = weight_side(mep, rt, args, dev, stream) if args.ffn_dim > 0 else None
 
     # The same step captured once into a CUDA graph and replayed: the launches of a step
     # go to the GPU as one unit (this matters most for small, launch-bound workloads).
@@ -580,6 +632,7 @@ def run_gpu(args, w):
             "gpu_launches": launches,
             "clocks": clk.summary(),
             "plan_stats": rt.pb.stats_dict(),
+            "replica_weights": weights,
         }
         print(json.dumps(line), flush=True)
     if pg:
@@ -604,6 +657,9 @@ def main():
                          "still comes from the eager steps); 0: eager only")
     ap.add_argument("--epilogue", default="none", choices=["none", "add_rmsnorm"],
                     help="add_rmsnorm: combine fused with residual add + RMSNorm")
+    ap.add_argument("--ffn-dim", type=int, default=0,
+                    help="> 0: also time the replica weight prefetch and gradient reduce with "
+                         "experts of H x ffn_dim (MoonEP's benchmark uses 2048), B = E/R")
     ap.add_argument("--tokens-per-rank", type=int, default=0,
                     help="override S (a smaller case of the same workload, e.g. for profiling)")
     args = ap.parse_args()

@@ -72,9 +72,13 @@ def lib() -> ctypes.CDLL:
         L.mep_combine_int8.argtypes = [P, P, i64, P, P, i64, i32, i64, P, P]
         L.mep_combine_add_rmsnorm.argtypes = [P, i64, P, P, i64, i32, i64, P, P, ctypes.c_float,
                                               P, P, P, P]
+        L.mep_prefetch_plan.argtypes = [P, P, i32, i32, i32, i32, P, P, P]
+        L.mep_prefetch_weights.argtypes = [P, P, i32, i32, i32, i64, P, P]
+        L.mep_grad_reduce.argtypes = [P, P, P, i32, i32, i32, i64, P]
         for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
                   "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8",
-                  "mep_combine_add_rmsnorm"]:
+                  "mep_combine_add_rmsnorm", "mep_prefetch_plan", "mep_prefetch_weights",
+                  "mep_grad_reduce"]:
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -237,6 +241,41 @@ def mep_combine_add_rmsnorm(y: torch.Tensor, pos: torch.Tensor, gates: torch.Ten
         _stream(stream))
     _ok(rc, "mep_combine_add_rmsnorm")
     return x_out, y_out, rstd_out
+
+
+def mep_prefetch_plan(plan: PlanBuffers, R: int, E: int, B: int, slot_expert: torch.Tensor,
+                      rep_weight: torch.Tensor, stream=None):
+    """Slots of the prefetched replicas and the weight row of every replica."""
+    cap = plan.rep_key.shape[1]
+    rc = lib().mep_prefetch_plan(_ptr(plan.rep_count, torch.int32, "rep_count"),
+                                 _ptr(plan.rep_key, torch.int32, "rep_key"), R, E, cap, B,
+                                 _ptr(slot_expert, torch.int32, "slot_expert") if B > 0 else None,
+                                 _ptr(rep_weight, torch.int32, "rep_weight"), _stream(stream))
+    _ok(rc, "mep_prefetch_plan")
+    return slot_expert, rep_weight
+
+
+def mep_prefetch_weights(w_home: torch.Tensor, slot_expert: torch.Tensor, R: int, B: int,
+                         w_slots: torch.Tensor, stream=None):
+    E = w_home.shape[0]
+    D = w_home.numel() // E
+    rc = lib().mep_prefetch_weights(_ptr(w_home, torch.bfloat16, "w_home"),
+                                    _ptr(slot_expert, torch.int32, "slot_expert"), E, R, B, D,
+                                    _ptr(w_slots, torch.bfloat16, "w_slots"), _stream(stream))
+    _ok(rc, "mep_prefetch_weights")
+    return w_slots
+
+
+def mep_grad_reduce(grad_home: torch.Tensor, grad_slots: torch.Tensor, slot_expert: torch.Tensor,
+                    R: int, B: int, stream=None):
+    E = grad_home.shape[0]
+    D = grad_home.numel() // E
+    rc = lib().mep_grad_reduce(_ptr(grad_home, torch.float32, "grad_home"),
+                               _ptr(grad_slots, torch.float32, "grad_slots"),
+                               _ptr(slot_expert, torch.int32, "slot_expert"), E, R, B, D,
+                               _stream(stream))
+    _ok(rc, "mep_grad_reduce")
+    return grad_home, grad_slots
 
 
 MEP_PLAN_STATIC_WS_BYTES = 4 << 20

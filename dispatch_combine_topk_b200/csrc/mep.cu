@@ -375,6 +375,66 @@ mep_status_t mep_combine_add_rmsnorm(const uint16_t *y, int64_t rows, const int3
     return launched();
 }
 
+mep_status_t mep_prefetch_plan(const int32_t *rep_count, const int32_t *rep_key, int32_t R, int32_t E, int32_t cap,
+                               int32_t B, int32_t *slot_expert, int32_t *rep_weight, mep_stream_t stream)
+{
+    if (!rep_count || !rep_key || !rep_weight || (B > 0 && !slot_expert)) return MEP_ERR_NULLPTR;
+    if (R < 1 || E < 1 || E > MEP_MAX_KEYS || R > MEP_MAX_KEYS || cap < 1 || cap > MEP_MAX_KEYS || B < 0 ||
+        (int64_t)R * B > MEP_MAX_SLOTS)
+        return MEP_ERR_SHAPE;
+    if (E % R != 0) return MEP_ERR_VALUE;
+    mep::k_prefetch_plan<<<(unsigned)mep::ceil_div(R, 128), 128, 0, (cudaStream_t)stream>>>(
+        rep_count, rep_key, R, E, cap, B, slot_expert, rep_weight);
+    return launched();
+}
+
+mep_status_t mep_prefetch_weights(const uint16_t *w_home, const int32_t *slot_expert, int32_t E, int32_t R,
+                                  int32_t B, int64_t D, uint16_t *w_slots, mep_stream_t stream)
+{
+    if ((int64_t)R * B > 0 && (!w_home || !slot_expert || !w_slots)) return MEP_ERR_NULLPTR;
+    if (E < 1 || R < 1 || B < 0 || D < 1 || (int64_t)R * B > MEP_MAX_SLOTS) return MEP_ERR_SHAPE;
+    if ((int64_t)R * B == 0) return MEP_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t per = (int64_t)sm_count() * 8;   // CTAs per slot, before the cap below
+    if (D % 8 == 0 && aligned(w_home, 16) && aligned(w_slots, 16)) {
+        const int64_t D8 = D / 8;
+        int64_t gx = mep::ceil_div(D8, 256 * 4);
+        if (gx > per) gx = per;
+        dim3 grid((unsigned)(gx > 0 ? gx : 1), (unsigned)(R * B));
+        mep::k_prefetch_weights<<<grid, 256, 0, s>>>((const uint4 *)w_home, slot_expert, E, D8, (uint4 *)w_slots);
+    } else {
+        int64_t gx = mep::ceil_div(D, 256 * 4);
+        if (gx > per) gx = per;
+        dim3 grid((unsigned)(gx > 0 ? gx : 1), (unsigned)(R * B));
+        mep::k_prefetch_weights_scalar<<<grid, 256, 0, s>>>(w_home, slot_expert, E, D, w_slots);
+    }
+    return launched();
+}
+
+mep_status_t mep_grad_reduce(float *grad_home, float *grad_slots, const int32_t *slot_expert, int32_t E, int32_t R,
+                             int32_t B, int64_t D, mep_stream_t stream)
+{
+    if ((int64_t)R * B > 0 && (!grad_home || !grad_slots || !slot_expert)) return MEP_ERR_NULLPTR;
+    if (E < 1 || E > 65535 || R < 1 || B < 0 || D < 1 || (int64_t)R * B > MEP_MAX_SLOTS) return MEP_ERR_SHAPE;
+    if ((int64_t)R * B == 0) return MEP_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int32_t RB = R * B;
+    const int64_t per = (int64_t)sm_count() * 4;
+    if (D % 4 == 0 && aligned(grad_home, 16) && aligned(grad_slots, 16)) {
+        const int64_t D4 = D / 4;
+        int64_t gx = mep::ceil_div(D4, 256 * 4 * mep::kReduceUnroll);
+        if (gx > per) gx = per;
+        dim3 grid((unsigned)(gx > 0 ? gx : 1), (unsigned)E);
+        mep::k_grad_reduce<<<grid, 256, 0, s>>>((float4 *)grad_home, (float4 *)grad_slots, slot_expert, RB, D4);
+    } else {
+        int64_t gx = mep::ceil_div(D, 256 * 4);
+        if (gx > per) gx = per;
+        dim3 grid((unsigned)(gx > 0 ? gx : 1), (unsigned)E);
+        mep::k_grad_reduce_scalar<<<grid, 256, 0, s>>>(grad_home, grad_slots, slot_expert, RB, D);
+    }
+    return launched();
+}
+
 mep_status_t mep_selftest_bounded_wait(int32_t max_polls, int32_t *timed_out, mep_stream_t stream)
 {
     if (!timed_out) return MEP_ERR_NULLPTR;

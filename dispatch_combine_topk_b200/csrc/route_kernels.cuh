@@ -847,6 +847,185 @@ k_combine_add_rmsnorm_scalar(const uint16_t *__restrict__ y, const int32_t *__re
     }
 }
 
+// ----------------------------------- replica weight prefetch and grad reduce (f2, f3)
+
+// One thread per rank: walk its replicas in order; a replica of an expert homed on
+// another rank takes the next free slot while slots remain (weight row E + r*B + b),
+// otherwise it reads the home row e; home replicas read row e.
+__global__ void k_prefetch_plan(const int32_t *__restrict__ rep_count, const int32_t *__restrict__ rep_key, int32_t R,
+                                int32_t E, int32_t cap, int32_t B, int32_t *__restrict__ slot_expert,
+                                int32_t *__restrict__ rep_weight)
+{
+    const int32_t r = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= R) return;
+    const int32_t per_rank = E / R;
+    for (int32_t b = 0; b < B; b++) slot_expert[(int64_t)r * B + b] = -1;
+    for (int32_t j = 0; j < cap; j++) rep_weight[(int64_t)r * cap + j] = -1;
+    int32_t n = rep_count[r];
+    if (n < 0 || n > cap) {
+        flag_error(0x1);
+        n = n < 0 ? 0 : cap;
+    }
+    int32_t used = 0;
+    for (int32_t j = 0; j < n; j++) {
+        const int32_t e = rep_key[(int64_t)r * cap + j];
+        if (e < 0 || e >= E) {
+            flag_error(0x1);
+            continue;
+        }
+        int32_t row = e;
+        if (e / per_rank != r && used < B) {
+            slot_expert[(int64_t)r * B + used] = e;
+            row = E + r * B + used;
+            used++;
+        }
+        rep_weight[(int64_t)r * cap + j] = row;
+    }
+}
+
+// w_slots[s, :] = w_home[slot_expert[s], :]; blockIdx.y = slot, CTAs of a slot stride
+// over its 16-byte chunks. Unused slots (-1) exit at once.
+__global__ void __launch_bounds__(256)
+k_prefetch_weights(const uint4 *__restrict__ w_home, const int32_t *__restrict__ slot_expert, int32_t E, int64_t D8,
+                   uint4 *__restrict__ w_slots)
+{
+    const int32_t e = slot_expert[blockIdx.y];
+    if (e < 0) return;
+    if (e >= E) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(0x1);
+        return;
+    }
+    const uint4 *src = w_home + (int64_t)e * D8;
+    uint4 *dst = w_slots + (int64_t)blockIdx.y * D8;
+    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < D8; c += (int64_t)gridDim.x * blockDim.x)
+        st_v4(dst + c, ld_stream(src + c));
+}
+
+__global__ void __launch_bounds__(256)
+k_prefetch_weights_scalar(const uint16_t *__restrict__ w_home, const int32_t *__restrict__ slot_expert, int32_t E,
+                          int64_t D, uint16_t *__restrict__ w_slots)
+{
+    const int32_t e = slot_expert[blockIdx.y];
+    if (e < 0) return;
+    if (e >= E) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(0x1);
+        return;
+    }
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < D; i += (int64_t)gridDim.x * blockDim.x)
+        w_slots[(int64_t)blockIdx.y * D + i] = w_home[(int64_t)e * D + i];
+}
+
+// The slots holding expert e, in ascending order, compacted into list (shared memory,
+// at most `max_list` entries kept). Called by every thread; returns the count.
+__device__ __forceinline__ int32_t slots_of_expert(const int32_t *__restrict__ slot_expert, int32_t RB, int32_t e,
+                                                   int32_t *list, int32_t max_list, int32_t *warp_cnt)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int32_t total = 0;
+    for (int32_t base = 0; base < RB; base += blockDim.x) {
+        const int32_t s = base + threadIdx.x;
+        const bool hit = s < RB && slot_expert[s] == e;
+        const uint32_t m = __ballot_sync(0xffffffffu, hit);
+        if (lane == 0) warp_cnt[warp] = __popc(m);
+        __syncthreads();
+        int32_t before = total;
+        for (int w = 0; w < warp; w++) before += warp_cnt[w];
+        int32_t round_total = 0;
+        for (int w = 0; w < nw; w++) round_total += warp_cnt[w];
+        if (hit) {
+            const int32_t at = before + __popc(m & lanemask_lt());
+            if (at < max_list) list[at] = s;
+        }
+        total += round_total;
+        __syncthreads();
+    }
+    return total;
+}
+
+// grad_home[e, :] += grad_slots[s, :] over e's slots in ascending order (fp32, one
+// rounding per addition), then those slots are zeroed. blockIdx.y = expert; CTAs of an
+// expert stride over 16-byte chunks (4 floats). Experts without a slot do nothing.
+constexpr int kMaxSlotsPerExpert = 1024;
+constexpr int kReduceUnroll = 4;   // 16-byte chunks per thread in flight
+
+__global__ void __launch_bounds__(256)
+k_grad_reduce(float4 *__restrict__ grad_home, float4 *__restrict__ grad_slots, const int32_t *__restrict__ slot_expert,
+              int32_t RB, int64_t D4)
+{
+    __shared__ int32_t list[kMaxSlotsPerExpert];
+    __shared__ int32_t warp_cnt[32];
+    const int32_t e = blockIdx.y;
+    const int32_t n = slots_of_expert(slot_expert, RB, e, list, kMaxSlotsPerExpert, warp_cnt);
+    if (n == 0) return;
+    const int32_t m = n < kMaxSlotsPerExpert ? n : kMaxSlotsPerExpert;
+    if (n > kMaxSlotsPerExpert && blockIdx.x == 0 && threadIdx.x == 0) flag_error(0x1);
+    float4 *home = grad_home + (int64_t)e * D4;
+    const int64_t step = (int64_t)gridDim.x * blockDim.x * kReduceUnroll;
+    const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int64_t c0 = (int64_t)blockIdx.x * blockDim.x * kReduceUnroll + threadIdx.x; c0 < D4; c0 += step) {
+        float4 acc[kReduceUnroll];
+#pragma unroll
+        for (int u = 0; u < kReduceUnroll; u++) {
+            const int64_t c = c0 + (int64_t)u * blockDim.x;
+            acc[u] = c < D4 ? home[c] : zero;
+        }
+        // all of the expert's slots are read before any is cleared, so the loads of
+        // consecutive slots need not wait for stores to the same array
+#pragma unroll 2
+        for (int32_t i = 0; i < m; i++) {
+            const float4 *slot = grad_slots + (int64_t)list[i] * D4;
+            float4 v[kReduceUnroll];
+#pragma unroll
+            for (int u = 0; u < kReduceUnroll; u++) {
+                const int64_t c = c0 + (int64_t)u * blockDim.x;
+                v[u] = c < D4 ? slot[c] : zero;
+            }
+#pragma unroll
+            for (int u = 0; u < kReduceUnroll; u++) {
+                acc[u].x = __fadd_rn(acc[u].x, v[u].x);
+                acc[u].y = __fadd_rn(acc[u].y, v[u].y);
+                acc[u].z = __fadd_rn(acc[u].z, v[u].z);
+                acc[u].w = __fadd_rn(acc[u].w, v[u].w);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kReduceUnroll; u++) {
+            const int64_t c = c0 + (int64_t)u * blockDim.x;
+            if (c < D4) home[c] = acc[u];
+        }
+        for (int32_t i = 0; i < m; i++) {
+            float4 *slot = grad_slots + (int64_t)list[i] * D4;
+#pragma unroll
+            for (int u = 0; u < kReduceUnroll; u++) {
+                const int64_t c = c0 + (int64_t)u * blockDim.x;
+                if (c < D4) slot[c] = zero;
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256)
+k_grad_reduce_scalar(float *__restrict__ grad_home, float *__restrict__ grad_slots, const int32_t *__restrict__ slot_expert,
+                     int32_t RB, int64_t D)
+{
+    __shared__ int32_t list[kMaxSlotsPerExpert];
+    __shared__ int32_t warp_cnt[32];
+    const int32_t e = blockIdx.y;
+    const int32_t n = slots_of_expert(slot_expert, RB, e, list, kMaxSlotsPerExpert, warp_cnt);
+    if (n == 0) return;
+    const int32_t m = n < kMaxSlotsPerExpert ? n : kMaxSlotsPerExpert;
+    if (n > kMaxSlotsPerExpert && blockIdx.x == 0 && threadIdx.x == 0) flag_error(0x1);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < D; i += (int64_t)gridDim.x * blockDim.x) {
+        float acc = grad_home[(int64_t)e * D + i];
+        for (int32_t j = 0; j < m; j++) {
+            const int64_t k = (int64_t)list[j] * D + i;
+            acc = __fadd_rn(acc, grad_slots[k]);
+            grad_slots[k] = 0.0f;
+        }
+        grad_home[(int64_t)e * D + i] = acc;
+    }
+}
+
 // --------------------------------------------------------------- wait self-test
 
 // Waits, with the library's bounded wait, on an mbarrier that nothing ever completes:

@@ -216,6 +216,58 @@ mep_status_t mep_combine_add_rmsnorm(const uint16_t *y, int64_t rows, const int3
                                      uint16_t *x_out, uint16_t *y_out, float *rstd_out,
                                      mep_stream_t stream);
 
+/* Most prefetch slots over all ranks (R * B) of the prefetch and grad-reduce calls. */
+#define MEP_MAX_SLOTS 65535
+
+/*
+ * f2 — replica weight prefetch: where every replica of the plan reads its expert's
+ * weights (MoonEP memory contract; twodots.gr article on MoonEP: weights [E+B, H, H'],
+ * rows 0..E-1 the ranks' own experts, rows E..E+B-1 per-rank prefetch slots; B = E/R
+ * for training, 3-4 for inference; a rank with more remote experts than slots reads the
+ * rest from their home rank). On one GPU the weights are one array of E + R*B rows:
+ * rows [0, E) the home experts (expert e at row e, on rank e / (E/R)), rows E + r*B + b
+ * rank r's slots.
+ * mep_prefetch_plan walks each rank's replicas (rep_count, rep_key from mep_plan) in
+ * order: a replica of an expert homed elsewhere takes the rank's next free slot while
+ * slots remain (slot_expert[r, b] = e, rep_weight = E + r*B + b), otherwise it reads
+ * the home row e; home replicas read row e.
+ * rep_count int32 [R]; rep_key int32 [R, cap]; outputs slot_expert int32 [R, B]
+ * (-1 = unused) and rep_weight int32 [R, cap] (-1 past rep_count).
+ * Errors: NULL pointer; R, E or cap outside [1, MEP_MAX_KEYS], B < 0, R*B > MEP_MAX_SLOTS
+ * (MEP_ERR_SHAPE); E % R != 0 (MEP_ERR_VALUE). A count or key out of range sets
+ * MEP_DERR_KEY_RANGE.
+ */
+mep_status_t mep_prefetch_plan(const int32_t *rep_count, const int32_t *rep_key, int32_t R,
+                               int32_t E, int32_t cap, int32_t B, int32_t *slot_expert,
+                               int32_t *rep_weight, mep_stream_t stream);
+
+/*
+ * f2 — the prefetch copy: w_slots[s, :] = w_home[slot_expert[s], :] for every used slot
+ * s of the R*B slots (unused slots are left as they are). D bf16 elements per expert
+ * (H * H'). w_home bf16 [E, D]; slot_expert int32 [R*B]; w_slots bf16 [R*B, D].
+ * Errors: NULL pointer; E < 1, R < 1, B < 0, D < 1, R*B > MEP_MAX_SLOTS (MEP_ERR_SHAPE).
+ * A slot expert >= E is skipped and sets MEP_DERR_KEY_RANGE.
+ */
+mep_status_t mep_prefetch_weights(const uint16_t *w_home, const int32_t *slot_expert, int32_t E,
+                                  int32_t R, int32_t B, int64_t D, uint16_t *w_slots,
+                                  mep_stream_t stream);
+
+/*
+ * f3 — replica gradient reduce (MoonEP: the gradients of prefetched copies go to a
+ * separate reduce buffer [R, B, H, H']; the home rank reads the slots of its experts,
+ * adds them into its parameter gradient and clears them before the next microbatch).
+ * For every expert e and element i, in fp32, over the slots s with slot_expert[s] == e
+ * in ascending s (rank, then slot):
+ *   grad_home[e, i] = (...(grad_home[e, i] + grad_slots[s0, i]) + grad_slots[s1, i]) ...
+ * then those slots are set to zero. Unused slots are left as they are.
+ * grad_home fp32 [E, D]; grad_slots fp32 [R*B, D]; slot_expert int32 [R*B].
+ * Errors: NULL pointer; E outside [1, 65535], R < 1, B < 0, D < 1, R*B > MEP_MAX_SLOTS
+ * (MEP_ERR_SHAPE). More than 1024 slots holding one expert sets MEP_DERR_KEY_RANGE
+ * (only the first 1024 are added).
+ */
+mep_status_t mep_grad_reduce(float *grad_home, float *grad_slots, const int32_t *slot_expert,
+                             int32_t E, int32_t R, int32_t B, int64_t D, mep_stream_t stream);
+
 /*
  * Diagnostic: checks the failure path of the kernels' bounded waits on this GPU.
  * Launches one CTA that waits, with the same bounded mbarrier wait the staged int8
