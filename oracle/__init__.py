@@ -47,6 +47,8 @@ def _configure(L):
     L.orc_grad_reduce.argtypes = [P, P, P, i32, i32, i32, i64]
     for name in ["orc_prefetch_plan", "orc_prefetch_weights", "orc_grad_reduce"]:
         getattr(L, name).restype = ctypes.c_int
+    L.orc_dispatch_int8_smooth.argtypes = [P, P, P, i64, i32, i64, P, i32, i64, P, P]
+    L.orc_dispatch_int8_smooth.restype = ctypes.c_int
     for name in ["orc_histogram", "orc_plan_balanced", "orc_plan_grouped",
                  "orc_update_expert", "orc_dispatch", "orc_dispatch_int8", "orc_combine"]:
         getattr(L, name).restype = ctypes.c_int
@@ -319,3 +321,17 @@ def grad_reduce(grad_home, grad_slots, slot_expert, R: int, B: int):
     se = _c(slot_expert, np.int32).ravel()
     _check(lib().orc_grad_reduce(_p(gh), _p(gs), _p(se), E, R, B, D), "grad_reduce")
     return gh, gs
+
+
+def dispatch_int8_smooth(x_bits, ids, pos, K: int, smooth, rows: int):
+    """int8 dispatch with per-expert smoothing scales: codes and scale per slot."""
+    x = _c(x_bits, np.uint16)
+    T, H = x.shape
+    ids = _c(ids, np.int32).ravel()
+    pos = _c(pos, np.int32).ravel()
+    sm = _c(smooth, np.float32)
+    q = np.zeros((rows, H), np.int8)
+    sc = np.zeros(rows, np.float32)
+    _check(lib().orc_dispatch_int8_smooth(_p(x), _p(ids), _p(pos), T, K, H, _p(sm), sm.shape[0], rows,
+                                          _p(q), _p(sc)), "dispatch_int8_smooth")
+    return q, sc

@@ -636,3 +636,57 @@ int orc_grad_reduce(float *grad_home, float *grad_slots, const int32_t *slot_exp
     }
     return ORC_OK;
 }
+
+/* --------------------------------------------- f1: smooth-quantised int8 dispatch */
+
+/*
+ * Dispatch with per-expert smoothing before the dynamic int8 quantisation (the
+ * optional scales of shape (moeExpertNum, H), fp32, that aclnnMoeDistributeDispatch
+ * takes when quantMode > 0: gitcode ops-transformer aclnnMoeUpdateExpert doc, 调用示例;
+ * hiascend aclnnMoeDistributeDispatchSetup doc, scalesOptional). Reading: for every kept
+ * slot n of token g with expert e = ids[n],
+ *   xs_h  = fl(x_h * smooth[e, h])          (binary32)
+ *   amax  = max_h |xs_h|,  scale = amax / 127,
+ *   q_h   = clamp(round_half_even(xs_h / scale), -127, 127)   (q = 0 when amax == 0)
+ *   recv_q[pos[n], :] = q,  recv_scale[pos[n]] = scale.
+ * The codes and scale are per slot. The decisions are taken in binary32, as on the GPU.
+ */
+int orc_dispatch_int8_smooth(const uint16_t *x, const int32_t *ids, const int32_t *pos, int64_t T, int32_t K,
+                             int64_t H, const float *smooth, int32_t n_experts, int64_t rows, int8_t *recv_q,
+                             float *recv_scale)
+{
+    if (T < 0 || K <= 0 || H <= 0 || rows < 0 || n_experts <= 0) return ORC_EARG;
+    float *xs = (float *)malloc((size_t)H * sizeof(float));
+    if (!xs) return ORC_EARG;
+    for (int64_t n = 0; n < T * K; n++) {
+        int64_t p = pos[n];
+        if (p < 0) continue;
+        int32_t e = ids[n];
+        if (p >= rows || e < 0 || e >= n_experts) {
+            free(xs);
+            return ORC_EDATA;
+        }
+        const uint16_t *row = x + (n / K) * H;
+        float amax = 0.0f;
+        for (int64_t h = 0; h < H; h++) {
+            float v = bf16_bits_to_float(row[h]) * smooth[(int64_t)e * H + h];
+            xs[h] = v;
+            float a = fabsf(v);
+            if (a > amax) amax = a;
+        }
+        float scale = amax / 127.0f;
+        recv_scale[p] = scale;
+        for (int64_t h = 0; h < H; h++) {
+            int8_t q = 0;
+            if (scale != 0.0f) {
+                float r = nearbyintf(xs[h] / scale);
+                if (r > 127.0f) r = 127.0f;
+                if (r < -127.0f) r = -127.0f;
+                q = (int8_t)r;
+            }
+            recv_q[p * H + h] = q;
+        }
+    }
+    free(xs);
+    return ORC_OK;
+}

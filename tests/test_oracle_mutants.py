@@ -83,6 +83,11 @@ MUTANTS = [
     ("grad reduce leaves the slots uncleared",
      "        for (int64_t i = 0; i < D; i++) grad_slots[s * D + i] = 0.0f;\n", "",
      ["test_oracle_prefetch.test_grad_reduce_conserves_integer_gradients"]),
+    ("smooth quantisation uses the first expert's scales",
+     "float v = bf16_bits_to_float(row[h]) * smooth[(int64_t)e * H + h];",
+     "float v = bf16_bits_to_float(row[h]) * smooth[h];",
+     ["test_oracle_smooth.test_power_of_two_scales_commute_with_quantisation",
+      "test_oracle_smooth.test_per_slot_bounds"]),
     ("combine skips the last slot",
      "                acc = acc + prod;", "                if (k + 1 < K) acc = acc + prod;",
      ["test_oracle_numerics.test_combine_k1_is_one_rounded_product",
