@@ -75,10 +75,11 @@ def lib() -> ctypes.CDLL:
         L.mep_prefetch_plan.argtypes = [P, P, i32, i32, i32, i32, P, P, P]
         L.mep_prefetch_weights.argtypes = [P, P, i32, i32, i32, i64, P, P]
         L.mep_grad_reduce.argtypes = [P, P, P, i32, i32, i32, i64, P]
+        L.mep_dispatch_int8_smooth.argtypes = [P, P, P, i64, i32, i64, P, i32, P, P, i64, P]
         for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
                   "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8",
                   "mep_combine_add_rmsnorm", "mep_prefetch_plan", "mep_prefetch_weights",
-                  "mep_grad_reduce"]:
+                  "mep_grad_reduce", "mep_dispatch_int8_smooth"]:
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -276,6 +277,21 @@ def mep_grad_reduce(grad_home: torch.Tensor, grad_slots: torch.Tensor, slot_expe
                                _stream(stream))
     _ok(rc, "mep_grad_reduce")
     return grad_home, grad_slots
+
+
+def mep_dispatch_int8_smooth(x: torch.Tensor, ids: torch.Tensor, pos: torch.Tensor, K: int,
+                             smooth: torch.Tensor, recv: torch.Tensor, recv_scale: torch.Tensor,
+                             stream=None):
+    """int8 dispatch with per-expert smoothing scales (codes and scale per slot)."""
+    T, H = x.shape
+    rc = lib().mep_dispatch_int8_smooth(_ptr(x, torch.bfloat16, "x"), _ptr(ids, torch.int32, "ids"),
+                                        _ptr(pos, torch.int32, "pos"), T, K, H,
+                                        _ptr(smooth, torch.float32, "smooth"), smooth.shape[0],
+                                        _ptr(recv, torch.int8, "recv"),
+                                        _ptr(recv_scale, torch.float32, "recv_scale"), recv.shape[0],
+                                        _stream(stream))
+    _ok(rc, "mep_dispatch_int8_smooth")
+    return recv, recv_scale
 
 
 MEP_PLAN_STATIC_WS_BYTES = 4 << 20

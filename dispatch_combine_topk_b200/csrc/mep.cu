@@ -435,6 +435,32 @@ mep_status_t mep_grad_reduce(float *grad_home, float *grad_slots, const int32_t 
     return launched();
 }
 
+mep_status_t mep_dispatch_int8_smooth(const uint16_t *x, const int32_t *ids, const int32_t *pos, int64_t T,
+                                      int32_t K, int64_t H, const float *smooth, int32_t n_experts, int8_t *recv,
+                                      float *recv_scale, int64_t rows, mep_stream_t stream)
+{
+    if (T > 0 && (!x || !ids || !pos || !smooth || (rows > 0 && (!recv || !recv_scale)))) return MEP_ERR_NULLPTR;
+    if (T < 0 || K < 1 || K > MEP_MAX_K || H < 1 || rows < 0 || n_experts < 1 || T * K >= ((int64_t)1 << 31))
+        return MEP_ERR_SHAPE;
+    if (T == 0) return MEP_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int grid = token_grid(T, 8);
+    const int64_t H8 = H / 8;
+    const bool vec = H % 8 == 0 && aligned(x, 16) && aligned(recv, 8) && aligned(smooth, 16);
+    const int64_t per_thread = mep::ceil_div(H8, 256);
+    if (vec && per_thread <= 4) {
+        mep::k_dispatch_int8_smooth<4><<<grid, 256, 0, s>>>((const uint4 *)x, ids, pos, T, K, H8, (const float4 *)smooth,
+                                                           n_experts, rows, (uint2 *)recv, recv_scale);
+    } else if (vec && per_thread <= 8) {
+        mep::k_dispatch_int8_smooth<8><<<grid, 256, 0, s>>>((const uint4 *)x, ids, pos, T, K, H8, (const float4 *)smooth,
+                                                           n_experts, rows, (uint2 *)recv, recv_scale);
+    } else {
+        mep::k_dispatch_int8_smooth_scalar<<<grid, 256, 0, s>>>(x, ids, pos, T, K, H, smooth, n_experts, rows, recv,
+                                                               recv_scale);
+    }
+    return launched();
+}
+
 mep_status_t mep_selftest_bounded_wait(int32_t max_polls, int32_t *timed_out, mep_stream_t stream)
 {
     if (!timed_out) return MEP_ERR_NULLPTR;

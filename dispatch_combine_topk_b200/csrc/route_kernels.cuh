@@ -847,6 +847,143 @@ k_combine_add_rmsnorm_scalar(const uint16_t *__restrict__ y, const int32_t *__re
     }
 }
 
+// ------------------------------------------ smooth-quantised int8 dispatch (f1)
+
+// Block-wide max of one non-negative float per thread (every thread gets it); red holds
+// 33 floats of shared memory. Ends with a barrier.
+__device__ __forceinline__ float block_max(float v, float *red)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int d = 16; d > 0; d >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, d));
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        float t = lane < nw ? red[lane] : 0.0f;
+        for (int d = 16; d > 0; d >>= 1) t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, d));
+        if (lane == 0) red[32] = t;
+    }
+    __syncthreads();
+    return red[32];
+}
+
+// One CTA per token; the token's row (up to kChunks 8-column chunks per thread) stays in
+// registers. For every kept slot: xs = fl(x * smooth[e]) with e the slot's expert, amax
+// over the row (block reduction), scale = amax / 127, codes round_half_even(xs / scale)
+// clamped to [-127, 127], stored 8 bytes per chunk with the slot's scale.
+template <int kChunks>
+__global__ void __launch_bounds__(256)
+k_dispatch_int8_smooth(const uint4 *__restrict__ x, const int32_t *__restrict__ ids, const int32_t *__restrict__ pos,
+                       int64_t T, int K, int64_t H8, const float4 *__restrict__ smooth, int32_t n_experts,
+                       int64_t rows, uint2 *__restrict__ recv, float *__restrict__ recv_scale)
+{
+    __shared__ int32_t sp[kMaxK];
+    __shared__ int32_t se[kMaxK];
+    __shared__ float red[33];
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        load_token_rows(pos, t, K, rows, sp);
+        if (threadIdx.x < K) {
+            int32_t e = ids[t * K + threadIdx.x];
+            if (e < 0 || e >= n_experts) {
+                flag_error(0x1);
+                e = -1;
+            }
+            se[threadIdx.x] = e;
+        }
+        float xr[kChunks][8];
+#pragma unroll
+        for (int i = 0; i < kChunks; i++) {
+            const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
+            if (c < H8) {
+                const uint4 v = x[t * H8 + c];
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    xr[i][2 * j] = bf16lo(w[j]);
+                    xr[i][2 * j + 1] = bf16hi(w[j]);
+                }
+            }
+        }
+        __syncthreads();
+        for (int k = 0; k < K; k++) {
+            const int32_t p = sp[k], e = se[k];
+            if (p < 0 || e < 0) continue;                 // uniform over the block
+            const float4 *srow = smooth + (int64_t)e * H8 * 2;
+            float xs[kChunks][8];
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < kChunks; i++) {
+                const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
+                if (c < H8) {
+                    const float4 s0 = srow[2 * c], s1 = srow[2 * c + 1];
+                    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        xs[i][j] = __fmul_rn(xr[i][j], sv[j]);
+                        amax = fmaxf(amax, fabsf(xs[i][j]));
+                    }
+                }
+            }
+            amax = block_max(amax, red);
+            const float scale = __fdiv_rn(amax, 127.0f);
+            if (threadIdx.x == 0) recv_scale[p] = scale;
+#pragma unroll
+            for (int i = 0; i < kChunks; i++) {
+                const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
+                if (c < H8) {
+                    uint2 q;
+                    q.x = q8x4(xs[i][0], xs[i][1], xs[i][2], xs[i][3], scale);
+                    q.y = q8x4(xs[i][4], xs[i][5], xs[i][6], xs[i][7], scale);
+                    recv[(int64_t)p * H8 + c] = q;
+                }
+            }
+            __syncthreads();                               // red is reused by the next slot
+        }
+    }
+}
+
+// Element version for any H and alignment: two passes per slot over x and the scales.
+__global__ void __launch_bounds__(256)
+k_dispatch_int8_smooth_scalar(const uint16_t *__restrict__ x, const int32_t *__restrict__ ids,
+                              const int32_t *__restrict__ pos, int64_t T, int K, int64_t H,
+                              const float *__restrict__ smooth, int32_t n_experts, int64_t rows,
+                              int8_t *__restrict__ recv, float *__restrict__ recv_scale)
+{
+    __shared__ int32_t sp[kMaxK];
+    __shared__ int32_t se[kMaxK];
+    __shared__ float red[33];
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        load_token_rows(pos, t, K, rows, sp);
+        if (threadIdx.x < K) {
+            int32_t e = ids[t * K + threadIdx.x];
+            if (e < 0 || e >= n_experts) {
+                flag_error(0x1);
+                e = -1;
+            }
+            se[threadIdx.x] = e;
+        }
+        __syncthreads();
+        for (int k = 0; k < K; k++) {
+            const int32_t p = sp[k], e = se[k];
+            if (p < 0 || e < 0) continue;
+            float amax = 0.0f;
+            for (int64_t h = threadIdx.x; h < H; h += blockDim.x)
+                amax = fmaxf(amax, fabsf(__fmul_rn(bf16lo(x[t * H + h]), smooth[(int64_t)e * H + h])));
+            amax = block_max(amax, red);
+            const float scale = __fdiv_rn(amax, 127.0f);
+            if (threadIdx.x == 0) recv_scale[p] = scale;
+            for (int64_t h = threadIdx.x; h < H; h += blockDim.x) {
+                int r = 0;
+                if (scale != 0.0f) {
+                    const float v = __fmul_rn(bf16lo(x[t * H + h]), smooth[(int64_t)e * H + h]);
+                    r = max(-127, min(127, __float2int_rn(__fdiv_rn(v, scale))));
+                }
+                recv[(int64_t)p * H + h] = (int8_t)r;
+            }
+            __syncthreads();
+        }
+    }
+}
+
 // ----------------------------------- replica weight prefetch and grad reduce (f2, f3)
 
 // One thread per rank: walk its replicas in order; a replica of an expert homed on

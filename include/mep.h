@@ -187,6 +187,27 @@ mep_status_t mep_combine_int8(const int8_t *yq, const float *y_scale, int64_t ro
                               const int32_t *pos, const float *gates, int64_t T, int32_t K,
                               int64_t H, uint16_t *out, mep_stream_t stream);
 
+/*
+ * f1 — int8 dispatch with per-expert smoothing scales (the optional scales of shape
+ * (moeExpertNum, H), fp32, that aclnnMoeDistributeDispatch takes when quantMode > 0:
+ * gitcode ops-transformer aclnnMoeUpdateExpert doc, 调用示例; hiascend
+ * aclnnMoeDistributeDispatchSetup doc, scalesOptional). For every kept slot n of token
+ * g with expert e = ids[n] (the expert id the smoothing row belongs to):
+ *   xs_h  = fl(float(x[g, h]) * smooth[e, h]),   amax = max_h |xs_h|,
+ *   scale = amax / 127,   q_h = clamp(round_half_even(xs_h / scale), -127, 127)
+ *   (q = 0 when amax == 0);   recv[pos[n], :] = q,   recv_scale[pos[n]] = scale.
+ * Unlike mep_dispatch with quant 1, codes and scale are per slot (the smoothing depends
+ * on the expert). x bf16 [T, H]; ids int32 [T*K]; pos int32 [T*K]; smooth fp32
+ * [n_experts, H]; recv int8 [rows, H]; recv_scale fp32 [rows].
+ * Errors: NULL pointer; T < 0, K outside [1, MEP_MAX_K], H < 1, rows < 0, n_experts < 1
+ * (MEP_ERR_SHAPE). An id outside [0, n_experts) skips the slot and sets
+ * MEP_DERR_KEY_RANGE; a pos outside [-1, rows) as mep_dispatch.
+ */
+mep_status_t mep_dispatch_int8_smooth(const uint16_t *x, const int32_t *ids, const int32_t *pos,
+                                      int64_t T, int32_t K, int64_t H, const float *smooth,
+                                      int32_t n_experts, int8_t *recv, float *recv_scale,
+                                      int64_t rows, mep_stream_t stream);
+
 /* Largest hidden size of mep_combine_add_rmsnorm (one fp32 row in shared memory). */
 #define MEP_RMSNORM_MAX_H 49152
 
