@@ -19,9 +19,11 @@
  *    stream) and never synchronise the host, so a chain plan -> dispatch -> combine
  *    needs no host round trip (MoonEP's static shapes remove per-layer host syncs:
  *    twodots.gr article on MoonEP, static-shapes paragraph). Only mep_get_error
- *    synchronises. mep_plan, mep_update_expert, mep_dispatch, mep_dequantize and
- *    mep_combine can be captured into a CUDA graph and replayed on new inputs, once each
- *    has been called eagerly on the device (the first call sets kernel attributes).
+ *    synchronises. mep_histogram, mep_plan, mep_update_expert, mep_dispatch,
+ *    mep_dispatch_int8_smooth, mep_dequantize, mep_combine, mep_combine_int8,
+ *    mep_combine_add_rmsnorm, mep_prefetch_plan, mep_prefetch_weights and mep_grad_reduce
+ *    can be captured into a CUDA graph and replayed on new inputs, once each has been
+ *    called eagerly on the device (the first call sets kernel attributes).
  *  - A call first checks its arguments on the host and returns a status without
  *    launching anything when one is wrong: MEP_ERR_NULLPTR / MEP_ERR_DTYPE /
  *    MEP_ERR_SHAPE / MEP_ERR_VALUE mirror the aclnn codes 161001 (null tensor),

@@ -90,3 +90,76 @@ def test_graph_replay_matches_eager(name, S):
                                b.view(torch.int16) if b.dtype == torch.bfloat16 else b)
     del g
     assert mep.mep_get_error() == 0
+
+
+def test_graph_replay_of_the_other_calls():
+    """Histogram, int8 combine, the fused RMSNorm epilogue, the smooth-quantised
+    dispatch, the prefetch plan and copy, and the gradient reduce, captured once and
+    replayed on new inputs, equal eager calls."""
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w = synth.scaled(synth.get("r8"), S=128)
+    B, D = w.E // w.R, 4096
+    ids0, gates0, x0 = _inputs(w, 5)
+    ids_d = torch.from_numpy(ids0).to(dev).view(-1)
+    g_d = torch.from_numpy(gates0).to(dev).view(-1)
+    x_d = x0.to(dev)
+    smooth = torch.rand((w.E, w.H), device=dev) + 0.5
+    res = torch.randn((w.T, w.H), device=dev).to(torch.bfloat16)
+    gam = torch.ones(w.H, device=dev).to(torch.bfloat16)
+    hist = torch.empty(w.E, dtype=torch.int32, device=dev)
+    pb = mep.PlanBuffers.allocate(w.R, w.E, w.S, w.K, dev)
+    q = torch.empty((w.N, w.H), dtype=torch.int8, device=dev)
+    sc = torch.empty(w.N, dtype=torch.float32, device=dev)
+    recv = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
+    o1 = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
+    xo, yo = torch.empty_like(o1), torch.empty_like(o1)
+    rstd = torch.empty(w.T, dtype=torch.float32, device=dev)
+    se = torch.empty((w.R, B), dtype=torch.int32, device=dev)
+    rw = torch.empty((w.R, w.E), dtype=torch.int32, device=dev)
+    w_home = torch.randn((w.E, D), device=dev).to(torch.bfloat16)
+    w_slots = torch.zeros((w.R * B, D), dtype=torch.bfloat16, device=dev)
+    gh0 = torch.randn((w.E, D), device=dev)
+    gs0 = torch.randn((w.R * B, D), device=dev)
+    gh, gs = gh0.clone(), gs0.clone()
+
+    def step(s):
+        mep.mep_histogram(ids_d, w.E, hist, stream=s)
+        mep.mep_plan(ids_d, w.R, w.E, w.S, w.K, pb, stream=s)
+        mep.mep_dispatch_int8_smooth(x_d, ids_d, pb.pos, w.K, smooth, q, sc, stream=s)
+        mep.mep_combine_int8(q, sc, pb.pos, g_d, w.K, o1, stream=s)
+        mep.mep_dispatch(x_d, pb.pos, w.K, recv, stream=s)
+        mep.mep_combine_add_rmsnorm(recv, pb.pos, g_d, w.K, res, gam, 1e-6, xo, yo, rstd, stream=s)
+        mep.mep_prefetch_plan(pb, w.R, w.E, B, se, rw, stream=s)
+        mep.mep_prefetch_weights(w_home, se, w.R, B, w_slots, stream=s)
+        mep.mep_grad_reduce(gh, gs, se, w.R, B, stream=s)
+
+    outs = [hist, pb.pos, q, sc, o1, xo, yo, rstd, se, rw, w_slots, gh, gs]
+    s = torch.cuda.Stream(dev)
+    with torch.cuda.stream(s):
+        step(s)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step(s)
+    for seed in (6, 7):
+        ids, gates, x = _inputs(w, seed)
+        ids_d.copy_(torch.from_numpy(ids).view(-1))
+        g_d.copy_(torch.from_numpy(gates).view(-1))
+        x_d.copy_(x)
+        gh.copy_(gh0)
+        gs.copy_(gs0)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        got = [t.clone() for t in outs]
+        gh.copy_(gh0)
+        gs.copy_(gs0)
+        with torch.cuda.stream(s):
+            step(s)
+        s.synchronize()
+        for a, b in zip(got, outs):
+            assert torch.equal(a.view(torch.int16) if a.dtype == torch.bfloat16 else a,
+                               b.view(torch.int16) if b.dtype == torch.bfloat16 else b)
+    del g
+    assert mep.mep_get_error() == 0
