@@ -9,6 +9,8 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <mutex>
+
 #include "mep.h"
 #include "common.cuh"
 #include "plan_kernels.cuh"
@@ -22,19 +24,15 @@ constexpr int kMaxDevices = 64;
 // Shared memory the staged int8 dispatch may use per CTA.
 constexpr int kBulkSmemMax = 200 * 1024;
 int g_sm_count[kMaxDevices];
-bool g_attrs_set[kMaxDevices];
+std::once_flag g_device_once[kMaxDevices];
 
-// SM count of the current device (cached), and one-time kernel attributes.
-int sm_count()
+// One-time set-up of a device: its SM count and the kernels' shared-memory limits.
+void device_setup(int dev)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-    if (g_sm_count[dev] == 0) {
-        int n = 0;
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        g_sm_count[dev] = n > 0 ? n : 148;
-    }
-    if (!g_attrs_set[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_sm_count[dev] = n > 0 ? n : 148;
+    {
         const int big = 200 * 1024;
         cudaFuncSetAttribute(mep::k_rank, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
         cudaFuncSetAttribute(mep::k_tile_count, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
@@ -49,8 +47,16 @@ int sm_count()
         cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
         cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
         cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_scalar, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
-        g_attrs_set[dev] = true;
     }
+}
+
+// SM count of the current device; the first call on a device runs its set-up (once,
+// also when several host threads call at the same time).
+int sm_count()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    std::call_once(g_device_once[dev], device_setup, dev);
     return g_sm_count[dev];
 }
 

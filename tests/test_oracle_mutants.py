@@ -59,7 +59,7 @@ MUTANTS = [
      "float r = nearbyintf(v);", "float r = roundf(v);",
      ["test_oracle_numerics.test_quant_half_even_golden"]),
     ("quantisation scale over 128",
-     "float scale = amax / 127.0f;", "float scale = amax / 128.0f;",
+     "float scale = amax / 127.0f;\n    *scale_out = scale;", "float scale = amax / 128.0f;\n    *scale_out = scale;",
      ["test_oracle_numerics.test_quant_half_even_golden", "test_oracle_numerics.test_quant_properties"]),
     ("bf16 conversion truncates",
      "u = u + 0x7fffu + keep_lsb;", "u = u;",
