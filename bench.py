@@ -412,6 +412,18 @@ class Route:
         return {"plan": plan, "dispatch": disp, "combine": comb}
 
 
+def maxvio(rt):
+    """maxvio = max load / mean load - 1: over ranks before the plan (experts on their
+    home ranks) and after it (the rows each rank receives), and over experts."""
+    w, st = rt.w, rt.pb.stats_dict()
+    mean_rank = w.S * w.K
+    n_keys = rt.pb.hist.numel()
+    out = {"rank_before": st["max_load"] / mean_rank - 1.0,
+           "rank_after": st["max_chunk"] / mean_rank - 1.0,
+           "expert": st["max_hist"] / (st["n_kept"] / n_keys) - 1.0 if st["n_kept"] else None}
+    return out
+
+
 def weight_side(mep, rt, args, dev, stream):
     """The replica weight prefetch and the replica gradient reduce of the step's plan,
     with B = E/R slots per rank (MoonEP's training setting) and experts of H x ffn_dim.
@@ -664,6 +676,7 @@ def run_gpu(args, w):
             "gpu_launches": launches,
             "clocks": clk.summary(),
             "plan_stats": rt.pb.stats_dict(),
+            "maxvio": maxvio(rt),
             "replica_weights": weights,
         }
         print(json.dumps(line), flush=True)

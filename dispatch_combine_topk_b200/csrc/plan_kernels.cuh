@@ -20,8 +20,11 @@
 
 namespace mep {
 
+#ifndef MEP_PLAN_WARP_ROUNDS
+#define MEP_PLAN_WARP_ROUNDS 8                   // 32-slot rounds per warp in a tile
+#endif
 constexpr int kPlanWarps = 8;                    // warps per tile CTA
-constexpr int kPlanTile = kPlanWarps * 32 * 8;   // 2048 slots per tile, 256 per warp
+constexpr int kPlanTile = kPlanWarps * 32 * MEP_PLAN_WARP_ROUNDS;   // 2048 slots by default
 
 // Key of slot n: the id, or -1 when the slot is dropped or its id is out of range.
 __device__ __forceinline__ int32_t slot_key(const int32_t *ids, const uint8_t *keep, int64_t n,
