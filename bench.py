@@ -73,14 +73,26 @@ def kernel_source_hash(name: str) -> str:
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch, from the ncu captures
 # summarised in profiles/, scaled to the full workload by the rows routed (a capture on
-# S=1024 of the r8 workload routes a quarter of its rows).
+# a quarter or a sixteenth of the tokens per rank routes that share of the rows).
 TRAFFIC = {
     ("k_dispatch_warp", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 998.09e6, "src": "0a17c397b27cf663",
-        "note": "profiles/k_dispatch_warp_r8_s1024.md: 998.1 MB at S=1024, x4"},
+        "bytes": 4 * 998.24e6, "src": "09eb46386adf6b89",
+        "note": "profiles/traffic_dominant_kernels.md: 998.2 MB at S=1024, x4"},
     ("k_combine_v8", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 1009.43e6, "src": "a9d5f41e42e115fa",
-        "note": "profiles/k_combine_v8_r8_s1024.md: 1009.4 MB at S=1024, x4"},
+        "bytes": 4 * 1005.02e6, "src": "a9b213675638d967",
+        "note": "profiles/traffic_dominant_kernels.md: 1005.0 MB at S=1024, x4"},
+    ("k_dispatch_int8_staged", "int8_r32_e256_s8192_k8_h7168"): {
+        "bytes": 16 * 1115.87e6, "src": "cdff245baaa9e16b",
+        "note": "profiles/traffic_dominant_kernels.md: 1115.9 MB at S=512, x16"},
+    ("k_combine_int8_v16", "int8_r32_e256_s8192_k8_h7168"): {
+        "bytes": 16 * 1117.06e6, "src": "bcf572dd17035aa7",
+        "note": "profiles/traffic_dominant_kernels.md: 1117.1 MB at S=512, x16"},
+    ("k_dispatch_warp", "skew_r64_e512_s2048_k8_h4096"): {
+        "bytes": 4 * 2357.43e6, "src": "09eb46386adf6b89",
+        "note": "profiles/traffic_dominant_kernels.md: 2357.4 MB at S=512, x4"},
+    ("k_combine_v8", "skew_r64_e512_s2048_k8_h4096"): {
+        "bytes": 4 * 2364.92e6, "src": "a9b213675638d967",
+        "note": "profiles/traffic_dominant_kernels.md: 2364.9 MB at S=512, x4"},
 }
 
 
