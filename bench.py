@@ -496,7 +496,7 @@ def run_gpu(args, w):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     pg = None
-    if world > 1:
+    if world > 1 or ("MASTER_ADDR" in os.environ and "RANK" in os.environ):   # under torchrun
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -554,7 +554,9 @@ def run_gpu(args, w):
     graph_ms = None
     if args.graph:
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
+        # thread-local capture: other threads (NCCL's watchdog, the clock sampler) may
+        # make CUDA calls while this thread captures
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
             rt.step(stream)
         with torch.cuda.stream(stream):
             for _ in range(3):
