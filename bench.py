@@ -50,24 +50,47 @@ def load_peaks():
 CSRC = os.path.join(ROOT, "dispatch_combine_topk_b200", "csrc")
 
 
+def _device_functions():
+    """name -> source text of every function defined in the library's CUDA headers."""
+    import re
+
+    funcs = {}
+    for fn in ("common.cuh", "tma.cuh", "plan_kernels.cuh", "route_kernels.cuh"):
+        src = open(os.path.join(CSRC, fn)).read()
+        for m in re.finditer(r"\n(?:template <[^>]*>\n)?(?:__global__|__device__|__host__ __device__)\b", src):
+            brace = src.find("{", m.end())
+            end = src.find("\n}\n", brace)
+            if brace < 0 or end < 0:
+                continue
+            header = re.sub(r"__launch_bounds__\s*\([^)]*\)", "", src[m.end():brace])
+            name = re.search(r"(\w+)\s*\(", header)
+            if name:
+                funcs.setdefault(name.group(1), src[m.start():end + 3])
+    return funcs
+
+
 def kernel_source_hash(name: str) -> str:
-    """sha256 of a kernel's own source text (from its declaration to its closing brace)
-    plus the shared helpers, so that a captured traffic figure is only reported for the
-    kernel it was measured on."""
+    """sha256 of a kernel's source text and of every library function it calls (found
+    by name, transitively), so that a captured traffic figure is only reported for the
+    code it was measured on."""
     import hashlib
     import re
 
-    h = hashlib.sha256()
-    for fn in ("route_kernels.cuh", "plan_kernels.cuh"):
-        src = open(os.path.join(CSRC, fn)).read()
-        m = re.search(r"\n(?:template <[^>]*>\n)?__global__[^\n]*\n?" + re.escape(name) + r"\(", src)
-        if m:
-            end = src.index("\n}\n", m.start())
-            h.update(src[m.start():end + 3].encode())
-            break
-    else:
+    funcs = _device_functions()
+    if name not in funcs:
         return ""
-    h.update(open(os.path.join(CSRC, "common.cuh")).read().encode())
+    seen, todo = set(), [name]
+    while todo:
+        f = todo.pop()
+        if f in seen:
+            continue
+        seen.add(f)
+        for ident in set(re.findall(r"\b(\w+)\s*[<(]", funcs[f])):
+            if ident in funcs and ident not in seen:
+                todo.append(ident)
+    h = hashlib.sha256()
+    for f in sorted(seen):
+        h.update(funcs[f].encode())
     return h.hexdigest()[:16]
 
 
@@ -76,23 +99,23 @@ def kernel_source_hash(name: str) -> str:
 # a quarter or a sixteenth of the tokens per rank routes that share of the rows).
 TRAFFIC = {
     ("k_dispatch_warp", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 998.24e6, "src": "09eb46386adf6b89",
-        "note": "profiles/traffic_dominant_kernels.md: 998.2 MB at S=1024, x4"},
+        "bytes": 4 * 998.05e6, "src": "17b1506c97a87d55",
+        "note": "profiles/traffic_dominant_kernels.md: 998.05 MB at S=1024, x4"},
     ("k_combine_v8", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 1005.02e6, "src": "a9b213675638d967",
-        "note": "profiles/traffic_dominant_kernels.md: 1005.0 MB at S=1024, x4"},
+        "bytes": 4 * 1005.70e6, "src": "b8d0144407f8df74",
+        "note": "profiles/traffic_dominant_kernels.md: 1005.70 MB at S=1024, x4"},
     ("k_dispatch_int8_staged", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1115.87e6, "src": "cdff245baaa9e16b",
-        "note": "profiles/traffic_dominant_kernels.md: 1115.9 MB at S=512, x16"},
+        "bytes": 16 * 1115.86e6, "src": "cf5ee39cf4a3516f",
+        "note": "profiles/traffic_dominant_kernels.md: 1115.86 MB at S=512, x16"},
     ("k_combine_int8_v16", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1117.06e6, "src": "bcf572dd17035aa7",
-        "note": "profiles/traffic_dominant_kernels.md: 1117.1 MB at S=512, x16"},
+        "bytes": 16 * 1116.82e6, "src": "567d09ad603be0a8",
+        "note": "profiles/traffic_dominant_kernels.md: 1116.82 MB at S=512, x16"},
     ("k_dispatch_warp", "skew_r64_e512_s2048_k8_h4096"): {
-        "bytes": 4 * 2357.43e6, "src": "09eb46386adf6b89",
-        "note": "profiles/traffic_dominant_kernels.md: 2357.4 MB at S=512, x4"},
+        "bytes": 4 * 2357.84e6, "src": "17b1506c97a87d55",
+        "note": "profiles/traffic_dominant_kernels.md: 2357.84 MB at S=512, x4"},
     ("k_combine_v8", "skew_r64_e512_s2048_k8_h4096"): {
-        "bytes": 4 * 2364.92e6, "src": "a9b213675638d967",
-        "note": "profiles/traffic_dominant_kernels.md: 2364.9 MB at S=512, x4"},
+        "bytes": 4 * 2364.80e6, "src": "b8d0144407f8df74",
+        "note": "profiles/traffic_dominant_kernels.md: 2364.80 MB at S=512, x4"},
 }
 
 

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "mep.h"   // the MEP_DERR_* bits the kernels set
+
 namespace mep {
 
 // Sticky per-device word of data errors (MEP_DERR_* bits), read by mep_get_error.

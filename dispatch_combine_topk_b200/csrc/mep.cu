@@ -240,7 +240,7 @@ mep_status_t mep_dispatch(const uint16_t *x, const int32_t *pos, int64_t T, int3
             mep::k_dispatch_warp<<<(int)(ctas < cap ? ctas : cap), 256, 0, s>>>((const uint4 *)x, pos, T, K, H / 8,
                                                                               rows, (uint4 *)recv);
         } else {
-            mep::k_dispatch_copy<uint16_t><<<grid, 256, 0, s>>>(x, pos, T, K, H, rows, (uint16_t *)recv);
+            mep::k_dispatch_elem<<<grid, 256, 0, s>>>(x, pos, T, K, H, rows, (uint16_t *)recv);
         }
     } else {
         const size_t staged_smem = (size_t)mep::kDispatchSmemHead + 4 * (size_t)H * 2 + 2 * (size_t)H;

@@ -34,7 +34,7 @@ __device__ __forceinline__ int32_t slot_key(const int32_t *ids, const uint8_t *k
     if (keep && !keep[n]) return -1;
     int32_t e = ids[n];
     if (e < 0 || e >= n_keys) {
-        flag_error(0x1);
+        flag_error(MEP_DERR_KEY_RANGE);
         return -1;
     }
     return e;

@@ -32,25 +32,25 @@ __global__ void k_update_expert(const int32_t *__restrict__ ids, const int32_t *
         uint8_t act = 1;
         if (active) {
             act = active[i] ? 1 : 0;
-            if (i > 0 && act && !active[i - 1]) flag_error(0x8);
+            if (i > 0 && act && !active[i - 1]) flag_error(MEP_DERR_MASK);
         }
         for (int32_t k = 0; k < K; k++) {
             const int32_t e = ids[i * K + k];
             int32_t inst = -1;
             if (e < 0 || e >= E) {
-                flag_error(0x1);
+                flag_error(MEP_DERR_KEY_RANGE);
             } else {
                 const int32_t *row = table + (int64_t)e * F;
                 const int32_t c = row[0];
                 if (c < 1 || c > F - 1) {
-                    flag_error(0x4);
+                    flag_error(MEP_DERR_TABLE);
                 } else {
                     int64_t col;
                     if (c == 1) col = 1;
                     else if (mode == 0) col = local_rank / ((world_size + c - 1) / c) + 1;
                     else col = (i % c) + 1;
                     const int32_t v = row[col];   // col <= c <= F-1: inside the row
-                    if (v < 0 || v >= 1024) flag_error(0x4);
+                    if (v < 0 || v >= 1024) flag_error(MEP_DERR_TABLE);
                     else inst = v;
                 }
             }
@@ -76,7 +76,7 @@ __device__ __forceinline__ void load_token_rows(const int32_t *__restrict__ pos,
     if (threadIdx.x < K) {
         int32_t p = pos[t * K + threadIdx.x];
         if (p < -1 || (int64_t)p >= rows) {
-            flag_error(0x2);
+            flag_error(MEP_DERR_ROW_RANGE);
             p = -1;
         }
         sp[threadIdx.x] = p;
@@ -87,26 +87,20 @@ __device__ __forceinline__ void load_token_rows(const int32_t *__restrict__ pos,
 
 // bf16 copy for unaligned buffers or H % 8 != 0: recv[pos[t*K+k], :] = x[t, :], one CTA
 // per token, one element per access.
-template <typename V>
 __global__ void __launch_bounds__(256)
-k_dispatch_copy(const V *__restrict__ x, const int32_t *__restrict__ pos, int64_t T, int K,
-                int64_t HV, int64_t rows, V *__restrict__ recv)
+k_dispatch_elem(const uint16_t *__restrict__ x, const int32_t *__restrict__ pos, int64_t T, int K, int64_t H,
+                int64_t rows, uint16_t *__restrict__ recv)
 {
     __shared__ int32_t sp[kMaxK];
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         load_token_rows(pos, t, K, rows, sp);
         __syncthreads();
-        const V *src = x + t * HV;
-        for (int64_t c = threadIdx.x; c < HV; c += blockDim.x) {
-            V v;
-            if constexpr (sizeof(V) == 16) v = ld_stream(reinterpret_cast<const uint4 *>(src + c));
-            else v = src[c];
+        const uint16_t *src = x + t * H;
+        for (int64_t h = threadIdx.x; h < H; h += blockDim.x) {
+            const uint16_t v = src[h];
             for (int k = 0; k < K; k++) {
                 const int32_t p = sp[k];
-                if (p >= 0) {
-                    if constexpr (sizeof(V) == 16) st_v4(reinterpret_cast<uint4 *>(recv + (int64_t)p * HV + c), v);
-                    else recv[(int64_t)p * HV + c] = v;
-                }
+                if (p >= 0) recv[(int64_t)p * H + h] = v;
             }
         }
         __syncthreads();
@@ -137,7 +131,7 @@ k_dispatch_warp(const uint4 *__restrict__ x, const int32_t *__restrict__ pos, in
         if (lane < K) {
             mine = pos[t * K + lane];
             if (mine < -1 || (int64_t)mine >= rows) {
-                flag_error(0x2);
+                flag_error(MEP_DERR_ROW_RANGE);
                 mine = -1;
             }
         }
@@ -268,7 +262,7 @@ k_dispatch_int8_staged(const uint16_t *__restrict__ x, const int32_t *__restrict
         if (lane < K) {
             int32_t p = pos[t * K + lane];
             if (p < -1 || (int64_t)p >= rows) {
-                flag_error(0x2);
+                flag_error(MEP_DERR_ROW_RANGE);
                 p = -1;
             }
             srow[s * 32 + lane] = p;
@@ -283,7 +277,7 @@ k_dispatch_int8_staged(const uint16_t *__restrict__ x, const int32_t *__restrict
         const bool ok = mbar_wait_bounded(&bar[s], (uint32_t)((i / kStages) & 1));
         if (!__syncthreads_and(ok)) {
             if (tid == 0) {
-                flag_error(0x10);
+                flag_error(MEP_DERR_TIMEOUT);
                 for (int64_t j = i + 1; j < n && j < i + kStages; j++)
                     mbar_wait_bounded(&bar[j % kStages], (uint32_t)((j / kStages) & 1));
             }
@@ -408,6 +402,49 @@ k_dequant_scalar(const int8_t *__restrict__ q, const float *__restrict__ scale, 
 
 // ------------------------------------------------------------------- combine (a5)
 
+// acc[0..8) = sum over kept slots k (ascending) of fl(sg[k] * y[sp[k], chunk c]) in fp32,
+// each product and sum rounded on its own. All K 16-byte loads of the chunk are issued
+// before the first add (compile-time K); with KC = 0 the runtime K loop is used.
+template <int KC>
+__device__ __forceinline__ void combine_chunk8(const uint4 *__restrict__ y, const int32_t *sp, const float *sg,
+                                               int K, int64_t H8, int64_t c, float acc[8])
+{
+#pragma unroll
+    for (int j = 0; j < 8; j++) acc[j] = 0.0f;
+    if constexpr (KC > 0) {
+        uint4 v[KC];
+#pragma unroll
+        for (int k = 0; k < KC; k++) {
+            const int32_t p = sp[k];
+            v[k] = p >= 0 ? ld_stream(y + (int64_t)p * H8 + c) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < KC; k++) {
+            if (sp[k] < 0) continue;
+            const float g = sg[k];
+            const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                acc[2 * j] = __fadd_rn(acc[2 * j], __fmul_rn(g, bf16lo(w[j])));
+                acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], __fmul_rn(g, bf16hi(w[j])));
+            }
+        }
+    } else {
+        for (int k = 0; k < K; k++) {
+            const int32_t p = sp[k];
+            if (p < 0) continue;
+            const uint4 vv = ld_stream(y + (int64_t)p * H8 + c);
+            const float g = sg[k];
+            const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                acc[2 * j] = __fadd_rn(acc[2 * j], __fmul_rn(g, bf16lo(w[j])));
+                acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], __fmul_rn(g, bf16hi(w[j])));
+            }
+        }
+    }
+}
+
 // out[t, :] = bf16( sum_k fl(gate[t,k] * y[pos[t,k], :]) ), fp32, ascending k, no FMA.
 // All K 16-byte loads of a chunk are issued before the first add.
 template <int KC>
@@ -426,40 +463,7 @@ k_combine_v8(const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
         __syncthreads();
         for (int64_t c = threadIdx.x; c < H8; c += blockDim.x) {
             float acc[8];
-#pragma unroll
-            for (int j = 0; j < 8; j++) acc[j] = 0.0f;
-            if constexpr (kFixed) {
-                uint4 v[KC];
-#pragma unroll
-                for (int k = 0; k < KC; k++) {
-                    const int32_t p = sp[k];
-                    v[k] = p >= 0 ? ld_stream(y + (int64_t)p * H8 + c) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int k = 0; k < KC; k++) {
-                    if (sp[k] < 0) continue;
-                    const float g = sg[k];
-                    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        acc[2 * j] = __fadd_rn(acc[2 * j], __fmul_rn(g, bf16lo(w[j])));
-                        acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], __fmul_rn(g, bf16hi(w[j])));
-                    }
-                }
-            } else {
-                for (int k = 0; k < K; k++) {
-                    const int32_t p = sp[k];
-                    if (p < 0) continue;
-                    const uint4 vv = ld_stream(y + (int64_t)p * H8 + c);
-                    const float g = sg[k];
-                    const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        acc[2 * j] = __fadd_rn(acc[2 * j], __fmul_rn(g, bf16lo(w[j])));
-                        acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], __fmul_rn(g, bf16hi(w[j])));
-                    }
-                }
-            }
+            combine_chunk8<KC>(y, sp, sg, K, H8, c, acc);
             uint4 o;
             o.x = pack_bf16x2(acc[0], acc[1]);
             o.y = pack_bf16x2(acc[2], acc[3]);
@@ -736,40 +740,7 @@ k_combine_add_rmsnorm_v8(const uint4 *__restrict__ y, const int32_t *__restrict_
         float ss = 0.0f;
         for (int64_t c = threadIdx.x; c < H8; c += blockDim.x) {
             float acc[8];
-#pragma unroll
-            for (int j = 0; j < 8; j++) acc[j] = 0.0f;
-            if constexpr (kFixed) {
-                uint4 v[KC];
-#pragma unroll
-                for (int k = 0; k < KC; k++) {
-                    const int32_t p = sp[k];
-                    v[k] = p >= 0 ? ld_stream(y + (int64_t)p * H8 + c) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int k = 0; k < KC; k++) {
-                    if (sp[k] < 0) continue;
-                    const float g = sg[k];
-                    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        acc[2 * j] = __fadd_rn(acc[2 * j], __fmul_rn(g, bf16lo(w[j])));
-                        acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], __fmul_rn(g, bf16hi(w[j])));
-                    }
-                }
-            } else {
-                for (int k = 0; k < K; k++) {
-                    const int32_t p = sp[k];
-                    if (p < 0) continue;
-                    const uint4 vv = ld_stream(y + (int64_t)p * H8 + c);
-                    const float g = sg[k];
-                    const uint32_t w[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        acc[2 * j] = __fadd_rn(acc[2 * j], __fmul_rn(g, bf16lo(w[j])));
-                        acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], __fmul_rn(g, bf16hi(w[j])));
-                    }
-                }
-            }
+            combine_chunk8<KC>(y, sp, sg, K, H8, c, acc);
             const uint4 r = ld_stream(residual + t * H8 + c);
             const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
             uint32_t xo[4];
@@ -884,7 +855,7 @@ k_dispatch_int8_smooth(const uint4 *__restrict__ x, const int32_t *__restrict__ 
         if (threadIdx.x < K) {
             int32_t e = ids[t * K + threadIdx.x];
             if (e < 0 || e >= n_experts) {
-                flag_error(0x1);
+                flag_error(MEP_DERR_KEY_RANGE);
                 e = -1;
             }
             se[threadIdx.x] = e;
@@ -956,7 +927,7 @@ k_dispatch_int8_smooth_scalar(const uint16_t *__restrict__ x, const int32_t *__r
         if (threadIdx.x < K) {
             int32_t e = ids[t * K + threadIdx.x];
             if (e < 0 || e >= n_experts) {
-                flag_error(0x1);
+                flag_error(MEP_DERR_KEY_RANGE);
                 e = -1;
             }
             se[threadIdx.x] = e;
@@ -1000,14 +971,14 @@ __global__ void k_prefetch_plan(const int32_t *__restrict__ rep_count, const int
     for (int32_t j = 0; j < cap; j++) rep_weight[(int64_t)r * cap + j] = -1;
     int32_t n = rep_count[r];
     if (n < 0 || n > cap) {
-        flag_error(0x1);
+        flag_error(MEP_DERR_KEY_RANGE);
         n = n < 0 ? 0 : cap;
     }
     int32_t used = 0;
     for (int32_t j = 0; j < n; j++) {
         const int32_t e = rep_key[(int64_t)r * cap + j];
         if (e < 0 || e >= E) {
-            flag_error(0x1);
+            flag_error(MEP_DERR_KEY_RANGE);
             continue;
         }
         int32_t row = e;
@@ -1029,7 +1000,7 @@ k_prefetch_weights(const uint4 *__restrict__ w_home, const int32_t *__restrict__
     const int32_t e = slot_expert[blockIdx.y];
     if (e < 0) return;
     if (e >= E) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(0x1);
+        if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(MEP_DERR_KEY_RANGE);
         return;
     }
     const uint4 *src = w_home + (int64_t)e * D8;
@@ -1045,7 +1016,7 @@ k_prefetch_weights_scalar(const uint16_t *__restrict__ w_home, const int32_t *__
     const int32_t e = slot_expert[blockIdx.y];
     if (e < 0) return;
     if (e >= E) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(0x1);
+        if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(MEP_DERR_KEY_RANGE);
         return;
     }
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < D; i += (int64_t)gridDim.x * blockDim.x)
@@ -1095,7 +1066,7 @@ k_grad_reduce(float4 *__restrict__ grad_home, float4 *__restrict__ grad_slots, c
     const int32_t n = slots_of_expert(slot_expert, RB, e, list, kMaxSlotsPerExpert, warp_cnt);
     if (n == 0) return;
     const int32_t m = n < kMaxSlotsPerExpert ? n : kMaxSlotsPerExpert;
-    if (n > kMaxSlotsPerExpert && blockIdx.x == 0 && threadIdx.x == 0) flag_error(0x1);
+    if (n > kMaxSlotsPerExpert && blockIdx.x == 0 && threadIdx.x == 0) flag_error(MEP_DERR_KEY_RANGE);
     float4 *home = grad_home + (int64_t)e * D4;
     const int64_t step = (int64_t)gridDim.x * blockDim.x * kReduceUnroll;
     const float4 zero = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -1151,7 +1122,7 @@ k_grad_reduce_scalar(float *__restrict__ grad_home, float *__restrict__ grad_slo
     const int32_t n = slots_of_expert(slot_expert, RB, e, list, kMaxSlotsPerExpert, warp_cnt);
     if (n == 0) return;
     const int32_t m = n < kMaxSlotsPerExpert ? n : kMaxSlotsPerExpert;
-    if (n > kMaxSlotsPerExpert && blockIdx.x == 0 && threadIdx.x == 0) flag_error(0x1);
+    if (n > kMaxSlotsPerExpert && blockIdx.x == 0 && threadIdx.x == 0) flag_error(MEP_DERR_KEY_RANGE);
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < D; i += (int64_t)gridDim.x * blockDim.x) {
         float acc = grad_home[(int64_t)e * D + i];
         for (int32_t j = 0; j < m; j++) {
@@ -1178,7 +1149,7 @@ __global__ void k_selftest_wait(int max_polls, int32_t *timed_out)
     __syncthreads();
     const bool ok = mbar_wait_bounded(&bar, 0, max_polls);
     if (threadIdx.x == 0) {
-        if (!ok) flag_error(0x10);
+        if (!ok) flag_error(MEP_DERR_TIMEOUT);
         *timed_out = ok ? 0 : 1;
     }
 }
