@@ -107,9 +107,9 @@ TRAFFIC = {
     ("k_dispatch_int8_staged", "int8_r32_e256_s8192_k8_h7168"): {
         "bytes": 16 * 1115.86e6, "src": "cf5ee39cf4a3516f",
         "note": "profiles/traffic_dominant_kernels.md: 1115.86 MB at S=512, x16"},
-    ("k_combine_int8_v16", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1116.82e6, "src": "567d09ad603be0a8",
-        "note": "profiles/traffic_dominant_kernels.md: 1116.82 MB at S=512, x16"},
+    ("k_combine_int8_warp", "int8_r32_e256_s8192_k8_h7168"): {
+        "bytes": 16 * 1117.18e6, "src": "d852eb58236fe244",
+        "note": "profiles/traffic_dominant_kernels.md: 1117.18 MB at S=512, x16"},
     ("k_dispatch_warp", "skew_r64_e512_s2048_k8_h4096"): {
         "bytes": 4 * 2357.84e6, "src": "17b1506c97a87d55",
         "note": "profiles/traffic_dominant_kernels.md: 2357.84 MB at S=512, x4"},
@@ -301,7 +301,7 @@ class Route:
     workload) -> combine. The identity expert returns the dispatched rows; on the int8
     workload they stay int8 and the combine reads the codes and scales
     (mep_combine_int8, the same result as dequantising first).
-    Mapping workload: mep_update_expert for every rank -> grouped plan over the physical
+    Mapping workload: mep_update_expert_ranks (every rank, one launch) -> grouped plan over the physical
     instances -> dispatch -> combine.
     """
 
@@ -346,16 +346,12 @@ class Route:
     def plan(self, s):
         w, mep = self.w, self.mep
         if w.mapping:
-            g2 = self.gates.view(w.T, w.K)
-            ids2 = self.ids.view(w.T, w.K)
-            for r in range(w.R):
-                sl = slice(r * w.S, (r + 1) * w.S)
-                mep.mep_update_expert(ids2[sl], self.table, g2[sl], self.thr, self.active[sl], r, w.R,
-                                      0, self.bids[sl], self.bmask[sl], stream=s)
+            mep.mep_update_expert_ranks(self.ids.view(w.T, w.K), self.table, self.gates.view(w.T, w.K),
+                                        self.thr, self.active, w.R, 0, self.bids, self.bmask, stream=s)
             mep.mep_plan(self.bids.view(-1), w.R, self.n_keys, w.S, w.K, self.pb,
                          mode=mep.MEP_PLAN_GROUPED, keys_per_rank=w.place_per_rank,
                          keep=self.bmask.view(-1), stream=s)
-            return w.R + 4
+            return 1 + 4
         mep.mep_plan(self.ids, w.R, w.E, w.S, w.K, self.pb, stream=s)
         return 4
 
@@ -419,12 +415,12 @@ class Route:
                 return "k_combine_add_rmsnorm_v8" if w.H % 8 == 0 else "k_combine_add_rmsnorm_scalar"
             if w.quant:
                 if w.H % 16 == 0:
-                    return "k_combine_int8_v16"
+                    return "k_combine_int8_warp"
                 return "k_combine_int8_v8" if w.H % 8 == 0 else "k_combine_int8_scalar"
             return "k_combine_v8" if w.H % 8 == 0 else "k_combine_scalar"
         if w.quant:
             return "k_dispatch_int8_staged" if w.H % 16 == 0 else "k_dispatch_int8"
-        return "k_dispatch_warp" if w.H % 8 == 0 else "k_dispatch_copy"
+        return "k_dispatch_warp" if w.H % 8 == 0 else "k_dispatch_elem"
 
     def working_set_bytes(self) -> int:
         return (self.x.numel() * 2 + self.recv.numel() * self.recv.element_size() +

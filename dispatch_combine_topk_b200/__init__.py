@@ -76,10 +76,11 @@ def lib() -> ctypes.CDLL:
         L.mep_prefetch_weights.argtypes = [P, P, i32, i32, i32, i64, P, P]
         L.mep_grad_reduce.argtypes = [P, P, P, i32, i32, i32, i64, P]
         L.mep_dispatch_int8_smooth.argtypes = [P, P, P, i64, i32, i64, P, i32, P, P, i64, P]
+        L.mep_update_expert_ranks.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i64, P, P, P]
         for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
                   "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8",
                   "mep_combine_add_rmsnorm", "mep_prefetch_plan", "mep_prefetch_weights",
-                  "mep_grad_reduce", "mep_dispatch_int8_smooth"]:
+                  "mep_grad_reduce", "mep_dispatch_int8_smooth", "mep_update_expert_ranks"]:
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -184,6 +185,28 @@ def mep_update_expert(expert_ids: torch.Tensor, eplb_table: torch.Tensor,
                                  _ptr(balanced_active_mask, torch.uint8, "balanced_active_mask"),
                                  _stream(stream))
     _ok(rc, "mep_update_expert")
+    return balanced_expert_ids, balanced_active_mask
+
+
+def mep_update_expert_ranks(expert_ids: torch.Tensor, eplb_table: torch.Tensor,
+                            expert_scales: Optional[torch.Tensor],
+                            pruning_threshold: Optional[torch.Tensor],
+                            active_mask: Optional[torch.Tensor], world_size: int, balance_mode: int,
+                            balanced_expert_ids: torch.Tensor, balanced_active_mask: torch.Tensor,
+                            stream=None):
+    """mep_update_expert for every simulated rank in one launch (rows = world_size blocks)."""
+    rows, K = expert_ids.shape
+    E, F = eplb_table.shape
+    rc = lib().mep_update_expert_ranks(_ptr(expert_ids, torch.int32, "expert_ids"),
+                                       _ptr(eplb_table, torch.int32, "eplb_table"),
+                                       _ptr(expert_scales, torch.float32, "expert_scales"),
+                                       _ptr(pruning_threshold, torch.float32, "pruning_threshold"),
+                                       _ptr(active_mask, torch.uint8, "active_mask"), rows // world_size,
+                                       K, E, F, world_size, balance_mode,
+                                       _ptr(balanced_expert_ids, torch.int32, "balanced_expert_ids"),
+                                       _ptr(balanced_active_mask, torch.uint8, "balanced_active_mask"),
+                                       _stream(stream))
+    _ok(rc, "mep_update_expert_ranks")
     return balanced_expert_ids, balanced_active_mask
 
 

@@ -50,6 +50,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// bf16(p), round to nearest even, as an fp32 value: the packed conversion with a zero
+// low half leaves the bf16 bits in the high half, which read as fp32 are that value.
+__device__ __forceinline__ float round_bf16(float p) { return __uint_as_float(pack_bf16x2(0.0f, p)); }
+
 // Two binary32 additions / multiplications in one instruction (sm_100 packed f32x2),
 // each rounded to nearest even on its own: the same results as __fadd_rn / __fmul_rn
 // on each half. Use them only where no packed multiply feeds an addition: such a pair

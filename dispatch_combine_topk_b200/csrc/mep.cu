@@ -82,6 +82,19 @@ inline int token_grid(int64_t T, int per_sm)
     return (int)(g > 0 ? g : 1);
 }
 
+// Grid of at most `want` CTAs, capped at the number the GPU holds resident at once (for
+// grid-stride kernels whose CTAs should all start in the first wave).
+template <typename Kernel>
+int resident_grid(Kernel kernel, int threads, int64_t want)
+{
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    const int64_t cap = (int64_t)sm_count() * per_sm;
+    const int64_t g = want < cap ? want : cap;
+    return (int)(g > 0 ? g : 1);
+}
+
 inline int elem_grid(int64_t total, int threads)
 {
     int64_t g = (total + threads - 1) / threads;
@@ -215,8 +228,36 @@ mep_status_t mep_update_expert(const int32_t *expert_ids, const int32_t *eplb_ta
     int64_t g = (BS + threads - 1) / threads;
     int cap = sm_count() * 4;
     mep::k_update_expert<<<(unsigned)(g < cap ? g : cap), threads, 0, s>>>(
-        expert_ids, eplb_table, expert_scales, pruning_threshold, active_mask, BS, K, n_experts, F,
-        local_rank_id, world_size, balance_mode, balanced_expert_ids, balanced_active_mask);
+        expert_ids, eplb_table, expert_scales, pruning_threshold, active_mask, BS, BS, local_rank_id, K,
+        n_experts, F, world_size, balance_mode, balanced_expert_ids, balanced_active_mask);
+    return launched();
+}
+
+mep_status_t mep_update_expert_ranks(const int32_t *expert_ids, const int32_t *eplb_table,
+                                     const float *expert_scales, const float *pruning_threshold,
+                                     const uint8_t *active_mask, int64_t BS, int32_t K, int32_t n_experts,
+                                     int32_t F, int64_t world_size, int64_t balance_mode,
+                                     int32_t *balanced_expert_ids, uint8_t *balanced_active_mask,
+                                     mep_stream_t stream)
+{
+    if (!expert_ids || !eplb_table || !balanced_expert_ids || !balanced_active_mask)
+        return MEP_ERR_NULLPTR;
+    if ((expert_scales == nullptr) != (pruning_threshold == nullptr)) return MEP_ERR_NULLPTR;
+    if (active_mask && !expert_scales) return MEP_ERR_NULLPTR;
+    if (BS < 1 || K < 1 || K > 16 || n_experts < 1 || n_experts > 1024 || K > n_experts)
+        return MEP_ERR_SHAPE;
+    if (world_size < 1 || F < 2 || F > world_size + 1) return MEP_ERR_SHAPE;
+    if (balance_mode != 0 && balance_mode != 1) return MEP_ERR_VALUE;
+    if (balance_mode == 0 && (world_size < 2 || world_size > 768)) return MEP_ERR_VALUE;
+    if (BS * world_size * K >= ((int64_t)1 << 31)) return MEP_ERR_SHAPE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int threads = 128;
+    const int64_t rows = BS * world_size;
+    int64_t g = (rows + threads - 1) / threads;
+    int cap = sm_count() * 4;
+    mep::k_update_expert<<<(unsigned)(g < cap ? g : cap), threads, 0, s>>>(
+        expert_ids, eplb_table, expert_scales, pruning_threshold, active_mask, rows, BS, 0, K, n_experts, F,
+        world_size, balance_mode, balanced_expert_ids, balanced_active_mask);
     return launched();
 }
 
@@ -320,15 +361,20 @@ mep_status_t mep_combine_int8(const int8_t *yq, const float *y_scale, int64_t ro
         const uint4 *yv = (const uint4 *)yq;
         uint4 *ov = (uint4 *)out;
         const int64_t H16 = H / 16;
-        const int g16 = token_grid(T, 16);
+        using kernel_t = void (*)(const uint4 *, const float *, const int32_t *, const float *, int64_t, int,
+                                  int64_t, int64_t, uint4 *);
+        kernel_t kern;
         switch (K) {
-        case 1: mep::k_combine_int8_v16<1><<<g16, 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16, rows, ov); break;
-        case 2: mep::k_combine_int8_v16<2><<<g16, 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16, rows, ov); break;
-        case 4: mep::k_combine_int8_v16<4><<<g16, 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16, rows, ov); break;
-        case 6: mep::k_combine_int8_v16<6><<<g16, 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16, rows, ov); break;
-        case 8: mep::k_combine_int8_v16<8><<<g16, 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16, rows, ov); break;
-        default: mep::k_combine_int8_v16<0><<<g16, 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16, rows, ov); break;
+        case 1: kern = mep::k_combine_int8_warp<1>; break;
+        case 2: kern = mep::k_combine_int8_warp<2>; break;
+        case 4: kern = mep::k_combine_int8_warp<4>; break;
+        case 6: kern = mep::k_combine_int8_warp<6>; break;
+        case 8: kern = mep::k_combine_int8_warp<8>; break;
+        default: kern = mep::k_combine_int8_warp<0>; break;
         }
+        // one warp per token, grid-stride: as many CTAs as can be resident at once
+        kern<<<resident_grid(kern, 128, mep::ceil_div(T, 4)), 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16,
+                                                                           rows, ov);
     } else if (H % 8 == 0 && aligned(yq, 8) && aligned(out, 16)) {
         const uint2 *yv = (const uint2 *)yq;
         uint4 *ov = (uint4 *)out;

@@ -20,22 +20,26 @@ constexpr int kMaxK = 32;
 // ceil(world_size / count) + 1 (by rank) or (token mod count) + 1 (by token).
 // Pruning: v = sum_k fl(scale[k] * thr[k]) in fp32, ascending k, no FMA; a slot stays
 // active iff the token is active and !(scale[k] < v).
+// Rows are blocks of rows_per_rank tokens: row g belongs to rank rank0 + g / rows_per_rank
+// and is that rank's token i = g % rows_per_rank (one block for a single rank).
 __global__ void k_update_expert(const int32_t *__restrict__ ids, const int32_t *__restrict__ table,
                                 const float *__restrict__ scales, const float *__restrict__ thr,
-                                const uint8_t *__restrict__ active, int64_t BS, int32_t K,
-                                int32_t E, int32_t F, int64_t local_rank, int64_t world_size,
+                                const uint8_t *__restrict__ active, int64_t rows, int64_t rows_per_rank,
+                                int64_t rank0, int32_t K, int32_t E, int32_t F, int64_t world_size,
                                 int64_t mode, int32_t *__restrict__ out_ids,
                                 uint8_t *__restrict__ out_mask)
 {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < BS;
-         i += (int64_t)gridDim.x * blockDim.x) {
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < rows;
+         g += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = g % rows_per_rank;
+        const int64_t local_rank = rank0 + g / rows_per_rank;
         uint8_t act = 1;
         if (active) {
-            act = active[i] ? 1 : 0;
-            if (i > 0 && act && !active[i - 1]) flag_error(MEP_DERR_MASK);
+            act = active[g] ? 1 : 0;
+            if (i > 0 && act && !active[g - 1]) flag_error(MEP_DERR_MASK);
         }
         for (int32_t k = 0; k < K; k++) {
-            const int32_t e = ids[i * K + k];
+            const int32_t e = ids[g * K + k];
             int32_t inst = -1;
             if (e < 0 || e >= E) {
                 flag_error(MEP_DERR_KEY_RANGE);
@@ -54,15 +58,15 @@ __global__ void k_update_expert(const int32_t *__restrict__ ids, const int32_t *
                     else inst = v;
                 }
             }
-            out_ids[i * K + k] = inst;
+            out_ids[g * K + k] = inst;
         }
         if (scales) {
             float v = 0.0f;
-            for (int32_t k = 0; k < K; k++) v = __fadd_rn(v, __fmul_rn(scales[i * K + k], thr[k]));
+            for (int32_t k = 0; k < K; k++) v = __fadd_rn(v, __fmul_rn(scales[g * K + k], thr[k]));
             for (int32_t k = 0; k < K; k++)
-                out_mask[i * K + k] = (act && !(scales[i * K + k] < v)) ? 1 : 0;
+                out_mask[g * K + k] = (act && !(scales[g * K + k] < v)) ? 1 : 0;
         } else {
-            for (int32_t k = 0; k < K; k++) out_mask[i * K + k] = act;
+            for (int32_t k = 0; k < K; k++) out_mask[g * K + k] = act;
         }
     }
 }
@@ -537,24 +541,17 @@ k_combine_int8_v8(const uint2 *__restrict__ yq, const float *__restrict__ yscale
             // Codes to floats without the conversion unit: with the sign bit flipped a
             // code q is the byte q + 128, which a byte permute places in the mantissa of
             // 1.5 * 2^23; subtracting 1.5 * 2^23 + 128 gives q exactly. The bf16
-            // rounding of fl(q * scale) is one packed round-to-nearest-even conversion
-            // per two values.
+            // rounding of fl(q * scale) is one conversion per value that leaves the
+            // rounded value readable as fp32 (round_bf16), with nothing to unpack.
             auto add = [&](const uint2 &v, float g, float sc) {
                 const uint32_t w[2] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u};
 #pragma unroll
                 for (int h = 0; h < 2; h++) {
-                    float p[4];
 #pragma unroll
                     for (int j = 0; j < 4; j++) {
                         const float qf = __uint_as_float(__byte_perm(w[h], 0x4B400000u, 0x7650u + j)) - 12583040.0f;
-                        p[j] = __fmul_rn(qf, sc);
+                        acc[4 * h + j] = __fadd_rn(acc[4 * h + j], __fmul_rn(g, round_bf16(__fmul_rn(qf, sc))));
                     }
-                    const uint32_t b01 = pack_bf16x2(p[0], p[1]);
-                    const uint32_t b23 = pack_bf16x2(p[2], p[3]);
-                    acc[4 * h + 0] = __fadd_rn(acc[4 * h + 0], __fmul_rn(g, bf16lo(b01)));
-                    acc[4 * h + 1] = __fadd_rn(acc[4 * h + 1], __fmul_rn(g, bf16hi(b01)));
-                    acc[4 * h + 2] = __fadd_rn(acc[4 * h + 2], __fmul_rn(g, bf16lo(b23)));
-                    acc[4 * h + 3] = __fadd_rn(acc[4 * h + 3], __fmul_rn(g, bf16hi(b23)));
                 }
             };
             if constexpr (kFixed) {
@@ -585,85 +582,113 @@ k_combine_int8_v8(const uint2 *__restrict__ yq, const float *__restrict__ yscale
     }
 }
 
-// Same sum with 16 codes per slot per thread (one 16-byte load per slot, K of them in
-// flight per chunk): the path for H % 16 == 0 and 16-byte aligned buffers.
+// acc[j] (columns 2j, 2j+1 of a 16-column chunk) += fl(g * bf16(fl(q * sc))) for the 16
+// codes in v. Codes become floats as in k_combine_int8_v8 (byte permute into 1.5 * 2^23);
+// the exact bias subtraction and the code * scale product run on pairs of columns
+// (packed f32x2, each half rounded on its own).
+__device__ __forceinline__ void add_int8_x16(float2 (&acc)[8], const uint4 &v, float g, float sc)
+{
+    const uint32_t w[4] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u, v.z ^ 0x80808080u, v.w ^ 0x80808080u};
+    const float2 s2 = make_float2(sc, sc);
+    const float2 nb = make_float2(-12583040.0f, -12583040.0f);
+#pragma unroll
+    for (int h = 0; h < 4; h++) {
+#pragma unroll
+        for (int j = 0; j < 4; j += 2) {
+            const float2 qb = make_float2(__uint_as_float(__byte_perm(w[h], 0x4B400000u, 0x7650u + j)),
+                                          __uint_as_float(__byte_perm(w[h], 0x4B400000u, 0x7651u + j)));
+            const float2 p = mul2_rn(add2_rn(qb, nb), s2);
+            // the gate product is packed, the sum scalar: a packed multiply feeding a
+            // packed add may be fused into one rounding, which the sum's definition (two
+            // roundings) does not allow
+            const float2 gy = mul2_rn(make_float2(g, g), make_float2(round_bf16(p.x), round_bf16(p.y)));
+            float2 &a = acc[2 * h + j / 2];
+            a.x = __fadd_rn(a.x, gy.x);
+            a.y = __fadd_rn(a.y, gy.y);
+        }
+    }
+}
+
+__device__ __forceinline__ void store_bf16x16(uint4 *dst, const float2 (&acc)[8])
+{
+    uint4 o0, o1;
+    o0.x = pack_bf16x2(acc[0].x, acc[0].y);
+    o0.y = pack_bf16x2(acc[1].x, acc[1].y);
+    o0.z = pack_bf16x2(acc[2].x, acc[2].y);
+    o0.w = pack_bf16x2(acc[3].x, acc[3].y);
+    o1.x = pack_bf16x2(acc[4].x, acc[4].y);
+    o1.y = pack_bf16x2(acc[5].x, acc[5].y);
+    o1.z = pack_bf16x2(acc[6].x, acc[6].y);
+    o1.w = pack_bf16x2(acc[7].x, acc[7].y);
+    st_v4(dst, o0);
+    st_v4(dst + 1, o1);
+}
+
+// The combine of int8 rows for H % 16 == 0 and 16-byte aligned buffers (the same sum as
+// k_combine_int8_v8, 16 codes per slot per lane), one warp per token: lane k < K holds slot k's
+// row, gate and scale, which the other lanes take by shuffle once per token. There is no
+// block barrier, and the slot values stay in registers across the token's column chunks.
 template <int KC>
 __global__ void __launch_bounds__(128)
-k_combine_int8_v16(const uint4 *__restrict__ yq, const float *__restrict__ yscale, const int32_t *__restrict__ pos,
-                   const float *__restrict__ gates, int64_t T, int Krt, int64_t H16, int64_t rows,
-                   uint4 *__restrict__ out)
+k_combine_int8_warp(const uint4 *__restrict__ yq, const float *__restrict__ yscale, const int32_t *__restrict__ pos,
+                    const float *__restrict__ gates, int64_t T, int Krt, int64_t H16, int64_t rows,
+                    uint4 *__restrict__ out)
 {
     constexpr bool kFixed = KC > 0;
-    __shared__ int32_t sp[kMaxK];
-    __shared__ float sg[kMaxK];
-    __shared__ float ss[kMaxK];
     const int K = kFixed ? KC : Krt;
-    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-        load_token_rows(pos, t, K, rows, sp);
-        if (threadIdx.x < K) sg[threadIdx.x] = gates[t * K + threadIdx.x];
-        __syncthreads();
-        if (threadIdx.x < K) ss[threadIdx.x] = sp[threadIdx.x] >= 0 ? yscale[sp[threadIdx.x]] : 0.0f;
-        __syncthreads();
-        for (int64_t c = threadIdx.x; c < H16; c += blockDim.x) {
-            float2 acc[8];
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+        int32_t mine = -1;
+        float g_mine = 0.0f, s_mine = 0.0f;
+        if (lane < K) {
+            mine = pos[t * K + lane];
+            if (mine < -1 || (int64_t)mine >= rows) {
+                flag_error(MEP_DERR_ROW_RANGE);
+                mine = -1;
+            }
+            g_mine = gates[t * K + lane];
+            if (mine >= 0) s_mine = yscale[mine];
+        }
+        uint4 *dst = out + t * 2 * H16;
+        if constexpr (kFixed) {
+            int32_t pk[KC];
+            float gk[KC], sk[KC];
 #pragma unroll
-            for (int j = 0; j < 8; j++) acc[j] = make_float2(0.0f, 0.0f);
-            // codes -> floats as in k_combine_int8_v8 (byte permute into 1.5 * 2^23); the
-            // exact bias subtraction and the code * scale product run on pairs of columns
-            // (packed f32x2, each half rounded on its own)
-            const float2 bias = make_float2(12583040.0f, 12583040.0f);
-            auto add = [&](const uint4 &v, float g, float sc) {
-                const uint32_t w[4] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u, v.z ^ 0x80808080u,
-                                       v.w ^ 0x80808080u};
-                const float2 g2 = make_float2(g, g), s2 = make_float2(sc, sc);
+            for (int k = 0; k < KC; k++) {
+                pk[k] = __shfl_sync(0xffffffffu, mine, k);
+                gk[k] = __shfl_sync(0xffffffffu, g_mine, k);
+                sk[k] = __shfl_sync(0xffffffffu, s_mine, k);
+            }
+            for (int64_t c = lane; c < H16; c += 32) {
+                float2 acc[8];
 #pragma unroll
-                for (int h = 0; h < 4; h++) {
-#pragma unroll
-                    for (int j = 0; j < 4; j += 2) {
-                        const float2 qb = make_float2(__uint_as_float(__byte_perm(w[h], 0x4B400000u, 0x7650u + j)),
-                                                      __uint_as_float(__byte_perm(w[h], 0x4B400000u, 0x7651u + j)));
-                        const float2 qf = add2_rn(qb, make_float2(-bias.x, -bias.y));
-                        const float2 p = mul2_rn(qf, s2);
-                        const uint32_t bb = pack_bf16x2(p.x, p.y);
-                        // gate product and sum stay scalar: a packed multiply feeding a
-                        // packed add may be fused into one rounding, which the sum's
-                        // definition (two roundings) does not allow
-                        float2 &a = acc[2 * h + j / 2];
-                        a.x = __fadd_rn(a.x, __fmul_rn(g2.x, bf16lo(bb)));
-                        a.y = __fadd_rn(a.y, __fmul_rn(g2.y, bf16hi(bb)));
-                    }
-                }
-            };
-            if constexpr (kFixed) {
+                for (int j = 0; j < 8; j++) acc[j] = make_float2(0.0f, 0.0f);
                 uint4 v[KC];
 #pragma unroll
-                for (int k = 0; k < KC; k++) {
-                    const int32_t p = sp[k];
-                    v[k] = p >= 0 ? ld_stream(yq + (int64_t)p * H16 + c) : make_uint4(0, 0, 0, 0);
-                }
+                for (int k = 0; k < KC; k++)
+                    v[k] = pk[k] >= 0 ? ld_stream(yq + (int64_t)pk[k] * H16 + c) : make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int k = 0; k < KC; k++)
-                    if (sp[k] >= 0) add(v[k], sg[k], ss[k]);
-            } else {
-                for (int k = 0; k < K; k++) {
-                    const int32_t p = sp[k];
-                    if (p < 0) continue;
-                    add(ld_stream(yq + (int64_t)p * H16 + c), sg[k], ss[k]);
-                }
+                    if (pk[k] >= 0) add_int8_x16(acc, v[k], gk[k], sk[k]);
+                store_bf16x16(dst + 2 * c, acc);
             }
-            uint4 o0, o1;
-            o0.x = pack_bf16x2(acc[0].x, acc[0].y);
-            o0.y = pack_bf16x2(acc[1].x, acc[1].y);
-            o0.z = pack_bf16x2(acc[2].x, acc[2].y);
-            o0.w = pack_bf16x2(acc[3].x, acc[3].y);
-            o1.x = pack_bf16x2(acc[4].x, acc[4].y);
-            o1.y = pack_bf16x2(acc[5].x, acc[5].y);
-            o1.z = pack_bf16x2(acc[6].x, acc[6].y);
-            o1.w = pack_bf16x2(acc[7].x, acc[7].y);
-            st_v4(out + t * 2 * H16 + 2 * c, o0);
-            st_v4(out + t * 2 * H16 + 2 * c + 1, o1);
+        } else {
+            // warp-uniform trip count: every lane reaches the shuffles
+            for (int64_t base = 0; base < H16; base += 32) {
+                const int64_t c = base + lane;
+                float2 acc[8];
+#pragma unroll
+                for (int j = 0; j < 8; j++) acc[j] = make_float2(0.0f, 0.0f);
+                for (int k = 0; k < K; k++) {
+                    const int32_t p = __shfl_sync(0xffffffffu, mine, k);
+                    const float g = __shfl_sync(0xffffffffu, g_mine, k);
+                    const float sc = __shfl_sync(0xffffffffu, s_mine, k);
+                    if (p >= 0 && c < H16) add_int8_x16(acc, ld_stream(yq + (int64_t)p * H16 + c), g, sc);
+                }
+                if (c < H16) store_bf16x16(dst + 2 * c, acc);
+            }
         }
-        __syncthreads();
     }
 }
 

@@ -19,7 +19,7 @@
  *    stream) and never synchronise the host, so a chain plan -> dispatch -> combine
  *    needs no host round trip (MoonEP's static shapes remove per-layer host syncs:
  *    twodots.gr article on MoonEP, static-shapes paragraph). Only mep_get_error
- *    synchronises. mep_histogram, mep_plan, mep_update_expert, mep_dispatch,
+ *    synchronises. mep_histogram, mep_plan, mep_update_expert, mep_update_expert_ranks, mep_dispatch,
  *    mep_dispatch_int8_smooth, mep_dequantize, mep_combine, mep_combine_int8,
  *    mep_combine_add_rmsnorm, mep_prefetch_plan, mep_prefetch_weights and mep_grad_reduce
  *    can be captured into a CUDA graph and replayed on new inputs, once each has been
@@ -376,6 +376,24 @@ mep_status_t mep_update_expert(const int32_t *expert_ids, const int32_t *eplb_ta
                                int64_t world_size, int64_t balance_mode,
                                int32_t *balanced_expert_ids, uint8_t *balanced_active_mask,
                                mep_stream_t stream);
+
+/*
+ * a3 for every simulated rank at once: the same mapping and pruning as
+ * mep_update_expert, applied to the world_size ranks' tokens in one launch. Rows are
+ * world_size blocks of BS tokens: row g belongs to rank r = g / BS (its local_rank_id)
+ * and is that rank's token i = g % BS; the result equals world_size calls of
+ * mep_update_expert, one per block.
+ * expert_ids int32 [world_size*BS, K]; expert_scales fp32 [world_size*BS, K] or NULL;
+ * active_mask uint8 [world_size*BS] or NULL (every 1 before every 0 within each rank's
+ * block); other arguments, outputs and errors as mep_update_expert (without
+ * local_rank_id).
+ */
+mep_status_t mep_update_expert_ranks(const int32_t *expert_ids, const int32_t *eplb_table,
+                                     const float *expert_scales, const float *pruning_threshold,
+                                     const uint8_t *active_mask, int64_t BS, int32_t K,
+                                     int32_t n_experts, int32_t F, int64_t world_size,
+                                     int64_t balance_mode, int32_t *balanced_expert_ids,
+                                     uint8_t *balanced_active_mask, mep_stream_t stream);
 
 /*
  * a4 — dispatch: every kept slot's token row written straight to its final row of the

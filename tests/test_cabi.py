@@ -83,6 +83,21 @@ def test_update_expert_argument_checks(L):
     assert call(ws=1) == 4           # F=2 <= ws+1 is fine; ws < 2 in mode 0 -> VALUE
 
 
+def test_update_expert_ranks_argument_checks(L):
+    P = FAKE
+
+    def call(scales=None, thr=None, act=None, BS=4, K=2, E=8, F=2, ws=2, mode=0):
+        return L.mep_update_expert_ranks(P, P, scales, thr, act, BS, K, E, F, ws, mode, P, P, None)
+    assert call(scales=P) == 1
+    assert call(act=P) == 1
+    assert call(BS=0) == 3
+    assert call(K=3, E=2) == 3
+    assert call(F=4) == 3
+    assert call(mode=2) == 4
+    assert call(ws=1) == 4
+    assert call(BS=1 << 25, K=16, ws=8) == 3      # rows * K past int32
+
+
 def test_dispatch_combine_argument_checks(L):
     P = FAKE
     assert L.mep_dispatch(P, P, 4, 2, 64, 2, P, P, 8, None) == 2         # DTYPE

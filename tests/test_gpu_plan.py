@@ -117,6 +117,62 @@ def test_update_expert_and_grouped_plan_parity(mode):
     assert_plan_equal(pb, p, w.R)
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+def test_update_expert_ranks_matches_per_rank_oracle(mode):
+    """One launch over every rank's block equals the oracle called rank by rank."""
+    w = synth.get("map")
+    ids, gates = synth.router(w)
+    table, thr, active = synth.mapping_inputs(w)
+    bi = torch.empty((w.T, w.K), dtype=torch.int32, device=dev())
+    bm = torch.empty((w.T, w.K), dtype=torch.uint8, device=dev())
+    mep.mep_update_expert_ranks(torch.from_numpy(ids).to(dev()), torch.from_numpy(table).to(dev()),
+                                torch.from_numpy(gates).to(dev()), torch.from_numpy(thr).to(dev()),
+                                torch.from_numpy(active.astype(np.uint8)).to(dev()), w.R, mode, bi, bm)
+    _, _, oi, om = _mapping_all_ranks(w, mode, gpu=False)
+    assert np.array_equal(bi.cpu().numpy(), oi) and np.array_equal(bm.cpu().numpy().astype(bool), om)
+    assert mep.mep_get_error() == 0
+
+
+@pytest.mark.parametrize("ws,BS,K,E,F", [(2, 1, 1, 1, 2), (3, 37, 3, 9, 3), (7, 129, 4, 16, 5)])
+def test_update_expert_ranks_ragged_no_pruning(ws, BS, K, E, F):
+    """Ragged block sizes, no scales: every slot is mapped and kept."""
+    rng = np.random.default_rng(ws * 100 + BS)
+    ids = np.stack([rng.permutation(E)[:K] for _ in range(ws * BS)]).astype(np.int32)
+    table = np.zeros((E, F), np.int32)
+    for e in range(E):
+        c = int(rng.integers(1, F))
+        table[e, 0] = c
+        table[e, 1:1 + c] = rng.integers(0, ws * 4, c)
+    for mode in (0, 1) if ws >= 2 else (1,):
+        bi = torch.empty((ws * BS, K), dtype=torch.int32, device=dev())
+        bm = torch.empty((ws * BS, K), dtype=torch.uint8, device=dev())
+        mep.mep_update_expert_ranks(torch.from_numpy(ids).to(dev()), torch.from_numpy(table).to(dev()),
+                                    None, None, None, ws, mode, bi, bm)
+        for r in range(ws):
+            sl = slice(r * BS, (r + 1) * BS)
+            o, m = oracle.update_expert(ids[sl], table, None, None, None, r, ws, mode)
+            assert np.array_equal(bi.cpu().numpy()[sl], o)
+            assert np.array_equal(bm.cpu().numpy()[sl].astype(bool), m)
+    assert mep.mep_get_error() == 0
+
+
+def test_update_expert_ranks_mask_is_per_rank_block():
+    """A 0 then 1 across a rank boundary is allowed; inside one rank's block it is flagged."""
+    ids = torch.tensor([[0, 1], [1, 0], [0, 1], [1, 0]], dtype=torch.int32, device=dev())
+    table = torch.tensor([[1, 0, 0], [2, 1, 0]], dtype=torch.int32, device=dev())
+    sc = torch.full((4, 2), 0.5, dtype=torch.float32, device=dev())
+    thr = torch.zeros(2, dtype=torch.float32, device=dev())
+    bi = torch.empty_like(ids)
+    bm = torch.empty((4, 2), dtype=torch.uint8, device=dev())
+    mep.mep_update_expert_ranks(ids, table, sc, thr, torch.tensor([1, 0, 1, 1], dtype=torch.uint8,
+                                                                    device=dev()), 2, 0, bi, bm)
+    assert mep.mep_get_error() == 0
+    assert bm.cpu().tolist() == [[1, 1], [0, 0], [1, 1], [1, 1]]
+    mep.mep_update_expert_ranks(ids, table, sc, thr, torch.tensor([1, 1, 0, 1], dtype=torch.uint8,
+                                                                    device=dev()), 2, 0, bi, bm)
+    assert mep.mep_get_error() & mep.DERR_MASK
+
+
 def test_update_expert_hand_tables(golden_dir):
     import json, os
     g = json.load(open(os.path.join(golden_dir, "update_expert_hand.json")))
