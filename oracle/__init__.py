@@ -43,6 +43,8 @@ def _configure(L):
                                           P, P, P, P]
     L.orc_combine_add_rmsnorm.restype = ctypes.c_int
     L.orc_prefetch_plan.argtypes = [P, P, i32, i32, i32, i32, P, P]
+    L.orc_dedup_plan.argtypes = [P, i64, i32, P, i32, P, P, P, P, P, i64]
+    L.orc_expand.argtypes = [P, P, i64, P, i64, i64, P, P]
     L.orc_prefetch_weights.argtypes = [P, P, i32, i32, i32, i64, P]
     L.orc_grad_reduce.argtypes = [P, P, P, i32, i32, i32, i64]
     for name in ["orc_prefetch_plan", "orc_prefetch_weights", "orc_grad_reduce"]:
@@ -335,3 +337,42 @@ def dispatch_int8_smooth(x_bits, ids, pos, K: int, smooth, rows: int):
     _check(lib().orc_dispatch_int8_smooth(_p(x), _p(ids), _p(pos), T, K, H, _p(sm), sm.shape[0], rows,
                                           _p(q), _p(sc)), "dispatch_int8_smooth")
     return q, sc
+
+
+@dataclasses.dataclass
+class Dedup:
+    """One row per (token, destination rank): the send list, every slot's row, the
+    ranks' first rows, the token of every row and every plan row's source row."""
+    dsend: np.ndarray      # int32 [N]
+    dpos: np.ndarray       # int32 [N]
+    drank_off: np.ndarray  # int32 [R+1]
+    dtok: np.ndarray       # int32 [N] (-1 past drank_off[R])
+    gidx: np.ndarray       # int32 [len(pos)] (-1 past rank_off[R])
+
+
+def dedup_plan(pos, K: int, rank_off) -> Dedup:
+    pos = _c(pos, np.int32).ravel()
+    rank_off = _c(rank_off, np.int32).ravel()
+    N = pos.size
+    R = rank_off.size - 1
+    out = Dedup(np.empty(N, np.int32), np.empty(N, np.int32), np.empty(R + 1, np.int32),
+                np.empty(N, np.int32), np.empty(N, np.int32))
+    _check(lib().orc_dedup_plan(_p(pos), N, K, _p(rank_off), R, _p(out.dsend), _p(out.dpos),
+                                _p(out.drank_off), _p(out.dtok), _p(out.gidx), N), "dedup_plan")
+    return out
+
+
+def expand(src, gidx, rows: int, src_scale=None, dst=None, dst_scale=None):
+    """dst[p] = src[gidx[p]] for gidx[p] >= 0 (rows of any dtype; scales optional).
+    Returns dst (and dst_scale when scales are given)."""
+    src = np.ascontiguousarray(src)
+    gidx = _c(gidx, np.int32).ravel()
+    out = np.zeros((rows,) + src.shape[1:], src.dtype) if dst is None else np.array(dst, copy=True)
+    row_bytes = int(src.dtype.itemsize * np.prod(src.shape[1:]))
+    sc_in = None if src_scale is None else _c(src_scale, np.float32)
+    sc_out = None
+    if sc_in is not None:
+        sc_out = np.zeros(rows, np.float32) if dst_scale is None else np.array(dst_scale, np.float32, copy=True)
+    _check(lib().orc_expand(_p(src), None if sc_in is None else _p(sc_in), src.shape[0], _p(gidx), rows,
+                            row_bytes, _p(out), None if sc_out is None else _p(sc_out)), "expand")
+    return out if sc_out is None else (out, sc_out)

@@ -690,3 +690,86 @@ int orc_dispatch_int8_smooth(const uint16_t *x, const int32_t *ids, const int32_
     free(xs);
     return ORC_OK;
 }
+
+/* ------------------------------------- f1: one row per (token, destination rank) */
+
+/* Rank that owns row p of a plan: the r with rank_off[r] <= p < rank_off[r+1]. */
+static int32_t rank_of_row(const int32_t *rank_off, int32_t R, int64_t p)
+{
+    for (int32_t r = 0; r < R; r++)
+        if (p >= rank_off[r] && p < rank_off[r + 1]) return r;
+    return -1;
+}
+
+/*
+ * Deduplicated dispatch encoding (the MoonEP API reference, section 5.2 on
+ * communication performance, names a bounds check of a "dedup encoding"). Reading: a
+ * token whose kept slots land on one destination rank several times (several of its
+ * experts, or replicas, live there) crosses to that rank once. The rank's deduplicated
+ * receive rows hold its tokens in ascending global token order.
+ *
+ * For every rank r in ascending order, for every token g in ascending order: if any
+ * kept slot of g has its plan row on rank r, g takes the next deduplicated row u:
+ *   dtok[u] = g;  dsend[n0] = u for the first such slot n0 (the send list);
+ *   dpos[n] = u and gidx[pos[n]] = u for every such slot n.
+ * drank_off[r] = the first deduplicated row of rank r, drank_off[R] = the row count.
+ * Unset entries are -1. gidx has one entry per plan row (gidx_len >= rank_off[R]).
+ */
+int orc_dedup_plan(const int32_t *pos, int64_t N, int32_t K, const int32_t *rank_off, int32_t R,
+                   int32_t *dsend, int32_t *dpos, int32_t *drank_off, int32_t *dtok, int32_t *gidx,
+                   int64_t gidx_len)
+{
+    if (K <= 0 || N < 0 || N % K != 0 || R <= 0) return ORC_EARG;
+    if (rank_off[0] != 0) return ORC_EDATA;
+    for (int32_t r = 0; r < R; r++)
+        if (rank_off[r + 1] < rank_off[r]) return ORC_EDATA;
+    if (gidx_len < rank_off[R]) return ORC_EARG;
+    for (int64_t n = 0; n < N; n++) {
+        if (pos[n] < -1 || pos[n] >= rank_off[R]) return ORC_EDATA;
+        dsend[n] = -1;
+        dpos[n] = -1;
+        dtok[n] = -1;
+    }
+    for (int64_t i = 0; i < gidx_len; i++) gidx[i] = -1;
+    const int64_t T = N / K;
+    int32_t u = 0;
+    for (int32_t r = 0; r < R; r++) {
+        drank_off[r] = u;
+        for (int64_t g = 0; g < T; g++) {
+            int64_t first = -1;
+            for (int32_t k = 0; k < K; k++) {
+                const int64_t n = g * K + k;
+                if (pos[n] < 0 || rank_of_row(rank_off, R, pos[n]) != r) continue;
+                if (first < 0) {
+                    first = n;
+                    dsend[n] = u;
+                    dtok[u] = (int32_t)g;
+                }
+                dpos[n] = u;
+                gidx[pos[n]] = u;
+            }
+            if (first >= 0) u++;
+        }
+    }
+    drank_off[R] = u;
+    return ORC_OK;
+}
+
+/*
+ * Expansion on the receiving rank: dst[p, :] = src[gidx[p], :] (row_bytes bytes per
+ * row) and, with scales, dst_scale[p] = src_scale[gidx[p]], for every row p with
+ * gidx[p] >= 0; other rows are left as they are.
+ */
+int orc_expand(const uint8_t *src, const float *src_scale, int64_t src_rows, const int32_t *gidx, int64_t rows,
+               int64_t row_bytes, uint8_t *dst, float *dst_scale)
+{
+    if (rows < 0 || row_bytes <= 0 || src_rows < 0) return ORC_EARG;
+    for (int64_t p = 0; p < rows; p++) {
+        const int64_t u = gidx[p];
+        if (u < 0) continue;
+        if (u >= src_rows) return ORC_EDATA;
+        memcpy(dst + p * row_bytes, src + u * row_bytes, (size_t)row_bytes);
+        if (src_scale && dst_scale) dst_scale[p] = src_scale[u];
+    }
+    return ORC_OK;
+}

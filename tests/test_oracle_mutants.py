@@ -92,6 +92,24 @@ MUTANTS = [
      "                acc = acc + prod;", "                if (k + 1 < K) acc = acc + prod;",
      ["test_oracle_numerics.test_combine_k1_is_one_rounded_product",
       ("test_oracle_numerics.test_combine_equal_power_of_two_gates_is_exact", {"K": 4})]),
+    ("dedup: a rank's row range includes the next rank's first row",
+     "if (p >= rank_off[r] && p < rank_off[r + 1]) return r;",
+     "if (p >= rank_off[r] && p <= rank_off[r + 1]) return r;",
+     ["test_oracle_dedup.test_dedup_hand_example"]),
+    ("dedup: every slot is put on the send list",
+     "                if (first < 0) {\n                    first = n;",
+     "                if (1) {\n                    first = n;",
+     ["test_oracle_dedup.test_dedup_hand_example",
+      ("test_oracle_dedup.test_dedup_balanced_plans", {"R": 4, "E": 16, "S": 37, "K": 3})]),
+    ("dedup: a rank's rows in descending token order",
+     "        for (int64_t g = 0; g < T; g++) {\n            int64_t first = -1;",
+     "        for (int64_t g = T - 1; g >= 0; g--) {\n            int64_t first = -1;",
+     ["test_oracle_dedup.test_dedup_hand_example",
+      ("test_oracle_dedup.test_dedup_balanced_plans", {"R": 2, "E": 4, "S": 3, "K": 2})]),
+    ("expansion copies the first row's scale",
+     "if (src_scale && dst_scale) dst_scale[p] = src_scale[u];",
+     "if (src_scale && dst_scale) dst_scale[p] = src_scale[0];",
+     ["test_oracle_dedup.test_expand_copies_rows_and_scales"]),
 ]
 
 
