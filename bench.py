@@ -303,11 +303,16 @@ class Route:
     (mep_combine_int8, the same result as dequantising first).
     Mapping workload: mep_update_expert_ranks (every rank, one launch) -> grouped plan over the physical
     instances -> dispatch -> combine.
+    With dedup, the plan is followed by the deduplicated encoding (mep_dedup_plan), the
+    dispatch sends one row per (token, destination rank) along its send list, and an
+    expand phase (mep_expand) rebuilds the expert-grouped rows on the receiving side.
     """
 
-    def __init__(self, mep, w, dev, epilogue: str = "none"):
+    def __init__(self, mep, w, dev, epilogue: str = "none", dedup: bool = False):
         self.mep, self.w, self.dev = mep, w, dev
         self.epilogue = epilogue
+        self.dedup = dedup
+        self.n_sent = None
         ids, gates = synth.router(w)
         x = synth.hidden(w)
         self.host = dict(ids=torch.from_numpy(ids).view(-1), gates=torch.from_numpy(gates).view(-1), x=x)
@@ -341,7 +346,19 @@ class Route:
             else:
                 self.recv = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
                 self.y = self.recv
+        if dedup:
+            # the send buffer holds at most one row per slot; the plan decides how many
+            self.db = mep.DedupBuffers.allocate(w.R, w.S, w.K, dev)
+            self.sent = torch.empty((w.N, w.H), dtype=self.recv.dtype, device=dev)
+            self.sent_scale = torch.empty(w.N, dtype=torch.float32, device=dev) if w.quant else None
         torch.cuda.synchronize()
+
+    def phases(self):
+        """The step's phases in launch order (each timed with its own CUDA events)."""
+        ph = [("plan", self.plan), ("dispatch", self.dispatch)]
+        if self.dedup:
+            ph.append(("expand", self.expand))
+        return ph + [("combine", self.combine)]
 
     def plan(self, s):
         w, mep = self.w, self.mep
@@ -351,16 +368,30 @@ class Route:
             mep.mep_plan(self.bids.view(-1), w.R, self.n_keys, w.S, w.K, self.pb,
                          mode=mep.MEP_PLAN_GROUPED, keys_per_rank=w.place_per_rank,
                          keep=self.bmask.view(-1), stream=s)
-            return 1 + 4
-        mep.mep_plan(self.ids, w.R, w.E, w.S, w.K, self.pb, stream=s)
-        return 4
+            n = 1 + 4
+        else:
+            mep.mep_plan(self.ids, w.R, w.E, w.S, w.K, self.pb, stream=s)
+            n = 4
+        if self.dedup:
+            mep.mep_dedup_plan(self.pb.pos, self.pb.rank_off, w.R, w.S, w.K, self.db, stream=s)
+            n += 6
+        return n
 
     def dispatch(self, s):
         w = self.w
+        pos, recv, scale = self.pb.pos, self.recv, (self.scale if w.quant else None)
+        if self.dedup:
+            pos, recv, scale = self.db.dsend, self.sent, self.sent_scale
         if w.quant:
-            self.mep.mep_dispatch(self.x, self.pb.pos, w.K, self.recv, self.scale, quant=1, stream=s)
+            self.mep.mep_dispatch(self.x, pos, w.K, recv, scale, quant=1, stream=s)
         else:
-            self.mep.mep_dispatch(self.x, self.pb.pos, w.K, self.recv, stream=s)
+            self.mep.mep_dispatch(self.x, pos, w.K, recv, stream=s)
+        return 1
+
+    def expand(self, s):
+        """Receiving side of the deduplicated dispatch: sent rows -> expert-grouped rows."""
+        self.mep.mep_expand(self.sent, self.db.gidx, self.recv, src_scale=self.sent_scale,
+                            dst_scale=self.scale if self.w.quant else None, stream=s)
         return 1
 
     def combine(self, s):
@@ -378,17 +409,14 @@ class Route:
         return 1
 
     def step(self, s, ev=None):
+        """One step; ev (len(phases()) + 1 events) brackets the phases."""
+        n = 0
+        for i, (_, run) in enumerate(self.phases()):
+            if ev is not None:
+                ev[i].record(s)
+            n += run(s)
         if ev is not None:
-            ev[0].record(s)
-        n = self.plan(s)
-        if ev is not None:
-            ev[1].record(s)
-        n += self.dispatch(s)
-        if ev is not None:
-            ev[2].record(s)
-        n += self.combine(s)
-        if ev is not None:
-            ev[3].record(s)
+            ev[-1].record(s)
         return n
 
     def result_ok(self) -> bool:
@@ -418,13 +446,24 @@ class Route:
                     return "k_combine_int8_warp"
                 return "k_combine_int8_v8" if w.H % 8 == 0 else "k_combine_int8_scalar"
             return "k_combine_v8" if w.H % 8 == 0 else "k_combine_scalar"
+        if step == "expand":
+            return "k_expand_warp" if w.H % 16 == 0 or (not w.quant and w.H % 8 == 0) else "k_expand_bytes"
         if w.quant:
             return "k_dispatch_int8_staged" if w.H % 16 == 0 else "k_dispatch_int8"
         return "k_dispatch_warp" if w.H % 8 == 0 else "k_dispatch_elem"
 
     def working_set_bytes(self) -> int:
-        return (self.x.numel() * 2 + self.recv.numel() * self.recv.element_size() +
-                self.out.numel() * 2 + self.ids.numel() * 8)
+        b = (self.x.numel() * 2 + self.recv.numel() * self.recv.element_size() +
+             self.out.numel() * 2 + self.ids.numel() * 8)
+        if self.dedup:
+            b += self.sent.numel() * self.sent.element_size()
+        return b
+
+    def sent_rows(self) -> int:
+        """Rows the deduplicated dispatch sends (read once, after the first plan)."""
+        if self.n_sent is None:
+            self.n_sent = int(self.db.drank_off[-1].item())
+        return self.n_sent
 
     def bytes(self):
         """Algorithmic bytes per launch of dispatch and combine, and of the plan."""
@@ -440,7 +479,27 @@ class Route:
         if self.epilogue == "add_rmsnorm":
             comb += 2 * w.T * row + 4 * w.T + row   # residual in, normalised rows out, rstd, gamma
         plan = 16 * w.N
-        return {"plan": plan, "dispatch": disp, "combine": comb}
+        out = {"plan": plan, "dispatch": disp, "combine": comb}
+        if self.dedup:
+            # send: x in, one row (and scale) per (token, rank) out; expand: every
+            # expert-grouped row gathered from its sent row (read and write), gidx
+            qrow = w.H if w.quant else row
+            u = self.sent_rows()
+            out["dispatch"] = w.T * row + u * qrow + (4 * u if w.quant else 0) + 4 * w.N
+            out["expand"] = 2 * n_rows * qrow + (8 * n_rows if w.quant else 0) + 4 * n_rows
+            out["plan"] += 24 * w.N
+        return out
+
+
+def dedup_summary(rt):
+    """Rows the deduplicated dispatch sends against the slots it serves: the bytes that
+    would cross to other ranks with and without the dedup encoding."""
+    w = rt.w
+    u = rt.sent_rows()
+    kept = int(rt.pb.stats_dict()["n_kept"])
+    qrow = w.H if w.quant else 2 * w.H
+    return {"rows_sent": u, "slots": kept, "ratio": u / kept if kept else None,
+            "transport_bytes": u * qrow, "transport_bytes_without_dedup": kept * qrow}
 
 
 def maxvio(rt):
@@ -524,7 +583,10 @@ def run_gpu(args, w):
     # every rank routes its own independent batch (different seed)
     if args.epilogue != "none" and (w.quant or w.mapping):
         raise SystemExit("--epilogue applies to the balanced bf16 workloads")
-    rt = Route(mep, rank_workload(w, rank), dev, args.epilogue)
+    if args.dedup and w.mapping:
+        raise SystemExit("--dedup applies to the balanced workloads")
+    rt = Route(mep, rank_workload(w, rank), dev, args.epilogue, dedup=bool(args.dedup))
+    names = [n for n, _ in rt.phases()]
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -532,7 +594,7 @@ def run_gpu(args, w):
     stream.synchronize()
     mep.mep_get_error(clear=True)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # A working set that fits in L2 is flushed between steps (a 256 MB write, outside
     # the step's events); larger ones are not.
@@ -558,13 +620,11 @@ def run_gpu(args, w):
     if flush is None:
         ms = start.elapsed_time(end)
     else:
-        ms = float(sum(e[0].elapsed_time(e[3]) for e in evs))
+        ms = float(sum(e[0].elapsed_time(e[-1]) for e in evs))
     err = mep.mep_get_error(clear=True)
     if err:
         raise RuntimeError(f"device error word {err:#x} after the timed steps")
-    t_plan = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
-    t_disp = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
-    t_comb = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+    t_phase = {n: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs])) for i, n in enumerate(names)}
     ms_eager = max_over_ranks(ms, pg, dev) / args.steps
     weights = weight_side(mep, rt, args, dev, stream) if args.ffn_dim > 0 else None
 
@@ -665,12 +725,14 @@ def run_gpu(args, w):
     if rank == 0:
         peak, peak_kind = load_peaks()
         ab = rt.bytes()
-        dom = "dispatch" if t_disp >= t_comb else "combine"
-        t_dom = t_disp if dom == "dispatch" else t_comb
+        moving = [n for n in names if n != "plan"]          # the HBM-bound phases
+        dom = max(moving, key=lambda n: t_phase[n])
+        t_dom = t_phase[dom]
         achieved = ab[dom] / (t_dom * 1e-3) / 1e9
         kname = rt.kernel_name(dom)
         traffic, traffic_note = captured_traffic(kname, w.name)
-        dc_gbs = (ab["dispatch"] + ab["combine"]) / ((t_disp + t_comb) * 1e-3) / 1e9
+        t_move = sum(t_phase[n] for n in moving)
+        dc_gbs = sum(ab[n] for n in moving) / (t_move * 1e-3) / 1e9
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             v, desc, _ = oracle_sample(w, cpu_sample_S(w, args.cpu_div))
@@ -686,14 +748,14 @@ def run_gpu(args, w):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int8" if w.quant else "bf16", "data": "synthetic",
             "config": {"workload": w.name, "R": w.R, "E": w.E, "S": w.S, "K": w.K, "H": w.H,
-                       "epilogue": args.epilogue,
+                       "epilogue": args.epilogue, "dedup": bool(args.dedup),
                        "token_slots_per_gpu": w.N, "seed": w.seed, "parallelism": f"replicas{world}",
                        "l2": (f"working set {rt.working_set_bytes() / 1e6:.0f} MB "
                               + ("< 2x L2 (126 MB): L2 flushed between steps (256 MB write, "
                                  "not timed)" if flush is not None else
                                  "> 2x L2 (126 MB): inputs larger than L2, no flush"))},
-            "breakdown_ms": {"plan": t_plan, "dispatch": t_disp, "combine": t_comb},
-            "dispatch_combine": {"token_slots_per_s": w.N / ((t_disp + t_comb) * 1e-3),
+            "breakdown_ms": t_phase,
+            "dispatch_combine": {"token_slots_per_s": w.N / (t_move * 1e-3),
                                  "hbm_gbs": dc_gbs, "frac_of_peak": dc_gbs / peak,
                                  "frac_of_8tbs_nominal": dc_gbs / 8000.0},
             "roofline": {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": peak,
@@ -711,6 +773,7 @@ def run_gpu(args, w):
             "plan_stats": rt.pb.stats_dict(),
             "maxvio": maxvio(rt),
             "replica_weights": weights,
+            "dedup": dedup_summary(rt) if args.dedup else None,
         }
         print(json.dumps(line), flush=True)
     if pg:
@@ -733,6 +796,9 @@ def main():
     ap.add_argument("--graph", type=int, default=1,
                     help="1: time the step as a replayed CUDA graph (per-kernel breakdown "
                          "still comes from the eager steps); 0: eager only")
+    ap.add_argument("--dedup", type=int, default=0,
+                    help="1: send one row per (token, destination rank) and expand on the "
+                         "receiving side (mep_dedup_plan, mep_expand)")
     ap.add_argument("--epilogue", default="none", choices=["none", "add_rmsnorm"],
                     help="add_rmsnorm: combine fused with residual add + RMSNorm")
     ap.add_argument("--ffn-dim", type=int, default=0,

@@ -77,10 +77,15 @@ def lib() -> ctypes.CDLL:
         L.mep_grad_reduce.argtypes = [P, P, P, i32, i32, i32, i64, P]
         L.mep_dispatch_int8_smooth.argtypes = [P, P, P, i64, i32, i64, P, i32, P, P, i64, P]
         L.mep_update_expert_ranks.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i64, P, P, P]
+        L.mep_dedup_workspace_size.argtypes = [i32, i32, i32]
+        L.mep_dedup_workspace_size.restype = ctypes.c_size_t
+        L.mep_dedup_plan.argtypes = [P, P, i32, i32, i32, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.mep_expand.argtypes = [P, P, i64, P, i64, i64, i32, P, P, P]
         for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
                   "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8",
                   "mep_combine_add_rmsnorm", "mep_prefetch_plan", "mep_prefetch_weights",
-                  "mep_grad_reduce", "mep_dispatch_int8_smooth", "mep_update_expert_ranks"]:
+                  "mep_grad_reduce", "mep_dispatch_int8_smooth", "mep_update_expert_ranks",
+                  "mep_dedup_plan", "mep_expand"]:
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -166,6 +171,56 @@ def mep_plan(ids: torch.Tensor, R: int, n_keys: int, S: int, K: int, out: PlanBu
                         _ptr(out.workspace), out.workspace.numel(), _stream(stream))
     _ok(rc, "mep_plan")
     return out
+
+
+def mep_dedup_workspace_size(R: int, S: int, K: int) -> int:
+    return int(lib().mep_dedup_workspace_size(R, S, K))
+
+
+@dataclasses.dataclass
+class DedupBuffers:
+    """Device outputs of mep_dedup_plan: one row per (token, destination rank)."""
+
+    dsend: torch.Tensor      # int32 [N]  row of each pair's first slot (the send list), else -1
+    dpos: torch.Tensor       # int32 [N]  row of every kept slot
+    drank_off: torch.Tensor  # int32 [R+1]
+    dtok: torch.Tensor       # int32 [N]  token of every row, -1 past drank_off[R]
+    gidx: torch.Tensor       # int32 [N]  row holding the token of every plan row
+    workspace: torch.Tensor  # uint8, 256-byte aligned
+
+    @staticmethod
+    def allocate(R: int, S: int, K: int, device=None) -> "DedupBuffers":
+        dev = device or torch.device("cuda", torch.cuda.current_device())
+        N = R * S * K
+        z = lambda n: torch.empty(n, dtype=torch.int32, device=dev)
+        ws = torch.empty(max(256, mep_dedup_workspace_size(R, S, K)), dtype=torch.uint8, device=dev)
+        return DedupBuffers(z(N), z(N), z(R + 1), z(N), z(N), ws)
+
+
+def mep_dedup_plan(pos: torch.Tensor, rank_off: torch.Tensor, R: int, S: int, K: int, out: DedupBuffers,
+                   stream=None) -> DedupBuffers:
+    if pos.numel() != R * S * K or rank_off.numel() != R + 1:
+        raise ValueError("pos must hold R*S*K slots and rank_off R+1 offsets")
+    rc = lib().mep_dedup_plan(_ptr(pos, torch.int32, "pos"), _ptr(rank_off, torch.int32, "rank_off"), R, S, K,
+                              _ptr(out.dsend), _ptr(out.dpos), _ptr(out.drank_off), _ptr(out.dtok),
+                              _ptr(out.gidx), _ptr(out.workspace), out.workspace.numel(), _stream(stream))
+    _ok(rc, "mep_dedup_plan")
+    return out
+
+
+def mep_expand(src: torch.Tensor, gidx: torch.Tensor, dst: torch.Tensor, src_scale: Optional[torch.Tensor] = None,
+               dst_scale: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """dst[p] = src[gidx[p]] for gidx[p] >= 0: bf16 rows, or int8 rows with their scales."""
+    quant = 1 if src.dtype == torch.int8 else 0
+    want = torch.int8 if quant else torch.bfloat16
+    rows, H = dst.shape
+    if src.dim() != 2 or src.shape[1] != H or gidx.numel() != rows:
+        raise ValueError("src [rows_src, H], dst [rows, H] and gidx [rows] must agree")
+    rc = lib().mep_expand(_ptr(src, want, "src"), _ptr(src_scale, torch.float32, "src_scale"), src.shape[0],
+                          _ptr(gidx, torch.int32, "gidx"), rows, H, quant, _ptr(dst, want, "dst"),
+                          _ptr(dst_scale, torch.float32, "dst_scale"), _stream(stream))
+    _ok(rc, "mep_expand")
+    return dst
 
 
 def mep_update_expert(expert_ids: torch.Tensor, eplb_table: torch.Tensor,

@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "plan_kernels.cuh"
 #include "route_kernels.cuh"
+#include "dedup_kernels.cuh"
 
 namespace {
 
@@ -518,6 +519,80 @@ mep_status_t mep_selftest_bounded_wait(int32_t max_polls, int32_t *timed_out, me
     if (!timed_out) return MEP_ERR_NULLPTR;
     if (max_polls < 1 || max_polls > mep::kWaitPolls) return MEP_ERR_VALUE;
     mep::k_selftest_wait<<<1, 32, 0, (cudaStream_t)stream>>>(max_polls, timed_out);
+    return launched();
+}
+
+// ------------------------------------------------ f1: one row per (token, destination rank)
+
+size_t mep_dedup_workspace_size(int32_t R, int32_t S, int32_t K)
+{
+    if (R < 1 || S < 1 || K < 1) return 0;
+    const int64_t N = (int64_t)R * S * K;
+    const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
+    return align256(sizeof(int32_t) * (size_t)N) + align256((size_t)N) +
+           align256(sizeof(int32_t) * (size_t)tiles * R) + align256(sizeof(int32_t) * (size_t)R);
+}
+
+mep_status_t mep_dedup_plan(const int32_t *pos, const int32_t *rank_off, int32_t R, int32_t S, int32_t K,
+                            int32_t *dsend, int32_t *dpos, int32_t *drank_off, int32_t *dtok, int32_t *gidx,
+                            void *workspace, size_t workspace_bytes, mep_stream_t stream)
+{
+    if (!pos || !rank_off || !dsend || !dpos || !drank_off || !dtok || !gidx) return MEP_ERR_NULLPTR;
+    if (R < 1 || S < 1 || K < 1 || K > MEP_MAX_K || R > MEP_MAX_KEYS) return MEP_ERR_SHAPE;
+    const int64_t N = (int64_t)R * S * K;
+    if (N >= ((int64_t)1 << 31)) return MEP_ERR_SHAPE;
+    const size_t need = mep_dedup_workspace_size(R, S, K);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return MEP_ERR_WORKSPACE;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    const int sms = sm_count();
+    const int64_t T = (int64_t)R * S;
+    const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
+    unsigned char *w = (unsigned char *)workspace;
+    int32_t *dkey = (int32_t *)w;
+    w += align256(sizeof(int32_t) * (size_t)N);
+    uint8_t *dkeep = (uint8_t *)w;
+    w += align256((size_t)N);
+    int32_t *tile_cnt = (int32_t *)w;
+    w += align256(sizeof(int32_t) * (size_t)tiles * R);
+    int32_t *count = (int32_t *)w;
+
+    if (cudaMemsetAsync(dtok, 0xff, sizeof(int32_t) * (size_t)N, s) != cudaSuccess) return launched();
+    if (cudaMemsetAsync(gidx, 0xff, sizeof(int32_t) * (size_t)N, s) != cudaSuccess) return launched();
+    const int64_t tg = mep::ceil_div(T, 256), tcap = (int64_t)sms * 8;
+    const unsigned tgrid = (unsigned)(tg < tcap ? tg : tcap);
+    const size_t off_smem = sizeof(int32_t) * (size_t)(R + 1);
+    const int threads = mep::kPlanWarps * 32;
+    mep::k_dedup_keys<<<tgrid, 256, off_smem, s>>>(pos, rank_off, R, T, K, dkey, dkeep);
+    mep::k_tile_count<<<(unsigned)tiles, threads, sizeof(int32_t) * R, s>>>(dkey, dkeep, N, R, tile_cnt);
+    mep::k_scan_cols<<<(unsigned)mep::ceil_div(R, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, R, count);
+    const size_t rank_smem = sizeof(int32_t) * ((size_t)mep::kPlanWarps * R + R + 1 + 33);
+    mep::k_rank<<<(unsigned)tiles, threads, rank_smem, s>>>(dkey, dkeep, N, R, tile_cnt, count, dsend);
+    mep::k_dedup_offsets<<<1, 1024, sizeof(int32_t) * (size_t)(R + 1 + 33), s>>>(count, R, drank_off);
+    mep::k_dedup_finish<<<tgrid, 256, off_smem, s>>>(pos, rank_off, R, T, K, dsend, dpos, dtok, gidx);
+    return launched();
+}
+
+mep_status_t mep_expand(const void *src, const float *src_scale, int64_t src_rows, const int32_t *gidx,
+                        int64_t rows, int64_t H, int32_t quant, void *dst, float *dst_scale, mep_stream_t stream)
+{
+    if (quant != 0 && quant != 1) return MEP_ERR_DTYPE;
+    if (rows < 0 || src_rows < 0 || H < 1) return MEP_ERR_SHAPE;
+    if (rows == 0) return MEP_OK;
+    if (!gidx || !dst || (!src && src_rows > 0)) return MEP_ERR_NULLPTR;
+    if (quant == 1 && (!dst_scale || (!src_scale && src_rows > 0))) return MEP_ERR_NULLPTR;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t row_bytes = quant == 1 ? H : 2 * H;
+    const float *ss = quant == 1 ? src_scale : nullptr;
+    float *ds = quant == 1 ? dst_scale : nullptr;
+    if (row_bytes % 16 == 0 && aligned(src, 16) && aligned(dst, 16)) {
+        const unsigned g = (unsigned)resident_grid(mep::k_expand_warp, 256, mep::ceil_div(rows, 8));
+        mep::k_expand_warp<<<g, 256, 0, s>>>((const uint4 *)src, ss, src_rows, gidx, rows, row_bytes / 16,
+                                             (uint4 *)dst, ds);
+    } else {
+        mep::k_expand_bytes<<<token_grid(rows, 8), 256, 0, s>>>((const uint8_t *)src, ss, src_rows, gidx, rows,
+                                                              row_bytes, (uint8_t *)dst, ds);
+    }
     return launched();
 }
 

@@ -19,8 +19,9 @@
  *    stream) and never synchronise the host, so a chain plan -> dispatch -> combine
  *    needs no host round trip (MoonEP's static shapes remove per-layer host syncs:
  *    twodots.gr article on MoonEP, static-shapes paragraph). Only mep_get_error
- *    synchronises. mep_histogram, mep_plan, mep_update_expert, mep_update_expert_ranks, mep_dispatch,
- *    mep_dispatch_int8_smooth, mep_dequantize, mep_combine, mep_combine_int8,
+ *    synchronises. mep_histogram, mep_plan, mep_update_expert, mep_update_expert_ranks,
+ *    mep_dedup_plan, mep_dispatch, mep_expand, mep_dispatch_int8_smooth, mep_dequantize,
+ *    mep_combine, mep_combine_int8,
  *    mep_combine_add_rmsnorm, mep_prefetch_plan, mep_prefetch_weights and mep_grad_reduce
  *    can be captured into a CUDA graph and replayed on new inputs, once each has been
  *    called eagerly on the device (the first call sets kernel attributes).
@@ -415,6 +416,53 @@ mep_status_t mep_update_expert_ranks(const int32_t *expert_ids, const int32_t *e
 mep_status_t mep_dispatch(const uint16_t *x, const int32_t *pos, int64_t T, int32_t K,
                           int64_t H, int32_t quant, void *recv, float *recv_scale,
                           int64_t rows, mep_stream_t stream);
+
+/*
+ * f1 — one dispatch row per (token, destination rank). The MoonEP API reference
+ * (stapisi.com), section 5.2 on communication performance, names a bounds-checked
+ * "dedup encoding". Reading: a token whose kept slots land on one destination rank
+ * several times (several of its experts, or replicas, live there) crosses to that rank
+ * once, and the rank expands it to its expert-grouped rows locally.
+ *
+ * From a plan (pos, rank_off of mep_plan, either mode): the destination rank of kept
+ * slot n is the r with rank_off[r] <= pos[n] < rank_off[r+1]. Rank r's deduplicated
+ * rows are [drank_off[r], drank_off[r+1]) and hold, in ascending global token order,
+ * the tokens g with at least one kept slot on r. Outputs (device, overwritten):
+ *   dsend     int32 [N]    row of the first slot of each (token, rank) pair, -1 for
+ *                          every other slot: the send list (mep_dispatch(x, dsend, ...)
+ *                          writes each pair's row once)
+ *   dpos      int32 [N]    row of every kept slot (shared by a pair's slots), -1 dropped
+ *   drank_off int32 [R+1]  first row of every rank, drank_off[R] = the row count U
+ *   dtok      int32 [N]    token of every row, -1 from U on
+ *   gidx      int32 [N]    for every plan row p < rank_off[R], the row holding its token:
+ *                          gidx[pos[n]] = dpos[n]; -1 elsewhere (mep_expand's index)
+ * Bounds the encoding keeps: a rank's rows <= min(T, its plan rows); tokens with a kept
+ * slot <= U <= kept slots.
+ * Workspace: at least mep_dedup_workspace_size(R, S, K) bytes, 256-byte aligned.
+ * Errors: NULL pointer; R, S, K < 1, K > MEP_MAX_K, R > MEP_MAX_KEYS, N >= 2^31
+ * (MEP_ERR_SHAPE); workspace (MEP_ERR_WORKSPACE). A pos outside [-1, min(rank_off[R],
+ * N)) counts as dropped and sets MEP_DERR_ROW_RANGE. rank_off must be non-decreasing
+ * from 0 (as mep_plan writes it).
+ */
+size_t mep_dedup_workspace_size(int32_t R, int32_t S, int32_t K);
+mep_status_t mep_dedup_plan(const int32_t *pos, const int32_t *rank_off, int32_t R, int32_t S, int32_t K,
+                            int32_t *dsend, int32_t *dpos, int32_t *drank_off, int32_t *dtok, int32_t *gidx,
+                            void *workspace, size_t workspace_bytes, mep_stream_t stream);
+
+/*
+ * f1 — expansion on the receiving rank: dst[p, :] = src[gidx[p], :] for every row p in
+ * [0, rows) with gidx[p] >= 0 (other rows are left untouched); with quant == 1 also
+ * dst_scale[p] = src_scale[gidx[p]]. After mep_dedup_plan and a dispatch with its send
+ * list, this gives exactly the rows the plain dispatch writes.
+ * quant 0: src, dst bf16 [.., H]; quant 1: int8 [.., H] with fp32 scales [..] (required).
+ * src has src_rows rows; gidx int32 [rows].
+ * Errors: quant outside {0,1} (MEP_ERR_DTYPE); rows, src_rows < 0, H < 1
+ * (MEP_ERR_SHAPE); NULL pointer (MEP_ERR_NULLPTR). A gidx at or past src_rows is
+ * skipped and sets MEP_DERR_ROW_RANGE.
+ */
+mep_status_t mep_expand(const void *src, const float *src_scale, int64_t src_rows, const int32_t *gidx,
+                        int64_t rows, int64_t H, int32_t quant, void *dst, float *dst_scale,
+                        mep_stream_t stream);
 
 /*
  * Identity expert on int8 rows: y[r, h] = bf16_rne(fl(float(q[r,h]) * scale[r])).

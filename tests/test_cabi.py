@@ -98,6 +98,35 @@ def test_update_expert_ranks_argument_checks(L):
     assert call(BS=1 << 25, K=16, ws=8) == 3      # rows * K past int32
 
 
+def test_dedup_and_expand_argument_checks(L):
+    P = FAKE
+    wsb = L.mep_dedup_workspace_size(8, 4096, 8)
+    assert wsb >= 8 * 4096 * 8 * 5
+    assert L.mep_dedup_workspace_size(0, 1, 1) == 0
+
+    def dedup(pos=P, R=2, S=4, K=2, ws=P, wsb=1 << 20, out=P):
+        return L.mep_dedup_plan(pos, P, R, S, K, out, P, P, P, P, ws, wsb, None)
+    assert dedup(pos=None) == 1
+    assert dedup(out=None) == 1
+    assert dedup(R=0) == 3
+    assert dedup(K=33) == 3
+    assert dedup(R=5000) == 3
+    assert dedup(R=1 << 16, S=1 << 16) == 3
+    assert dedup(ws=None) == 5
+    assert dedup(wsb=16) == 5
+    assert dedup(ws=ctypes.c_void_p(0x1008)) == 5
+
+    def expand(src=P, ss=None, src_rows=4, gidx=P, rows=4, H=8, quant=0, dst=P, ds=None):
+        return L.mep_expand(src, ss, src_rows, gidx, rows, H, quant, dst, ds, None)
+    assert expand(quant=2) == 2
+    assert expand(rows=-1) == 3
+    assert expand(H=0) == 3
+    assert expand(rows=0) == 0                  # nothing to do: no launch
+    assert expand(gidx=None) == 1
+    assert expand(quant=1, ss=P) == 1           # int8 rows need both scale arrays
+    assert expand(quant=1, ds=P) == 1
+
+
 def test_dispatch_combine_argument_checks(L):
     P = FAKE
     assert L.mep_dispatch(P, P, 4, 2, 64, 2, P, P, 8, None) == 2         # DTYPE
