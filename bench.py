@@ -54,9 +54,11 @@ def _device_functions():
     """name -> source text of every function defined in the library's CUDA headers."""
     import re
 
+    import glob
+
     funcs = {}
-    for fn in ("common.cuh", "tma.cuh", "plan_kernels.cuh", "route_kernels.cuh"):
-        src = open(os.path.join(CSRC, fn)).read()
+    for path in sorted(glob.glob(os.path.join(CSRC, "*.cuh"))):
+        src = open(path).read()
         for m in re.finditer(r"\n(?:template <[^>]*>\n)?(?:__global__|__device__|__host__ __device__)\b", src):
             brace = src.find("{", m.end())
             end = src.find("\n}\n", brace)
@@ -110,6 +112,9 @@ TRAFFIC = {
     ("k_combine_int8_warp", "int8_r32_e256_s8192_k8_h7168"): {
         "bytes": 16 * 1117.18e6, "src": "d852eb58236fe244",
         "note": "profiles/traffic_dominant_kernels.md: 1117.18 MB at S=512, x16"},
+    ("k_expand_warp", "r8_e64_s4096_k8_h7168"): {
+        "bytes": 4 * 1793.81e6, "src": "a12dc9427177590d",
+        "note": "profiles/dedup_r8.md: 1793.81 MB at S=1024, x4 (--dedup 1)"},
     ("k_dispatch_warp", "skew_r64_e512_s2048_k8_h4096"): {
         "bytes": 4 * 2357.84e6, "src": "17b1506c97a87d55",
         "note": "profiles/traffic_dominant_kernels.md: 2357.84 MB at S=512, x4"},
