@@ -240,7 +240,7 @@ def oracle_sample(w, S_sample):
     dt = parts["plan"] + parts["dispatch"] + parts["combine"]
     desc = (f"oracle {'mapping+grouped plan' if ws.mapping else 'plan'}+"
             f"{'int8 ' if ws.quant else ''}dispatch+combine on R={ws.R} E={ws.E} S={ws.S} K={ws.K} "
-            f"H={ws.H} ({ws.N} token-slots; S reduced from {w.S}); "
+            f"H={ws.H} ({ws.N} token-slots" + (f"; S reduced from {w.S}" if ws.S < w.S else "; the whole workload") + "); "
             + " ".join(f"{k} {v:.3f}s" for k, v in parts.items()))
     return ws.N / dt, desc, dt
 
@@ -570,6 +570,108 @@ def weight_side(mep, rt, args, dev, stream):
     return out
 
 
+def e2e_route_host(mep, rt, w, dev, steps, pg):
+    """End to end through the C ABI with host buffers: each step is one mep_route_host
+    call (upload from pinned host memory, plan, dispatch, combine, download to pinned
+    host memory, all on one stream). Three device buffer sets on three streams take the
+    steps in turn, so one step's upload, another's kernels and a third's download overlap
+    on the full-duplex link."""
+    h = {k: v.contiguous().pin_memory() for k, v in rt.host.items()}
+    quant = 1 if w.quant else 0
+    sets = [mep.RouteBuffers.allocate(w.R, w.E, w.S, w.K, w.H, quant, dev) for _ in range(3)]
+    structs = [b.c_struct() for b in sets]
+    outs = [torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    streams = [torch.cuda.Stream(dev) for _ in range(3)]
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def run(n):
+        torch.cuda.synchronize()
+        first, last = ev(), ev()
+        first.record(streams[0])
+        for j in (1, 2):
+            streams[j].wait_event(first)
+        for i in range(n):
+            j = i % 3
+            mep.mep_route_host(sets[j], h["ids"], h["gates"], h["x"], outs[j], stream=streams[j],
+                               c_struct=structs[j])
+        for j in (1, 2):
+            done = ev()
+            done.record(streams[j])
+            streams[0].wait_event(done)
+        last.record(streams[0])
+        torch.cuda.synchronize()
+        return first.elapsed_time(last)
+
+    run(3)
+    if pg:
+        pg.barrier()
+    ms = max_over_ranks(run(steps) / steps, pg, dev)
+    ok = torch.equal(outs[(steps - 1) % 3].float(), rt.out.cpu().float())
+    h2d = sum(v.numel() * v.element_size() for v in h.values())
+    d2h = outs[0].numel() * 2
+    del sets
+    return ms, ok, h2d, d2h, ("one mep_route_host call per step (C ABI, pinned host buffers): upload, "
+                              "plan, dispatch, combine, download on one stream; three device buffer sets "
+                              "on three streams in turn")
+
+
+def e2e_pipeline(rt, w, dev, stream, steps, pg):
+    """End to end through the binding's calls for the steps mep_route_host does not cover
+    (the mapping workload, the fused epilogue, the deduplicated dispatch): every step
+    copies its inputs from pinned host memory to the device, routes them, and copies its
+    result back to pinned host memory. Double-buffered device inputs/outputs on three
+    streams (host-to-device, compute, device-to-host), so that step i+1's upload, step
+    i's routing and step i-1's download overlap on the full-duplex link."""
+    h = {k: v.pin_memory() for k, v in rt.host.items()}
+    out_h = [torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    slots = [dict(ids=rt.ids, gates=rt.gates, x=rt.x, out=rt.out)]
+    slots.append({k: torch.empty_like(v) for k, v in slots[0].items()})
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def e2e_run(n):
+        in_done, comp_done, out_done = [], [], []
+        first, last = ev(), ev()
+        first.record(s_in)
+        for i in range(n):
+            b = slots[i % 2]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(comp_done[i - 2])      # slot i%2 inputs consumed
+                b["ids"].copy_(h["ids"], non_blocking=True)
+                b["gates"].copy_(h["gates"], non_blocking=True)
+                b["x"].copy_(h["x"], non_blocking=True)
+                in_done.append(ev())
+                in_done[-1].record(s_in)
+            stream.wait_event(in_done[i])
+            if i >= 2:
+                stream.wait_event(out_done[i - 2])         # slot i%2 output downloaded
+            rt.ids, rt.gates, rt.x, rt.out = b["ids"], b["gates"], b["x"], b["out"]
+            with torch.cuda.stream(stream):
+                rt.step(stream)
+            comp_done.append(ev())
+            comp_done[-1].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[i])
+                out_h[i % 2].copy_(b["out"], non_blocking=True)
+                out_done.append(ev())
+                out_done[-1].record(s_out)
+        last.record(s_out)
+        torch.cuda.synchronize()
+        return first.elapsed_time(last)
+
+    e2e_run(3)
+    if pg:
+        pg.barrier()
+    ms = max_over_ranks(e2e_run(steps) / steps, pg, dev)
+    ok = rt.result_ok() and torch.equal(out_h[(steps - 1) % 2].float(), rt.out.cpu().float())
+    h2d = sum(v.numel() * v.element_size() for v in h.values())
+    d2h = out_h[0].numel() * 2
+    return ms, ok, h2d, d2h, ("binding calls with copies from and to pinned host memory: uploads, "
+                              "routing and downloads of consecutive steps overlap (two device buffer "
+                              "sets, three streams)")
+
+
 def run_gpu(args, w):
     import dispatch_combine_topk_b200 as mep
 
@@ -675,57 +777,11 @@ def run_gpu(args, w):
     ms_step = graph_ms if graph_ms is not None else ms_eager
     ok_device = rt.result_ok()
 
-    # End to end through the public calls: every step copies its inputs from pinned host
-    # memory to the device, routes them, and copies its result back to pinned host
-    # memory. Double-buffered device inputs/outputs on three streams (host-to-device,
-    # compute, device-to-host), so that step i+1's upload, step i's routing and step
-    # i-1's download overlap on the full-duplex link.
-    h = {k: v.pin_memory() for k, v in rt.host.items()}
-    out_h = [torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     e2e_steps = max(4, min(args.steps, 20))
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    slots = [dict(ids=rt.ids, gates=rt.gates, x=rt.x, out=rt.out)]
-    slots.append({k: torch.empty_like(v) for k, v in slots[0].items()})
-    ev = lambda: torch.cuda.Event(enable_timing=True)
-
-    def e2e_run(n):
-        in_done, comp_done, out_done = [], [], []
-        first, last = ev(), ev()
-        first.record(s_in)
-        for i in range(n):
-            b = slots[i % 2]
-            with torch.cuda.stream(s_in):
-                if i >= 2:
-                    s_in.wait_event(comp_done[i - 2])      # slot i%2 inputs consumed
-                b["ids"].copy_(h["ids"], non_blocking=True)
-                b["gates"].copy_(h["gates"], non_blocking=True)
-                b["x"].copy_(h["x"], non_blocking=True)
-                in_done.append(ev())
-                in_done[-1].record(s_in)
-            stream.wait_event(in_done[i])
-            if i >= 2:
-                stream.wait_event(out_done[i - 2])         # slot i%2 output downloaded
-            rt.ids, rt.gates, rt.x, rt.out = b["ids"], b["gates"], b["x"], b["out"]
-            with torch.cuda.stream(stream):
-                rt.step(stream)
-            comp_done.append(ev())
-            comp_done[-1].record(stream)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(comp_done[i])
-                out_h[i % 2].copy_(b["out"], non_blocking=True)
-                out_done.append(ev())
-                out_done[-1].record(s_out)
-        last.record(s_out)
-        torch.cuda.synchronize()
-        return first.elapsed_time(last)
-
-    e2e_run(3)
-    if pg:
-        pg.barrier()
-    e2e_ms = max_over_ranks(e2e_run(e2e_steps) / e2e_steps, pg, dev)
-    ok_e2e = rt.result_ok() and torch.equal(out_h[(e2e_steps - 1) % 2].float(), rt.out.cpu().float())
-    h2d = sum(v.numel() * v.element_size() for v in h.values())
-    d2h = out_h[0].numel() * 2
+    if not w.mapping and args.epilogue == "none" and not args.dedup:
+        e2e_ms, ok_e2e, h2d, d2h, how = e2e_route_host(mep, rt, w, dev, e2e_steps, pg)
+    else:
+        e2e_ms, ok_e2e, h2d, d2h, how = e2e_pipeline(rt, w, dev, stream, e2e_steps, pg)
 
     if rank == 0:
         peak, peak_kind = load_peaks()
@@ -770,8 +826,7 @@ def run_gpu(args, w):
             "cpu_baseline": cpu,
             "e2e": {"value": world * w.N / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                    "pipelining": "uploads, routing and downloads of consecutive steps overlap "
-                                  "(two device buffer sets, three streams)"},
+                    "path": how},
             "result_check": {"device": ok_device, "e2e": ok_e2e},
             "gpu_launches": launches,
             "clocks": clk.summary(),

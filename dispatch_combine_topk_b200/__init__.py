@@ -43,6 +43,16 @@ class MepError(RuntimeError):
         super().__init__(f"{what}: {name}{extra}")
 
 
+class _RouteBuffersC(ctypes.Structure):
+    """mep_route_buffers_t of include/mep.h."""
+    _fields_ = [("R", ctypes.c_int32), ("E", ctypes.c_int32), ("S", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("H", ctypes.c_int64), ("quant", ctypes.c_int32)] + \
+               [(n, ctypes.c_void_p) for n in ("ids", "gates", "x", "recv", "recv_scale", "out", "pos", "hist",
+                                               "rank_off", "load", "rep_count", "rep_key", "rep_cu", "stats",
+                                               "workspace")] + \
+               [("workspace_bytes", ctypes.c_size_t)]
+
+
 _lib = None
 
 
@@ -81,11 +91,12 @@ def lib() -> ctypes.CDLL:
         L.mep_dedup_workspace_size.restype = ctypes.c_size_t
         L.mep_dedup_plan.argtypes = [P, P, i32, i32, i32, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.mep_expand.argtypes = [P, P, i64, P, i64, i64, i32, P, P, P]
+        L.mep_route_host.argtypes = [ctypes.POINTER(_RouteBuffersC), P, P, P, P, P]
         for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
                   "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8",
                   "mep_combine_add_rmsnorm", "mep_prefetch_plan", "mep_prefetch_weights",
                   "mep_grad_reduce", "mep_dispatch_int8_smooth", "mep_update_expert_ranks",
-                  "mep_dedup_plan", "mep_expand"]:
+                  "mep_dedup_plan", "mep_expand", "mep_route_host"]:
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -394,3 +405,68 @@ def mep_plan_static_ws(ids: torch.Tensor, R: int, n_keys: int, S: int, K: int, o
     _ok(rc, "mep_plan_static_ws")
     return out
 
+
+
+@dataclasses.dataclass
+class RouteBuffers:
+    """Device buffers of one routing round trip from host memory (mep_route_host)."""
+
+    R: int
+    E: int
+    S: int
+    K: int
+    H: int
+    quant: int
+    ids: torch.Tensor                   # int32 [N]
+    gates: torch.Tensor                 # fp32 [N]
+    x: torch.Tensor                     # bf16 [T, H]
+    recv: torch.Tensor                  # bf16 or int8 [N, H]
+    recv_scale: Optional[torch.Tensor]  # fp32 [N] (int8)
+    out: torch.Tensor                   # bf16 [T, H]
+    plan: PlanBuffers
+
+    @staticmethod
+    def allocate(R: int, E: int, S: int, K: int, H: int, quant: int = 0, device=None) -> "RouteBuffers":
+        dev = device or torch.device("cuda", torch.cuda.current_device())
+        T, N = R * S, R * S * K
+        return RouteBuffers(
+            R, E, S, K, H, quant,
+            torch.empty(N, dtype=torch.int32, device=dev), torch.empty(N, dtype=torch.float32, device=dev),
+            torch.empty((T, H), dtype=torch.bfloat16, device=dev),
+            torch.empty((N, H), dtype=torch.int8 if quant else torch.bfloat16, device=dev),
+            torch.empty(N, dtype=torch.float32, device=dev) if quant else None,
+            torch.empty((T, H), dtype=torch.bfloat16, device=dev),
+            PlanBuffers.allocate(R, E, S, K, dev))
+
+    def c_struct(self) -> _RouteBuffersC:
+        p = lambda t: None if t is None else t.data_ptr()
+        pb = self.plan
+        return _RouteBuffersC(self.R, self.E, self.S, self.K, self.H, self.quant, p(self.ids), p(self.gates),
+                              p(self.x), p(self.recv), p(self.recv_scale), p(self.out), p(pb.pos), p(pb.hist),
+                              p(pb.rank_off), p(pb.load), p(pb.rep_count), p(pb.rep_key), p(pb.rep_cu),
+                              p(pb.stats), p(pb.workspace), pb.workspace.numel())
+
+
+def _host_ptr(t: torch.Tensor, dtype, name: str):
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def mep_route_host(rb: RouteBuffers, ids_h: torch.Tensor, gates_h: torch.Tensor, x_h: torch.Tensor,
+                   out_h: torch.Tensor, stream=None, c_struct: Optional[_RouteBuffersC] = None) -> torch.Tensor:
+    """Upload, plan, dispatch, combine (identity expert), download: one C call, all
+    enqueued on `stream`. Pinned host tensors keep it asynchronous."""
+    T, N = rb.R * rb.S, rb.R * rb.S * rb.K
+    if ids_h.numel() != N or gates_h.numel() != N or tuple(x_h.shape) != (T, rb.H) or tuple(out_h.shape) != (T, rb.H):
+        raise ValueError("host tensors must match the buffers' shapes")
+    cs = c_struct if c_struct is not None else rb.c_struct()
+    rc = lib().mep_route_host(ctypes.byref(cs), _host_ptr(ids_h, torch.int32, "ids_h"),
+                              _host_ptr(gates_h, torch.float32, "gates_h"), _host_ptr(x_h, torch.bfloat16, "x_h"),
+                              _host_ptr(out_h, torch.bfloat16, "out_h"), _stream(stream))
+    _ok(rc, "mep_route_host")
+    return out_h

@@ -596,6 +596,42 @@ mep_status_t mep_expand(const void *src, const float *src_scale, int64_t src_row
     return launched();
 }
 
+// ------------------------------------------------- one round trip from host memory
+
+mep_status_t mep_route_host(const mep_route_buffers_t *b, const int32_t *ids_h, const float *gates_h,
+                            const uint16_t *x_h, uint16_t *out_h, mep_stream_t stream)
+{
+    if (!b || !ids_h || !gates_h || !x_h || !out_h) return MEP_ERR_NULLPTR;
+    if (!b->ids || !b->gates || !b->x || !b->recv || !b->out) return MEP_ERR_NULLPTR;
+    if (b->quant != 0 && b->quant != 1) return MEP_ERR_DTYPE;
+    if (b->R < 1 || b->S < 1 || b->K < 1 || b->H < 1) return MEP_ERR_SHAPE;
+    const int64_t T = (int64_t)b->R * b->S, N = T * b->K;
+    if (N >= ((int64_t)1 << 31)) return MEP_ERR_SHAPE;
+    cudaStream_t s = (cudaStream_t)stream;
+    auto copy = [&](void *dst, const void *src, size_t bytes, cudaMemcpyKind kind) -> mep_status_t {
+        if (cudaMemcpyAsync(dst, src, bytes, kind, s) != cudaSuccess) return launched();
+        return MEP_OK;
+    };
+    mep_status_t st;
+    if ((st = copy(b->ids, ids_h, sizeof(int32_t) * (size_t)N, cudaMemcpyHostToDevice)) != MEP_OK) return st;
+    if ((st = copy(b->gates, gates_h, sizeof(float) * (size_t)N, cudaMemcpyHostToDevice)) != MEP_OK) return st;
+    if ((st = copy(b->x, x_h, sizeof(uint16_t) * (size_t)(T * b->H), cudaMemcpyHostToDevice)) != MEP_OK)
+        return st;
+    st = mep_plan(b->ids, nullptr, b->R, b->E, b->S, b->K, MEP_PLAN_BALANCED, 0, b->pos, b->hist, b->rank_off,
+                  b->load, b->rep_count, b->rep_key, b->rep_cu, b->stats, b->workspace, b->workspace_bytes,
+                  stream);
+    if (st != MEP_OK) return st;
+    st = mep_dispatch(b->x, b->pos, T, b->K, b->H, b->quant, b->recv, b->recv_scale, N, stream);
+    if (st != MEP_OK) return st;
+    if (b->quant == 0)
+        st = mep_combine((const uint16_t *)b->recv, N, b->pos, b->gates, T, b->K, b->H, b->out, stream);
+    else
+        st = mep_combine_int8((const int8_t *)b->recv, b->recv_scale, N, b->pos, b->gates, T, b->K, b->H,
+                              b->out, stream);
+    if (st != MEP_OK) return st;
+    return copy(out_h, b->out, sizeof(uint16_t) * (size_t)(T * b->H), cudaMemcpyDeviceToHost);
+}
+
 }  // extern "C"
 
 

@@ -490,6 +490,42 @@ mep_status_t mep_combine(const uint16_t *y, int64_t rows, const int32_t *pos,
                          const float *gates, int64_t T, int32_t K, int64_t H, uint16_t *out,
                          mep_stream_t stream);
 
+/*
+ * One routing round trip of a batch that lives in host memory: upload, balanced plan,
+ * dispatch, combine of the dispatched rows (the identity expert), download. This is the
+ * composition mep_plan -> mep_dispatch -> mep_combine (or mep_combine_int8 for int8
+ * rows) with its host<->device copies, all enqueued on `stream`; nothing synchronises.
+ * With pinned (page-locked) host buffers the call returns at once and consecutive calls
+ * on different streams with different buffer sets overlap their copies and kernels;
+ * pageable host buffers make the copies synchronous. The device buffers are the
+ * caller's (the call allocates nothing); they and the host buffers must not be touched
+ * until the stream has passed the call.
+ */
+typedef struct {
+    int32_t R, E, S, K;          /* ranks, experts (E % R == 0), tokens per rank, top-K */
+    int64_t H;                   /* hidden size */
+    int32_t quant;               /* 0: bf16 rows; 1: per-token int8 rows + scales */
+    int32_t *ids;                /* [N] int32, N = R*S*K */
+    float *gates;                /* [N] fp32 */
+    uint16_t *x;                 /* [T, H] bf16, T = R*S */
+    void *recv;                  /* [N, H] bf16 (quant 0) or int8 (quant 1) */
+    float *recv_scale;           /* [N] fp32 (quant 1), else NULL */
+    uint16_t *out;               /* [T, H] bf16 */
+    int32_t *pos, *hist, *rank_off, *load, *rep_count, *rep_key, *rep_cu;   /* as mep_plan */
+    mep_plan_stats_t *stats;
+    void *workspace;             /* mep_plan_workspace_size(R, E, S, K) bytes, 256-aligned */
+    size_t workspace_bytes;
+} mep_route_buffers_t;
+
+/*
+ * ids_h int32 [N], gates_h fp32 [N], x_h bf16 [T, H] (host, read); out_h bf16 [T, H]
+ * (host, written). Errors: NULL pointers (MEP_ERR_NULLPTR); quant outside {0,1}
+ * (MEP_ERR_DTYPE); then whatever mep_plan, mep_dispatch or the combine return; a failed
+ * copy (MEP_ERR_CUDA). Nothing after a failing step is enqueued.
+ */
+mep_status_t mep_route_host(const mep_route_buffers_t *dev, const int32_t *ids_h, const float *gates_h,
+                            const uint16_t *x_h, uint16_t *out_h, mep_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

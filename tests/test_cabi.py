@@ -147,3 +147,36 @@ def test_dispatch_combine_argument_checks(L):
     assert L.mep_selftest_bounded_wait(10, None, None) == 1
     assert L.mep_selftest_bounded_wait(0, P, None) == 4
     assert L.mep_selftest_bounded_wait(1 << 23, P, None) == 4
+
+
+def test_route_buffers_struct_layout_matches_the_header(tmp_path):
+    """The binding's ctypes mirror of mep_route_buffers_t has the header's layout
+    (size and field offsets as gcc lays the struct out)."""
+    import subprocess
+    import dispatch_combine_topk_b200 as mep
+    C = mep._RouteBuffersC
+    names = [f[0] for f in C._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"mep.h\"\nint main(void){\n"
+                   "printf(\"%zu\\n\", sizeof(mep_route_buffers_t));\n" +
+                   "".join(f'printf("%zu\\n", offsetof(mep_route_buffers_t, {n}));\n' for n in names) +
+                   "return 0;}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    assert got[0] == ctypes.sizeof(C)
+    assert got[1:] == [getattr(C, n).offset for n in names]
+
+
+def test_route_host_argument_checks(L):
+    import dispatch_combine_topk_b200 as mep
+    P = FAKE
+    b = mep._RouteBuffersC(2, 4, 2, 2, 8, 0, *([0x1000] * 15), 1 << 20)
+    assert L.mep_route_host(None, P, P, P, P, None) == 1
+    assert L.mep_route_host(ctypes.byref(b), None, P, P, P, None) == 1
+    b.quant = 3
+    assert L.mep_route_host(ctypes.byref(b), P, P, P, P, None) == 2
+    b.quant, b.R = 0, 0
+    assert L.mep_route_host(ctypes.byref(b), P, P, P, P, None) == 3
+    b.R, b.ids = 2, None
+    assert L.mep_route_host(ctypes.byref(b), P, P, P, P, None) == 1
