@@ -1,8 +1,9 @@
 /*
  * A C caller of libmep, with no Python involved: plan, dispatch and combine of a small
- * balanced workload through the C ABI of include/mep.h, checked against closed forms
- * (every rank receives exactly S*K rows; with gates summing to one, the identity expert
- * gives every token back). Prints "route_roundtrip ok" and exits 0 on success.
+ * balanced workload through the C ABI of include/mep.h, then the same round trip from
+ * host memory in one mep_route_host call, checked against closed forms (every rank
+ * receives exactly S*K rows; with gates summing to one, the identity expert gives every
+ * token back). Prints "route_roundtrip ok" and exits 0 on success.
  */
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -95,6 +96,22 @@ int main(void)
     for (int r = 0; r < R; r++) CHECK(count[r] == S * K && rank_off[r] == r * S * K);
     CHECK(stats.max_chunk == S * K && stats.n_kept == N && stats.redundant <= R - 1);
     CHECK(memcmp(out, x, sizeof(uint16_t) * T * H) == 0);
+    /* the same round trip from host memory in one call (pageable buffers: the copies
+       are synchronous, the kernels still run on the stream) */
+    uint16_t *out2 = malloc(sizeof(uint16_t) * T * H);
+    memset(out2, 0xff, sizeof(uint16_t) * T * H);
+    CHECK(cudaMemset(d_out, 0, sizeof(uint16_t) * T * H) == cudaSuccess);
+    mep_route_buffers_t rb;
+    memset(&rb, 0, sizeof rb);
+    rb.R = R; rb.E = E; rb.S = S; rb.K = K; rb.H = H; rb.quant = 0;
+    rb.ids = d_ids; rb.gates = d_g; rb.x = d_x; rb.recv = d_recv; rb.recv_scale = NULL; rb.out = d_out;
+    rb.pos = d_pos; rb.hist = d_hist; rb.rank_off = d_roff; rb.load = d_load; rb.rep_count = d_rc;
+    rb.rep_key = d_rk; rb.rep_cu = d_rcu; rb.stats = d_stats; rb.workspace = d_ws; rb.workspace_bytes = ws;
+    CHECK(mep_route_host(&rb, ids, gates, x, out2, st) == MEP_OK);
+    CHECK(cudaStreamSynchronize(st) == cudaSuccess);
+    CHECK(memcmp(out2, x, sizeof(uint16_t) * T * H) == 0);
+    rb.quant = 5;
+    CHECK(mep_route_host(&rb, ids, gates, x, out2, st) == MEP_ERR_DTYPE);
     /* argument errors come back without touching the device */
     CHECK(mep_dispatch(d_x, d_pos, T, K, H, 7, d_recv, NULL, N, st) == MEP_ERR_DTYPE);
     CHECK(mep_plan(NULL, NULL, R, E, S, K, 0, 0, d_pos, d_hist, d_roff, NULL, d_rc, d_rk, d_rcu, d_stats, d_ws,
