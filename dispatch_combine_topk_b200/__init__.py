@@ -114,6 +114,24 @@ def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor"):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _need(ok: bool, what: str):
+    """Shape check of the binding: the C calls cannot see the sizes of device buffers,
+    so a tensor too small for the call is refused here, before anything is launched."""
+    if not ok:
+        raise ValueError(what)
+
+
+def _n(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.numel()
+
+
+def _check_plan_buffers(out: "PlanBuffers", R: int, n_keys: int, N: int):
+    _need(_n(out.pos) >= N and _n(out.hist) >= n_keys and _n(out.rank_off) >= R + 1
+          and (out.load is None or _n(out.load) >= R) and _n(out.rep_count) >= R
+          and _n(out.rep_key) >= R * n_keys and _n(out.rep_cu) >= R * (n_keys + 1) and _n(out.stats) >= 8,
+          "plan buffers too small for (R, n_keys, S, K): allocate them with PlanBuffers.allocate")
+
+
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
@@ -132,6 +150,7 @@ def mep_get_error(clear: bool = True) -> int:
 
 
 def mep_histogram(ids: torch.Tensor, n_keys: int, hist: torch.Tensor, stream=None):
+    _need(_n(hist) >= n_keys, "hist must hold n_keys counts")
     _ok(lib().mep_histogram(_ptr(ids, torch.int32, "ids"), ids.numel(), n_keys,
                             _ptr(hist, torch.int32, "hist"), _stream(stream)), "mep_histogram")
     return hist
@@ -175,6 +194,8 @@ def mep_plan(ids: torch.Tensor, R: int, n_keys: int, S: int, K: int, out: PlanBu
              keep: Optional[torch.Tensor] = None, stream=None) -> PlanBuffers:
     if ids.numel() != R * S * K:
         raise ValueError("ids must hold R*S*K slots")
+    _need(keep is None or keep.numel() == R * S * K, "keep must hold R*S*K flags")
+    _check_plan_buffers(out, R, n_keys, R * S * K)
     rc = lib().mep_plan(_ptr(ids, torch.int32, "ids"), _ptr(keep, torch.uint8, "keep"), R, n_keys,
                         S, K, mode, keys_per_rank, _ptr(out.pos), _ptr(out.hist),
                         _ptr(out.rank_off), _ptr(out.load), _ptr(out.rep_count),
@@ -212,6 +233,9 @@ def mep_dedup_plan(pos: torch.Tensor, rank_off: torch.Tensor, R: int, S: int, K:
                    stream=None) -> DedupBuffers:
     if pos.numel() != R * S * K or rank_off.numel() != R + 1:
         raise ValueError("pos must hold R*S*K slots and rank_off R+1 offsets")
+    N = R * S * K
+    _need(min(_n(out.dsend), _n(out.dpos), _n(out.dtok), _n(out.gidx)) >= N and _n(out.drank_off) >= R + 1,
+          "dedup buffers too small: allocate them with DedupBuffers.allocate")
     rc = lib().mep_dedup_plan(_ptr(pos, torch.int32, "pos"), _ptr(rank_off, torch.int32, "rank_off"), R, S, K,
                               _ptr(out.dsend), _ptr(out.dpos), _ptr(out.drank_off), _ptr(out.dtok),
                               _ptr(out.gidx), _ptr(out.workspace), out.workspace.numel(), _stream(stream))
@@ -227,11 +251,22 @@ def mep_expand(src: torch.Tensor, gidx: torch.Tensor, dst: torch.Tensor, src_sca
     rows, H = dst.shape
     if src.dim() != 2 or src.shape[1] != H or gidx.numel() != rows:
         raise ValueError("src [rows_src, H], dst [rows, H] and gidx [rows] must agree")
+    _need(dst.dtype == src.dtype, "src and dst must have the same dtype")
+    if quant:
+        _need(_n(src_scale) >= src.shape[0] and _n(dst_scale) >= rows, "int8 rows need src and dst scales")
     rc = lib().mep_expand(_ptr(src, want, "src"), _ptr(src_scale, torch.float32, "src_scale"), src.shape[0],
                           _ptr(gidx, torch.int32, "gidx"), rows, H, quant, _ptr(dst, want, "dst"),
                           _ptr(dst_scale, torch.float32, "dst_scale"), _stream(stream))
     _ok(rc, "mep_expand")
     return dst
+
+
+def _check_mapping(ids, scales, thr, active, out_ids, out_mask):
+    rows, K = ids.shape
+    _need(scales is None or tuple(scales.shape) == (rows, K), "expert_scales must match expert_ids")
+    _need(thr is None or thr.numel() == K, "pruning_threshold must hold K values")
+    _need(active is None or active.numel() == rows, "active_mask must hold one flag per token")
+    _need(_n(out_ids) >= rows * K and _n(out_mask) >= rows * K, "outputs must hold one entry per slot")
 
 
 def mep_update_expert(expert_ids: torch.Tensor, eplb_table: torch.Tensor,
@@ -241,6 +276,8 @@ def mep_update_expert(expert_ids: torch.Tensor, eplb_table: torch.Tensor,
                       balanced_active_mask: torch.Tensor, stream=None):
     BS, K = expert_ids.shape
     E, F = eplb_table.shape
+    _check_mapping(expert_ids, expert_scales, pruning_threshold, active_mask, balanced_expert_ids,
+                   balanced_active_mask)
     rc = lib().mep_update_expert(_ptr(expert_ids, torch.int32, "expert_ids"),
                                  _ptr(eplb_table, torch.int32, "eplb_table"),
                                  _ptr(expert_scales, torch.float32, "expert_scales"),
@@ -263,6 +300,9 @@ def mep_update_expert_ranks(expert_ids: torch.Tensor, eplb_table: torch.Tensor,
     """mep_update_expert for every simulated rank in one launch (rows = world_size blocks)."""
     rows, K = expert_ids.shape
     E, F = eplb_table.shape
+    _need(world_size >= 1 and rows % world_size == 0, "expert_ids must hold world_size blocks of BS tokens")
+    _check_mapping(expert_ids, expert_scales, pruning_threshold, active_mask, balanced_expert_ids,
+                   balanced_active_mask)
     rc = lib().mep_update_expert_ranks(_ptr(expert_ids, torch.int32, "expert_ids"),
                                        _ptr(eplb_table, torch.int32, "eplb_table"),
                                        _ptr(expert_scales, torch.float32, "expert_scales"),
@@ -281,6 +321,9 @@ def mep_dispatch(x: torch.Tensor, pos: torch.Tensor, K: int, recv: torch.Tensor,
     T, H = x.shape
     want = torch.int8 if quant == 1 else torch.bfloat16
     rows = recv.shape[0]
+    _need(pos.numel() == T * K, "pos must hold T*K slots")
+    _need(recv.dim() == 2 and recv.shape[1] == H, "recv must be [rows, H]")
+    _need(quant != 1 or _n(recv_scale) >= rows, "int8 dispatch needs recv_scale [rows]")
     rc = lib().mep_dispatch(_ptr(x, torch.bfloat16, "x"), _ptr(pos, torch.int32, "pos"), T, K, H,
                             quant, _ptr(recv, want, "recv"),
                             _ptr(recv_scale, torch.float32, "recv_scale"), rows, _stream(stream))
@@ -290,14 +333,21 @@ def mep_dispatch(x: torch.Tensor, pos: torch.Tensor, K: int, recv: torch.Tensor,
 
 def mep_dequantize(q: torch.Tensor, scale: torch.Tensor, y: torch.Tensor, stream=None):
     rows, H = q.shape
+    _need(_n(scale) >= rows and tuple(y.shape) == (rows, H), "scale [rows] and y [rows, H] must match q")
     _ok(lib().mep_dequantize(_ptr(q, torch.int8, "q"), _ptr(scale, torch.float32, "scale"), rows, H,
                              _ptr(y, torch.bfloat16, "y"), _stream(stream)), "mep_dequantize")
     return y
 
 
+def _check_combine(y, pos, gates, T, K, H):
+    _need(y.dim() == 2 and y.shape[1] == H, "y must be [rows, H] with out's H")
+    _need(pos.numel() == T * K and gates.numel() == T * K, "pos and gates must hold T*K slots")
+
+
 def mep_combine(y: torch.Tensor, pos: torch.Tensor, gates: torch.Tensor, K: int,
                 out: torch.Tensor, stream=None):
     T, H = out.shape
+    _check_combine(y, pos, gates, T, K, H)
     rc = lib().mep_combine(_ptr(y, torch.bfloat16, "y"), y.shape[0], _ptr(pos, torch.int32, "pos"),
                            _ptr(gates, torch.float32, "gates"), T, K, H,
                            _ptr(out, torch.bfloat16, "out"), _stream(stream))
@@ -309,6 +359,8 @@ def mep_combine_int8(yq: torch.Tensor, y_scale: torch.Tensor, pos: torch.Tensor,
                      K: int, out: torch.Tensor, stream=None):
     """Combine of int8 rows with per-row scales (dequantisation fused into the sum)."""
     T, H = out.shape
+    _check_combine(yq, pos, gates, T, K, H)
+    _need(_n(y_scale) >= yq.shape[0], "y_scale must hold one scale per row")
     rc = lib().mep_combine_int8(_ptr(yq, torch.int8, "yq"), _ptr(y_scale, torch.float32, "y_scale"),
                                 yq.shape[0], _ptr(pos, torch.int32, "pos"),
                                 _ptr(gates, torch.float32, "gates"), T, K, H,
@@ -323,6 +375,9 @@ def mep_combine_add_rmsnorm(y: torch.Tensor, pos: torch.Tensor, gates: torch.Ten
                             stream=None):
     """Combine, residual add and RMSNorm in one kernel (see include/mep.h)."""
     T, H = x_out.shape
+    _check_combine(y, pos, gates, T, K, H)
+    _need(tuple(residual.shape) == (T, H) and tuple(y_out.shape) == (T, H) and gamma.numel() == H
+          and _n(rstd_out) >= T, "residual, y_out [T, H], gamma [H] and rstd_out [T] must match")
     rc = lib().mep_combine_add_rmsnorm(
         _ptr(y, torch.bfloat16, "y"), y.shape[0], _ptr(pos, torch.int32, "pos"),
         _ptr(gates, torch.float32, "gates"), T, K, H, _ptr(residual, torch.bfloat16, "residual"),
@@ -337,6 +392,9 @@ def mep_prefetch_plan(plan: PlanBuffers, R: int, E: int, B: int, slot_expert: to
                       rep_weight: torch.Tensor, stream=None):
     """Slots of the prefetched replicas and the weight row of every replica."""
     cap = plan.rep_key.shape[1]
+    _need(plan.rep_key.shape[0] >= R and _n(plan.rep_count) >= R, "plan buffers must cover R ranks")
+    _need(B == 0 or _n(slot_expert) >= R * B, "slot_expert must hold R*B slots")
+    _need(_n(rep_weight) >= R * cap, "rep_weight must be [R, cap]")
     rc = lib().mep_prefetch_plan(_ptr(plan.rep_count, torch.int32, "rep_count"),
                                  _ptr(plan.rep_key, torch.int32, "rep_key"), R, E, cap, B,
                                  _ptr(slot_expert, torch.int32, "slot_expert") if B > 0 else None,
@@ -349,6 +407,7 @@ def mep_prefetch_weights(w_home: torch.Tensor, slot_expert: torch.Tensor, R: int
                          w_slots: torch.Tensor, stream=None):
     E = w_home.shape[0]
     D = w_home.numel() // E
+    _need(_n(slot_expert) >= R * B and _n(w_slots) >= R * B * D, "slot_expert [R*B] and w_slots [R*B, ...] needed")
     rc = lib().mep_prefetch_weights(_ptr(w_home, torch.bfloat16, "w_home"),
                                     _ptr(slot_expert, torch.int32, "slot_expert"), E, R, B, D,
                                     _ptr(w_slots, torch.bfloat16, "w_slots"), _stream(stream))
@@ -360,6 +419,8 @@ def mep_grad_reduce(grad_home: torch.Tensor, grad_slots: torch.Tensor, slot_expe
                     R: int, B: int, stream=None):
     E = grad_home.shape[0]
     D = grad_home.numel() // E
+    _need(_n(slot_expert) >= R * B and _n(grad_slots) >= R * B * D,
+          "slot_expert [R*B] and grad_slots [R*B, ...] needed")
     rc = lib().mep_grad_reduce(_ptr(grad_home, torch.float32, "grad_home"),
                                _ptr(grad_slots, torch.float32, "grad_slots"),
                                _ptr(slot_expert, torch.int32, "slot_expert"), E, R, B, D,
@@ -373,6 +434,10 @@ def mep_dispatch_int8_smooth(x: torch.Tensor, ids: torch.Tensor, pos: torch.Tens
                              stream=None):
     """int8 dispatch with per-expert smoothing scales (codes and scale per slot)."""
     T, H = x.shape
+    _need(ids.numel() == T * K and pos.numel() == T * K, "ids and pos must hold T*K slots")
+    _need(smooth.dim() == 2 and smooth.shape[1] == H, "smooth must be [experts, H]")
+    _need(recv.dim() == 2 and recv.shape[1] == H and _n(recv_scale) >= recv.shape[0],
+          "recv [rows, H] and recv_scale [rows] needed")
     rc = lib().mep_dispatch_int8_smooth(_ptr(x, torch.bfloat16, "x"), _ptr(ids, torch.int32, "ids"),
                                         _ptr(pos, torch.int32, "pos"), T, K, H,
                                         _ptr(smooth, torch.float32, "smooth"), smooth.shape[0],
@@ -398,6 +463,8 @@ def mep_plan_static_ws(ids: torch.Tensor, R: int, n_keys: int, S: int, K: int, o
         f.restype = ctypes.c_int
     if ids.numel() != R * S * K:
         raise ValueError("ids must hold R*S*K slots")
+    _need(keep is None or keep.numel() == R * S * K, "keep must hold R*S*K flags")
+    _check_plan_buffers(out, R, n_keys, R * S * K)
     rc = f(_ptr(ids, torch.int32, "ids"), _ptr(keep, torch.uint8, "keep"), R, n_keys, S, K, mode,
            keys_per_rank, _ptr(out.pos), _ptr(out.hist), _ptr(out.rank_off), _ptr(out.load),
            _ptr(out.rep_count), _ptr(out.rep_key), _ptr(out.rep_cu), _ptr(out.stats),
