@@ -90,3 +90,36 @@ def test_combine_add_rmsnorm_full_r8():
         _check(bits(x_out[ti:ti + 1]), bits(y_out[ti:ti + 1]), rstd[ti:ti + 1].cpu().numpy(),
                xr, ye, rr, w.H)
     assert mep.mep_get_error() == 0
+
+
+@pytest.mark.parametrize("H", [49152, 49144, 49151])
+def test_combine_add_rmsnorm_largest_rows(H):
+    """The widest rows the fused kernel takes (H = MEP_RMSNORM_MAX_H = 49,152 floats of
+    shared memory), ragged widths just below it (vector and element paths); one past it
+    is refused."""
+    rng = np.random.default_rng(H)
+    T, K, rows, eps = 5, 4, 12, 1e-6
+    g = torch.Generator().manual_seed(H)
+    y = torch.randn(rows, H, generator=g).to(torch.bfloat16)
+    res = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    gam = (1.0 + 0.2 * torch.randn(H, generator=g)).to(torch.bfloat16)
+    pos = rng.integers(0, rows, T * K).astype(np.int32)
+    pos[3] = -1
+    gates = rng.random(T * K).astype(np.float32)
+    x_out = torch.empty((T, H), dtype=torch.bfloat16, device=dev())
+    y_out = torch.empty_like(x_out)
+    rstd = torch.empty(T, dtype=torch.float32, device=dev())
+    mep.mep_combine_add_rmsnorm(y.to(dev()), torch.from_numpy(pos).to(dev()), torch.from_numpy(gates).to(dev()),
+                                K, res.to(dev()), gam.to(dev()), eps, x_out, y_out, rstd)
+    xr, _, ye, rr = oracle.combine_add_rmsnorm(bits(y), pos, gates, K, bits(res), bits(gam), eps)
+    _check(bits(x_out), bits(y_out), rstd.cpu().numpy(), xr, ye, rr, H)
+    assert mep.mep_get_error() == 0
+    H1 = 49153
+    with pytest.raises(mep.MepError) as e:
+        mep.mep_combine_add_rmsnorm(torch.zeros((rows, H1), dtype=torch.bfloat16, device=dev()),
+                                    torch.from_numpy(pos).to(dev()), torch.from_numpy(gates).to(dev()), K,
+                                    torch.zeros((T, H1), dtype=torch.bfloat16, device=dev()),
+                                    torch.zeros(H1, dtype=torch.bfloat16, device=dev()), eps,
+                                    torch.empty((T, H1), dtype=torch.bfloat16, device=dev()),
+                                    torch.empty((T, H1), dtype=torch.bfloat16, device=dev()), rstd)
+    assert e.value.status == 3
