@@ -30,7 +30,7 @@ DERR_TABLE = 0x4
 DERR_MASK = 0x8
 
 STATUS = {0: "MEP_OK", 1: "MEP_ERR_NULLPTR", 2: "MEP_ERR_DTYPE", 3: "MEP_ERR_SHAPE",
-          4: "MEP_ERR_VALUE", 5: "MEP_ERR_WORKSPACE", 6: "MEP_ERR_CUDA"}
+          4: "MEP_ERR_VALUE", 5: "MEP_ERR_WORKSPACE", 6: "MEP_ERR_CUDA", 7: "MEP_ERR_TIMEOUT"}
 
 
 class MepError(RuntimeError):
@@ -92,11 +92,12 @@ def lib() -> ctypes.CDLL:
         L.mep_dedup_plan.argtypes = [P, P, i32, i32, i32, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.mep_expand.argtypes = [P, P, i64, P, i64, i64, i32, P, P, P]
         L.mep_route_host.argtypes = [ctypes.POINTER(_RouteBuffersC), P, P, P, P, P]
+        L.mep_stream_synchronize_timeout.argtypes = [P, i32]
         for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
                   "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8",
                   "mep_combine_add_rmsnorm", "mep_prefetch_plan", "mep_prefetch_weights",
                   "mep_grad_reduce", "mep_dispatch_int8_smooth", "mep_update_expert_ranks",
-                  "mep_dedup_plan", "mep_expand", "mep_route_host"]:
+                  "mep_dedup_plan", "mep_expand", "mep_route_host", "mep_stream_synchronize_timeout"]:
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -147,6 +148,16 @@ def mep_get_error(clear: bool = True) -> int:
     code = ctypes.c_int32(0)
     _ok(lib().mep_get_error(ctypes.byref(code), int(clear)), "mep_get_error")
     return code.value
+
+
+def mep_stream_synchronize_timeout(timeout_ms: int, stream=None) -> bool:
+    """Wait for the stream's work for at most timeout_ms: True when it finished, False
+    on time-out (the work keeps running). Raises MepError on a CUDA error."""
+    rc = lib().mep_stream_synchronize_timeout(_stream(stream), int(timeout_ms))
+    if rc == 7:
+        return False
+    _ok(rc, "mep_stream_synchronize_timeout")
+    return True
 
 
 def mep_histogram(ids: torch.Tensor, n_keys: int, hist: torch.Tensor, stream=None):

@@ -9,7 +9,9 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <chrono>
 #include <mutex>
+#include <thread>
 
 #include "mep.h"
 #include "common.cuh"
@@ -120,6 +122,7 @@ const char *mep_status_string(mep_status_t s)
     case MEP_ERR_VALUE: return "MEP_ERR_VALUE: an argument value is outside its range";
     case MEP_ERR_WORKSPACE: return "MEP_ERR_WORKSPACE: workspace NULL, too small or misaligned";
     case MEP_ERR_CUDA: return "MEP_ERR_CUDA: a CUDA call failed";
+    case MEP_ERR_TIMEOUT: return "MEP_ERR_TIMEOUT: the stream's work did not finish in time";
     }
     return "unknown mep_status_t";
 }
@@ -512,6 +515,25 @@ mep_status_t mep_dispatch_int8_smooth(const uint16_t *x, const int32_t *ids, con
                                                                recv_scale);
     }
     return launched();
+}
+
+mep_status_t mep_stream_synchronize_timeout(mep_stream_t stream, int32_t timeout_ms)
+{
+    if (timeout_ms < 0) return MEP_ERR_VALUE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const auto t0 = std::chrono::steady_clock::now();
+    for (;;) {
+        const cudaError_t e = cudaStreamQuery(s);
+        if (e == cudaSuccess) return MEP_OK;
+        if (e != cudaErrorNotReady) {
+            t_last_cuda_error = (int32_t)e;
+            return MEP_ERR_CUDA;
+        }
+        // "not ready" is no failure: keep it out of the error a later launch checks
+        if (cudaPeekAtLastError() == cudaErrorNotReady) (void)cudaGetLastError();
+        if (std::chrono::steady_clock::now() - t0 >= std::chrono::milliseconds(timeout_ms)) return MEP_ERR_TIMEOUT;
+        std::this_thread::sleep_for(std::chrono::microseconds(50));
+    }
 }
 
 mep_status_t mep_selftest_bounded_wait(int32_t max_polls, int32_t *timed_out, mep_stream_t stream)

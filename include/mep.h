@@ -62,7 +62,8 @@ typedef enum {
     MEP_ERR_SHAPE = 3,     /* a size outside the supported range (cf. 561002) */
     MEP_ERR_VALUE = 4,     /* an argument value outside its range (cf. 561002) */
     MEP_ERR_WORKSPACE = 5, /* workspace NULL, too small or not 256-byte aligned */
-    MEP_ERR_CUDA = 6       /* a CUDA call failed; the CUDA error is in mep_last_cuda_error() */
+    MEP_ERR_CUDA = 6,      /* a CUDA call failed; the CUDA error is in mep_last_cuda_error() */
+    MEP_ERR_TIMEOUT = 7    /* mep_stream_synchronize_timeout: the work did not finish in time */
 } mep_status_t;
 
 /* Bits of the device error word (see mep_get_error). */
@@ -291,6 +292,17 @@ mep_status_t mep_prefetch_weights(const uint16_t *w_home, const int32_t *slot_ex
  */
 mep_status_t mep_grad_reduce(float *grad_home, float *grad_slots, const int32_t *slot_expert,
                              int32_t E, int32_t R, int32_t B, int64_t D, mep_stream_t stream);
+
+/*
+ * Waits for the work enqueued on `stream` with a time limit: the timeout-bounded stream
+ * synchronisation of the aclnnMoeUpdateExpert doc's sample (调用示例,
+ * aclrtSynchronizeStreamWithTimeout(stream, 10000)). Polls the stream about every 50 us.
+ * Returns MEP_OK once the work has finished; MEP_ERR_TIMEOUT when it is still running
+ * after timeout_ms milliseconds (nothing is cancelled: the work keeps running, and a
+ * later call may still see it finish); MEP_ERR_CUDA when the stream reports an error
+ * (the CUDA error is in mep_last_cuda_error()). timeout_ms < 0 is MEP_ERR_VALUE.
+ */
+mep_status_t mep_stream_synchronize_timeout(mep_stream_t stream, int32_t timeout_ms);
 
 /*
  * Diagnostic: checks the failure path of the kernels' bounded waits on this GPU.

@@ -34,8 +34,8 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_status_strings_and_version(L):
     assert L.mep_version() >> 16 == 1
-    for code in range(7):
-        assert L.mep_status_string(code)
+    for code in range(8):
+        assert L.mep_status_string(code) and b"unknown" not in L.mep_status_string(code)
     assert b"unknown" in L.mep_status_string(99)
 
 
@@ -180,3 +180,7 @@ def test_route_host_argument_checks(L):
     assert L.mep_route_host(ctypes.byref(b), P, P, P, P, None) == 3
     b.R, b.ids = 2, None
     assert L.mep_route_host(ctypes.byref(b), P, P, P, P, None) == 1
+
+
+def test_stream_synchronize_timeout_argument_check(L):
+    assert L.mep_stream_synchronize_timeout(None, -1) == 4

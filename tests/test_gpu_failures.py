@@ -58,3 +58,35 @@ def test_selftest_arguments():
     one = torch.zeros(1, dtype=torch.int32, device=dev())
     assert f(0, ctypes.c_void_p(one.data_ptr()), None) == 4
     assert f(10, None, None) == 1
+
+
+def test_stream_synchronize_timeout_gives_up_then_sees_the_work_finish():
+    """A host wait with a time limit on work that outlasts it: the wait reports the
+    time-out, the work goes on, a later wait sees it finish, and the library still
+    routes correctly afterwards."""
+    torch.cuda.set_device(0)
+    mep.mep_get_error(clear=True)
+    f = mep.lib().mep_selftest_bounded_wait
+    f.argtypes = [ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    s = torch.cuda.Stream(dev())
+    flags = torch.full((8,), -1, dtype=torch.int32, device=dev())
+    torch.cuda.synchronize()
+    for i in range(8):       # each launch polls its barrier 2^22 times before giving up
+        assert f(1 << 22, ctypes.c_void_p(flags[i:].data_ptr()), ctypes.c_void_p(s.cuda_stream)) == 0
+    assert mep.mep_stream_synchronize_timeout(1, stream=s) is False
+    assert mep.mep_stream_synchronize_timeout(120000, stream=s) is True
+    assert flags.cpu().tolist() == [1] * 8
+    assert mep.mep_get_error(clear=True) & MEP_DERR_TIMEOUT
+    # an idle stream is done at once, and launches after a time-out still succeed
+    assert mep.mep_stream_synchronize_timeout(0, stream=s) is True
+    rng = np.random.default_rng(6)
+    T, K, H = 20, 2, 64
+    x = torch.randn((T, H), generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    pos = rng.permutation(T * K).astype(np.int32)
+    recv = torch.empty((T * K, H), dtype=torch.bfloat16, device=dev())
+    with torch.cuda.stream(s):
+        mep.mep_dispatch(x.to(dev()), torch.from_numpy(pos).to(dev()), K, recv, stream=s)
+    assert mep.mep_stream_synchronize_timeout(60000, stream=s) is True
+    assert np.array_equal(bits(recv), oracle.dispatch(bits(x), pos, K, T * K))
+    assert mep.mep_get_error() == 0
