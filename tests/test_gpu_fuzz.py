@@ -75,3 +75,64 @@ def test_fuzz_whole_path(seed):
     mep.mep_expand(sent, db.gidx, back)
     assert np.array_equal(bits(back), oracle.dispatch(xb, p.pos, K, N))
     assert mep.mep_get_error() == 0
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_fuzz_mapping_grouped_path(seed):
+    """Random eplb tables, both balance modes, pruning and active prefixes: the mapping of
+    every rank in one launch, the grouped plan over the physical instances, then dispatch
+    and combine with the dropped slots, all compared whole with the oracle."""
+    torch.cuda.set_device(0)
+    mep.mep_get_error(clear=True)
+    rng = np.random.default_rng(20_000 + seed)
+    mode = int(rng.integers(0, 2))
+    ws = int(rng.integers(2, 17))
+    ppr = int(rng.integers(1, 40))
+    n_keys = ws * ppr
+    E = int(rng.integers(1, 300))
+    K = int(rng.integers(1, min(16, E) + 1))
+    F = int(rng.integers(2, min(ws + 1, 6) + 1))
+    BS = int(rng.integers(1, 200))
+    H = int(rng.choice([8, 64, 130, 256]))
+    table = np.full((E, F), -1, np.int32)
+    for e in range(E):
+        c = int(rng.integers(1, F))
+        table[e, 0] = c
+        table[e, 1:1 + c] = rng.choice(n_keys, c, replace=False)
+    T = ws * BS
+    ids = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
+    sc = np.sort(rng.random((T, K)).astype(np.float32), axis=1)[:, ::-1].copy()
+    thr = (rng.random(K) * 0.3).astype(np.float32)
+    active = np.zeros(T, bool)
+    for r in range(ws):
+        active[r * BS: r * BS + int(rng.integers(0, BS + 1))] = True
+    bi = torch.empty((T, K), dtype=torch.int32, device=dev())
+    bm = torch.empty((T, K), dtype=torch.uint8, device=dev())
+    mep.mep_update_expert_ranks(torch.from_numpy(ids).to(dev()), torch.from_numpy(table).to(dev()),
+                                torch.from_numpy(sc).to(dev()), torch.from_numpy(thr).to(dev()),
+                                torch.from_numpy(active.astype(np.uint8)).to(dev()), ws, mode, bi, bm)
+    oi = np.empty_like(ids)
+    om = np.empty(ids.shape, bool)
+    for r in range(ws):
+        sl = slice(r * BS, (r + 1) * BS)
+        oi[sl], om[sl] = oracle.update_expert(ids[sl], table, sc[sl], thr, active[sl], r, ws, mode)
+    assert np.array_equal(bi.cpu().numpy(), oi)
+    assert np.array_equal(bm.cpu().numpy().astype(bool), om)
+
+    pb = mep.PlanBuffers.allocate(ws, n_keys, BS, K, dev())
+    mep.mep_plan(bi.view(-1), ws, n_keys, BS, K, pb, mode=mep.MEP_PLAN_GROUPED, keys_per_rank=ppr,
+                 keep=bm.view(-1))
+    p = oracle.plan_grouped(oi.ravel(), om.ravel(), ws, n_keys, ppr, BS, K)
+    assert_plan_equal(pb, p, ws)
+
+    N = T * K
+    x = torch.randn((T, H), generator=torch.Generator().manual_seed(seed)).to(torch.bfloat16)
+    recv = torch.zeros((N, H), dtype=torch.bfloat16, device=dev())
+    mep.mep_dispatch(x.to(dev()), pb.pos, K, recv)
+    y_ref = oracle.dispatch(bits(x), p.pos, K, N)
+    assert np.array_equal(bits(recv), y_ref)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev())
+    gates = sc.ravel()
+    mep.mep_combine(recv, pb.pos, torch.from_numpy(gates).to(dev()), K, out)
+    assert np.array_equal(bits(out), oracle.combine(y_ref, p.pos, gates, K))
+    assert mep.mep_get_error() == 0
