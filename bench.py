@@ -313,10 +313,11 @@ class Route:
     expand phase (mep_expand) rebuilds the expert-grouped rows on the receiving side.
     """
 
-    def __init__(self, mep, w, dev, epilogue: str = "none", dedup: bool = False):
+    def __init__(self, mep, w, dev, epilogue: str = "none", dedup: bool = False, smooth: bool = False):
         self.mep, self.w, self.dev = mep, w, dev
         self.epilogue = epilogue
         self.dedup = dedup
+        self.smooth = smooth
         self.n_sent = None
         ids, gates = synth.router(w)
         x = synth.hidden(w)
@@ -348,6 +349,10 @@ class Route:
             if w.quant:
                 self.recv = torch.empty((w.N, w.H), dtype=torch.int8, device=dev)
                 self.scale = torch.empty(w.N, dtype=torch.float32, device=dev)
+                if smooth:
+                    # per-expert smoothing scales, one per channel: exp(N(0, 0.25^2)), seeded
+                    g = torch.Generator().manual_seed(w.seed * 1000 + 7)
+                    self.smooth_scales = torch.exp(0.25 * torch.randn((w.E, w.H), generator=g)).to(dev)
             else:
                 self.recv = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
                 self.y = self.recv
@@ -387,7 +392,10 @@ class Route:
         pos, recv, scale = self.pb.pos, self.recv, (self.scale if w.quant else None)
         if self.dedup:
             pos, recv, scale = self.db.dsend, self.sent, self.sent_scale
-        if w.quant:
+        if w.quant and self.smooth:
+            self.mep.mep_dispatch_int8_smooth(self.x, self.ids, pos, w.K, self.smooth_scales, recv, scale,
+                                              stream=s)
+        elif w.quant:
             self.mep.mep_dispatch(self.x, pos, w.K, recv, scale, quant=1, stream=s)
         else:
             self.mep.mep_dispatch(self.x, pos, w.K, recv, stream=s)
@@ -433,6 +441,12 @@ class Route:
             return torch.equal(self.out.float(), ref) and bool(torch.isfinite(self.y_norm.float()).all())
         if w.mapping:
             return bool(torch.isfinite(self.out.float()).all())
+        if w.quant and self.smooth:
+            # codes and scale per slot: every kept slot's row reaches +-127 (or is all zero),
+            # checked on 256 sampled rows; the combine output is finite
+            rows = torch.randint(0, w.N, (256,), generator=torch.Generator().manual_seed(3)).to(self.dev)
+            amax = self.recv[rows].abs().amax(dim=1)
+            return bool(((amax == 127) | (amax == 0)).all()) and bool(torch.isfinite(self.out.float()).all())
         if w.quant:
             first = self.pb.pos.view(w.T, w.K)[:, 0].long()
             y_first = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=self.dev)
@@ -453,6 +467,8 @@ class Route:
             return "k_combine_v8" if w.H % 8 == 0 else "k_combine_scalar"
         if step == "expand":
             return "k_expand_warp" if w.H % 16 == 0 or (not w.quant and w.H % 8 == 0) else "k_expand_bytes"
+        if w.quant and self.smooth:
+            return "k_dispatch_int8_smooth" if w.H % 8 == 0 else "k_dispatch_int8_smooth_scalar"
         if w.quant:
             return "k_dispatch_int8_staged" if w.H % 16 == 0 else "k_dispatch_int8"
         return "k_dispatch_warp" if w.H % 8 == 0 else "k_dispatch_elem"
@@ -477,6 +493,8 @@ class Route:
         n_rows = int(self.pb.stats_dict()["n_kept"])
         if w.quant:
             disp = w.T * row + n_rows * w.H + 4 * n_rows + 4 * w.N
+            if self.smooth:
+                disp += 4 * w.N + 4 * w.E * w.H              # expert ids, smoothing scales
             comb = n_rows * w.H + 4 * n_rows + w.T * row + 8 * w.N
         else:
             disp = w.T * row + n_rows * row + 4 * w.N
@@ -692,7 +710,10 @@ def run_gpu(args, w):
         raise SystemExit("--epilogue applies to the balanced bf16 workloads")
     if args.dedup and w.mapping:
         raise SystemExit("--dedup applies to the balanced workloads")
-    rt = Route(mep, rank_workload(w, rank), dev, args.epilogue, dedup=bool(args.dedup))
+    if args.smooth and not w.quant:
+        raise SystemExit("--smooth applies to the int8 workload")
+    rt = Route(mep, rank_workload(w, rank), dev, args.epilogue, dedup=bool(args.dedup),
+               smooth=bool(args.smooth))
     names = [n for n, _ in rt.phases()]
     stream = torch.cuda.Stream(dev)
     with torch.cuda.stream(stream):
@@ -778,7 +799,7 @@ def run_gpu(args, w):
     ok_device = rt.result_ok()
 
     e2e_steps = max(4, min(args.steps, 20))
-    if not w.mapping and args.epilogue == "none" and not args.dedup:
+    if not w.mapping and args.epilogue == "none" and not args.dedup and not args.smooth:
         e2e_ms, ok_e2e, h2d, d2h, how = e2e_route_host(mep, rt, w, dev, e2e_steps, pg)
     else:
         e2e_ms, ok_e2e, h2d, d2h, how = e2e_pipeline(rt, w, dev, stream, e2e_steps, pg)
@@ -809,7 +830,7 @@ def run_gpu(args, w):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int8" if w.quant else "bf16", "data": "synthetic",
             "config": {"workload": w.name, "R": w.R, "E": w.E, "S": w.S, "K": w.K, "H": w.H,
-                       "epilogue": args.epilogue, "dedup": bool(args.dedup),
+                       "epilogue": args.epilogue, "dedup": bool(args.dedup), "smooth": bool(args.smooth),
                        "token_slots_per_gpu": w.N, "seed": w.seed, "parallelism": f"replicas{world}",
                        "l2": (f"working set {rt.working_set_bytes() / 1e6:.0f} MB "
                               + ("< 2x L2 (126 MB): L2 flushed between steps (256 MB write, "
@@ -859,6 +880,9 @@ def main():
     ap.add_argument("--dedup", type=int, default=0,
                     help="1: send one row per (token, destination rank) and expand on the "
                          "receiving side (mep_dedup_plan, mep_expand)")
+    ap.add_argument("--smooth", type=int, default=0,
+                    help="1 (int8 workload): per-expert smoothing scales before the int8 "
+                         "quantisation, codes and scale per slot (mep_dispatch_int8_smooth)")
     ap.add_argument("--epilogue", default="none", choices=["none", "add_rmsnorm"],
                     help="add_rmsnorm: combine fused with residual add + RMSNorm")
     ap.add_argument("--ffn-dim", type=int, default=0,

@@ -504,7 +504,23 @@ mep_status_t mep_dispatch_int8_smooth(const uint16_t *x, const int32_t *ids, con
     const int64_t H8 = H / 8;
     const bool vec = H % 8 == 0 && aligned(x, 16) && aligned(recv, 8) && aligned(smooth, 16);
     const int64_t per_thread = mep::ceil_div(H8, 256);
-    if (vec && per_thread <= 4) {
+    using smooth_k_t = void (*)(const uint4 *, const int32_t *, const int32_t *, int64_t, int64_t, const float4 *,
+                                int32_t, int64_t, uint2 *, float *);
+    smooth_k_t fused = nullptr;
+    if (vec && per_thread <= 8) {
+        const bool c4 = per_thread <= 4;
+        switch (K) {
+        case 2: fused = c4 ? mep::k_dispatch_int8_smooth_k<2, 4> : mep::k_dispatch_int8_smooth_k<2, 8>; break;
+        case 4: fused = c4 ? mep::k_dispatch_int8_smooth_k<4, 4> : mep::k_dispatch_int8_smooth_k<4, 8>; break;
+        case 8: fused = c4 ? mep::k_dispatch_int8_smooth_k<8, 4> : mep::k_dispatch_int8_smooth_k<8, 8>; break;
+        default: break;
+        }
+    }
+    if (fused) {
+        // the K slots of a token together; the grid is what the GPU holds resident
+        fused<<<resident_grid(fused, 256, T), 256, 0, s>>>((const uint4 *)x, ids, pos, T, H8, (const float4 *)smooth,
+                                                          n_experts, rows, (uint2 *)recv, recv_scale);
+    } else if (vec && per_thread <= 4) {
         mep::k_dispatch_int8_smooth<4><<<grid, 256, 0, s>>>((const uint4 *)x, ids, pos, T, K, H8, (const float4 *)smooth,
                                                            n_experts, rows, (uint2 *)recv, recv_scale);
     } else if (vec && per_thread <= 8) {

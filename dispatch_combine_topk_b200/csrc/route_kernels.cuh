@@ -159,7 +159,8 @@ k_dispatch_warp(const uint4 *__restrict__ x, const int32_t *__restrict__ pos, in
     }
 }
 
-// Quantise 8 fp32 values to int8 with the per-token scale; packed little-endian.
+// Quantise 4 fp32 values to int8 with the per-token scale; packed little-endian:
+// q = clamp(round_half_even(fl(v / scale)), -127, 127), q = 0 when scale == 0.
 __device__ __forceinline__ uint32_t q8x4(float a, float b, float c, float d, float scale)
 {
     auto q = [scale](float v) -> uint32_t {
@@ -171,6 +172,45 @@ __device__ __forceinline__ uint32_t q8x4(float a, float b, float c, float d, flo
         return (uint32_t)(r & 0xff);
     };
     return q(a) | (q(b) << 8) | (q(c) << 16) | (q(d) << 24);
+}
+
+// 1 / scale for q8x8: 0 when scale is 0 (every value of such a row is 0), and -1 when
+// 1 / scale overflows (scale below about 2.9e-39, a subnormal): such rows take the IEEE
+// quotient.
+__device__ __forceinline__ float quant_inv(float scale)
+{
+    if (scale == 0.0f) return 0.0f;
+    const float inv = __frcp_rn(scale);
+    return isinf(inv) ? -1.0f : inv;
+}
+
+// The codes of q8x4 for eight values (two packed words), with inv = quant_inv(scale) and
+// the values of a row whose amax gave scale = fl(amax / 127) (the smoothing dispatches).
+// Each quotient is taken as y = fl(v * inv). |v / scale| < 127.0001 (scale is within one
+// rounding of amax / 127, also when it is subnormal with 1 / scale finite) and inv is
+// within 2^-24 of 1 / scale, so |y - v/scale| < 2^-16 and |y - fl(v/scale)| < 2^-15:
+// unless y lies within 2^-15 of a half-integer, y and the correctly rounded quotient round
+// to the same integer, which is in [-127, 127] without a clamp. y + 1.5 * 2^23 rounds y
+// half-to-even to an integer whose two's-complement low byte is the code. When any of
+// the eight lies that close to a half-integer (about 1 group in 2000), or the row's
+// 1 / scale overflows, all eight take the IEEE quotient of q8x4 instead.
+__device__ __forceinline__ uint2 q8x8(const float (&v)[8], float scale, float inv)
+{
+    constexpr float kShift = 12582912.0f;             // 1.5 * 2^23
+    constexpr float kNearHalf = 0.5f - 0x1p-15f;
+    uint32_t b[8];
+    bool exact = inv < 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        const float y = __fmul_rn(v[j], inv);
+        const float t = __fadd_rn(y, kShift);
+        exact |= fabsf(__fsub_rn(y, __fsub_rn(t, kShift))) >= kNearHalf;
+        b[j] = __float_as_uint(t);
+    }
+    if (exact)
+        return make_uint2(q8x4(v[0], v[1], v[2], v[3], scale), q8x4(v[4], v[5], v[6], v[7], scale));
+    return make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410),
+                      __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410));
 }
 
 // Per-token dynamic int8: one CTA per token, pass 1 reduces amax over the row, pass 2
@@ -920,20 +960,115 @@ k_dispatch_int8_smooth(const uint4 *__restrict__ x, const int32_t *__restrict__ 
                 }
             }
             amax = block_max(amax, red);
-            const float scale = __fdiv_rn(amax, 127.0f);
+            const float scale = __fdiv_rn(amax, 127.0f), inv = quant_inv(scale);
             if (threadIdx.x == 0) recv_scale[p] = scale;
 #pragma unroll
             for (int i = 0; i < kChunks; i++) {
                 const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
-                if (c < H8) {
-                    uint2 q;
-                    q.x = q8x4(xs[i][0], xs[i][1], xs[i][2], xs[i][3], scale);
-                    q.y = q8x4(xs[i][4], xs[i][5], xs[i][6], xs[i][7], scale);
-                    recv[(int64_t)p * H8 + c] = q;
-                }
+                if (c < H8) recv[(int64_t)p * H8 + c] = q8x8(xs[i], scale, inv);
             }
             __syncthreads();                               // red is reused by the next slot
         }
+    }
+}
+
+// The same codes with the K slots of a token taken together (K fixed at KC): pass 1
+// forms, slot by slot, each thread's maximum of |fl(x * smooth[e_k])| and its warp
+// maximum (every smoothing row read once); one block barrier later the K scales follow
+// from the warps' maxima; pass 2 forms each product again (the smoothing rows a second
+// time, from L2) and stores the codes. Two block barriers per token instead of two per
+// slot. Both passes walk the slots in a loop that is not unrolled, which keeps the code
+// short and the registers at 64 (4 CTAs per SM).
+template <int KC, int kChunks>
+__global__ void __launch_bounds__(256)
+k_dispatch_int8_smooth_k(const uint4 *__restrict__ x, const int32_t *__restrict__ ids, const int32_t *__restrict__ pos,
+                         int64_t T, int64_t H8, const float4 *__restrict__ smooth, int32_t n_experts, int64_t rows,
+                         uint2 *__restrict__ recv, float *__restrict__ recv_scale)
+{
+    __shared__ int32_t sp[KC], se[KC];
+    __shared__ float red[8][KC];                      // 256 threads = 8 warps
+    __shared__ float ssc[KC];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        if (threadIdx.x < KC) {
+            int32_t p = pos[t * KC + threadIdx.x];
+            if (p < -1 || (int64_t)p >= rows) {
+                flag_error(MEP_DERR_ROW_RANGE);
+                p = -1;
+            }
+            int32_t e = ids[t * KC + threadIdx.x];
+            if (e < 0 || e >= n_experts) {
+                flag_error(MEP_DERR_KEY_RANGE);
+                e = -1;
+            }
+            sp[threadIdx.x] = p;
+            se[threadIdx.x] = e;
+        }
+        float xr[kChunks][8];
+#pragma unroll
+        for (int i = 0; i < kChunks; i++) {
+            const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
+            if (c < H8) {
+                const uint4 v = x[t * H8 + c];
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    xr[i][2 * j] = bf16lo(w[j]);
+                    xr[i][2 * j + 1] = bf16hi(w[j]);
+                }
+            }
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int k = 0; k < KC; k++) {
+            float amax = 0.0f;
+            const int32_t e = se[k];
+            if (sp[k] >= 0 && e >= 0) {
+                const float4 *srow = smooth + (int64_t)e * H8 * 2;
+#pragma unroll
+                for (int i = 0; i < kChunks; i++) {
+                    const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
+                    if (c < H8) {
+                        const float4 s0 = srow[2 * c], s1 = srow[2 * c + 1];
+                        const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+                        for (int j = 0; j < 8; j++) amax = fmaxf(amax, fabsf(__fmul_rn(xr[i][j], sv[j])));
+                    }
+                }
+            }
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+            if (lane == 0) red[warp][k] = amax;
+        }
+        __syncthreads();
+        if (threadIdx.x < KC) {
+            float m = 0.0f;
+            for (int w = 0; w < 8; w++) m = fmaxf(m, red[w][threadIdx.x]);
+            const float scale = __fdiv_rn(m, 127.0f);
+            ssc[threadIdx.x] = scale;
+            if (sp[threadIdx.x] >= 0 && se[threadIdx.x] >= 0) recv_scale[sp[threadIdx.x]] = scale;
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int k = 0; k < KC; k++) {                    // one slot at a time: a short loop body
+            const int32_t p = sp[k], e = se[k];
+            if (p < 0 || e < 0) continue;
+            const float scale = ssc[k], inv = quant_inv(scale);
+            const float4 *srow = smooth + (int64_t)e * H8 * 2;
+#pragma unroll
+            for (int i = 0; i < kChunks; i++) {
+                const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
+                if (c < H8) {
+                    const float4 s0 = srow[2 * c], s1 = srow[2 * c + 1];
+                    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+                    float xs[8];
+#pragma unroll
+                    for (int j = 0; j < 8; j++) xs[j] = __fmul_rn(xr[i][j], sv[j]);
+                    recv[(int64_t)p * H8 + c] = q8x8(xs, scale, inv);
+                }
+            }
+        }
+        __syncthreads();                                   // sp, se, ssc and red are reused
     }
 }
 

@@ -77,18 +77,24 @@ def test_combine_random_rows_every_k(K):
 
 
 def test_quant_edge_rows():
-    """Zero rows (scale 0), exact ties (scale 1), outliers, denormal-range values."""
+    """Zero rows (scale 0), exact ties (scale 1), outliers, denormal-range values: rows
+    whose scale is subnormal with 1/scale finite or overflowing, and the largest bf16."""
     H, K = 64, 2
-    x = torch.zeros((4, H), dtype=torch.float32)
+    T = 8
+    x = torch.zeros((T, H), dtype=torch.float32)
     x[1, :12] = torch.tensor([127.0, 2.5, 3.5, -2.5, -3.5, 0.5, 1.5, -0.5, 0.0, 126.5, -127.0, 0.25])
     x[2] = torch.linspace(-3000, 3000, H)
     x[3] = torch.linspace(-1e-37, 1e-37, H)
+    x[4] = torch.linspace(-1e-36, 1e-36, H)          # scale subnormal, 1/scale finite
+    x[5] = torch.linspace(-4e-37, 4e-37, H)          # scale close to where 1/scale overflows
+    x[6, :3] = torch.tensor([9.2e-41, -1.84e-40, 0.0])  # bf16 subnormals: 1/scale overflows
+    x[7] = torch.linspace(-1.0, 1.0, H) * 3.38e38    # near the largest finite bf16
     xb16 = x.to(torch.bfloat16)
-    pos = np.arange(4 * K, dtype=np.int32)
-    recv = torch.zeros((4 * K, H), dtype=torch.int8, device=dev())
-    sc = torch.zeros(4 * K, dtype=torch.float32, device=dev())
+    pos = np.arange(T * K, dtype=np.int32)
+    recv = torch.zeros((T * K, H), dtype=torch.int8, device=dev())
+    sc = torch.zeros(T * K, dtype=torch.float32, device=dev())
     mep.mep_dispatch(xb16.to(dev()), torch.from_numpy(pos).to(dev()), K, recv, sc, quant=1)
-    q_ref, s_ref = oracle.dispatch_int8(bits(xb16), pos, K, 4 * K)
+    q_ref, s_ref = oracle.dispatch_int8(bits(xb16), pos, K, T * K)
     assert np.array_equal(recv.cpu().numpy(), q_ref)
     assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
     assert recv[0:2].abs().max().item() == 0 and sc[0].item() == 0.0   # token 0: zero row
