@@ -101,8 +101,8 @@ def kernel_source_hash(name: str) -> str:
 # a quarter or a sixteenth of the tokens per rank routes that share of the rows).
 TRAFFIC = {
     ("k_dispatch_warp", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 998.05e6, "src": "17b1506c97a87d55",
-        "note": "profiles/traffic_dominant_kernels.md: 998.05 MB at S=1024, x4"},
+        "bytes": 4 * 998.22e6, "src": "2bdb2659ae3ccd32",
+        "note": "profiles/traffic_dominant_kernels.md: 998.22 MB at S=1024, x4"},
     ("k_combine_v8", "r8_e64_s4096_k8_h7168"): {
         "bytes": 4 * 1005.70e6, "src": "b8d0144407f8df74",
         "note": "profiles/traffic_dominant_kernels.md: 1005.70 MB at S=1024, x4"},
@@ -116,8 +116,8 @@ TRAFFIC = {
         "bytes": 4 * 1793.81e6, "src": "a12dc9427177590d",
         "note": "profiles/dedup_r8.md: 1793.81 MB at S=1024, x4 (--dedup 1)"},
     ("k_dispatch_warp", "skew_r64_e512_s2048_k8_h4096"): {
-        "bytes": 4 * 2357.84e6, "src": "17b1506c97a87d55",
-        "note": "profiles/traffic_dominant_kernels.md: 2357.84 MB at S=512, x4"},
+        "bytes": 4 * 2357.51e6, "src": "2bdb2659ae3ccd32",
+        "note": "profiles/traffic_dominant_kernels.md: 2357.51 MB at S=512, x4"},
     ("k_combine_v8", "skew_r64_e512_s2048_k8_h4096"): {
         "bytes": 4 * 2364.80e6, "src": "b8d0144407f8df74",
         "note": "profiles/traffic_dominant_kernels.md: 2364.80 MB at S=512, x4"},

@@ -279,8 +279,8 @@ mep_status_t mep_dispatch(const uint16_t *x, const int32_t *pos, int64_t T, int3
     const int grid = token_grid(T, 8);
     if (quant == 0) {
         if (H % 8 == 0 && aligned(x, 16) && aligned(recv, 16)) {
-            // one warp per token, 8 warps per CTA, up to 64 CTAs per SM in waves
-            const int64_t ctas = mep::ceil_div(T, 8);
+            // one warp per half token row, 8 warps per CTA, up to 64 CTAs per SM in waves
+            const int64_t ctas = mep::ceil_div(2 * T, 8);
             const int64_t cap = (int64_t)sm_count() * 64;
             mep::k_dispatch_warp<<<(int)(ctas < cap ? ctas : cap), 256, 0, s>>>((const uint4 *)x, pos, T, K, H / 8,
                                                                               rows, (uint4 *)recv);

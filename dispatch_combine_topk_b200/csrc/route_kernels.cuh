@@ -111,7 +111,8 @@ k_dispatch_elem(const uint16_t *__restrict__ x, const int32_t *__restrict__ pos,
     }
 }
 
-// bf16 copy, one warp per token (the default path).
+// bf16 copy, one warp per half token row (the default path): work item i is row half
+// i % 2 of token i / 2, so the last wave of warps is half as coarse as whole rows.
 //
 // A warp reads its token's K row indices once (lane k holds slot k, broadcast with
 // shuffles), then walks the row in 16-byte chunks, kUnroll chunks per lane in flight,
@@ -130,7 +131,9 @@ k_dispatch_warp(const uint4 *__restrict__ x, const int32_t *__restrict__ pos, in
 {
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+    const int64_t per = (H8 + 1) / 2;
+    for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < 2 * T; it += nwarps) {
+        const int64_t t = it >> 1;
         int32_t mine = -1;
         if (lane < K) {
             mine = pos[t * K + lane];
@@ -140,20 +143,21 @@ k_dispatch_warp(const uint4 *__restrict__ x, const int32_t *__restrict__ pos, in
             }
         }
         const uint4 *src = x + t * H8;
+        const int64_t lo = (it & 1) * per, hi = (it & 1) ? H8 : per;
         // warp-uniform trip count: every lane reaches the shuffles below
-        for (int64_t base = 0; base < H8; base += 32 * kDispatchUnroll) {
+        for (int64_t base = lo; base < hi; base += 32 * kDispatchUnroll) {
             const int64_t c0 = base + lane;
             uint4 v[kDispatchUnroll];
 #pragma unroll
             for (int u = 0; u < kDispatchUnroll; u++)
-                if (c0 + 32 * u < H8) v[u] = ld_stream(src + c0 + 32 * u);
+                if (c0 + 32 * u < hi) v[u] = ld_stream(src + c0 + 32 * u);
             for (int k = 0; k < K; k++) {
                 const int32_t p = __shfl_sync(0xffffffffu, mine, k);
                 if (p < 0) continue;
                 uint4 *dst = recv + (int64_t)p * H8;
 #pragma unroll
                 for (int u = 0; u < kDispatchUnroll; u++)
-                    if (c0 + 32 * u < H8) st_v4(dst + c0 + 32 * u, v[u]);
+                    if (c0 + 32 * u < hi) st_v4(dst + c0 + 32 * u, v[u]);
             }
         }
     }
