@@ -217,6 +217,37 @@ __device__ __forceinline__ uint2 q8x8(const float (&v)[8], float scale, float in
                       __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410));
 }
 
+// q8x8 with the products and the rounding arithmetic on pairs of values (packed f32x2,
+// each half rounded on its own): xs = fl(x * s), y = fl(xs * inv), t = fl(y + 1.5*2^23),
+// r = t - 1.5*2^23, d = y - r. No product here feeds a sum whose rounding matters: had a
+// pair of them been fused, t would round the exact xs * inv, which is still within the
+// bound, and d only decides whether to take the IEEE quotient.
+__device__ __forceinline__ uint2 q8x8_packed(const float (&x)[8], const float (&s)[8], float scale, float inv)
+{
+    const float2 kShift = make_float2(12582912.0f, 12582912.0f), kNegShift = make_float2(-12582912.0f, -12582912.0f);
+    const float2 inv2 = make_float2(inv, inv);
+    float xs[8];
+    uint32_t b[8];
+    float dmax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const float2 v = mul2_rn(make_float2(x[2 * j], x[2 * j + 1]), make_float2(s[2 * j], s[2 * j + 1]));
+        const float2 y = mul2_rn(v, inv2);
+        const float2 t = add2_rn(y, kShift);
+        const float2 r = add2_rn(t, kNegShift);
+        const float2 d = add2_rn(y, make_float2(-r.x, -r.y));
+        dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+        xs[2 * j] = v.x;
+        xs[2 * j + 1] = v.y;
+        b[2 * j] = __float_as_uint(t.x);
+        b[2 * j + 1] = __float_as_uint(t.y);
+    }
+    if (inv < 0.0f || dmax >= 0.5f - 0x1p-15f)
+        return make_uint2(q8x4(xs[0], xs[1], xs[2], xs[3], scale), q8x4(xs[4], xs[5], xs[6], xs[7], scale));
+    return make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410),
+                      __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410));
+}
+
 // Per-token dynamic int8: one CTA per token, pass 1 reduces amax over the row, pass 2
 // re-reads the row (from L1/L2) and writes the K copies of the codes and the scale.
 // Needs H % 8 == 0 and 16-byte aligned x, 8-byte aligned recv.
@@ -1036,7 +1067,11 @@ k_dispatch_int8_smooth_k(const uint4 *__restrict__ x, const int32_t *__restrict_
                         const float4 s0 = srow[2 * c], s1 = srow[2 * c + 1];
                         const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-                        for (int j = 0; j < 8; j++) amax = fmaxf(amax, fabsf(__fmul_rn(xr[i][j], sv[j])));
+                        for (int j = 0; j < 4; j++) {
+                            const float2 v = mul2_rn(make_float2(xr[i][2 * j], xr[i][2 * j + 1]),
+                                                     make_float2(sv[2 * j], sv[2 * j + 1]));
+                            amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
+                        }
                     }
                 }
             }
@@ -1065,10 +1100,7 @@ k_dispatch_int8_smooth_k(const uint4 *__restrict__ x, const int32_t *__restrict_
                 if (c < H8) {
                     const float4 s0 = srow[2 * c], s1 = srow[2 * c + 1];
                     const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-                    float xs[8];
-#pragma unroll
-                    for (int j = 0; j < 8; j++) xs[j] = __fmul_rn(xr[i][j], sv[j]);
-                    recv[(int64_t)p * H8 + c] = q8x8(xs, scale, inv);
+                    recv[(int64_t)p * H8 + c] = q8x8_packed(xr[i], sv, scale, inv);
                 }
             }
         }
