@@ -125,3 +125,39 @@ def test_generated_mapping_workload_properties():
             assert not mask[~act].any()
             # prefix property: once a slot is pruned every later slot is too
             assert np.all(np.diff(mask.astype(np.int8), axis=1) <= 0)
+
+
+def test_grouped_receive_rows_within_the_setup_docs_bound():
+    """The receive buffer bound of the aclnnMoeDistributeDispatchSetup doc (约束说明 5, A):
+    a rank may receive at most BS * world_size * min(experts on the rank, K) token-slots,
+    since every source rank sends BS tokens and a token's K distinct experts put at most
+    min(local instances, K) of its slots on one rank. The grouped plan after the mapping
+    keeps within it on the mapping workload in both modes, and under random tables with
+    every token active and nothing pruned."""
+    w = synth.get("map")
+    ids, gates = synth.router(w)
+    table, thr, active = synth.mapping_inputs(w)
+    n_keys = w.R * w.place_per_rank
+    bound = w.S * w.R * min(w.place_per_rank, w.K)
+    for mode in (0, 1):
+        keys = np.empty_like(ids)
+        keep = np.empty(ids.shape, bool)
+        for r in range(w.R):
+            sl = slice(r * w.S, (r + 1) * w.S)
+            keys[sl], keep[sl] = oracle.update_expert(ids[sl], table, gates[sl], thr, active[sl], r, w.R, mode)
+        p = oracle.plan_grouped(keys.ravel(), keep.ravel(), w.R, n_keys, w.place_per_rank, w.S, w.K)
+        assert np.diff(p.rank_off).max() <= bound
+    rng = np.random.default_rng(11)
+    for _ in range(20):
+        ws, kpr, BS = int(rng.integers(2, 6)), int(rng.integers(1, 4)), int(rng.integers(1, 30))
+        E = ws * kpr
+        K = int(rng.integers(1, min(E, 8) + 1))
+        # each expert one instance, a random permutation of the physical slots
+        table = np.full((E, 2), -1, np.int32)
+        table[:, 0] = 1
+        table[:, 1] = rng.permutation(E)
+        ids = np.stack([rng.choice(E, K, replace=False) for _ in range(ws * BS)]).astype(np.int32)
+        keys = np.concatenate([oracle.update_expert(ids[r * BS:(r + 1) * BS], table, None, None, None, r, ws, 0)[0]
+                               for r in range(ws)])
+        p = oracle.plan_grouped(keys.ravel(), None, ws, E, kpr, BS, K)
+        assert np.diff(p.rank_off).max() <= BS * ws * min(kpr, K)
