@@ -18,8 +18,9 @@
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
  *    stream) and never synchronise the host, so a chain plan -> dispatch -> combine
  *    needs no host round trip (MoonEP's static shapes remove per-layer host syncs:
- *    twodots.gr article on MoonEP, static-shapes paragraph). Only mep_get_error
- *    synchronises. mep_histogram, mep_plan, mep_update_expert, mep_update_expert_ranks,
+ *    twodots.gr article on MoonEP, static-shapes paragraph). Only mep_get_error and
+ *    mep_stream_synchronize_timeout wait for the device (and mep_route_host's copies
+ *    when its host buffers are pageable). mep_histogram, mep_plan, mep_update_expert, mep_update_expert_ranks,
  *    mep_dedup_plan, mep_dispatch, mep_expand, mep_dispatch_int8_smooth, mep_dequantize,
  *    mep_combine, mep_combine_int8,
  *    mep_combine_add_rmsnorm, mep_prefetch_plan, mep_prefetch_weights and mep_grad_reduce
