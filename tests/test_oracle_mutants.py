@@ -106,6 +106,29 @@ MUTANTS = [
      "        for (int64_t g = T - 1; g >= 0; g--) {\n            int64_t first = -1;",
      ["test_oracle_dedup.test_dedup_hand_example",
       ("test_oracle_dedup.test_dedup_balanced_plans", {"R": 2, "E": 4, "S": 3, "K": 2})]),
+    ("rmsnorm without eps",
+     "        double r = 1.0 / sqrt(ss / (double)H + eps);",
+     "        double r = 1.0 / sqrt(ss / (double)H);",
+     ["test_oracle_rmsnorm.test_rmsnorm_constant_rows_closed_form",
+      "test_oracle_rmsnorm.test_rmsnorm_matches_torch_float64"]),
+    ("rmsnorm mean over H - 1",
+     "        double r = 1.0 / sqrt(ss / (double)H + eps);",
+     "        double r = 1.0 / sqrt(ss / (double)(H - 1) + eps);",
+     ["test_oracle_rmsnorm.test_rmsnorm_constant_rows_closed_form",
+      "test_oracle_rmsnorm.test_rmsnorm_matches_torch_float64"]),
+    ("rmsnorm without gamma",
+     "            double v = x[h] * r * (double)bf16_bits_to_float(gamma[h]);",
+     "            double v = x[h] * r;",
+     ["test_oracle_rmsnorm.test_rmsnorm_matches_torch_float64"]),
+    ("rmsnorm drops the residual from x",
+     "            x[h] = (double)bf16_bits_to_float(c[g * H + h]) + (double)bf16_bits_to_float(residual[g * H + h]);",
+     "            x[h] = (double)bf16_bits_to_float(c[g * H + h]);",
+     ["test_oracle_rmsnorm.test_rmsnorm_dropped_token_is_the_residual",
+      "test_oracle_rmsnorm.test_rmsnorm_matches_torch_float64"]),
+    ("binary64 to bf16 through binary32 (two roundings)",
+     "        r = ldexp(nearbyint(ldexp(m, 8)), e - 8);   /* 8 significant bits */",
+     "        r = ldexp(nearbyint(ldexp((double)(float)m, 8)), e - 8);",
+     ["test_oracle_rmsnorm.test_double_to_bf16_single_rounding"]),
     ("expansion copies the first row's scale",
      "if (src_scale && dst_scale) dst_scale[p] = src_scale[u];",
      "if (src_scale && dst_scale) dst_scale[p] = src_scale[0];",
