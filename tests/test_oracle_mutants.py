@@ -106,6 +106,22 @@ MUTANTS = [
      "        for (int64_t g = T - 1; g >= 0; g--) {\n            int64_t first = -1;",
      ["test_oracle_dedup.test_dedup_hand_example",
       ("test_oracle_dedup.test_dedup_balanced_plans", {"R": 2, "E": 4, "S": 3, "K": 2})]),
+    ("pruning ignores the active mask",
+     "                out_mask[i * K + k] = (uint8_t)(act && !(scales[i * K + k] < v));",
+     "                out_mask[i * K + k] = (uint8_t)(!(scales[i * K + k] < v));",
+     ["test_oracle_update_expert.test_pruning_hand_example",
+      "test_oracle_update_expert.test_generated_mapping_workload_properties"]),
+    ("grouped plan ranks instances by modulo",
+     "                sl[m].rank = key / keys_per_rank;", "                sl[m].rank = key % R;",
+     ["test_oracle_plan.test_grouped_plan_packs_kept_slots_by_instance"]),
+    ("dequantisation truncates to bf16",
+     "            y[r * H + h] = orc_float_to_bf16(v);",
+     "            { uint32_t u; memcpy(&u, &v, sizeof u); y[r * H + h] = (uint16_t)(u >> 16); }",
+     ["test_oracle_numerics.test_dequantize_is_rounded_product"]),
+    ("prefetch copies the first expert into every slot",
+     "        for (int64_t i = 0; i < D; i++) w_slots[s * D + i] = w_home[(int64_t)e * D + i];",
+     "        for (int64_t i = 0; i < D; i++) w_slots[s * D + i] = w_home[i];",
+     [("test_oracle_prefetch.test_prefetch_properties", {"name": "r8", "B": 8})]),
     ("rmsnorm without eps",
      "        double r = 1.0 / sqrt(ss / (double)H + eps);",
      "        double r = 1.0 / sqrt(ss / (double)H);",
