@@ -9,6 +9,7 @@ import oracle
 import synth
 from gpu_helpers import assert_plan_equal, dev, gpu_plan_balanced, gpu_plan_grouped
 from plan_checks import check_balanced_plan
+from dedup_checks import check_dedup
 
 pytestmark = pytest.mark.gpu
 
@@ -214,3 +215,26 @@ def test_grouped_plan_all_dropped_and_ragged():
                  np.ones(R * S * K, np.uint8)]:
         pb = gpu_plan_grouped(keys, keep, R, R * kpr, kpr, S, K)
         assert_plan_equal(pb, oracle.plan_grouped(keys, keep, R, R * kpr, kpr, S, K), R)
+
+
+def test_plan_and_dedup_at_the_largest_rank_and_key_counts():
+    """R = n_keys = MEP_MAX_KEYS (4096 ranks of one expert each): the plan and its replica
+    tables bit for bit against the oracle, the dedup encoding against every property an
+    encoding of that plan must have (the oracle's rank-by-rank construction is too slow at
+    4096 ranks); and one rank past the limit is refused."""
+    R = E = 4096
+    S, K = 2, 2
+    rng = np.random.default_rng(4096)
+    ids = np.stack([rng.choice(E, K, replace=False) for _ in range(R * S)]).astype(np.int32).ravel()
+    pb = gpu_plan_balanced(ids, R, E, S, K)
+    p = oracle.plan_balanced(ids, R, E, S, K)
+    assert_plan_equal(pb, p, R)
+    db = mep.DedupBuffers.allocate(R, S, K, dev())
+    mep.mep_dedup_plan(pb.pos, pb.rank_off, R, S, K, db)
+    check_dedup(p.pos, K, p.rank_off, oracle.Dedup(*[getattr(db, n).cpu().numpy() for n in
+                                                     ("dsend", "dpos", "drank_off", "dtok", "gidx")]))
+    assert mep.mep_get_error() == 0
+    with pytest.raises(mep.MepError) as e:
+        mep.mep_plan(torch.zeros((R + 1) * S * K, dtype=torch.int32, device=dev()), R + 1, E + 1, S, K,
+                     mep.PlanBuffers.allocate(R + 1, E + 1, S, K, dev()))
+    assert e.value.status == 3
