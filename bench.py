@@ -248,8 +248,8 @@ def oracle_sample(w, S_sample):
 def cpu_sample_S(w, div: int) -> int:
     """Tokens per rank of the CPU sample: S/div, and small enough that the host copy of
     the receive rows stays under 2^31 elements."""
-    cap = max(1, -(-w.N * w.H // (1 << 31)))
-    return max(1, w.S // max(div, cap))
+    fit = ((1 << 31) - 1) // (w.R * w.K * w.H)
+    return max(1, min(w.S // max(div, 1), fit))
 
 
 def run_reference(args, w):
