@@ -421,7 +421,8 @@ mep_status_t mep_update_expert_ranks(const int32_t *expert_ids, const int32_t *e
  *                recv[pos[n], :] = q (int8), recv_scale[pos[n]] = scale.
  * x bf16 [T, H]; pos int32 [T*K] (-1 = dropped); recv bf16 or int8 [rows, H];
  * recv_scale fp32 [rows] (quant == 1 only, else ignored). Rows no slot points at are
- * left untouched.
+ * left untouched. For quant == 1 the row must be finite: a NaN or infinity in it leaves
+ * that row's codes unspecified.
  * Errors: NULL pointer; T < 0, K outside [1, MEP_MAX_K], H < 1, rows < 0,
  * T*K >= 2^31 (MEP_ERR_SHAPE); quant outside {0,1} (MEP_ERR_DTYPE). A pos outside
  * [-1, rows) is skipped and sets MEP_DERR_ROW_RANGE.
