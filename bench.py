@@ -527,14 +527,11 @@ def dedup_summary(rt):
 
 def maxvio(rt):
     """maxvio = max load / mean load - 1: over ranks before the plan (experts on their
-    home ranks) and after it (the rows each rank receives), and over experts."""
-    w, st = rt.w, rt.pb.stats_dict()
-    mean_rank = w.S * w.K
-    n_keys = rt.pb.hist.numel()
-    out = {"rank_before": st["max_load"] / mean_rank - 1.0,
-           "rank_after": st["max_chunk"] / mean_rank - 1.0,
-           "expert": st["max_hist"] / (st["n_kept"] / n_keys) - 1.0 if st["n_kept"] else None}
-    return out
+    home ranks) and after it (the rows each rank receives), and over experts, from the
+    plan summary through the library's mep_maxvio."""
+    w = rt.w
+    out = rt.mep.mep_maxvio(rt.pb.stats, w.S, w.K, rt.pb.hist.numel())
+    return {k: (None if v != v else v) for k, v in out.items()}     # NaN (no slot kept) -> null
 
 
 def weight_side(mep, rt, args, dev, stream):

@@ -93,11 +93,13 @@ def lib() -> ctypes.CDLL:
         L.mep_expand.argtypes = [P, P, i64, P, i64, i64, i32, P, P, P]
         L.mep_route_host.argtypes = [ctypes.POINTER(_RouteBuffersC), P, P, P, P, P]
         L.mep_stream_synchronize_timeout.argtypes = [P, i32]
+        L.mep_maxvio.argtypes = [P, i32, i32, i32, P, P, P]
         for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
                   "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8",
                   "mep_combine_add_rmsnorm", "mep_prefetch_plan", "mep_prefetch_weights",
                   "mep_grad_reduce", "mep_dispatch_int8_smooth", "mep_update_expert_ranks",
-                  "mep_dedup_plan", "mep_expand", "mep_route_host", "mep_stream_synchronize_timeout"]:
+                  "mep_dedup_plan", "mep_expand", "mep_route_host", "mep_stream_synchronize_timeout",
+                  "mep_maxvio"]:
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -214,6 +216,17 @@ def mep_plan(ids: torch.Tensor, R: int, n_keys: int, S: int, K: int, out: PlanBu
                         _ptr(out.workspace), out.workspace.numel(), _stream(stream))
     _ok(rc, "mep_plan")
     return out
+
+
+def mep_maxvio(stats, S: int, K: int, n_keys: int) -> dict:
+    """maxvio before and after the plan, and over experts, from a plan summary (the
+    PlanBuffers' stats tensor on any device, or 8 ints); host arithmetic only."""
+    vals = (stats.tolist() if hasattr(stats, "tolist") else list(stats))[:8]
+    buf = (ctypes.c_int32 * 8)(*[int(v) for v in vals])
+    out = [ctypes.c_double(0.0) for _ in range(3)]
+    _ok(lib().mep_maxvio(ctypes.cast(buf, ctypes.c_void_p), S, K, n_keys, *[ctypes.byref(o) for o in out]),
+        "mep_maxvio")
+    return {"rank_before": out[0].value, "rank_after": out[1].value, "expert": out[2].value}
 
 
 def mep_dedup_workspace_size(R: int, S: int, K: int) -> int:

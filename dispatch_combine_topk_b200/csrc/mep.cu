@@ -10,6 +10,7 @@
 #include <stdio.h>
 
 #include <chrono>
+#include <cmath>
 #include <mutex>
 #include <thread>
 
@@ -668,6 +669,22 @@ mep_status_t mep_route_host(const mep_route_buffers_t *b, const int32_t *ids_h, 
                               b->out, stream);
     if (st != MEP_OK) return st;
     return copy(out_h, b->out, sizeof(uint16_t) * (size_t)(T * b->H), cudaMemcpyDeviceToHost);
+}
+
+// ------------------------------------------------------------ maxvio (host only)
+
+mep_status_t mep_maxvio(const mep_plan_stats_t *stats, int32_t S, int32_t K, int32_t n_keys,
+                        double *rank_before, double *rank_after, double *expert)
+{
+    if (!stats) return MEP_ERR_NULLPTR;
+    if (S < 1 || K < 1 || n_keys < 1) return MEP_ERR_SHAPE;
+    const double mean_rank = (double)S * (double)K;
+    if (rank_before) *rank_before = (double)stats->max_load / mean_rank - 1.0;
+    if (rank_after) *rank_after = (double)stats->max_chunk / mean_rank - 1.0;
+    if (expert)
+        *expert = stats->n_kept > 0 ? (double)stats->max_hist / ((double)stats->n_kept / (double)n_keys) - 1.0
+                                    : std::nan("");
+    return MEP_OK;
 }
 
 }  // extern "C"

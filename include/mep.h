@@ -84,7 +84,7 @@ typedef enum {
 
 /* Plan summary, written by mep_plan to device memory. All counts are exact integers;
  * maxvio = max_load / (S*K) - 1 (before planning) and max_chunk / (S*K) - 1 (after)
- * are left to the caller so that they are computed once, in double precision. */
+ * follow from it on the host, in double precision (mep_maxvio). */
 typedef struct {
     int32_t max_load;   /* max over ranks of the rows its home experts would receive */
     int32_t max_chunk;  /* max over ranks of the rows it receives under the plan */
@@ -95,6 +95,18 @@ typedef struct {
     int32_t n_ranks_used; /* ranks that receive at least one row */
     int32_t reserved;
 } mep_plan_stats_t;
+
+/*
+ * maxvio of a plan (MoonEP article, maxvio paragraph: the maximum load over the mean
+ * load, minus one), from the plan summary copied to host memory:
+ *   rank_before = max_load / (S*K) - 1    (every expert on its home rank)
+ *   rank_after  = max_chunk / (S*K) - 1   (the rows each rank receives; 0 when balanced)
+ *   expert      = max_hist / (n_kept / n_keys) - 1   (NaN when n_kept is 0)
+ * in double precision. Host only: no device call, no stream. Any output may be NULL.
+ * Errors: NULL stats (MEP_ERR_NULLPTR); S, K or n_keys below 1 (MEP_ERR_SHAPE).
+ */
+mep_status_t mep_maxvio(const mep_plan_stats_t *stats, int32_t S, int32_t K, int32_t n_keys,
+                        double *rank_before, double *rank_after, double *expert);
 
 /* Library version, (major << 16) | minor. */
 int32_t mep_version(void);

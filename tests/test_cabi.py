@@ -184,3 +184,33 @@ def test_route_host_argument_checks(L):
 
 def test_stream_synchronize_timeout_argument_check(L):
     assert L.mep_stream_synchronize_timeout(None, -1) == 4
+
+
+def test_maxvio_from_a_plan_summary(L, golden_dir):
+    """mep_maxvio is host arithmetic: on the plan hand example it gives the golden's
+    maxvio before (0.5) and after (0.0); on every balanced workload's oracle plan the
+    after-value is 0; an empty plan has no expert-level value; bad sizes are refused."""
+    import json
+    import math
+    import dispatch_combine_topk_b200 as mep
+    import oracle
+    import synth
+    g = json.load(open(os.path.join(golden_dir, "plan_hand_r2_e4_s2_k2.json")))
+    R, E, S, K = g["R"], g["E"], g["S"], g["K"]
+    p = oracle.plan_balanced(__import__("numpy").array(g["ids"], "int32").ravel(), R, E, S, K)
+    st = [p.max_load, p.max_chunk, p.redundant, p.prefetched, p.n_kept, p.max_hist, 0, 0]
+    m = mep.mep_maxvio(st, S, K, E)
+    assert m["rank_before"] == g["expected"]["maxvio_before"]
+    assert m["rank_after"] == g["expected"]["maxvio_after"]
+    assert m["expert"] == max(g["expected"]["hist"]) / (R * S * K / E) - 1.0
+    for name in ("tiny", "r8"):
+        w = synth.get(name)
+        ids, _ = synth.router(w)
+        p = oracle.plan_balanced(ids, w.R, w.E, w.S, w.K)
+        st = [p.max_load, p.max_chunk, p.redundant, p.prefetched, p.n_kept, p.max_hist, 0, 0]
+        m = mep.mep_maxvio(st, w.S, w.K, w.E)
+        assert m["rank_after"] == 0.0 and m["rank_before"] == p.maxvio_before(w.S, w.K)
+    assert math.isnan(mep.mep_maxvio([0] * 8, 2, 2, 4)["expert"])
+    assert L.mep_maxvio(None, 2, 2, 4, None, None, None) == 1
+    buf = (ctypes.c_int32 * 8)()
+    assert L.mep_maxvio(ctypes.cast(buf, ctypes.c_void_p), 0, 2, 4, None, None, None) == 3
