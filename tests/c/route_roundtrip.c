@@ -95,6 +95,9 @@ int main(void)
     }
     for (int r = 0; r < R; r++) CHECK(count[r] == S * K && rank_off[r] == r * S * K);
     CHECK(stats.max_chunk == S * K && stats.n_kept == N && stats.redundant <= R - 1);
+    double mv_before = -9.0, mv_after = -9.0;
+    CHECK(mep_maxvio(&stats, S, K, E, &mv_before, &mv_after, NULL) == MEP_OK);
+    CHECK(mv_after == 0.0 && mv_before == (double)stats.max_load / (double)(S * K) - 1.0);
     CHECK(memcmp(out, x, sizeof(uint16_t) * T * H) == 0);
     /* the same round trip from host memory in one call (pageable buffers: the copies
        are synchronous, the kernels still run on the stream) */
