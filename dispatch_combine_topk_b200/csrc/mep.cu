@@ -9,6 +9,7 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <atomic>
 #include <chrono>
 #include <cmath>
 #include <mutex>
@@ -699,7 +700,8 @@ mep_status_t mep_maxvio(const mep_plan_stats_t *stats, int32_t S, int32_t K, int
 static __device__ __align__(256) unsigned char g_plan_static_ws[MEP_PLAN_STATIC_WS_BYTES];
 
 namespace {
-void *g_plan_static_ws_addr[kMaxDevices];   // device address of g_plan_static_ws, per device
+// device address of g_plan_static_ws, per device (host threads may look it up at once)
+std::atomic<void *> g_plan_static_ws_addr[kMaxDevices];
 }
 
 extern "C" mep_status_t mep_plan_static_ws(const int32_t *ids, const uint8_t *keep, int32_t R,
@@ -721,15 +723,15 @@ extern "C" mep_status_t mep_plan_static_ws(const int32_t *ids, const uint8_t *ke
         return MEP_ERR_CUDA;
     }
     if (dev < 0 || dev >= kMaxDevices) return MEP_ERR_VALUE;
-    void *ws = g_plan_static_ws_addr[dev];
+    void *ws = g_plan_static_ws_addr[dev].load(std::memory_order_acquire);
     if (!ws) {
-        // once per device, with that device current
+        // with that device current; threads that race here all find the same address
         e = cudaGetSymbolAddress(&ws, g_plan_static_ws);
         if (e != cudaSuccess || !ws) {
             t_last_cuda_error = (int32_t)(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
             return MEP_ERR_CUDA;
         }
-        g_plan_static_ws_addr[dev] = ws;
+        g_plan_static_ws_addr[dev].store(ws, std::memory_order_release);
     }
     return mep_plan(ids, keep, R, n_keys, S, K, mode, keys_per_rank, pos, hist, rank_off, load,
                     rep_count, rep_key, rep_cu, stats, ws, (size_t)MEP_PLAN_STATIC_WS_BYTES, stream);
