@@ -47,3 +47,30 @@ def test_mapping_table_is_well_formed():
     assert np.bincount(ids // w.place_per_rank).tolist() == [w.place_per_rank] * w.R
     assert thr.shape == (w.K,) and np.all((thr >= 0) & (thr < 0.1))
     assert active.reshape(w.R, w.S)[:, : w.n_active].all() and not active.reshape(w.R, w.S)[:, w.n_active:].any()
+
+
+def test_router_follows_the_zipf_bias():
+    """Experts with a larger Zipf bias receive more slots: the per-expert counts rank like
+    the bias (Spearman correlation), the first expert leads when there is no
+    permutation, and a permuted workload does not keep the identity order."""
+    for name, S in [("tiny", 128), ("r8", 256), ("int8", 256)]:
+        w = synth.scaled(synth.get(name), S=S)
+        ids, _ = synth.router(w)
+        h = np.bincount(ids.ravel(), minlength=w.E).astype(np.float64)
+        bias, rank = synth.zipf_bias(w)
+        rh = np.argsort(np.argsort(-h))
+        rb = np.argsort(np.argsort(-bias))
+        rho = np.corrcoef(rh, rb)[0, 1]
+        assert rho > 0.8, (name, rho)
+        if not w.permute:
+            assert h.argmax() == 0
+        else:
+            assert not np.array_equal(rank, np.arange(w.E))
+
+
+def test_hidden_rows_are_standard_normal_in_bf16():
+    w = synth.scaled(synth.get("r8"), S=8, H=1024)
+    x = synth.hidden(w).float()
+    assert abs(x.mean().item()) < 0.01 and abs(x.std().item() - 1.0) < 0.01
+    # every value is a bf16 number (rounded once from the fp32 draw)
+    assert torch.equal(x.to(torch.bfloat16).float(), x)
