@@ -163,6 +163,7 @@ def mep_stream_synchronize_timeout(timeout_ms: int, stream=None) -> bool:
 
 
 def mep_histogram(ids: torch.Tensor, n_keys: int, hist: torch.Tensor, stream=None):
+    """hist[e] = slots of ids equal to e (int32 [n_keys]); ids int32, any length."""
     _need(_n(hist) >= n_keys, "hist must hold n_keys counts")
     _ok(lib().mep_histogram(_ptr(ids, torch.int32, "ids"), ids.numel(), n_keys,
                             _ptr(hist, torch.int32, "hist"), _stream(stream)), "mep_histogram")
@@ -170,6 +171,7 @@ def mep_histogram(ids: torch.Tensor, n_keys: int, hist: torch.Tensor, stream=Non
 
 
 def mep_plan_workspace_size(R: int, n_keys: int, S: int, K: int) -> int:
+    """Bytes of scratch mep_plan needs for this shape (PlanBuffers.allocate uses it)."""
     return int(lib().mep_plan_workspace_size(R, n_keys, S, K))
 
 
@@ -205,6 +207,8 @@ class PlanBuffers:
 def mep_plan(ids: torch.Tensor, R: int, n_keys: int, S: int, K: int, out: PlanBuffers,
              mode: int = MEP_PLAN_BALANCED, keys_per_rank: int = 0,
              keep: Optional[torch.Tensor] = None, stream=None) -> PlanBuffers:
+    """The placement plan of R*S*K slots (balanced: every rank exactly S*K rows; grouped:
+    by physical instance with dropped slots) into `out` (see include/mep.h)."""
     if ids.numel() != R * S * K:
         raise ValueError("ids must hold R*S*K slots")
     _need(keep is None or keep.numel() == R * S * K, "keep must hold R*S*K flags")
@@ -230,6 +234,7 @@ def mep_maxvio(stats, S: int, K: int, n_keys: int) -> dict:
 
 
 def mep_dedup_workspace_size(R: int, S: int, K: int) -> int:
+    """Bytes of scratch mep_dedup_plan needs (DedupBuffers.allocate uses it)."""
     return int(lib().mep_dedup_workspace_size(R, S, K))
 
 
@@ -255,6 +260,9 @@ class DedupBuffers:
 
 def mep_dedup_plan(pos: torch.Tensor, rank_off: torch.Tensor, R: int, S: int, K: int, out: DedupBuffers,
                    stream=None) -> DedupBuffers:
+    """One row per (token, destination rank) from a plan's pos and rank_off: the send
+    list, every slot's row, the ranks' first rows, each row's token and the plan rows'
+    source rows (see include/mep.h)."""
     if pos.numel() != R * S * K or rank_off.numel() != R + 1:
         raise ValueError("pos must hold R*S*K slots and rank_off R+1 offsets")
     N = R * S * K
@@ -298,6 +306,8 @@ def mep_update_expert(expert_ids: torch.Tensor, eplb_table: torch.Tensor,
                       active_mask: Optional[torch.Tensor], local_rank_id: int, world_size: int,
                       balance_mode: int, balanced_expert_ids: torch.Tensor,
                       balanced_active_mask: torch.Tensor, stream=None):
+    """Logical -> physical expert ids through eplb_table (balance_mode 0 by rank, 1 by
+    token) and the pruning mask, for one rank's BS tokens."""
     BS, K = expert_ids.shape
     E, F = eplb_table.shape
     _check_mapping(expert_ids, expert_scales, pruning_threshold, active_mask, balanced_expert_ids,
@@ -342,6 +352,8 @@ def mep_update_expert_ranks(expert_ids: torch.Tensor, eplb_table: torch.Tensor,
 
 def mep_dispatch(x: torch.Tensor, pos: torch.Tensor, K: int, recv: torch.Tensor,
                  recv_scale: Optional[torch.Tensor] = None, quant: int = 0, stream=None):
+    """recv[pos[n]] = x[n // K] for every kept slot (bf16), or its per-token int8 codes
+    with the scale in recv_scale (quant=1). x bf16 [T, H], pos int32 [T*K], recv [rows, H]."""
     T, H = x.shape
     want = torch.int8 if quant == 1 else torch.bfloat16
     rows = recv.shape[0]
@@ -356,6 +368,7 @@ def mep_dispatch(x: torch.Tensor, pos: torch.Tensor, K: int, recv: torch.Tensor,
 
 
 def mep_dequantize(q: torch.Tensor, scale: torch.Tensor, y: torch.Tensor, stream=None):
+    """y = bf16(q * scale) row by row: the identity expert on int8 rows."""
     rows, H = q.shape
     _need(_n(scale) >= rows and tuple(y.shape) == (rows, H), "scale [rows] and y [rows, H] must match q")
     _ok(lib().mep_dequantize(_ptr(q, torch.int8, "q"), _ptr(scale, torch.float32, "scale"), rows, H,
@@ -370,6 +383,8 @@ def _check_combine(y, pos, gates, T, K, H):
 
 def mep_combine(y: torch.Tensor, pos: torch.Tensor, gates: torch.Tensor, K: int,
                 out: torch.Tensor, stream=None):
+    """out[t] = bf16(sum over kept k, ascending, of fl(gate * y[pos[t*K+k]])) in fp32.
+    y bf16 [rows, H], pos int32 [T*K], gates fp32 [T*K], out bf16 [T, H]."""
     T, H = out.shape
     _check_combine(y, pos, gates, T, K, H)
     rc = lib().mep_combine(_ptr(y, torch.bfloat16, "y"), y.shape[0], _ptr(pos, torch.int32, "pos"),
@@ -429,6 +444,7 @@ def mep_prefetch_plan(plan: PlanBuffers, R: int, E: int, B: int, slot_expert: to
 
 def mep_prefetch_weights(w_home: torch.Tensor, slot_expert: torch.Tensor, R: int, B: int,
                          w_slots: torch.Tensor, stream=None):
+    """w_slots[s] = w_home[slot_expert[s]] for every used slot (bf16 expert weights)."""
     E = w_home.shape[0]
     D = w_home.numel() // E
     _need(_n(slot_expert) >= R * B and _n(w_slots) >= R * B * D, "slot_expert [R*B] and w_slots [R*B, ...] needed")
@@ -441,6 +457,8 @@ def mep_prefetch_weights(w_home: torch.Tensor, slot_expert: torch.Tensor, R: int
 
 def mep_grad_reduce(grad_home: torch.Tensor, grad_slots: torch.Tensor, slot_expert: torch.Tensor,
                     R: int, B: int, stream=None):
+    """grad_home[e] += its slots in ascending (rank, slot) order (fp32), then the slots
+    are cleared."""
     E = grad_home.shape[0]
     D = grad_home.numel() // E
     _need(_n(slot_expert) >= R * B and _n(grad_slots) >= R * B * D,
