@@ -709,6 +709,10 @@ def run_gpu(args, w):
         raise SystemExit("--dedup applies to the balanced workloads")
     if args.smooth and not w.quant:
         raise SystemExit("--smooth applies to the int8 workload")
+    if args.smooth and args.dedup:
+        # smoothed codes belong to a slot's expert, so one row per (token, rank) cannot
+        # carry them for the other slots of that pair
+        raise SystemExit("--smooth and --dedup do not combine: smoothed codes are per slot")
     rt = Route(mep, rank_workload(w, rank), dev, args.epilogue, dedup=bool(args.dedup),
                smooth=bool(args.smooth))
     names = [n for n, _ in rt.phases()]
