@@ -456,7 +456,9 @@ mep_status_t mep_dispatch(const uint16_t *x, const int32_t *pos, int64_t T, int3
  * the tokens g with at least one kept slot on r. Outputs (device, overwritten):
  *   dsend     int32 [N]    row of the first slot of each (token, rank) pair, -1 for
  *                          every other slot: the send list (mep_dispatch(x, dsend, ...)
- *                          writes each pair's row once)
+ *                          writes each pair's row once, bf16 or per-token int8; the
+ *                          smoothing dispatch does not compose with it, its codes being
+ *                          per slot)
  *   dpos      int32 [N]    row of every kept slot (shared by a pair's slots), -1 dropped
  *   drank_off int32 [R+1]  first row of every rank, drank_off[R] = the row count U
  *   dtok      int32 [N]    token of every row, -1 from U on
