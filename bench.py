@@ -1,12 +1,15 @@
 """Benchmark of MoE expert-parallel token routing on B200.
 
 One step = the whole hot path over one batch: balanced plan (histogram, stable
-counting sort, replica tables) -> dispatch of bf16 rows into the R ranks' receive
+counting sort, replica tables) -> dispatch of the token rows into the R ranks' receive
 partitions -> combine of the identity expert's rows back into token order.
 
-Default workload: R=8 simulated EP ranks, E=64 experts, S=4096 tokens per rank, K=8,
-H=7168 bf16 (N = 262,144 token-slots per step). Inputs (x 470 MB, receive buffer
-3.76 GB) are larger than the 126 MB L2, so no flush is needed between steps.
+Default workload (the headline): R=32 simulated EP ranks, E=256 experts, S=8192 tokens
+per rank, K=8, H=7168, with per-token dynamic int8 dispatch and the combine of the int8
+rows (N = 2,097,152 token-slots per step). Inputs (x 3.76 GB, receive buffer 15 GB) are
+larger than the 126 MB L2, so no flush is needed between steps. After it, the other four
+workloads (tiny, r8, map, skew) are measured the same way, more briefly, and reported
+in the same line under `per_workload`.
 
 Prints one JSON line (rank 0). `value` = token-slots of all ranks per second of the
 slowest rank's device time. With --gpus N > 1 (torchrun), every rank routes its own
@@ -96,39 +99,67 @@ def kernel_source_hash(name: str) -> str:
     return h.hexdigest()[:16]
 
 
-# dram__bytes_read.sum + dram__bytes_write.sum per launch, from the ncu captures
-# summarised in profiles/, scaled to the full workload by the rows routed (a capture on
-# a quarter or a sixteenth of the tokens per rank routes that share of the rows).
+# dram__bytes_read.sum + dram__bytes_write.sum per launch, from one ncu capture of the
+# kernel on a smaller case of the same workload (inputs larger than L2), scaled to the
+# full workload by the rows routed: a capture on 1/4 or 1/16 of the tokens per rank
+# routes that share of the rows. "src" is the kernel's source hash when captured.
+_TRAFFIC_METRICS = "dram__bytes_read.sum + dram__bytes_write.sum"
 TRAFFIC = {
     ("k_dispatch_warp", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 998.22e6, "src": "2bdb2659ae3ccd32",
-        "note": "profiles/traffic_dominant_kernels.md: 998.22 MB at S=1024, x4"},
+        "bytes": 4 * 998.22e6, "src": "2bdb2659ae3ccd32", "case_S": 1024, "case_mb": 998.22},
     ("k_combine_v8", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 1005.70e6, "src": "b8d0144407f8df74",
-        "note": "profiles/traffic_dominant_kernels.md: 1005.70 MB at S=1024, x4"},
+        "bytes": 4 * 1005.70e6, "src": "b8d0144407f8df74", "case_S": 1024, "case_mb": 1005.70},
     ("k_dispatch_int8_staged", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1115.86e6, "src": "cf5ee39cf4a3516f",
-        "note": "profiles/traffic_dominant_kernels.md: 1115.86 MB at S=512, x16"},
+        "bytes": 16 * 1115.86e6, "src": "cf5ee39cf4a3516f", "case_S": 512, "case_mb": 1115.86},
     ("k_combine_int8_warp", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1117.18e6, "src": "d852eb58236fe244",
-        "note": "profiles/traffic_dominant_kernels.md: 1117.18 MB at S=512, x16"},
+        "bytes": 16 * 1117.18e6, "src": "d852eb58236fe244", "case_S": 512, "case_mb": 1117.18},
     ("k_expand_warp", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 1793.81e6, "src": "a12dc9427177590d",
-        "note": "profiles/dedup_r8.md: 1793.81 MB at S=1024, x4 (--dedup 1)"},
+        "bytes": 4 * 1793.81e6, "src": "a12dc9427177590d", "case_S": 1024, "case_mb": 1793.81},
     ("k_dispatch_warp", "skew_r64_e512_s2048_k8_h4096"): {
-        "bytes": 4 * 2357.51e6, "src": "2bdb2659ae3ccd32",
-        "note": "profiles/traffic_dominant_kernels.md: 2357.51 MB at S=512, x4"},
+        "bytes": 4 * 2357.51e6, "src": "2bdb2659ae3ccd32", "case_S": 512, "case_mb": 2357.51},
     ("k_combine_v8", "skew_r64_e512_s2048_k8_h4096"): {
-        "bytes": 4 * 2364.80e6, "src": "b8d0144407f8df74",
-        "note": "profiles/traffic_dominant_kernels.md: 2364.80 MB at S=512, x4"},
+        "bytes": 4 * 2364.80e6, "src": "b8d0144407f8df74", "case_S": 512, "case_mb": 2364.80},
 }
 
 
 def captured_traffic(kernel: str, workload: str):
+    """(bytes per full launch, capture descriptor), or (None, None) when the kernel has
+    no capture for this workload or its source changed since the capture."""
     t = TRAFFIC.get((kernel, workload))
     if not t or kernel_source_hash(kernel) != t["src"]:
         return None, None
-    return t["bytes"], t["note"]
+    w = synth.get(workload)
+    return t["bytes"], {"kernel": kernel, "workload": workload, "case_tokens_per_rank": t["case_S"],
+                        "metrics": _TRAFFIC_METRICS, "case_mb": t["case_mb"],
+                        "scale": w.S // t["case_S"], "kernel_src": t["src"]}
+
+
+def host_info() -> dict:
+    """The host the CPU baseline runs on: logical CPUs and the CPU model name."""
+    model = None
+    try:
+        import subprocess
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.lower().startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except Exception:
+        pass
+    if model is None:
+        try:
+            for line in open("/proc/cpuinfo"):
+                if line.lower().startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+        except OSError:
+            pass
+    mem_gb = None
+    try:
+        mem_gb = os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_PHYS_PAGES") / 2**30
+    except (ValueError, OSError):
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model, "host_mem_gib": mem_gb}
 
 
 # ------------------------------------------------------------------ clock sampler
@@ -271,11 +302,11 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * tot / max(1, args.steps), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8" if w.quant else "bf16", "data": "synthetic",
         "config": {"workload": w.name, "R": w.R, "E": w.E, "S": w.S, "K": w.K, "H": w.H,
                    "sample_S": S_sample, "seed": w.seed},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": desc},
+                         "sample": desc, **host_info()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -621,7 +652,7 @@ def e2e_route_host(mep, rt, w, dev, steps, pg):
     if pg:
         pg.barrier()
     ms = max_over_ranks(run(steps) / steps, pg, dev)
-    ok = torch.equal(outs[(steps - 1) % 3].float(), rt.out.cpu().float())
+    ok = torch.equal(outs[(steps - 1) % 3].view(torch.int16), rt.out.cpu().view(torch.int16))
     h2d = sum(v.numel() * v.element_size() for v in h.values())
     d2h = outs[0].numel() * 2
     del sets
@@ -687,6 +718,148 @@ def e2e_pipeline(rt, w, dev, stream, steps, pg):
                               "sets, three streams)")
 
 
+def time_route(mep, rt, args, dev, stream, pg, steps):
+    """Warm-up, eager timed steps (per-phase CUDA events) and, with --graph, timed replays
+    of the step captured as a CUDA graph (one event between replays). Returns a dict of
+    per-step device times (max over ranks for the job time) and per-phase means."""
+    names = [n for n, _ in rt.phases()]
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            rt.step(stream)
+    stream.synchronize()
+    mep.mep_get_error(clear=True, stream=stream)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # A working set that fits in L2 is flushed between steps (a 256 MB write, outside
+    # the step's events); larger ones are not.
+    flush = None
+    if rt.working_set_bytes() < 2 * L2_BYTES:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    launches = 0
+    local = dev.index or 0
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for i in range(steps):
+                if flush is not None:
+                    flush.fill_(i & 0xff)
+                launches += rt.step(stream, evs[i])
+            end.record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        eager_steps = [e[0].elapsed_time(e[-1]) for e in evs]
+        ms = start.elapsed_time(end) if flush is None else float(sum(eager_steps))
+        err = mep.mep_get_error(clear=True, stream=stream)
+        if err:
+            raise RuntimeError(f"device error word {err:#x} after the timed steps")
+        t_phase = {n: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs])) for i, n in enumerate(names)}
+        ms_eager = max_over_ranks(ms, pg, dev) / steps
+
+        # The same step captured once into a CUDA graph and replayed: the launches of a
+        # step go to the GPU as one unit (this matters most for small, launch-bound
+        # workloads).
+        graph_ms, graph_steps = None, None
+        if args.graph:
+            g = torch.cuda.CUDAGraph()
+            # thread-local capture: other threads (NCCL's watchdog, the clock sampler)
+            # may make CUDA calls while this thread captures
+            with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+                rt.step(stream)
+            with torch.cuda.stream(stream):
+                for _ in range(3):
+                    g.replay()
+            stream.synchronize()
+            if pg:
+                pg.barrier()
+            torch.cuda.synchronize()
+            gev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+            with torch.cuda.stream(stream):
+                if flush is None:
+                    for i in range(steps):
+                        gev[i].record(stream)
+                        g.replay()
+                    gev[steps].record(stream)
+                    stream.synchronize()
+                    graph_steps = [gev[i].elapsed_time(gev[i + 1]) for i in range(steps)]
+                    gms = gev[0].elapsed_time(gev[steps])
+                else:
+                    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    graph_steps = []
+                    for i in range(steps):
+                        flush.fill_(i & 0xff)
+                        g0.record(stream)
+                        g.replay()
+                        g1.record(stream)
+                        stream.synchronize()
+                        graph_steps.append(g0.elapsed_time(g1))
+                    gms = float(sum(graph_steps))
+            torch.cuda.synchronize()
+            if pg:
+                pg.barrier()
+            graph_ms = max_over_ranks(gms, pg, dev) / steps
+            err = mep.mep_get_error(clear=True, stream=stream)
+            if err:
+                raise RuntimeError(f"device error word {err:#x} after the graph replays")
+            del g
+    per_step = graph_steps if graph_steps is not None else eager_steps
+    return {
+        "names": names, "t_phase": t_phase, "launches": launches, "ms_eager": ms_eager, "graph_ms": graph_ms,
+        "ms_step": graph_ms if graph_ms is not None else ms_eager,
+        "step_ms": {"median": float(statistics.median(per_step)), "min": float(min(per_step)),
+                    "max": float(max(per_step)), "mean": float(np.mean(per_step)), "n": len(per_step),
+                    "of": "cuda_graph_replay" if graph_steps is not None else "eager"},
+        "flush": flush is not None, "clocks": clk.summary(),
+    }
+
+
+def roofline_of(rt, tm, peak, peak_kind):
+    """The dominant HBM-bound phase (the slower of the moving phases) against the peak,
+    with its algorithmic bytes; and the dispatch+combine rate over all moving phases."""
+    w = rt.w
+    ab = rt.bytes()
+    t_phase = tm["t_phase"]
+    moving = [n for n in tm["names"] if n != "plan"]
+    dom = max(moving, key=lambda n: t_phase[n])
+    achieved = ab[dom] / (t_phase[dom] * 1e-3) / 1e9
+    kname = rt.kernel_name(dom)
+    traffic, capture = captured_traffic(kname, w.name)
+    t_move = sum(t_phase[n] for n in moving)
+    dc_gbs = sum(ab[n] for n in moving) / (t_move * 1e-3) / 1e9
+    roof = {"kernel": kname, "phase": dom, "bound": "hbm", "achieved": achieved, "peak": peak,
+            "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "algorithmic_bytes": ab[dom],
+            "traffic": traffic, "traffic_capture": capture}
+    dc = {"token_slots_per_s": w.N / (t_move * 1e-3), "hbm_gbs": dc_gbs, "frac_of_peak": dc_gbs / peak,
+          "frac_of_8tbs_nominal": dc_gbs / 8000.0, "algorithmic_bytes": sum(ab[n] for n in moving)}
+    return roof, dc
+
+
+def per_workload_entry(mep, name, args, dev, stream, pg, peak, peak_kind):
+    """A shorter measurement of another workload for the `per_workload` block: the same
+    timing method (graph replays, per-phase eager events), no end-to-end leg."""
+    w = synth.get(name)
+    rt = Route(mep, w, dev)
+    steps = max(5, min(args.steps, 20))
+    tm = time_route(mep, rt, args, dev, stream, pg, steps)
+    roof, dc = roofline_of(rt, tm, peak, peak_kind)
+    entry = {
+        "workload": w.name, "token_slots": w.N, "ms_per_step": tm["ms_step"],
+        "token_slots_per_s": w.N / (tm["ms_step"] * 1e-3), "step_ms": tm["step_ms"],
+        "breakdown_ms": tm["t_phase"], "dispatch_combine": dc,
+        "roofline": {k: roof[k] for k in ("kernel", "phase", "achieved", "frac", "algorithmic_bytes", "traffic")},
+        "launches_per_step": tm["launches"] // steps, "result_check": rt.result_ok(), "flush": tm["flush"],
+        "clocks": tm["clocks"], "plan_stats": rt.pb.stats_dict(), "maxvio": maxvio(rt),
+    }
+    del rt
+    torch.cuda.empty_cache()
+    return entry
+
+
 def run_gpu(args, w):
     import dispatch_combine_topk_b200 as mep
 
@@ -715,88 +888,9 @@ def run_gpu(args, w):
         raise SystemExit("--smooth and --dedup do not combine: smoothed codes are per slot")
     rt = Route(mep, rank_workload(w, rank), dev, args.epilogue, dedup=bool(args.dedup),
                smooth=bool(args.smooth))
-    names = [n for n, _ in rt.phases()]
     stream = torch.cuda.Stream(dev)
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            rt.step(stream)
-    stream.synchronize()
-    mep.mep_get_error(clear=True)
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    # A working set that fits in L2 is flushed between steps (a 256 MB write, outside
-    # the step's events); larger ones are not.
-    flush = None
-    if rt.working_set_bytes() < 2 * L2_BYTES:
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    launches = 0
-    with ClockSampler(local) as clk:
-        with torch.cuda.stream(stream):
-            start.record(stream)
-            for i in range(args.steps):
-                if flush is not None:
-                    flush.fill_(i & 0xff)
-                launches += rt.step(stream, evs[i])
-            end.record(stream)
-        stream.synchronize()
-    torch.cuda.synchronize()
-    if pg:
-        pg.barrier()
-    if flush is None:
-        ms = start.elapsed_time(end)
-    else:
-        ms = float(sum(e[0].elapsed_time(e[-1]) for e in evs))
-    err = mep.mep_get_error(clear=True)
-    if err:
-        raise RuntimeError(f"device error word {err:#x} after the timed steps")
-    t_phase = {n: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs])) for i, n in enumerate(names)}
-    ms_eager = max_over_ranks(ms, pg, dev) / args.steps
+    tm = time_route(mep, rt, args, dev, stream, pg, args.steps)
     weights = weight_side(mep, rt, args, dev, stream) if args.ffn_dim > 0 else None
-
-    # The same step captured once into a CUDA graph and replayed: the launches of a step
-    # go to the GPU as one unit (this matters most for small, launch-bound workloads).
-    graph_ms = None
-    if args.graph:
-        g = torch.cuda.CUDAGraph()
-        # thread-local capture: other threads (NCCL's watchdog, the clock sampler) may
-        # make CUDA calls while this thread captures
-        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
-            rt.step(stream)
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                g.replay()
-        stream.synchronize()
-        if pg:
-            pg.barrier()
-        torch.cuda.synchronize()
-        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            if flush is None:
-                g0.record(stream)
-                for _ in range(args.steps):
-                    g.replay()
-                g1.record(stream)
-                stream.synchronize()
-                gms = g0.elapsed_time(g1)
-            else:
-                gms = 0.0
-                for i in range(args.steps):
-                    flush.fill_(i & 0xff)
-                    g0.record(stream)
-                    g.replay()
-                    g1.record(stream)
-                    stream.synchronize()
-                    gms += g0.elapsed_time(g1)
-        graph_ms = max_over_ranks(gms, pg, dev) / args.steps
-        err = mep.mep_get_error(clear=True)
-        if err:
-            raise RuntimeError(f"device error word {err:#x} after the graph replays")
-        del g
-    ms_step = graph_ms if graph_ms is not None else ms_eager
     ok_device = rt.result_ok()
 
     e2e_steps = max(4, min(args.steps, 20))
@@ -804,59 +898,63 @@ def run_gpu(args, w):
         e2e_ms, ok_e2e, h2d, d2h, how = e2e_route_host(mep, rt, w, dev, e2e_steps, pg)
     else:
         e2e_ms, ok_e2e, h2d, d2h, how = e2e_pipeline(rt, w, dev, stream, e2e_steps, pg)
+    torch.cuda.empty_cache()
 
+    line = None
+    peak, peak_kind = load_peaks()
     if rank == 0:
-        peak, peak_kind = load_peaks()
-        ab = rt.bytes()
-        moving = [n for n in names if n != "plan"]          # the HBM-bound phases
-        dom = max(moving, key=lambda n: t_phase[n])
-        t_dom = t_phase[dom]
-        achieved = ab[dom] / (t_dom * 1e-3) / 1e9
-        kname = rt.kernel_name(dom)
-        traffic, traffic_note = captured_traffic(kname, w.name)
-        t_move = sum(t_phase[n] for n in moving)
-        dc_gbs = sum(ab[n] for n in moving) / (t_move * 1e-3) / 1e9
+        roof, dc = roofline_of(rt, tm, peak, peak_kind)
+        ms_step = tm["ms_step"]
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             v, desc, _ = oracle_sample(w, cpu_sample_S(w, args.cpu_div))
-            cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+            cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc, **host_info()}
         line = {
             "metric": METRIC,
             "value": world * w.N / (ms_step * 1e-3),
             "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step,
-            "timing": {"mode": "cuda_graph_replay" if graph_ms is not None else "eager",
-                       "graph_ms_per_step": graph_ms, "eager_ms_per_step": ms_eager},
+            "step_ms": tm["step_ms"],
+            "timing": {"mode": "cuda_graph_replay" if tm["graph_ms"] is not None else "eager",
+                       "graph_ms_per_step": tm["graph_ms"], "eager_ms_per_step": tm["ms_eager"]},
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int8" if w.quant else "bf16", "data": "synthetic",
             "config": {"workload": w.name, "R": w.R, "E": w.E, "S": w.S, "K": w.K, "H": w.H,
+                       "quant": "per-token dynamic int8 dispatch, combine of the int8 rows" if w.quant else "none",
                        "epilogue": args.epilogue, "dedup": bool(args.dedup), "smooth": bool(args.smooth),
                        "token_slots_per_gpu": w.N, "seed": w.seed, "parallelism": f"replicas{world}",
                        "l2": (f"working set {rt.working_set_bytes() / 1e6:.0f} MB "
                               + ("< 2x L2 (126 MB): L2 flushed between steps (256 MB write, "
-                                 "not timed)" if flush is not None else
+                                 "not timed)" if tm["flush"] else
                                  "> 2x L2 (126 MB): inputs larger than L2, no flush"))},
-            "breakdown_ms": t_phase,
-            "dispatch_combine": {"token_slots_per_s": w.N / (t_move * 1e-3),
-                                 "hbm_gbs": dc_gbs, "frac_of_peak": dc_gbs / peak,
-                                 "frac_of_8tbs_nominal": dc_gbs / 8000.0},
-            "roofline": {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": peak,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "algorithmic_bytes": ab[dom], "traffic": traffic,
-                         "traffic_source": traffic_note},
+            "breakdown_ms": tm["t_phase"],
+            "dispatch_combine": dc,
+            "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": world * w.N / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "path": how},
             "result_check": {"device": ok_device, "e2e": ok_e2e},
-            "gpu_launches": launches,
-            "clocks": clk.summary(),
+            "gpu_launches": tm["launches"],
+            "clocks": tm["clocks"],
             "plan_stats": rt.pb.stats_dict(),
             "maxvio": maxvio(rt),
             "replica_weights": weights,
             "dedup": dedup_summary(rt) if args.dedup else None,
         }
+    del rt
+    torch.cuda.empty_cache()
+    # the other workloads, on every rank (each rank its own GPU), reported by rank 0
+    others = [n for n in args.per_workload.split(",") if n] if args.per_workload != "none" else []
+    per = {}
+    for name in others:
+        if synth.get(name).name == w.name:
+            continue
+        e = per_workload_entry(mep, name, args, dev, stream, pg, peak, peak_kind)
+        per[e["workload"]] = e
+    if line is not None:
+        line["per_workload"] = per or None
         print(json.dumps(line), flush=True)
     if pg:
         pg.barrier()
@@ -869,7 +967,10 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="mep", choices=["mep", "reference"])
-    ap.add_argument("--workload", default="r8")
+    ap.add_argument("--workload", default="int8")
+    ap.add_argument("--per-workload", default="tiny,r8,map,skew",
+                    help="comma-separated workloads measured after the main one and reported under "
+                         "per_workload (graph replays, no end-to-end leg); 'none' to skip")
     ap.add_argument("--ref-div", type=int, default=8,
                     help="--impl reference: the oracle routes S/ref_div tokens per rank per step")
     ap.add_argument("--cpu-div", type=int, default=1,

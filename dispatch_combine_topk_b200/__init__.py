@@ -28,6 +28,9 @@ DERR_KEY_RANGE = 0x1
 DERR_ROW_RANGE = 0x2
 DERR_TABLE = 0x4
 DERR_MASK = 0x8
+DERR_TIMEOUT = 0x10
+DERR_DRAIN = 0x20
+DERR_HIST = 0x40
 
 STATUS = {0: "MEP_OK", 1: "MEP_ERR_NULLPTR", 2: "MEP_ERR_DTYPE", 3: "MEP_ERR_SHAPE",
           4: "MEP_ERR_VALUE", 5: "MEP_ERR_WORKSPACE", 6: "MEP_ERR_CUDA", 7: "MEP_ERR_TIMEOUT"}
@@ -69,7 +72,7 @@ def lib() -> ctypes.CDLL:
         L.mep_status_string.argtypes = [ctypes.c_int]
         L.mep_status_string.restype = ctypes.c_char_p
         L.mep_last_cuda_error.restype = i32
-        L.mep_get_error.argtypes = [P, i32]
+        L.mep_get_error.argtypes = [P, P, i32]
         L.mep_histogram.argtypes = [P, i64, i32, P, P]
         L.mep_plan_workspace_size.argtypes = [i32, i32, i32, i32]
         L.mep_plan_workspace_size.restype = ctypes.c_size_t
@@ -94,12 +97,16 @@ def lib() -> ctypes.CDLL:
         L.mep_route_host.argtypes = [ctypes.POINTER(_RouteBuffersC), P, P, P, P, P]
         L.mep_stream_synchronize_timeout.argtypes = [P, i32]
         L.mep_maxvio.argtypes = [P, i32, i32, i32, P, P, P]
+        L.mep_plan_rank_workspace_size.argtypes = [i32, i32, i32, i32]
+        L.mep_plan_rank_workspace_size.restype = ctypes.c_size_t
+        L.mep_plan_rank.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.mep_plan_static_ws.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P]
         for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
                   "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8",
                   "mep_combine_add_rmsnorm", "mep_prefetch_plan", "mep_prefetch_weights",
                   "mep_grad_reduce", "mep_dispatch_int8_smooth", "mep_update_expert_ranks",
                   "mep_dedup_plan", "mep_expand", "mep_route_host", "mep_stream_synchronize_timeout",
-                  "mep_maxvio"]:
+                  "mep_maxvio", "mep_plan_rank", "mep_plan_static_ws"]:
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -145,10 +152,11 @@ def _ok(rc: int, what: str):
         raise MepError(rc, what)
 
 
-def mep_get_error(clear: bool = True) -> int:
-    """Sticky device error word of the current device (synchronises the device)."""
+def mep_get_error(clear: bool = True, stream=None) -> int:
+    """Sticky error word of the current device, read in order on `stream` (default: the
+    current stream); waits for that stream only. With clear, the bits read are cleared."""
     code = ctypes.c_int32(0)
-    _ok(lib().mep_get_error(ctypes.byref(code), int(clear)), "mep_get_error")
+    _ok(lib().mep_get_error(_stream(stream), ctypes.byref(code), int(clear)), "mep_get_error")
     return code.value
 
 
@@ -231,6 +239,48 @@ def mep_maxvio(stats, S: int, K: int, n_keys: int) -> dict:
     _ok(lib().mep_maxvio(ctypes.cast(buf, ctypes.c_void_p), S, K, n_keys, *[ctypes.byref(o) for o in out]),
         "mep_maxvio")
     return {"rank_before": out[0].value, "rank_after": out[1].value, "expert": out[2].value}
+
+
+def mep_plan_rank_workspace_size(R: int, E: int, S: int, K: int) -> int:
+    """Bytes of scratch mep_plan_rank needs for this shape."""
+    return int(lib().mep_plan_rank_workspace_size(R, E, S, K))
+
+
+@dataclasses.dataclass
+class RankPlanBuffers:
+    """Device outputs of mep_plan_rank: one EP rank's share of the balanced plan."""
+
+    pos: torch.Tensor         # int32 [S*K]: global row of each of this rank's slots
+    send_count: torch.Tensor  # int32 [R]
+    send_off: torch.Tensor    # int32 [R+1]
+    recv_count: torch.Tensor  # int32 [R]
+    recv_off: torch.Tensor    # int32 [R+1]
+    workspace: torch.Tensor   # uint8, 256-byte aligned
+
+    @staticmethod
+    def allocate(R: int, E: int, S: int, K: int, device=None) -> "RankPlanBuffers":
+        dev = device or torch.device("cuda", torch.cuda.current_device())
+        z = lambda n: torch.empty(n, dtype=torch.int32, device=dev)
+        ws = torch.empty(max(256, mep_plan_rank_workspace_size(R, E, S, K)), dtype=torch.uint8, device=dev)
+        return RankPlanBuffers(z(S * K), z(R), z(R + 1), z(R), z(R + 1), ws)
+
+
+def mep_plan_rank(ids: torch.Tensor, hist_all: torch.Tensor, R: int, E: int, S: int, K: int, rank: int,
+                  out: RankPlanBuffers, stream=None) -> RankPlanBuffers:
+    """Rank `rank`'s share of the balanced plan from the all-gathered per-rank histograms
+    hist_all (int32 [R, E]): the global rows of its S*K slots and the exchange counts."""
+    _need(ids.numel() == S * K, "ids must hold this rank's S*K slots")
+    _need(hist_all.numel() == R * E, "hist_all must be [R, E]")
+    _need(_n(out.pos) >= S * K and _n(out.send_count) >= R and _n(out.send_off) >= R + 1
+          and _n(out.recv_count) >= R and _n(out.recv_off) >= R + 1,
+          "rank plan buffers too small: allocate them with RankPlanBuffers.allocate")
+    rc = lib().mep_plan_rank(_ptr(ids, torch.int32, "ids"), _ptr(hist_all, torch.int32, "hist_all"), R, E, S, K,
+                             rank, _ptr(out.pos, torch.int32), _ptr(out.send_count, torch.int32),
+                             _ptr(out.send_off, torch.int32), _ptr(out.recv_count, torch.int32),
+                             _ptr(out.recv_off, torch.int32), _ptr(out.workspace), out.workspace.numel(),
+                             _stream(stream))
+    _ok(rc, "mep_plan_rank")
+    return out
 
 
 def mep_dedup_workspace_size(R: int, S: int, K: int) -> int:
@@ -499,10 +549,6 @@ def mep_plan_static_ws(ids: torch.Tensor, R: int, n_keys: int, S: int, K: int, o
     """mep_plan for callers that cannot allocate device memory: the scratch is a 4 MiB
     array inside libmep (``out.workspace`` is not used). See include/mep.h."""
     f = lib().mep_plan_static_ws
-    if f.argtypes is None:
-        P, i32 = ctypes.c_void_p, ctypes.c_int32
-        f.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P]
-        f.restype = ctypes.c_int
     if ids.numel() != R * S * K:
         raise ValueError("ids must hold R*S*K slots")
     _need(keep is None or keep.numel() == R * S * K, "keep must hold R*S*K flags")

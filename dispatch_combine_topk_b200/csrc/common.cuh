@@ -14,6 +14,9 @@ __device__ int32_t g_error_word;
 
 __device__ __forceinline__ void flag_error(int32_t bit) { atomicOr(&g_error_word, bit); }
 
+// Clears the given bits of the error word (the ones a reader has just reported).
+__global__ void k_clear_error_bits(int32_t bits) { atomicAnd(&g_error_word, ~bits); }
+
 __device__ __forceinline__ uint32_t lanemask_lt()
 {
     uint32_t m;

@@ -5,6 +5,7 @@
 // One translation unit on purpose: the device error word lives here and every kernel
 // reaches it without relocatable device code.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdio.h>
@@ -28,41 +29,109 @@ thread_local int32_t t_last_cuda_error = 0;
 constexpr int kMaxDevices = 64;
 // Shared memory the staged int8 dispatch may use per CTA.
 constexpr int kBulkSmemMax = 200 * 1024;
-int g_sm_count[kMaxDevices];
-std::once_flag g_device_once[kMaxDevices];
 
-// One-time set-up of a device: its SM count and the kernels' shared-memory limits.
-void device_setup(int dev)
+// ---------------------------------------------------------------- per-context state
+//
+// Kernel attributes (the dynamic shared-memory limits) and the device address of the
+// static plan scratch belong to a CUDA context, not to a device ordinal: after
+// cudaDeviceReset, or for a caller that makes its own driver context current, they
+// must be set up again. The current context is identified by its driver-assigned id
+// (cuCtxGetId, unique for the life of the process, also when a context is destroyed
+// and another takes its handle). The two driver calls are reached through the
+// runtime's entry-point query, so the library links only the CUDA runtime.
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+std::once_flag g_driver_once;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+void driver_entry_points()
 {
-    int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    g_sm_count[dev] = n > 0 ? n : 148;
-    {
-        const int big = 200 * 1024;
-        cudaFuncSetAttribute(mep::k_rank, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(mep::k_tile_count, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(mep::k_histogram, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(mep::k_plan_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-        cudaFuncSetAttribute(mep::k_dispatch_int8_staged<4, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kBulkSmemMax);
-        const int norm_smem = (int)(sizeof(float) * MEP_RMSNORM_MAX_H);
-        cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
-        cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<6>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
-        cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
-        cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
-        cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
-        cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_scalar, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
-    }
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_ctx_get_current = (CtxGetCurrentFn)f;
+    f = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_ctx_get_id = (CtxGetIdFn)f;
+    (void)cudaGetLastError();
 }
 
-// SM count of the current device; the first call on a device runs its set-up (once,
-// also when several host threads call at the same time).
+// Id of the context current on this host thread; false when there is none (or the
+// driver cannot say).
+bool current_context_id(unsigned long long *id)
+{
+    std::call_once(g_driver_once, driver_entry_points);
+    if (!g_ctx_get_current || !g_ctx_get_id) return false;
+    CUcontext c = nullptr;
+    if (g_ctx_get_current(&c) != CUDA_SUCCESS || !c) return false;
+    return g_ctx_get_id(c, id) == CUDA_SUCCESS;
+}
+
+struct DeviceState {
+    std::mutex m;
+    std::atomic<bool> ready{false};
+    std::atomic<unsigned long long> ctx_id{0};
+    int sm_count = 148;
+    void *plan_static_ws = nullptr;   // device address of g_plan_static_ws in ctx_id
+};
+DeviceState g_dev[kMaxDevices];
+
+// Lookup of the static plan scratch's device address (defined with the array below).
+cudaError_t plan_static_ws_lookup(void **addr);
+
+// Set-up of the current device in the current context: its SM count, the kernels'
+// shared-memory limits, the address of the static plan scratch. Runs again whenever
+// the current context differs from the one it last ran in (several host threads may
+// call at once). Without the driver's context id it runs once per device.
+DeviceState &device_state(int dev)
+{
+    DeviceState &st = g_dev[dev];
+    unsigned long long id = 0;
+    const bool have = current_context_id(&id);
+    if (st.ready.load(std::memory_order_acquire) && (!have || st.ctx_id.load(std::memory_order_relaxed) == id))
+        return st;
+    std::lock_guard<std::mutex> lock(st.m);
+    if (st.ready.load(std::memory_order_relaxed) && (!have || st.ctx_id.load(std::memory_order_relaxed) == id))
+        return st;
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    st.sm_count = n > 0 ? n : 148;
+    const int big = 200 * 1024;
+    cudaFuncSetAttribute(mep::k_rank, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_tile_count, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_histogram, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_plan_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_source_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_dispatch_int8_staged<4, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kBulkSmemMax);
+    const int norm_smem = (int)(sizeof(float) * MEP_RMSNORM_MAX_H);
+    cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
+    cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<6>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
+    cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
+    cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
+    cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_v8<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
+    cudaFuncSetAttribute(mep::k_combine_add_rmsnorm_scalar, cudaFuncAttributeMaxDynamicSharedMemorySize, norm_smem);
+    void *ws = nullptr;
+    if (plan_static_ws_lookup(&ws) != cudaSuccess) ws = nullptr;
+    st.plan_static_ws = ws;
+    (void)cudaGetLastError();
+    // the calls above made the device's context current if none was
+    unsigned long long id2 = 0;
+    st.ctx_id.store(current_context_id(&id2) ? id2 : 0, std::memory_order_relaxed);
+    st.ready.store(true, std::memory_order_release);
+    return st;
+}
+
+// SM count of the current device (running its set-up when needed).
 int sm_count()
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-    std::call_once(g_device_once[dev], device_setup, dev);
-    return g_sm_count[dev];
+    return device_state(dev).sm_count;
 }
 
 mep_status_t launched()
@@ -131,19 +200,24 @@ const char *mep_status_string(mep_status_t s)
 
 int32_t mep_last_cuda_error(void) { return t_last_cuda_error; }
 
-mep_status_t mep_get_error(int32_t *code, int32_t clear)
+mep_status_t mep_get_error(mep_stream_t stream, int32_t *code, int32_t clear)
 {
     if (!code) return MEP_ERR_NULLPTR;
-    cudaError_t e = cudaDeviceSynchronize();
-    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(code, mep::g_error_word, sizeof(int32_t));
-    if (e == cudaSuccess && clear) {
-        const int32_t zero = 0;
-        e = cudaMemcpyToSymbol(mep::g_error_word, &zero, sizeof(int32_t));
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t word = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&word, mep::g_error_word, sizeof(int32_t), 0,
+                                              cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess && clear && word) {
+        // clears only the bits read: a bit another stream sets meanwhile stays set
+        mep::k_clear_error_bits<<<1, 1, 0, s>>>(word);
+        e = cudaGetLastError();
     }
     if (e != cudaSuccess) {
         t_last_cuda_error = (int32_t)e;
         return MEP_ERR_CUDA;
     }
+    *code = word;
     return MEP_OK;
 }
 
@@ -170,12 +244,14 @@ size_t mep_plan_workspace_size(int32_t R, int32_t n_keys, int32_t S, int32_t K)
     return align256(sizeof(int32_t) * (size_t)tiles * n_keys);
 }
 
-mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_t n_keys,
-                      int32_t S, int32_t K, int32_t mode, int32_t keys_per_rank,
-                      int32_t *pos, int32_t *hist, int32_t *rank_off, int32_t *load,
-                      int32_t *rep_count, int32_t *rep_key, int32_t *rep_cu,
-                      mep_plan_stats_t *stats, void *workspace, size_t workspace_bytes,
-                      mep_stream_t stream)
+}  // extern "C"
+
+namespace {
+// The argument checks of mep_plan, without the workspace (shared with mep_plan_static_ws).
+mep_status_t plan_args(const int32_t *ids, const uint8_t *keep, int32_t R, int32_t n_keys, int32_t S, int32_t K,
+                       int32_t mode, int32_t keys_per_rank, const int32_t *pos, const int32_t *hist,
+                       const int32_t *rank_off, const int32_t *rep_count, const int32_t *rep_key,
+                       const int32_t *rep_cu, const mep_plan_stats_t *stats)
 {
     if (!ids || !pos || !hist || !rank_off || !rep_count || !rep_key || !rep_cu || !stats)
         return MEP_ERR_NULLPTR;
@@ -191,6 +267,23 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
     } else {
         return MEP_ERR_VALUE;
     }
+    return MEP_OK;
+}
+}  // namespace
+
+extern "C" {
+
+mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_t n_keys,
+                      int32_t S, int32_t K, int32_t mode, int32_t keys_per_rank,
+                      int32_t *pos, int32_t *hist, int32_t *rank_off, int32_t *load,
+                      int32_t *rep_count, int32_t *rep_key, int32_t *rep_cu,
+                      mep_plan_stats_t *stats, void *workspace, size_t workspace_bytes,
+                      mep_stream_t stream)
+{
+    const mep_status_t st = plan_args(ids, keep, R, n_keys, S, K, mode, keys_per_rank, pos, hist, rank_off,
+                                      rep_count, rep_key, rep_cu, stats);
+    if (st != MEP_OK) return st;
+    const int64_t N = (int64_t)R * S * K;
     const size_t need = mep_plan_workspace_size(R, n_keys, S, K);
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return MEP_ERR_WORKSPACE;
 
@@ -203,11 +296,54 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
     mep::k_tile_count<<<(unsigned)tiles, threads, sizeof(int32_t) * n_keys, s>>>(ids, keep, N, n_keys, tile_cnt);
     mep::k_scan_cols<<<(unsigned)mep::ceil_div(n_keys, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, n_keys, hist);
     const size_t rank_smem = sizeof(int32_t) * ((size_t)mep::kPlanWarps * n_keys + n_keys + 1 + 33);
-    mep::k_rank<<<(unsigned)tiles, threads, rank_smem, s>>>(ids, keep, N, n_keys, tile_cnt, hist, pos);
+    mep::k_rank<<<(unsigned)tiles, threads, rank_smem, s>>>(ids, keep, N, n_keys, tile_cnt, hist, nullptr,
+                                                            pos);
     const size_t meta_smem = sizeof(int32_t) * (size_t)(2 * (n_keys + 1) + (R + 1) + R);
     mep::k_plan_meta<<<1, 1024, meta_smem, s>>>(hist, R, n_keys, (int64_t)S * K, mode,
                                                 keys_per_rank, rank_off, load, rep_count, rep_key,
                                                 rep_cu, (int32_t *)stats);
+    return launched();
+}
+
+size_t mep_plan_rank_workspace_size(int32_t R, int32_t E, int32_t S, int32_t K)
+{
+    if (R < 1 || E < 1 || S < 1 || K < 1) return 0;
+    const int64_t tiles = mep::ceil_div((int64_t)S * K, mep::kPlanTile);
+    return align256(sizeof(int32_t) * (size_t)tiles * E) + 2 * align256(sizeof(int32_t) * (size_t)E);
+}
+
+mep_status_t mep_plan_rank(const int32_t *ids, const int32_t *hist_all, int32_t R, int32_t E, int32_t S,
+                           int32_t K, int32_t rank, int32_t *pos, int32_t *send_count, int32_t *send_off,
+                           int32_t *recv_count, int32_t *recv_off, void *workspace, size_t workspace_bytes,
+                           mep_stream_t stream)
+{
+    if (!ids || !hist_all || !pos || !send_count || !send_off || !recv_count || !recv_off) return MEP_ERR_NULLPTR;
+    if (R < 1 || S < 1 || K < 1 || K > MEP_MAX_K || E < 1 || E > MEP_MAX_KEYS || R > MEP_MAX_KEYS)
+        return MEP_ERR_SHAPE;
+    if ((int64_t)R * S * K >= ((int64_t)1 << 31)) return MEP_ERR_SHAPE;
+    if (E % R != 0 || rank < 0 || rank >= R) return MEP_ERR_VALUE;
+    const size_t need = mep_plan_rank_workspace_size(R, E, S, K);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return MEP_ERR_WORKSPACE;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    sm_count();
+    const int64_t N = (int64_t)S * K;   // this rank's slots
+    const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
+    unsigned char *w = (unsigned char *)workspace;
+    int32_t *tile_cnt = (int32_t *)w;
+    w += align256(sizeof(int32_t) * (size_t)tiles * E);
+    int32_t *hist_local = (int32_t *)w;
+    w += align256(sizeof(int32_t) * (size_t)E);
+    int32_t *key_base = (int32_t *)w;
+    const int threads = mep::kPlanWarps * 32;
+    mep::k_tile_count<<<(unsigned)tiles, threads, sizeof(int32_t) * E, s>>>(ids, nullptr, N, E, tile_cnt);
+    mep::k_scan_cols<<<(unsigned)mep::ceil_div(E, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, E, hist_local);
+    const size_t meta_smem = sizeof(int32_t) * (size_t)(2 * E + 1 + 2 * R);
+    mep::k_source_meta<<<1, 1024, meta_smem, s>>>(hist_all, hist_local, R, E, (int64_t)S * K, rank, key_base,
+                                                  send_count, send_off, recv_count, recv_off);
+    const size_t rank_smem = sizeof(int32_t) * ((size_t)mep::kPlanWarps * E + E + 1 + 33);
+    mep::k_rank<<<(unsigned)tiles, threads, rank_smem, s>>>(ids, nullptr, N, E, tile_cnt, hist_local, key_base,
+                                                            pos);
     return launched();
 }
 
@@ -607,7 +743,8 @@ mep_status_t mep_dedup_plan(const int32_t *pos, const int32_t *rank_off, int32_t
     mep::k_tile_count<<<(unsigned)tiles, threads, sizeof(int32_t) * R, s>>>(dkey, dkeep, N, R, tile_cnt);
     mep::k_scan_cols<<<(unsigned)mep::ceil_div(R, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, R, count);
     const size_t rank_smem = sizeof(int32_t) * ((size_t)mep::kPlanWarps * R + R + 1 + 33);
-    mep::k_rank<<<(unsigned)tiles, threads, rank_smem, s>>>(dkey, dkeep, N, R, tile_cnt, count, dsend);
+    mep::k_rank<<<(unsigned)tiles, threads, rank_smem, s>>>(dkey, dkeep, N, R, tile_cnt, count, nullptr,
+                                                            dsend);
     mep::k_dedup_offsets<<<1, 1024, sizeof(int32_t) * (size_t)(R + 1 + 33), s>>>(count, R, drank_off);
     mep::k_dedup_finish<<<tgrid, 256, off_smem, s>>>(pos, rank_off, R, T, K, dsend, dpos, dtok, gidx);
     return launched();
@@ -700,9 +837,9 @@ mep_status_t mep_maxvio(const mep_plan_stats_t *stats, int32_t S, int32_t K, int
 static __device__ __align__(256) unsigned char g_plan_static_ws[MEP_PLAN_STATIC_WS_BYTES];
 
 namespace {
-// device address of g_plan_static_ws, per device (host threads may look it up at once)
-std::atomic<void *> g_plan_static_ws_addr[kMaxDevices];
-}
+// With the context that owns the address current (device_state calls it at set-up).
+cudaError_t plan_static_ws_lookup(void **addr) { return cudaGetSymbolAddress(addr, g_plan_static_ws); }
+}  // namespace
 
 extern "C" mep_status_t mep_plan_static_ws(const int32_t *ids, const uint8_t *keep, int32_t R,
                                            int32_t n_keys, int32_t S, int32_t K, int32_t mode,
@@ -711,11 +848,11 @@ extern "C" mep_status_t mep_plan_static_ws(const int32_t *ids, const uint8_t *ke
                                            int32_t *rep_key, int32_t *rep_cu,
                                            mep_plan_stats_t *stats, mep_stream_t stream)
 {
-    if (!ids || !pos || !hist || !rank_off || !rep_count || !rep_key || !rep_cu || !stats)
-        return MEP_ERR_NULLPTR;
-    const size_t need = mep_plan_workspace_size(R, n_keys, S, K);
-    if (need == 0) return MEP_ERR_SHAPE;
-    if (need > (size_t)MEP_PLAN_STATIC_WS_BYTES) return MEP_ERR_WORKSPACE;
+    // mep_plan's own argument checks first, then the size of the array
+    const mep_status_t st = plan_args(ids, keep, R, n_keys, S, K, mode, keys_per_rank, pos, hist, rank_off,
+                                      rep_count, rep_key, rep_cu, stats);
+    if (st != MEP_OK) return st;
+    if (mep_plan_workspace_size(R, n_keys, S, K) > (size_t)MEP_PLAN_STATIC_WS_BYTES) return MEP_ERR_WORKSPACE;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) {
@@ -723,17 +860,13 @@ extern "C" mep_status_t mep_plan_static_ws(const int32_t *ids, const uint8_t *ke
         return MEP_ERR_CUDA;
     }
     if (dev < 0 || dev >= kMaxDevices) return MEP_ERR_VALUE;
-    void *ws = g_plan_static_ws_addr[dev].load(std::memory_order_acquire);
+    // the address in the current context: looked up at the context's set-up, again
+    // after a device reset or under another context
+    void *ws = device_state(dev).plan_static_ws;
     if (!ws) {
-        // with that device current; threads that race here all find the same address
-        e = cudaGetSymbolAddress(&ws, g_plan_static_ws);
-        if (e != cudaSuccess || !ws) {
-            t_last_cuda_error = (int32_t)(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
-            return MEP_ERR_CUDA;
-        }
-        g_plan_static_ws_addr[dev].store(ws, std::memory_order_release);
+        t_last_cuda_error = (int32_t)cudaErrorInvalidSymbol;
+        return MEP_ERR_CUDA;
     }
     return mep_plan(ids, keep, R, n_keys, S, K, mode, keys_per_rank, pos, hist, rank_off, load,
                     rep_count, rep_key, rep_cu, stats, ws, (size_t)MEP_PLAN_STATIC_WS_BYTES, stream);
 }
-

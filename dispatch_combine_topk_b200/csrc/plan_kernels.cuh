@@ -159,21 +159,28 @@ k_scan_cols(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys, int
 }
 
 // pos[n] = off[key] + (slots of key in earlier tiles) + (earlier slots of key in this
-// tile), off = exclusive prefix of hist over keys. Each warp owns an eighth of the
-// tile: it counts its sub-range per key, the CTA turns those counts into per-warp bases,
-// then each warp walks its sub-range again in order, ranking equal keys with match.any.
+// tile), off = exclusive prefix of hist over keys, or key_base[key] when key_base is
+// given (the first row of this caller's slots of each key). Each warp owns an eighth of
+// the tile: it counts its sub-range per key, the CTA turns those counts into per-warp
+// bases, then each warp walks its sub-range again in order, ranking equal keys with
+// match.any.
 // Dynamic shared memory: cnt [kPlanWarps][n_keys], off [n_keys + 1], scratch [33].
 __global__ void __launch_bounds__(kPlanWarps * 32)
 k_rank(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, int64_t N, int32_t n_keys,
        const int32_t *__restrict__ tile_base, const int32_t *__restrict__ hist,
-       int32_t *__restrict__ pos)
+       const int32_t *__restrict__ key_base, int32_t *__restrict__ pos)
 {
     extern __shared__ int32_t cnt[];
     int32_t *key_off = cnt + kPlanWarps * n_keys;
     int32_t *scan_scratch = key_off + n_keys + 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < kPlanWarps * n_keys; i += blockDim.x) cnt[i] = 0;
-    block_exclusive_scan(hist, n_keys, key_off, scan_scratch);
+    if (key_base) {
+        for (int i = threadIdx.x; i < n_keys; i += blockDim.x) key_off[i] = key_base[i];
+        __syncthreads();
+    } else {
+        block_exclusive_scan(hist, n_keys, key_off, scan_scratch);
+    }
     constexpr int kSub = kPlanTile / kPlanWarps;
     const int64_t lo = (int64_t)blockIdx.x * kPlanTile + warp * kSub;
     int32_t *mine = cnt + warp * n_keys;
@@ -345,6 +352,83 @@ k_plan_meta(const int32_t *__restrict__ hist, int32_t R,
         stats[6] = s_red[6];
         stats[7] = 0;
     }
+}
+
+// ------------------------------------------------ one rank's share of the plan (e)
+//
+// Each real GPU is one EP rank holding its own S tokens. With the per-rank histograms
+// of all R ranks gathered (hist_all [R, E], row r = rank r's slots per expert) every
+// rank knows where its slots go in the global balanced plan without seeing the others'
+// ids: the plan orders slots by (e, src, t, k), so the rows of rank `rank`'s slots of
+// expert e start at
+//   key_base[e] = off[e] + sum_{r < rank} hist_all[r, e],   off = exclusive scan over e
+//                                                             of sum_r hist_all[r, e],
+// and within them follow its own slot order (k_rank with key_base). Row p lands on
+// destination rank p / SK. One CTA also writes the exchange counts:
+//   send_count[d] = rows this rank writes into rank d's partition,
+//   recv_count[s] = rows rank s writes into this rank's partition,
+// with their exclusive prefixes (R + 1 entries each), and checks that row `rank` of
+// hist_all equals the histogram of this rank's ids (hist_local).
+// Dynamic shared memory: off [E + 1], send [R], recv [R].
+__global__ void __launch_bounds__(1024)
+k_source_meta(const int32_t *__restrict__ hist_all, const int32_t *__restrict__ hist_local, int32_t R,
+              int32_t E, int64_t SK, int32_t rank, int32_t *__restrict__ key_base,
+              int32_t *__restrict__ send_count, int32_t *__restrict__ send_off,
+              int32_t *__restrict__ recv_count, int32_t *__restrict__ recv_off)
+{
+    extern __shared__ int32_t smem[];
+    int32_t *off = smem;                 // E + 1
+    int32_t *tot = off + (E + 1);        // E (column totals, then reused)
+    int32_t *snd = tot + E;              // R
+    int32_t *rcv = snd + R;              // R
+    __shared__ int32_t scan_scratch[33];
+    for (int r = threadIdx.x; r < R; r += blockDim.x) {
+        snd[r] = 0;
+        rcv[r] = 0;
+    }
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int32_t t = 0, pre = 0;
+        for (int r = 0; r < R; r++) {
+            const int32_t h = hist_all[(int64_t)r * E + e];
+            if (r == rank) pre = t;
+            t += h;
+        }
+        tot[e] = t;
+        key_base[e] = pre;   // completed below
+        if (hist_all[(int64_t)rank * E + e] != hist_local[e]) flag_error(MEP_DERR_HIST);
+    }
+    __syncthreads();
+    block_exclusive_scan(tot, E, off, scan_scratch);
+    const int64_t lo = (int64_t)rank * SK, hi = lo + SK;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int64_t b = (int64_t)off[e] + key_base[e];
+        key_base[e] = (int32_t)b;
+        // this rank's rows of e, split over the destination partitions they cross
+        const int32_t h = hist_all[(int64_t)rank * E + e];
+        for (int64_t p = b; p < b + h;) {
+            const int64_t d = p / SK;
+            const int64_t end = min(b + h, (d + 1) * SK);
+            atomicAdd(&snd[d], (int32_t)(end - p));
+            p = end;
+        }
+        // every source's rows of e that land in this rank's partition
+        if (off[e + 1] > lo && off[e] < hi) {
+            int64_t p = off[e];
+            for (int r = 0; r < R; r++) {
+                const int32_t hr = hist_all[(int64_t)r * E + e];
+                const int64_t a = max(p, lo), z = min(p + hr, hi);
+                if (z > a) atomicAdd(&rcv[r], (int32_t)(z - a));
+                p += hr;
+            }
+        }
+    }
+    __syncthreads();
+    for (int r = threadIdx.x; r < R; r += blockDim.x) {
+        send_count[r] = snd[r];
+        recv_count[r] = rcv[r];
+    }
+    block_exclusive_scan(snd, R, send_off, scan_scratch);
+    block_exclusive_scan(rcv, R, recv_off, scan_scratch);
 }
 
 }  // namespace mep

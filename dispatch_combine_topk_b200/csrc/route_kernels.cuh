@@ -355,10 +355,14 @@ k_dispatch_int8_staged(const uint16_t *__restrict__ x, const int32_t *__restrict
         const int s = (int)(i % kStages);
         const bool ok = mbar_wait_bounded(&bar[s], (uint32_t)((i / kStages) & 1));
         if (!__syncthreads_and(ok)) {
+            // Drain every load still issued, the one that just ran out included, before
+            // the CTA leaves: its shared memory may go to the next CTA on this SM. A
+            // drain wait that runs out as well is recorded with its own bit.
             if (tid == 0) {
                 flag_error(MEP_DERR_TIMEOUT);
-                for (int64_t j = i + 1; j < n && j < i + kStages; j++)
-                    mbar_wait_bounded(&bar[j % kStages], (uint32_t)((j / kStages) & 1));
+                for (int64_t j = i; j < n && j < i + kStages; j++)
+                    if (!mbar_wait_bounded(&bar[j % kStages], (uint32_t)((j / kStages) & 1)))
+                        flag_error(MEP_DERR_DRAIN);
             }
             break;
         }

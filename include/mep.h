@@ -18,14 +18,17 @@
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
  *    stream) and never synchronise the host, so a chain plan -> dispatch -> combine
  *    needs no host round trip (MoonEP's static shapes remove per-layer host syncs:
- *    twodots.gr article on MoonEP, static-shapes paragraph). Only mep_get_error and
- *    mep_stream_synchronize_timeout wait for the device (and mep_route_host's copies
- *    when its host buffers are pageable). mep_histogram, mep_plan, mep_update_expert, mep_update_expert_ranks,
- *    mep_dedup_plan, mep_dispatch, mep_expand, mep_dispatch_int8_smooth, mep_dequantize,
- *    mep_combine, mep_combine_int8,
- *    mep_combine_add_rmsnorm, mep_prefetch_plan, mep_prefetch_weights and mep_grad_reduce
- *    can be captured into a CUDA graph and replayed on new inputs, once each has been
- *    called eagerly on the device (the first call sets kernel attributes).
+ *    twodots.gr article on MoonEP, static-shapes paragraph). Three calls wait:
+ *    mep_get_error waits for its `stream` (and that stream only);
+ *    mep_stream_synchronize_timeout waits for its `stream` with a time limit; and
+ *    mep_route_host's copies are synchronous when its host buffers are pageable.
+ *    No call synchronises the whole device. mep_histogram, mep_plan, mep_plan_rank,
+ *    mep_update_expert, mep_update_expert_ranks, mep_dedup_plan, mep_dispatch,
+ *    mep_expand, mep_dispatch_int8_smooth, mep_dequantize, mep_combine,
+ *    mep_combine_int8, mep_combine_add_rmsnorm, mep_prefetch_plan, mep_prefetch_weights
+ *    and mep_grad_reduce can be captured into a CUDA graph and replayed on new inputs,
+ *    once each has been called eagerly in the current context (the first call in a
+ *    context sets kernel attributes).
  *  - A call first checks its arguments on the host and returns a status without
  *    launching anything when one is wrong: MEP_ERR_NULLPTR / MEP_ERR_DTYPE /
  *    MEP_ERR_SHAPE / MEP_ERR_VALUE mirror the aclnn codes 161001 (null tensor),
@@ -73,6 +76,10 @@ typedef enum {
 #define MEP_DERR_TABLE     0x4  /* eplb_table: count outside [1, F-1] or instance id outside [0, 1024) */
 #define MEP_DERR_MASK      0x8  /* active_mask has a true after a false */
 #define MEP_DERR_TIMEOUT   0x10 /* a bounded wait inside a kernel ran out; that kernel stopped early */
+#define MEP_DERR_DRAIN     0x20 /* after such a time-out, waiting for the kernel's own copies in flight
+                                   ran out as well */
+#define MEP_DERR_HIST      0x40 /* mep_plan_rank: the gathered histogram row of this rank differs from
+                                   the histogram of its ids (the ranks' inputs disagree) */
 
 /* Plan modes. */
 #define MEP_PLAN_BALANCED 0
@@ -118,12 +125,20 @@ const char *mep_status_string(mep_status_t status);
 int32_t mep_last_cuda_error(void);
 
 /*
- * Reads the sticky device error word of the CURRENT device into *code (a host
- * pointer; 0 = no data error since the last clear), after synchronising the device.
- * With clear != 0 the word is reset to 0. Returns MEP_ERR_NULLPTR if code is NULL.
- * This is the only call that synchronises.
+ * Reads the sticky error word of the CURRENT device into *code (a host pointer; 0 = no
+ * data error since the last clear), in stream order: the read is enqueued on `stream`
+ * (a stream of the current device) and the call waits for that stream only, so it sees
+ * every kernel enqueued on `stream` before it. Work on other streams that has not
+ * finished may set bits later. With clear != 0 the bits it returns are cleared, also in
+ * stream order; a bit that work on another stream sets meanwhile stays set. The word is
+ * one per device, shared by all streams: which stream's kernel set a bit cannot be told
+ * apart (read it after each stream's work, or keep one stream per job).
+ * (The aclnn calls report in the same two steps: the call's status on the host, then the
+ * stream's result after a stream synchronisation; gitcode ops-transformer
+ * aclnnMoeUpdateExpert doc, 调用示例.)
+ * Errors: NULL code (MEP_ERR_NULLPTR); a failed copy or synchronisation (MEP_ERR_CUDA).
  */
-mep_status_t mep_get_error(int32_t *code, int32_t clear);
+mep_status_t mep_get_error(mep_stream_t stream, int32_t *code, int32_t clear);
 
 /*
  * a1 — per-expert histogram (tokens per expert: twodots.gr article on MoonEP, "six
@@ -186,6 +201,40 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
                       int32_t *rep_count, int32_t *rep_key, int32_t *rep_cu,
                       mep_plan_stats_t *stats, void *workspace, size_t workspace_bytes,
                       mep_stream_t stream);
+
+/*
+ * (e) — one expert-parallel rank's share of the balanced plan, for the layout in which
+ * every GPU is one EP rank holding its own S tokens (MoonEP zero-copy dispatch: every
+ * token row is written straight to its final, expert-grouped row on the destination
+ * rank; twodots.gr article on MoonEP, zero-copy paragraph). Each rank computes its
+ * per-expert histogram (mep_histogram of its own ids), the ranks all-gather them into
+ * hist_all, and each rank then places its own slots exactly where mep_plan over the
+ * ids of all ranks would: the plan orders slots by (e, src, t, k), so
+ *   pos[n] = off[e] + sum_{r < rank} hist_all[r, e] + #{m < n : ids[m] == e}
+ * for this rank's slot n = t*K + k with expert e, off the exclusive prefix over experts
+ * of sum_r hist_all[r, e]. Row p belongs to destination rank p / (S*K), at local row
+ * p mod (S*K) of its receive buffer.
+ * Inputs:  ids int32 [S*K] (this rank's slots); hist_all int32 [R, E] (row r = rank r's
+ *          histogram, the same on every rank); rank in [0, R).
+ * Outputs (device, overwritten):
+ *   pos        int32 [S*K]  global row of every slot of this rank
+ *   send_count int32 [R]    rows this rank writes into rank d's partition
+ *   send_off   int32 [R+1]  exclusive prefix of send_count (a send buffer packed by
+ *                           destination: slots in ascending pos)
+ *   recv_count int32 [R]    rows rank s writes into this rank's partition
+ *   recv_off   int32 [R+1]  exclusive prefix of recv_count; recv_off[R] = S*K
+ * Workspace: mep_plan_rank_workspace_size(R, E, S, K) bytes, 256-byte aligned.
+ * Errors: NULL pointer; R, S, K < 1, K > MEP_MAX_K, E outside [1, MEP_MAX_KEYS],
+ * R > MEP_MAX_KEYS, R*S*K >= 2^31 (MEP_ERR_SHAPE); E % R != 0, rank outside [0, R)
+ * (MEP_ERR_VALUE); workspace (MEP_ERR_WORKSPACE). Data errors: ids outside [0, E)
+ * (dropped, pos = -1, MEP_DERR_KEY_RANGE); row `rank` of hist_all differs from the
+ * histogram of ids (MEP_DERR_HIST: the ranks' inputs disagree, the rows are not a plan).
+ */
+size_t mep_plan_rank_workspace_size(int32_t R, int32_t E, int32_t S, int32_t K);
+mep_status_t mep_plan_rank(const int32_t *ids, const int32_t *hist_all, int32_t R, int32_t E,
+                           int32_t S, int32_t K, int32_t rank, int32_t *pos, int32_t *send_count,
+                           int32_t *send_off, int32_t *recv_count, int32_t *recv_off,
+                           void *workspace, size_t workspace_bytes, mep_stream_t stream);
 
 /*
  * a5 with int8 rows (quantised return path) — combine of per-row int8 codes with one
@@ -348,9 +397,11 @@ mep_status_t mep_selftest_bounded_wait(int32_t max_polls, int32_t *timed_out, me
  * outputs are still the caller's. This call allocates nothing: no cudaMalloc, no
  * cudaFree, no allocating library routine.
  *
- * Set-up: the first call on each device looks up the array's device address with
- * cudaGetSymbolAddress (for the device current at that call) and keeps it; make that
- * first call on a device before any stream capture.
+ * Set-up: the first call of the library in a CUDA context (the device's primary
+ * context, or a context the caller made current) looks up the array's device address
+ * with cudaGetSymbolAddress, with that context current, and keeps it for that context;
+ * after cudaDeviceReset, or under another context, the next call looks it up again.
+ * Make the first call in a context before any stream capture.
  * Sharing: all calls on a device use the same array, which keeps the contents of the
  * last call. The plan kernels write every scratch word before they read it, so nothing
  * has to be cleared between calls. Calls that overlap on the GPU (unordered streams)

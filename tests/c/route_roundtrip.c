@@ -80,7 +80,7 @@ int main(void)
     CHECK(mep_combine(d_recv, N, d_pos, d_g, T, K, H, d_out, st) == MEP_OK);
     CHECK(cudaStreamSynchronize(st) == cudaSuccess);
     int32_t derr = -1;
-    CHECK(mep_get_error(&derr, 1) == MEP_OK && derr == 0);
+    CHECK(mep_get_error(st, &derr, 1) == MEP_OK && derr == 0);
 
     CHECK(cudaMemcpy(pos, d_pos, sizeof(int32_t) * N, cudaMemcpyDeviceToHost) == cudaSuccess);
     CHECK(cudaMemcpy(rank_off, d_roff, sizeof(int32_t) * (R + 1), cudaMemcpyDeviceToHost) == cudaSuccess);

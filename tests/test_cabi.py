@@ -142,7 +142,7 @@ def test_dispatch_combine_argument_checks(L):
     assert L.mep_histogram(P, 10, 0, P, None) == 3
     assert L.mep_histogram(P, 10, 4, None, None) == 1
     assert L.mep_dequantize(None, P, 4, 8, P, None) == 1
-    assert L.mep_get_error(None, 0) == 1
+    assert L.mep_get_error(None, None, 0) == 1
     L.mep_selftest_bounded_wait.argtypes = [ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
     assert L.mep_selftest_bounded_wait(10, None, None) == 1
     assert L.mep_selftest_bounded_wait(0, P, None) == 4
@@ -214,3 +214,41 @@ def test_maxvio_from_a_plan_summary(L, golden_dir):
     assert L.mep_maxvio(None, 2, 2, 4, None, None, None) == 1
     buf = (ctypes.c_int32 * 8)()
     assert L.mep_maxvio(ctypes.cast(buf, ctypes.c_void_p), 0, 2, 4, None, None, None) == 3
+
+
+def test_static_ws_checks_arguments_before_its_size(L):
+    """mep_plan_static_ws reports mep_plan's argument errors first: a call that is both
+    invalid and larger than the 4 MiB array gets the argument's status, not
+    MEP_ERR_WORKSPACE (which is only for a valid plan that does not fit)."""
+    P = FAKE
+    big = dict(R=8, E=2048, S=32768, K=8)          # 2^21 slots x 2048 keys: 8 MiB of scratch
+    import dispatch_combine_topk_b200 as mep
+    assert mep.mep_plan_workspace_size(big["R"], big["E"], big["S"], big["K"]) > 4 << 20
+
+    def call(ids=P, keep=None, R=big["R"], E=big["E"], S=big["S"], K=big["K"], mode=0, kpr=0):
+        return L.mep_plan_static_ws(ids, keep, R, E, S, K, mode, kpr, P, P, P, None, P, P, P, P, None)
+    assert call(K=33) == 3                         # SHAPE, not WORKSPACE
+    assert call(E=2047) == 4                       # VALUE: E % R != 0
+    assert call(mode=9) == 4
+    assert call(keep=P) == 4
+    assert call(ids=None) == 1
+    assert call() == 5                             # valid, too large: WORKSPACE
+
+
+def test_plan_rank_argument_checks(L):
+    P = FAKE
+
+    def call(ids=P, hist=P, R=4, E=16, S=8, K=2, rank=0, ws=P, wsb=1 << 20):
+        return L.mep_plan_rank(ids, hist, R, E, S, K, rank, P, P, P, P, P, ws, wsb, None)
+    assert call(ids=None) == 1
+    assert call(hist=None) == 1
+    assert call(R=0) == 3
+    assert call(K=33) == 3
+    assert call(E=5000) == 3
+    assert call(E=18) == 4                         # E % R != 0
+    assert call(rank=4) == 4
+    assert call(rank=-1) == 4
+    assert call(ws=None) == 5
+    assert call(wsb=16) == 5
+    assert L.mep_plan_rank_workspace_size(0, 16, 8, 2) == 0
+    assert L.mep_plan_rank_workspace_size(4, 16, 8, 2) > 0

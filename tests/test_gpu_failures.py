@@ -90,3 +90,22 @@ def test_stream_synchronize_timeout_gives_up_then_sees_the_work_finish():
     assert mep.mep_stream_synchronize_timeout(60000, stream=s) is True
     assert np.array_equal(bits(recv), oracle.dispatch(bits(x), pos, K, T * K))
     assert mep.mep_get_error() == 0
+
+
+def test_error_word_is_read_in_stream_order():
+    """mep_get_error reads the word in order on the stream it is given, waiting for that
+    stream only: a data error set by a kernel enqueued just before on the same stream is
+    seen without any other synchronisation, and clearing it is ordered the same way."""
+    torch.cuda.set_device(0)
+    s = torch.cuda.Stream(dev())
+    torch.cuda.synchronize()
+    assert mep.mep_get_error(clear=True, stream=s) == 0
+    T, K, H = 4, 2, 64
+    x = torch.zeros((T, H), dtype=torch.bfloat16, device=dev())
+    pos = torch.tensor([0, 1, 2, 3, 4, 5, 6, 99], dtype=torch.int32, device=dev())
+    recv = torch.zeros((T * K, H), dtype=torch.bfloat16, device=dev())
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        mep.mep_dispatch(x, pos, K, recv, stream=s)
+        assert mep.mep_get_error(clear=True, stream=s) == mep.DERR_ROW_RANGE
+        assert mep.mep_get_error(clear=False, stream=s) == 0

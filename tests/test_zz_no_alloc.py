@@ -99,3 +99,25 @@ def test_static_scratch_plan_refuses_plans_larger_than_its_array():
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     rc = _entry()(_p(one), None, R, n_keys, S, K, 0, 0, *[_p(one)] * 8, stream)
     assert rc == MEP_ERR_WORKSPACE
+
+
+def test_static_scratch_plan_after_a_device_reset(tmp_path):
+    """The array's device address belongs to a CUDA context: after cudaDeviceReset the
+    library must look it up again. A C program (its own process, so the reset cannot
+    touch this one's context) plans with the static scratch and with a workspace, resets
+    the device, and plans both ways twice more; every output must match bit for bit."""
+    import os
+    import subprocess
+    from dispatch_combine_topk_b200 import build
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lib = build.build()
+    exe = tmp_path / "static_ws_reset"
+    cuda = "/usr/local/cuda"
+    subprocess.run(["gcc", "-O2", "-std=c11", os.path.join(root, "tests", "c", "static_ws_reset.c"),
+                    "-I", os.path.join(root, "include"), "-I", os.path.join(cuda, "include"),
+                    "-L", os.path.dirname(lib), "-lmep", "-L", os.path.join(cuda, "lib64"), "-lcudart",
+                    "-Wl,-rpath," + os.path.dirname(lib), "-Wl,-rpath," + os.path.join(cuda, "lib64"),
+                    "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert "static_ws_reset ok" in r.stdout
