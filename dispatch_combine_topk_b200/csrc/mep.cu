@@ -29,6 +29,10 @@ thread_local int32_t t_last_cuda_error = 0;
 constexpr int kMaxDevices = 64;
 // Shared memory the staged int8 dispatch may use per CTA.
 constexpr int kBulkSmemMax = 200 * 1024;
+// Plans of at most this many slots (and few enough keys for the shared memory below) run
+// as one CTA: below it the four-kernel plan is bound by launch latency.
+constexpr int64_t kSmallPlanMaxSlots = 32768;
+constexpr int kSmallPlanSmemMax = 200 * 1024;
 
 // ---------------------------------------------------------------- per-context state
 //
@@ -106,6 +110,7 @@ DeviceState &device_state(int dev)
     cudaFuncSetAttribute(mep::k_histogram, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     cudaFuncSetAttribute(mep::k_plan_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     cudaFuncSetAttribute(mep::k_source_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_plan_small, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallPlanSmemMax);
     cudaFuncSetAttribute(mep::k_dispatch_int8_staged<4, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kBulkSmemMax);
     const int norm_smem = (int)(sizeof(float) * MEP_RMSNORM_MAX_H);
@@ -289,6 +294,14 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
 
     cudaStream_t s = (cudaStream_t)stream;
     sm_count();
+    // small problems: the whole plan in one CTA (one launch instead of four)
+    const size_t small_smem = sizeof(int32_t) * (size_t)(34 * (int64_t)n_keys + 34);
+    if (N <= kSmallPlanMaxSlots && small_smem <= (size_t)kSmallPlanSmemMax) {
+        mep::k_plan_small<<<1, mep::kSmallPlanThreads, small_smem, s>>>(ids, keep, N, n_keys, R, (int64_t)S * K, mode,
+                                                                       keys_per_rank, pos, hist, rank_off, load,
+                                                                       rep_count, rep_key, rep_cu, (int32_t *)stats);
+        return launched();
+    }
     const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
     int32_t *tile_cnt = (int32_t *)workspace;
     const int threads = mep::kPlanWarps * 32;
@@ -644,6 +657,48 @@ mep_status_t mep_dispatch_int8_smooth(const uint16_t *x, const int32_t *ids, con
     const int64_t per_thread = mep::ceil_div(H8, 256);
     using smooth_k_t = void (*)(const uint4 *, const int32_t *, const int32_t *, int64_t, int64_t, const float4 *,
                                 int32_t, int64_t, uint2 *, float *);
+    // every smoothing row read once: a cluster of cl CTAs per token, four columns per
+    // thread, the smallest cl with at most kSmoothClMaxThreads threads per CTA
+    int cl = 0;
+    for (int c = 2; c <= 8 && !cl; c *= 2)
+        if (H % (128 * c) == 0 && H / (4 * c) <= mep::kSmoothClMaxThreads) cl = c;
+    if (cl && (K == 2 || K == 4 || K == 8) && aligned(x, 8) && aligned(smooth, 16) && aligned(recv, 4)) {
+        using cl_k_t = void (*)(const uint2 *, const int32_t *, const int32_t *, int64_t, int64_t, const float4 *,
+                                int32_t, int64_t, uint32_t *, float *);
+        cl_k_t kern = nullptr;
+#define MEP_SMOOTH_CL(KC_)                                                                          \
+    kern = cl == 2 ? mep::k_dispatch_int8_smooth_cl<KC_, 2>                                          \
+                   : (cl == 4 ? mep::k_dispatch_int8_smooth_cl<KC_, 4> : mep::k_dispatch_int8_smooth_cl<KC_, 8>)
+        if (K == 2) MEP_SMOOTH_CL(2);
+        else if (K == 4) MEP_SMOOTH_CL(4);
+        else MEP_SMOOTH_CL(8);
+#undef MEP_SMOOTH_CL
+        const int threads = (int)(H / (4 * cl));
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)cl;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.blockDim = dim3((unsigned)threads);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        // as many clusters as the GPU holds at once (never more than tokens)
+        int max_cl = 0;
+        cfg.gridDim = dim3((unsigned)(cl * sm_count()));
+        if (cudaOccupancyMaxActiveClusters(&max_cl, kern, &cfg) != cudaSuccess || max_cl < 1) {
+            (void)cudaGetLastError();
+            max_cl = sm_count() / cl;
+        }
+        const int64_t ncl = T < max_cl ? T : max_cl;
+        cfg.gridDim = dim3((unsigned)(cl * (ncl > 0 ? ncl : 1)));
+        if (cudaLaunchKernelEx(&cfg, kern, (const uint2 *)x, ids, pos, T, H / 4, (const float4 *)smooth, n_experts,
+                               rows, (uint32_t *)recv, recv_scale) != cudaSuccess)
+            return launched();
+        return launched();
+    }
     smooth_k_t fused = nullptr;
     if (vec && per_thread <= 8) {
         const bool c4 = per_thread <= 4;

@@ -231,16 +231,15 @@ __device__ __forceinline__ int32_t upper_bound_sh(const int32_t *a, int32_t n, i
     return lo;
 }
 
-// One CTA of 1024 threads: per-rank replica tables and the summary counts.
-// Dynamic shared memory: key_off (n_keys+1) + nz (n_keys+1) + rank_off (R+1) + e_lo (R).
-__global__ void __launch_bounds__(1024)
-k_plan_meta(const int32_t *__restrict__ hist, int32_t R,
-            int32_t n_keys, int64_t SK, int32_t mode, int32_t keys_per_rank,
-            int32_t *__restrict__ rank_off_out, int32_t *__restrict__ load_out,
-            int32_t *__restrict__ rep_count, int32_t *__restrict__ rep_key,
-            int32_t *__restrict__ rep_cu, int32_t *__restrict__ stats)
+// Per-rank replica tables and the summary counts, by one CTA of 1024 threads.
+// smem: key_off (n_keys+1) + nz (n_keys+1) + rank_off (R+1) + e_lo (R) ints.
+__device__ __forceinline__ void plan_meta(const int32_t *__restrict__ hist, int32_t R,
+                                          int32_t n_keys, int64_t SK, int32_t mode, int32_t keys_per_rank,
+                                          int32_t *__restrict__ rank_off_out, int32_t *__restrict__ load_out,
+                                          int32_t *__restrict__ rep_count, int32_t *__restrict__ rep_key,
+                                          int32_t *__restrict__ rep_cu, int32_t *__restrict__ stats,
+                                          int32_t *smem)
 {
-    extern __shared__ int32_t smem[];
     int32_t *koff = smem;                    // n_keys + 1
     int32_t *nz = koff + (n_keys + 1);       // n_keys + 1: exclusive count of non-empty keys
     int32_t *roff = nz + (n_keys + 1);       // R + 1
@@ -352,6 +351,90 @@ k_plan_meta(const int32_t *__restrict__ hist, int32_t R,
         stats[6] = s_red[6];
         stats[7] = 0;
     }
+}
+
+// Dynamic shared memory: as plan_meta.
+__global__ void __launch_bounds__(1024)
+k_plan_meta(const int32_t *__restrict__ hist, int32_t R,
+            int32_t n_keys, int64_t SK, int32_t mode, int32_t keys_per_rank,
+            int32_t *__restrict__ rank_off_out, int32_t *__restrict__ load_out,
+            int32_t *__restrict__ rep_count, int32_t *__restrict__ rep_key,
+            int32_t *__restrict__ rep_cu, int32_t *__restrict__ stats)
+{
+    extern __shared__ int32_t smem[];
+    plan_meta(hist, R, n_keys, SK, mode, keys_per_rank, rank_off_out, load_out, rep_count, rep_key, rep_cu, stats,
+              smem);
+}
+
+// The whole plan in one CTA of 1024 threads, for small problems (a few thousand slots,
+// where the four-kernel plan is bound by launch latency): the same stable counting
+// sort with a single tile. Each of the 32 warps owns a contiguous sub-range of the
+// slots: it counts its keys, the CTA turns the counts into per-warp bases (after hist
+// and its prefix over keys), each warp ranks its sub-range in order, then plan_meta
+// writes the replica tables. Writes hist to global memory before plan_meta reads it.
+// Dynamic shared memory: 33 * n_keys + n_keys + 1 + 33 ints (plan_meta reuses the start,
+// which n_keys >= R keeps inside the per-warp counts).
+constexpr int kSmallPlanThreads = 1024;
+
+__global__ void __launch_bounds__(kSmallPlanThreads)
+k_plan_small(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, int64_t N, int32_t n_keys,
+             int32_t R, int64_t SK, int32_t mode, int32_t keys_per_rank, int32_t *__restrict__ pos,
+             int32_t *__restrict__ hist, int32_t *__restrict__ rank_off_out, int32_t *__restrict__ load_out,
+             int32_t *__restrict__ rep_count, int32_t *__restrict__ rep_key, int32_t *__restrict__ rep_cu,
+             int32_t *__restrict__ stats)
+{
+    extern __shared__ int32_t smem[];
+    constexpr int kWarps = kSmallPlanThreads / 32;
+    int32_t *cnt = smem;                              // [kWarps][n_keys]
+    int32_t *key_off = cnt + kWarps * n_keys;         // n_keys + 1
+    int32_t *scan_scratch = key_off + n_keys + 1;     // 33
+    int32_t *tot = scan_scratch + 33;                 // n_keys: hist, kept for plan_meta
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < kWarps * n_keys; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+    const int64_t sub = ((N + kWarps - 1) / kWarps + 31) / 32 * 32;
+    const int64_t lo = (int64_t)warp * sub, hi = min(N, lo + sub);
+    int32_t *mine = cnt + warp * n_keys;
+    for (int64_t n0 = lo; n0 < hi; n0 += 32) {
+        int32_t key = slot_key(ids, keep, n0 + lane, hi, n_keys);
+        uint32_t peers = __match_any_sync(0xffffffffu, key);
+        if (key >= 0 && lane == __ffs(peers) - 1) mine[key] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    // per key: exclusive prefix over warps (in place) and the total
+    for (int e = threadIdx.x; e < n_keys; e += blockDim.x) {
+        int32_t run = 0;
+        for (int w = 0; w < kWarps; w++) {
+            const int32_t v = cnt[w * n_keys + e];
+            cnt[w * n_keys + e] = run;
+            run += v;
+        }
+        hist[e] = run;
+        tot[e] = run;
+    }
+    __syncthreads();
+    block_exclusive_scan(tot, n_keys, key_off, scan_scratch);
+    for (int e = threadIdx.x; e < n_keys; e += blockDim.x) {
+        const int32_t b = key_off[e];
+        for (int w = 0; w < kWarps; w++) cnt[w * n_keys + e] += b;
+    }
+    __syncthreads();
+    const uint32_t lt = lanemask_lt();
+    for (int64_t n0 = lo; n0 < hi; n0 += 32) {
+        const int64_t n = n0 + lane;
+        int32_t key = slot_key(ids, keep, n, hi, n_keys);
+        uint32_t peers = __match_any_sync(0xffffffffu, key);
+        int32_t p = -1;
+        if (key >= 0) p = mine[key] + __popc(peers & lt);
+        __syncwarp();
+        if (key >= 0 && lane == __ffs(peers) - 1) mine[key] += __popc(peers);
+        __syncwarp();
+        if (n < hi) pos[n] = p;
+    }
+    __syncthreads();
+    plan_meta(tot, R, n_keys, SK, mode, keys_per_rank, rank_off_out, load_out, rep_count, rep_key, rep_cu, stats,
+              smem);
 }
 
 // ------------------------------------------------ one rank's share of the plan (e)

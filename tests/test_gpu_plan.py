@@ -32,9 +32,14 @@ def test_histogram_parity_ragged_and_skewed():
     assert mep.mep_get_error() == 0
 
 
+# Plans of at most 32768 slots with few enough keys run as one CTA, the others as the
+# tiled four-kernel sort: the cases cover both, at and just past the boundary (ragged last
+# tile), and small plans whose keys are too many for the one-CTA path.
 @pytest.mark.parametrize("R,E,S,K", [
     (2, 4, 2, 2), (3, 9, 37, 3), (4, 12, 1000, 3), (4, 16, 128, 2), (8, 64, 300, 8),
     (1, 5, 17, 1), (16, 4096, 32, 4), (8, 4096, 512, 8), (5, 5, 2048, 1),
+    (4, 16, 2048, 4), (7, 7, 4681, 1), (2, 1024, 8192, 2), (3, 9, 3641, 3), (1, 2, 32769, 1),
+    (64, 1536, 8, 8),
 ])
 def test_plan_balanced_parity_random(R, E, S, K):
     rng = np.random.default_rng(R * 7919 + E * 31 + S)
@@ -207,9 +212,10 @@ def test_update_expert_data_errors_flag():
     assert mep.mep_get_error() & mep.DERR_KEY_RANGE
 
 
-def test_grouped_plan_all_dropped_and_ragged():
-    R, kpr, S, K = 4, 5, 333, 3
-    rng = np.random.default_rng(9)
+@pytest.mark.parametrize("R,kpr,S,K", [(4, 5, 333, 3), (4, 34, 3000, 3), (8, 34, 256, 8)])
+def test_grouped_plan_all_dropped_and_ragged(R, kpr, S, K):
+    """One-CTA plans (the first and last shapes) and a tiled one (36,000 slots)."""
+    rng = np.random.default_rng(9 + S)
     keys = rng.integers(0, R * kpr, R * S * K).astype(np.int32)
     for keep in [np.zeros(R * S * K, np.uint8), (rng.random(R * S * K) < 0.5).astype(np.uint8),
                  np.ones(R * S * K, np.uint8)]:

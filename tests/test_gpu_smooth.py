@@ -1,7 +1,10 @@
 """GPU parity of the int8 dispatch with per-expert smoothing scales against the oracle
-(codes and scales bit for bit; K in {2, 4, 8} takes the fused kernel, the others the
-per-slot one), and the special case of all-ones scales against the plain per-token int8
-dispatch on the full int8 workload."""
+(codes and scales bit for bit). K in {2, 4, 8} with H a multiple of 256 takes the
+cluster kernel (2, 4 or 8 CTAs per token), other K the per-slot kernel, other H the
+one-CTA kernels. The full int8 workload is compared whole, one rank partition at a time,
+and with all-ones scales against the plain per-token int8 dispatch."""
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import pytest
 import torch
@@ -35,7 +38,61 @@ def test_smooth_dispatch_matches_oracle(K, H):
     assert mep.mep_get_error() == 0
 
 
+@pytest.mark.parametrize("K,H", [(2, 4096), (4, 7168), (8, 4096), (8, 12288), (8, 7168)])
+def test_smooth_dispatch_many_tokens_per_cluster(K, H):
+    """More tokens than clusters resident on the GPU, so every cluster walks many tokens
+    (the shared buffers alternate by token parity); dropped slots and whole buffers."""
+    rng = np.random.default_rng(K * 13 + H)
+    T, E = 3001, 40
+    x = (torch.randn((T, H), generator=torch.Generator().manual_seed(H + K)) * 3).to(torch.bfloat16)
+    ids = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
+    rows = T * K + 5
+    pos = rng.permutation(rows)[: T * K].astype(np.int32)
+    pos[rng.random(T * K) < 0.1] = -1
+    sm = (10.0 ** rng.uniform(-1.5, 1.5, (E, H))).astype(np.float32)
+    q = torch.zeros((rows, H), dtype=torch.int8, device=dev())
+    sc = torch.zeros(rows, dtype=torch.float32, device=dev())
+    mep.mep_dispatch_int8_smooth(x.to(dev()), torch.from_numpy(ids).to(dev()).view(-1),
+                                 torch.from_numpy(pos).to(dev()), K, torch.from_numpy(sm).to(dev()), q, sc)
+    q_ref, s_ref = oracle.dispatch_int8_smooth(bits(x), ids, pos, K, sm, rows)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert mep.mep_get_error() == 0
+
+
+def test_smooth_dispatch_bad_ids_and_rows_are_skipped_and_flagged():
+    T, K, H, E = 64, 4, 4096, 8
+    rng = np.random.default_rng(5)
+    x = torch.randn((T, H), generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    ids = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
+    pos = np.arange(T * K, dtype=np.int32)
+    ids[3, 1] = E + 2                                      # expert out of range: slot skipped
+    sm = np.ones((E, H), np.float32)
+    q = torch.full((T * K + 1, H), 55, dtype=torch.int8, device=dev())
+    sc = torch.full((T * K + 1,), 7.0, dtype=torch.float32, device=dev())
+    mep.mep_dispatch_int8_smooth(x.to(dev()), torch.from_numpy(ids).to(dev()).view(-1),
+                                 torch.from_numpy(pos).to(dev()), K, torch.from_numpy(sm).to(dev()), q[: T * K],
+                                 sc[: T * K])
+    assert mep.mep_get_error() & mep.DERR_KEY_RANGE
+    assert bool((q[3 * K + 1] == 55).all()) and sc[3 * K + 1].item() == 7.0
+    assert bool((q[T * K] == 55).all())                     # the guard row is untouched
+    keep = np.ones(T * K, bool)
+    keep[3 * K + 1] = False
+    pos_ok = np.where(keep, pos, -1).astype(np.int32)
+    q_ref, s_ref = oracle.dispatch_int8_smooth(bits(x), np.where(ids < E, ids, 0), pos_ok, K, sm, T * K)
+    got = q[: T * K].cpu().numpy()
+    assert np.array_equal(got[keep], q_ref[keep])
+    pos_bad = pos.copy()
+    pos_bad[10] = T * K + 1                                # row out of range: slot skipped
+    mep.mep_dispatch_int8_smooth(x.to(dev()), torch.from_numpy(np.where(ids < E, ids, 0)).to(dev()).view(-1),
+                                 torch.from_numpy(pos_bad).to(dev()), K, torch.from_numpy(sm).to(dev()), q[: T * K],
+                                 sc[: T * K])
+    assert mep.mep_get_error() & mep.DERR_ROW_RANGE
+
+
 def test_smooth_dispatch_full_int8_workload():
+    """The whole int8 workload: every code and scale against the oracle, one rank
+    partition at a time; with all-ones scales, the plain per-token int8 dispatch."""
     w = synth.get("int8")
     ids, _ = synth.router(w)
     x = synth.hidden(w)
@@ -50,23 +107,34 @@ def test_smooth_dispatch_full_int8_workload():
     s0 = torch.empty_like(sc)
     mep.mep_dispatch(x_d, pb.pos, w.K, q0, s0, quant=1)
     assert torch.equal(q, q0) and torch.equal(sc.view(torch.int32), s0.view(torch.int32))
-    # per-expert scales: sampled tokens, every slot, against the oracle
+    del q0, s0
+    # per-expert scales: every slot against the oracle
     rng = np.random.default_rng(21)
     sm = (10.0 ** rng.uniform(-1, 1, (w.E, w.H))).astype(np.float32)
     mep.mep_dispatch_int8_smooth(x_d, ids_d, pb.pos, w.K, torch.from_numpy(sm).to(dev()), q, sc)
-    pos = pb.pos.cpu().numpy()
-    for t in np.unique(np.concatenate([[0, w.T - 1], rng.integers(0, w.T, 60)])):
-        sl = slice(t * w.K, (t + 1) * w.K)
-        q_ref, s_ref = oracle.dispatch_int8_smooth(bits(x[t:t + 1]), ids[t][None, :],
-                                                   np.arange(w.K, dtype=np.int32), w.K, sm, w.K)
-        rows = torch.from_numpy(pos[sl].astype(np.int64)).to(dev())
-        assert np.array_equal(q[rows].cpu().numpy(), q_ref)
-        assert np.array_equal(sc[rows].cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    torch.cuda.synchronize()
+    p = oracle.plan_balanced(ids, w.R, w.E, w.S, w.K)
+    assert np.array_equal(pb.pos.cpu().numpy(), p.pos)
+    xb = bits(x)
+    SK = w.S * w.K
+
+    def one(r):
+        lo, hi = r * SK, (r + 1) * SK
+        inside = (p.pos >= lo) & (p.pos < hi)
+        toks = np.unique(np.flatnonzero(inside) // w.K)
+        pos_r = np.where(inside, p.pos - lo, -1).astype(np.int32).reshape(-1, w.K)[toks]
+        q_ref, s_ref = oracle.dispatch_int8_smooth(xb[toks], ids[toks], pos_r, w.K, sm, SK)
+        assert np.array_equal(q[lo:hi].cpu().numpy(), q_ref), r
+        assert np.array_equal(sc[lo:hi].cpu().numpy().view(np.uint32), s_ref.view(np.uint32)), r
+        return r
+    with ThreadPoolExecutor(8) as ex:
+        assert sorted(ex.map(one, range(w.R))) == list(range(w.R))
     assert mep.mep_get_error() == 0
 
 
+@pytest.mark.parametrize("K", [1, 2])
 @pytest.mark.parametrize("amax", [381.0, 88.9, 1.0e-3, 5.0e30, 1.0e-36])
-def test_quantiser_at_and_next_to_half_integer_quotients(amax):
+def test_quantiser_at_and_next_to_half_integer_quotients(amax, K):
     """Codes of values whose quotient by the scale sits on or within a few ulps of a
     half-integer, where a quotient taken through the reciprocal could round the other
     way: with x = 1, the smoothing scales are the quantised values themselves. Column 0
@@ -82,17 +150,21 @@ def test_quantiser_at_and_next_to_half_integer_quotients(amax):
                 v = np.nextafter(v, np.float32(np.inf if j > 0 else -np.inf), dtype=np.float32)
             if abs(v) <= np.float32(amax):
                 vals.append(v)
-    H = (len(vals) + 7) // 8 * 8
-    sm = np.zeros((1, H), np.float32)
+    # K = 1: the per-slot kernel (H a multiple of 8); K = 2: the cluster kernel (H a
+    # multiple of 256), the second slot on a second expert holding the values reversed
+    H = (len(vals) + 7) // 8 * 8 if K == 1 else (len(vals) + 255) // 256 * 256
+    sm = np.zeros((K, H), np.float32)
     sm[0, :len(vals)] = vals
+    if K == 2:
+        sm[1, :len(vals)] = vals[::-1]
     x = torch.ones((1, H), dtype=torch.bfloat16)
-    ids = np.zeros((1, 1), np.int32)
-    pos = np.zeros(1, np.int32)
-    q = torch.zeros((1, H), dtype=torch.int8, device=dev())
-    s = torch.zeros(1, dtype=torch.float32, device=dev())
+    ids = np.arange(K, dtype=np.int32)[None, :]
+    pos = np.arange(K, dtype=np.int32)
+    q = torch.zeros((K, H), dtype=torch.int8, device=dev())
+    s = torch.zeros(K, dtype=torch.float32, device=dev())
     mep.mep_dispatch_int8_smooth(x.to(dev()), torch.from_numpy(ids).to(dev()).view(-1),
-                                 torch.from_numpy(pos).to(dev()), 1, torch.from_numpy(sm).to(dev()), q, s)
-    q_ref, s_ref = oracle.dispatch_int8_smooth(bits(x), ids, pos, 1, sm, 1)
+                                 torch.from_numpy(pos).to(dev()), K, torch.from_numpy(sm).to(dev()), q, s)
+    q_ref, s_ref = oracle.dispatch_int8_smooth(bits(x), ids, pos, K, sm, K)
     assert s_ref[0] == sc32
     assert np.array_equal(q.cpu().numpy(), q_ref)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
