@@ -409,10 +409,10 @@ class Route:
             mep.mep_plan(self.bids.view(-1), w.R, self.n_keys, w.S, w.K, self.pb,
                          mode=mep.MEP_PLAN_GROUPED, keys_per_rank=w.place_per_rank,
                          keep=self.bmask.view(-1), stream=s)
-            n = 1 + 4
+            n = 1 + mep.mep_plan_launches(w.R, self.n_keys, w.S, w.K)
         else:
             mep.mep_plan(self.ids, w.R, w.E, w.S, w.K, self.pb, stream=s)
-            n = 4
+            n = mep.mep_plan_launches(w.R, w.E, w.S, w.K)
         if self.dedup:
             mep.mep_dedup_plan(self.pb.pos, self.pb.rank_off, w.R, w.S, w.K, self.db, stream=s)
             n += 6
@@ -894,7 +894,9 @@ def run_gpu(args, w):
     ok_device = rt.result_ok()
 
     e2e_steps = max(4, min(args.steps, 20))
-    if not w.mapping and args.epilogue == "none" and not args.dedup and not args.smooth:
+    if args.no_e2e:
+        e2e_ms, ok_e2e, h2d, d2h, how = None, None, None, None, "skipped (--no-e2e)"
+    elif not w.mapping and args.epilogue == "none" and not args.dedup and not args.smooth:
         e2e_ms, ok_e2e, h2d, d2h, how = e2e_route_host(mep, rt, w, dev, e2e_steps, pg)
     else:
         e2e_ms, ok_e2e, h2d, d2h, how = e2e_pipeline(rt, w, dev, stream, e2e_steps, pg)
@@ -932,9 +934,9 @@ def run_gpu(args, w):
             "dispatch_combine": dc,
             "roofline": roof,
             "cpu_baseline": cpu,
-            "e2e": {"value": world * w.N / (e2e_ms * 1e-3), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                    "path": how},
+            "e2e": None if e2e_ms is None else {
+                "value": world * w.N / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "path": how},
             "result_check": {"device": ok_device, "e2e": ok_e2e},
             "gpu_launches": tm["launches"],
             "clocks": tm["clocks"],
@@ -976,6 +978,8 @@ def main():
     ap.add_argument("--cpu-div", type=int, default=1,
                     help="cpu_baseline: the oracle routes S/cpu_div tokens per rank once")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end leg (for profiling runs; the line then has no e2e)")
     ap.add_argument("--graph", type=int, default=1,
                     help="1: time the step as a replayed CUDA graph (per-kernel breakdown "
                          "still comes from the eager steps); 0: eager only")

@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.mep_histogram.argtypes = [P, i64, i32, P, P]
         L.mep_plan_workspace_size.argtypes = [i32, i32, i32, i32]
         L.mep_plan_workspace_size.restype = ctypes.c_size_t
+        L.mep_plan_launches.argtypes = [i32, i32, i32, i32]
+        L.mep_plan_launches.restype = i32
         L.mep_plan.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P,
                                ctypes.c_size_t, P]
         L.mep_update_expert.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i64, i64, P, P, P]
@@ -181,6 +183,11 @@ def mep_histogram(ids: torch.Tensor, n_keys: int, hist: torch.Tensor, stream=Non
 def mep_plan_workspace_size(R: int, n_keys: int, S: int, K: int) -> int:
     """Bytes of scratch mep_plan needs for this shape (PlanBuffers.allocate uses it)."""
     return int(lib().mep_plan_workspace_size(R, n_keys, S, K))
+
+
+def mep_plan_launches(R: int, n_keys: int, S: int, K: int) -> int:
+    """Kernels mep_plan launches for this shape (1: one CTA; 4: the tiled sort)."""
+    return int(lib().mep_plan_launches(R, n_keys, S, K))
 
 
 @dataclasses.dataclass

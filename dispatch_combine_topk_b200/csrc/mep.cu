@@ -29,9 +29,8 @@ thread_local int32_t t_last_cuda_error = 0;
 constexpr int kMaxDevices = 64;
 // Shared memory the staged int8 dispatch may use per CTA.
 constexpr int kBulkSmemMax = 200 * 1024;
-// Plans of at most this many slots (and few enough keys for the shared memory below) run
-// as one CTA: below it the four-kernel plan is bound by launch latency.
-constexpr int64_t kSmallPlanMaxSlots = 32768;
+// Plans of at most mep::kSmallPlanMaxSlots slots (and few enough keys for the shared
+// memory below) run as one CTA: there the four-kernel plan is bound by launch latency.
 constexpr int kSmallPlanSmemMax = 200 * 1024;
 
 // ---------------------------------------------------------------- per-context state
@@ -278,6 +277,21 @@ mep_status_t plan_args(const int32_t *ids, const uint8_t *keep, int32_t R, int32
 
 extern "C" {
 
+namespace {
+// Whether mep_plan runs as one CTA for this shape.
+bool plan_is_small(int64_t N, int32_t n_keys)
+{
+    const size_t small_smem = sizeof(int32_t) * (size_t)(34 * (int64_t)n_keys + 34);
+    return N <= mep::kSmallPlanMaxSlots && small_smem <= (size_t)kSmallPlanSmemMax;
+}
+}  // namespace
+
+int32_t mep_plan_launches(int32_t R, int32_t n_keys, int32_t S, int32_t K)
+{
+    if (R < 1 || S < 1 || K < 1 || n_keys < 1) return 0;
+    return plan_is_small((int64_t)R * S * K, n_keys) ? 1 : 4;
+}
+
 mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_t n_keys,
                       int32_t S, int32_t K, int32_t mode, int32_t keys_per_rank,
                       int32_t *pos, int32_t *hist, int32_t *rank_off, int32_t *load,
@@ -295,8 +309,8 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
     cudaStream_t s = (cudaStream_t)stream;
     sm_count();
     // small problems: the whole plan in one CTA (one launch instead of four)
-    const size_t small_smem = sizeof(int32_t) * (size_t)(34 * (int64_t)n_keys + 34);
-    if (N <= kSmallPlanMaxSlots && small_smem <= (size_t)kSmallPlanSmemMax) {
+    if (plan_is_small(N, n_keys)) {
+        const size_t small_smem = sizeof(int32_t) * (size_t)(34 * (int64_t)n_keys + 34);
         mep::k_plan_small<<<1, mep::kSmallPlanThreads, small_smem, s>>>(ids, keep, N, n_keys, R, (int64_t)S * K, mode,
                                                                        keys_per_rank, pos, hist, rank_off, load,
                                                                        rep_count, rep_key, rep_cu, (int32_t *)stats);
@@ -528,8 +542,9 @@ mep_status_t mep_combine_int8(const int8_t *yq, const float *y_scale, int64_t ro
         default: kern = mep::k_combine_int8_warp<0>; break;
         }
         // one warp per token, grid-stride: as many CTAs as can be resident at once
-        kern<<<resident_grid(kern, 128, mep::ceil_div(T, 4)), 128, 0, s>>>(yv, y_scale, pos, gates, T, K, H16,
-                                                                           rows, ov);
+        const int tpb = mep::kCombineInt8Threads;
+        kern<<<resident_grid(kern, tpb, mep::ceil_div(T, tpb / 32)), tpb, 0, s>>>(yv, y_scale, pos, gates, T, K, H16,
+                                                                                   rows, ov);
     } else if (H % 8 == 0 && aligned(yq, 8) && aligned(out, 16)) {
         const uint2 *yv = (const uint2 *)yq;
         uint4 *ov = (uint4 *)out;

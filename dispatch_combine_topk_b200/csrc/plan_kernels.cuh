@@ -366,15 +366,18 @@ k_plan_meta(const int32_t *__restrict__ hist, int32_t R,
               smem);
 }
 
-// The whole plan in one CTA of 1024 threads, for small problems (a few thousand slots,
+// The whole plan in one CTA of 1024 threads, for small problems (up to 16384 slots,
 // where the four-kernel plan is bound by launch latency): the same stable counting
 // sort with a single tile. Each of the 32 warps owns a contiguous sub-range of the
-// slots: it counts its keys, the CTA turns the counts into per-warp bases (after hist
-// and its prefix over keys), each warp ranks its sub-range in order, then plan_meta
-// writes the replica tables. Writes hist to global memory before plan_meta reads it.
+// slots, whose keys its lanes load at once into registers (up to kSmallPlanPerLane each,
+// every load in flight together); it counts its keys, the CTA turns the counts into
+// per-warp bases (after hist and its prefix over keys), each warp ranks its sub-range in
+// order, then plan_meta writes the replica tables.
 // Dynamic shared memory: 33 * n_keys + n_keys + 1 + 33 ints (plan_meta reuses the start,
 // which n_keys >= R keeps inside the per-warp counts).
 constexpr int kSmallPlanThreads = 1024;
+constexpr int kSmallPlanPerLane = 16;
+constexpr int64_t kSmallPlanMaxSlots = (int64_t)kSmallPlanThreads * kSmallPlanPerLane;
 
 __global__ void __launch_bounds__(kSmallPlanThreads)
 k_plan_small(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, int64_t N, int32_t n_keys,
@@ -392,11 +395,22 @@ k_plan_small(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < kWarps * n_keys; i += blockDim.x) cnt[i] = 0;
     __syncthreads();
-    const int64_t sub = ((N + kWarps - 1) / kWarps + 31) / 32 * 32;
+    const int64_t sub = ((N + kWarps - 1) / kWarps + 31) / 32 * 32;   // <= 32 * kSmallPlanPerLane
     const int64_t lo = (int64_t)warp * sub, hi = min(N, lo + sub);
     int32_t *mine = cnt + warp * n_keys;
-    for (int64_t n0 = lo; n0 < hi; n0 += 32) {
-        int32_t key = slot_key(ids, keep, n0 + lane, hi, n_keys);
+    // key + 1 (0 for a dropped slot; keys < 4096) in 16-bit halves, two per register
+    uint32_t kp[kSmallPlanPerLane / 2];
+#pragma unroll
+    for (int j = 0; j < kSmallPlanPerLane; j += 2) {
+        const int32_t k0 = lo + 32 * j < hi ? slot_key(ids, keep, lo + 32 * j + lane, hi, n_keys) : -1;
+        const int32_t k1 = lo + 32 * (j + 1) < hi ? slot_key(ids, keep, lo + 32 * (j + 1) + lane, hi, n_keys) : -1;
+        kp[j / 2] = (uint32_t)(k0 + 1) | ((uint32_t)(k1 + 1) << 16);
+    }
+    auto key_at = [&](int j) -> int32_t { return (int32_t)((kp[j / 2] >> (16 * (j & 1))) & 0xffffu) - 1; };
+#pragma unroll
+    for (int j = 0; j < kSmallPlanPerLane; j++) {
+        if (lo + 32 * j >= hi) break;                 // uniform over the warp
+        const int32_t key = key_at(j);
         uint32_t peers = __match_any_sync(0xffffffffu, key);
         if (key >= 0 && lane == __ffs(peers) - 1) mine[key] += __popc(peers);
         __syncwarp();
@@ -421,9 +435,11 @@ k_plan_small(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, 
     }
     __syncthreads();
     const uint32_t lt = lanemask_lt();
-    for (int64_t n0 = lo; n0 < hi; n0 += 32) {
-        const int64_t n = n0 + lane;
-        int32_t key = slot_key(ids, keep, n, hi, n_keys);
+#pragma unroll
+    for (int j = 0; j < kSmallPlanPerLane; j++) {
+        if (lo + 32 * j >= hi) break;
+        const int64_t n = lo + 32 * j + lane;
+        const int32_t key = key_at(j);
         uint32_t peers = __match_any_sync(0xffffffffu, key);
         int32_t p = -1;
         if (key >= 0) p = mine[key] + __popc(peers & lt);

@@ -32,13 +32,13 @@ def test_histogram_parity_ragged_and_skewed():
     assert mep.mep_get_error() == 0
 
 
-# Plans of at most 32768 slots with few enough keys run as one CTA, the others as the
+# Plans of at most 16384 slots with few enough keys run as one CTA, the others as the
 # tiled four-kernel sort: the cases cover both, at and just past the boundary (ragged last
 # tile), and small plans whose keys are too many for the one-CTA path.
 @pytest.mark.parametrize("R,E,S,K", [
     (2, 4, 2, 2), (3, 9, 37, 3), (4, 12, 1000, 3), (4, 16, 128, 2), (8, 64, 300, 8),
     (1, 5, 17, 1), (16, 4096, 32, 4), (8, 4096, 512, 8), (5, 5, 2048, 1),
-    (4, 16, 2048, 4), (7, 7, 4681, 1), (2, 1024, 8192, 2), (3, 9, 3641, 3), (1, 2, 32769, 1),
+    (4, 16, 1024, 4), (7, 7, 2340, 1), (2, 1024, 4096, 2), (3, 9, 1821, 3), (1, 2, 16385, 1),
     (64, 1536, 8, 8),
 ])
 def test_plan_balanced_parity_random(R, E, S, K):
