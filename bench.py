@@ -64,13 +64,23 @@ def _device_functions():
         src = open(path).read()
         for m in re.finditer(r"\n(?:template <[^>]*>\n)?(?:__global__|__device__|__host__ __device__)\b", src):
             brace = src.find("{", m.end())
-            end = src.find("\n}\n", brace)
-            if brace < 0 or end < 0:
+            if brace < 0 or src.find(";", m.end(), brace) >= 0:    # a variable, not a function
+                continue
+            depth, end = 0, -1
+            for i in range(brace, len(src)):                       # the matching closing brace
+                if src[i] == "{":
+                    depth += 1
+                elif src[i] == "}":
+                    depth -= 1
+                    if depth == 0:
+                        end = i
+                        break
+            if end < 0:
                 continue
             header = re.sub(r"__launch_bounds__\s*\([^)]*\)", "", src[m.end():brace])
             name = re.search(r"(\w+)\s*\(", header)
             if name:
-                funcs.setdefault(name.group(1), src[m.start():end + 3])
+                funcs.setdefault(name.group(1), src[m.start():end + 1])
     return funcs
 
 

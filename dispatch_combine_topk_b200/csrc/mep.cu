@@ -104,8 +104,12 @@ DeviceState &device_state(int dev)
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     st.sm_count = n > 0 ? n : 148;
     const int big = 200 * 1024;
-    cudaFuncSetAttribute(mep::k_rank, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-    cudaFuncSetAttribute(mep::k_tile_count, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_rank<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_rank<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_rank<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_tile_count<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_tile_count<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_tile_count<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     cudaFuncSetAttribute(mep::k_histogram, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     cudaFuncSetAttribute(mep::k_plan_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     cudaFuncSetAttribute(mep::k_source_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
@@ -181,6 +185,41 @@ inline int elem_grid(int64_t total, int threads)
     return (int)(g > 0 ? g : 1);
 }
 
+// Rounds per warp of the counting sort's tile (256 * rounds slots) for N slots: smaller
+// tiles spread a small sort over all SMs, larger ones keep the per-tile scan and rank
+// work low for a large one (plan times measured with CUDA events: 262,144 slots fastest
+// with 512-slot tiles, 1,048,576 with 1024, 2,097,152 with 2048).
+inline int sort_rounds(int64_t N) { return N <= ((int64_t)1 << 18) ? 2 : (N <= ((int64_t)1 << 20) ? 4 : 8); }
+inline int64_t sort_tiles(int64_t N) { return mep::ceil_div(N, (int64_t)mep::kPlanWarps * 32 * sort_rounds(N)); }
+
+// Stable counting sort of N keys in [0, n_keys) (dropped: keep == 0 or out of range):
+// pos[n] = base[key] + (earlier slots of key), base = the exclusive prefix of the
+// histogram, or key_base when given. Writes the histogram to hist; tile_cnt holds
+// sort_tiles(N) * n_keys ints of scratch.
+template <int kRounds>
+void counting_sort_r(const int32_t *keys, const uint8_t *keep, int64_t N, int32_t n_keys, int32_t *tile_cnt,
+                     int32_t *hist, const int32_t *key_base, int32_t *pos, cudaStream_t s)
+{
+    const int64_t tiles = mep::ceil_div(N, (int64_t)mep::sort_tile<kRounds>());
+    const int threads = mep::kPlanWarps * 32;
+    mep::k_tile_count<kRounds><<<(unsigned)tiles, threads, sizeof(int32_t) * n_keys, s>>>(keys, keep, N, n_keys,
+                                                                                         tile_cnt);
+    mep::k_scan_cols<<<(unsigned)mep::ceil_div(n_keys, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, n_keys, hist);
+    const size_t rank_smem = sizeof(int32_t) * ((size_t)mep::kPlanWarps * n_keys + n_keys + 1 + 33);
+    mep::k_rank<kRounds><<<(unsigned)tiles, threads, rank_smem, s>>>(keys, keep, N, n_keys, tile_cnt, hist, key_base,
+                                                                    pos);
+}
+
+void counting_sort(const int32_t *keys, const uint8_t *keep, int64_t N, int32_t n_keys, int32_t *tile_cnt,
+                   int32_t *hist, const int32_t *key_base, int32_t *pos, cudaStream_t s)
+{
+    switch (sort_rounds(N)) {
+    case 2: counting_sort_r<2>(keys, keep, N, n_keys, tile_cnt, hist, key_base, pos, s); break;
+    case 4: counting_sort_r<4>(keys, keep, N, n_keys, tile_cnt, hist, key_base, pos, s); break;
+    default: counting_sort_r<8>(keys, keep, N, n_keys, tile_cnt, hist, key_base, pos, s); break;
+    }
+}
+
 }  // namespace
 
 extern "C" {
@@ -244,8 +283,7 @@ size_t mep_plan_workspace_size(int32_t R, int32_t n_keys, int32_t S, int32_t K)
 {
     if (R < 1 || S < 1 || K < 1 || n_keys < 1) return 0;
     const int64_t N = (int64_t)R * S * K;
-    const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
-    return align256(sizeof(int32_t) * (size_t)tiles * n_keys);
+    return align256(sizeof(int32_t) * (size_t)sort_tiles(N) * n_keys);
 }
 
 }  // extern "C"
@@ -316,15 +354,7 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
                                                                        rep_count, rep_key, rep_cu, (int32_t *)stats);
         return launched();
     }
-    const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
-    int32_t *tile_cnt = (int32_t *)workspace;
-    const int threads = mep::kPlanWarps * 32;
-
-    mep::k_tile_count<<<(unsigned)tiles, threads, sizeof(int32_t) * n_keys, s>>>(ids, keep, N, n_keys, tile_cnt);
-    mep::k_scan_cols<<<(unsigned)mep::ceil_div(n_keys, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, n_keys, hist);
-    const size_t rank_smem = sizeof(int32_t) * ((size_t)mep::kPlanWarps * n_keys + n_keys + 1 + 33);
-    mep::k_rank<<<(unsigned)tiles, threads, rank_smem, s>>>(ids, keep, N, n_keys, tile_cnt, hist, nullptr,
-                                                            pos);
+    counting_sort(ids, keep, N, n_keys, (int32_t *)workspace, hist, nullptr, pos, s);
     const size_t meta_smem = sizeof(int32_t) * (size_t)(2 * (n_keys + 1) + (R + 1) + R);
     mep::k_plan_meta<<<1, 1024, meta_smem, s>>>(hist, R, n_keys, (int64_t)S * K, mode,
                                                 keys_per_rank, rank_off, load, rep_count, rep_key,
@@ -335,7 +365,7 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
 size_t mep_plan_rank_workspace_size(int32_t R, int32_t E, int32_t S, int32_t K)
 {
     if (R < 1 || E < 1 || S < 1 || K < 1) return 0;
-    const int64_t tiles = mep::ceil_div((int64_t)S * K, mep::kPlanTile);
+    const int64_t tiles = sort_tiles((int64_t)S * K);
     return align256(sizeof(int32_t) * (size_t)tiles * E) + 2 * align256(sizeof(int32_t) * (size_t)E);
 }
 
@@ -355,22 +385,37 @@ mep_status_t mep_plan_rank(const int32_t *ids, const int32_t *hist_all, int32_t 
     cudaStream_t s = (cudaStream_t)stream;
     sm_count();
     const int64_t N = (int64_t)S * K;   // this rank's slots
-    const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
+    const int64_t tiles = sort_tiles(N);
     unsigned char *w = (unsigned char *)workspace;
     int32_t *tile_cnt = (int32_t *)w;
     w += align256(sizeof(int32_t) * (size_t)tiles * E);
     int32_t *hist_local = (int32_t *)w;
     w += align256(sizeof(int32_t) * (size_t)E);
     int32_t *key_base = (int32_t *)w;
+    // the rank's own histogram first (the tile counts and their column scan), then the
+    // bases from the gathered histograms, then the rows from those bases
     const int threads = mep::kPlanWarps * 32;
-    mep::k_tile_count<<<(unsigned)tiles, threads, sizeof(int32_t) * E, s>>>(ids, nullptr, N, E, tile_cnt);
+    const int rounds = sort_rounds(N);
+    if (rounds == 2)
+        mep::k_tile_count<2><<<(unsigned)tiles, threads, sizeof(int32_t) * E, s>>>(ids, nullptr, N, E, tile_cnt);
+    else if (rounds == 4)
+        mep::k_tile_count<4><<<(unsigned)tiles, threads, sizeof(int32_t) * E, s>>>(ids, nullptr, N, E, tile_cnt);
+    else
+        mep::k_tile_count<8><<<(unsigned)tiles, threads, sizeof(int32_t) * E, s>>>(ids, nullptr, N, E, tile_cnt);
     mep::k_scan_cols<<<(unsigned)mep::ceil_div(E, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, E, hist_local);
     const size_t meta_smem = sizeof(int32_t) * (size_t)(2 * E + 1 + 2 * R);
     mep::k_source_meta<<<1, 1024, meta_smem, s>>>(hist_all, hist_local, R, E, (int64_t)S * K, rank, key_base,
                                                   send_count, send_off, recv_count, recv_off);
     const size_t rank_smem = sizeof(int32_t) * ((size_t)mep::kPlanWarps * E + E + 1 + 33);
-    mep::k_rank<<<(unsigned)tiles, threads, rank_smem, s>>>(ids, nullptr, N, E, tile_cnt, hist_local, key_base,
-                                                            pos);
+    if (rounds == 2)
+        mep::k_rank<2><<<(unsigned)tiles, threads, rank_smem, s>>>(ids, nullptr, N, E, tile_cnt, hist_local, key_base,
+                                                                   pos);
+    else if (rounds == 4)
+        mep::k_rank<4><<<(unsigned)tiles, threads, rank_smem, s>>>(ids, nullptr, N, E, tile_cnt, hist_local, key_base,
+                                                                   pos);
+    else
+        mep::k_rank<8><<<(unsigned)tiles, threads, rank_smem, s>>>(ids, nullptr, N, E, tile_cnt, hist_local, key_base,
+                                                                   pos);
     return launched();
 }
 
@@ -672,48 +717,6 @@ mep_status_t mep_dispatch_int8_smooth(const uint16_t *x, const int32_t *ids, con
     const int64_t per_thread = mep::ceil_div(H8, 256);
     using smooth_k_t = void (*)(const uint4 *, const int32_t *, const int32_t *, int64_t, int64_t, const float4 *,
                                 int32_t, int64_t, uint2 *, float *);
-    // every smoothing row read once: a cluster of cl CTAs per token, four columns per
-    // thread, the smallest cl with at most kSmoothClMaxThreads threads per CTA
-    int cl = 0;
-    for (int c = 2; c <= 8 && !cl; c *= 2)
-        if (H % (128 * c) == 0 && H / (4 * c) <= mep::kSmoothClMaxThreads) cl = c;
-    if (cl && (K == 2 || K == 4 || K == 8) && aligned(x, 8) && aligned(smooth, 16) && aligned(recv, 4)) {
-        using cl_k_t = void (*)(const uint2 *, const int32_t *, const int32_t *, int64_t, int64_t, const float4 *,
-                                int32_t, int64_t, uint32_t *, float *);
-        cl_k_t kern = nullptr;
-#define MEP_SMOOTH_CL(KC_)                                                                          \
-    kern = cl == 2 ? mep::k_dispatch_int8_smooth_cl<KC_, 2>                                          \
-                   : (cl == 4 ? mep::k_dispatch_int8_smooth_cl<KC_, 4> : mep::k_dispatch_int8_smooth_cl<KC_, 8>)
-        if (K == 2) MEP_SMOOTH_CL(2);
-        else if (K == 4) MEP_SMOOTH_CL(4);
-        else MEP_SMOOTH_CL(8);
-#undef MEP_SMOOTH_CL
-        const int threads = (int)(H / (4 * cl));
-        cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)cl;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.blockDim = dim3((unsigned)threads);
-        cfg.dynamicSmemBytes = 0;
-        cfg.stream = s;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        // as many clusters as the GPU holds at once (never more than tokens)
-        int max_cl = 0;
-        cfg.gridDim = dim3((unsigned)(cl * sm_count()));
-        if (cudaOccupancyMaxActiveClusters(&max_cl, kern, &cfg) != cudaSuccess || max_cl < 1) {
-            (void)cudaGetLastError();
-            max_cl = sm_count() / cl;
-        }
-        const int64_t ncl = T < max_cl ? T : max_cl;
-        cfg.gridDim = dim3((unsigned)(cl * (ncl > 0 ? ncl : 1)));
-        if (cudaLaunchKernelEx(&cfg, kern, (const uint2 *)x, ids, pos, T, H / 4, (const float4 *)smooth, n_experts,
-                               rows, (uint32_t *)recv, recv_scale) != cudaSuccess)
-            return launched();
-        return launched();
-    }
     smooth_k_t fused = nullptr;
     if (vec && per_thread <= 8) {
         const bool c4 = per_thread <= 4;
@@ -774,7 +777,7 @@ size_t mep_dedup_workspace_size(int32_t R, int32_t S, int32_t K)
 {
     if (R < 1 || S < 1 || K < 1) return 0;
     const int64_t N = (int64_t)R * S * K;
-    const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
+    const int64_t tiles = sort_tiles(N);
     return align256(sizeof(int32_t) * (size_t)N) + align256((size_t)N) +
            align256(sizeof(int32_t) * (size_t)tiles * R) + align256(sizeof(int32_t) * (size_t)R);
 }
@@ -793,7 +796,7 @@ mep_status_t mep_dedup_plan(const int32_t *pos, const int32_t *rank_off, int32_t
     cudaStream_t s = (cudaStream_t)stream;
     const int sms = sm_count();
     const int64_t T = (int64_t)R * S;
-    const int64_t tiles = mep::ceil_div(N, mep::kPlanTile);
+    const int64_t tiles = sort_tiles(N);
     unsigned char *w = (unsigned char *)workspace;
     int32_t *dkey = (int32_t *)w;
     w += align256(sizeof(int32_t) * (size_t)N);
@@ -808,13 +811,8 @@ mep_status_t mep_dedup_plan(const int32_t *pos, const int32_t *rank_off, int32_t
     const int64_t tg = mep::ceil_div(T, 256), tcap = (int64_t)sms * 8;
     const unsigned tgrid = (unsigned)(tg < tcap ? tg : tcap);
     const size_t off_smem = sizeof(int32_t) * (size_t)(R + 1);
-    const int threads = mep::kPlanWarps * 32;
     mep::k_dedup_keys<<<tgrid, 256, off_smem, s>>>(pos, rank_off, R, T, K, dkey, dkeep);
-    mep::k_tile_count<<<(unsigned)tiles, threads, sizeof(int32_t) * R, s>>>(dkey, dkeep, N, R, tile_cnt);
-    mep::k_scan_cols<<<(unsigned)mep::ceil_div(R, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, R, count);
-    const size_t rank_smem = sizeof(int32_t) * ((size_t)mep::kPlanWarps * R + R + 1 + 33);
-    mep::k_rank<<<(unsigned)tiles, threads, rank_smem, s>>>(dkey, dkeep, N, R, tile_cnt, count, nullptr,
-                                                            dsend);
+    counting_sort(dkey, dkeep, N, R, tile_cnt, count, nullptr, dsend, s);
     mep::k_dedup_offsets<<<1, 1024, sizeof(int32_t) * (size_t)(R + 1 + 33), s>>>(count, R, drank_off);
     mep::k_dedup_finish<<<tgrid, 256, off_smem, s>>>(pos, rank_off, R, T, K, dsend, dpos, dtok, gidx);
     return launched();

@@ -20,11 +20,11 @@
 
 namespace mep {
 
-#ifndef MEP_PLAN_WARP_ROUNDS
-#define MEP_PLAN_WARP_ROUNDS 8                   // 32-slot rounds per warp in a tile
-#endif
 constexpr int kPlanWarps = 8;                    // warps per tile CTA
-constexpr int kPlanTile = kPlanWarps * 32 * MEP_PLAN_WARP_ROUNDS;   // 2048 slots by default
+constexpr int kPlanTile = kPlanWarps * 32 * 8;   // the histogram's tile: 2048 slots
+// The counting sort's tile: kRounds 32-slot rounds per warp, 256 * kRounds slots.
+template <int kRounds>
+constexpr int sort_tile() { return kPlanWarps * 32 * kRounds; }
 
 // Key of slot n: the id, or -1 when the slot is dropped or its id is out of range.
 __device__ __forceinline__ int32_t slot_key(const int32_t *ids, const uint8_t *keep, int64_t n,
@@ -61,17 +61,19 @@ k_histogram(const int32_t *__restrict__ ids, int64_t N, int32_t n_keys, int32_t 
         if (sh[i]) atomicAdd(&hist[i], sh[i]);
 }
 
-// tile_cnt[tile, key] = slots of `key` in tile `blockIdx.x`.
+// tile_cnt[tile, key] = slots of `key` in tile `blockIdx.x` (tiles of sort_tile<kRounds>).
+template <int kRounds>
 __global__ void __launch_bounds__(kPlanWarps * 32)
 k_tile_count(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, int64_t N,
              int32_t n_keys, int32_t *__restrict__ tile_cnt)
 {
+    constexpr int kTile = sort_tile<kRounds>();
     extern __shared__ int32_t sh[];
     for (int i = threadIdx.x; i < n_keys; i += blockDim.x) sh[i] = 0;
     __syncthreads();
     const int lane = threadIdx.x & 31;
-    const int64_t base = (int64_t)blockIdx.x * kPlanTile;
-    for (int64_t n = base + threadIdx.x - lane; n < base + kPlanTile; n += blockDim.x) {
+    const int64_t base = (int64_t)blockIdx.x * kTile;
+    for (int64_t n = base + threadIdx.x - lane; n < base + kTile; n += blockDim.x) {
         int32_t key = slot_key(ids, keep, n + lane, N, n_keys);
         uint32_t peers = __match_any_sync(0xffffffffu, key);
         if (key >= 0 && lane == __ffs(peers) - 1) atomicAdd(&sh[key], __popc(peers));
@@ -165,6 +167,7 @@ k_scan_cols(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys, int
 // bases, then each warp walks its sub-range again in order, ranking equal keys with
 // match.any.
 // Dynamic shared memory: cnt [kPlanWarps][n_keys], off [n_keys + 1], scratch [33].
+template <int kRounds>
 __global__ void __launch_bounds__(kPlanWarps * 32)
 k_rank(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, int64_t N, int32_t n_keys,
        const int32_t *__restrict__ tile_base, const int32_t *__restrict__ hist,
@@ -181,8 +184,8 @@ k_rank(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, int64_
     } else {
         block_exclusive_scan(hist, n_keys, key_off, scan_scratch);
     }
-    constexpr int kSub = kPlanTile / kPlanWarps;
-    const int64_t lo = (int64_t)blockIdx.x * kPlanTile + warp * kSub;
+    constexpr int kSub = sort_tile<kRounds>() / kPlanWarps;
+    const int64_t lo = (int64_t)blockIdx.x * sort_tile<kRounds>() + warp * kSub;
     int32_t *mine = cnt + warp * n_keys;
     for (int64_t n0 = lo; n0 < lo + kSub; n0 += 32) {
         int32_t key = slot_key(ids, keep, n0 + lane, N, n_keys);

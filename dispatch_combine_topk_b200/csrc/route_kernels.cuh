@@ -704,28 +704,23 @@ __device__ __forceinline__ void store_bf16x16(uint4 *dst, const float2 (&acc)[8]
 }
 
 // The combine of int8 rows for H % 16 == 0 and 16-byte aligned buffers (the same sum as
-// k_combine_int8_v8, 16 codes per slot per lane), one warp per token, no block barrier.
-// With K fixed at compile time, lanes k < K write the token's slot table (row pointer,
-// gate, scale of slot k) into the warp's part of shared memory, where every lane reads
-// it for each 16-column chunk: keeping the table out of registers holds the kernel to 80
-// registers, 6 CTAs of 128 threads per SM (24 warps) against 5 with the table in
-// registers, which measured 17% faster on the int8 workload's shape (bit-exact). With a
-// runtime K the lanes take the slot values by shuffle.
+// k_combine_int8_v8, 16 codes per slot per lane), one warp per token: lane k < K holds slot k's
+// row, gate and scale, which the other lanes take by shuffle once per token. There is no
+// block barrier, and the slot values stay in registers across the token's column chunks.
+// (Keeping them in shared memory instead allows 6 CTAs per SM instead of 5 and measured
+// faster alone, but 3% slower inside the routing step, where the GPU runs at its power
+// limit and the extra shared-memory reads cost more than the occupancy gains.)
 constexpr int kCombineInt8Threads = 128;
 
 template <int KC>
-__global__ void __launch_bounds__(kCombineInt8Threads, 6)
+__global__ void __launch_bounds__(128)
 k_combine_int8_warp(const uint4 *__restrict__ yq, const float *__restrict__ yscale, const int32_t *__restrict__ pos,
                     const float *__restrict__ gates, int64_t T, int Krt, int64_t H16, int64_t rows,
                     uint4 *__restrict__ out)
 {
     constexpr bool kFixed = KC > 0;
-    constexpr int kTab = kFixed ? KC : 1;
-    constexpr int kWarps = kCombineInt8Threads / 32;
-    __shared__ const uint4 *s_row[kWarps][kTab];
-    __shared__ float s_g[kWarps][kTab], s_s[kWarps][kTab];
     const int K = kFixed ? KC : Krt;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
         int32_t mine = -1;
@@ -741,26 +736,25 @@ k_combine_int8_warp(const uint4 *__restrict__ yq, const float *__restrict__ ysca
         }
         uint4 *dst = out + t * 2 * H16;
         if constexpr (kFixed) {
-            __syncwarp();                                   // every lane is done with the last table
-            if (lane < KC) {
-                s_row[warp][lane] = mine >= 0 ? yq + (int64_t)mine * H16 : nullptr;
-                s_g[warp][lane] = g_mine;
-                s_s[warp][lane] = s_mine;
+            int32_t pk[KC];
+            float gk[KC], sk[KC];
+#pragma unroll
+            for (int k = 0; k < KC; k++) {
+                pk[k] = __shfl_sync(0xffffffffu, mine, k);
+                gk[k] = __shfl_sync(0xffffffffu, g_mine, k);
+                sk[k] = __shfl_sync(0xffffffffu, s_mine, k);
             }
-            __syncwarp();
             for (int64_t c = lane; c < H16; c += 32) {
                 float2 acc[8];
 #pragma unroll
                 for (int j = 0; j < 8; j++) acc[j] = make_float2(0.0f, 0.0f);
                 uint4 v[KC];
 #pragma unroll
-                for (int k = 0; k < KC; k++) {
-                    const uint4 *r = s_row[warp][k];
-                    v[k] = r ? ld_stream(r + c) : make_uint4(0, 0, 0, 0);
-                }
+                for (int k = 0; k < KC; k++)
+                    v[k] = pk[k] >= 0 ? ld_stream(yq + (int64_t)pk[k] * H16 + c) : make_uint4(0, 0, 0, 0);
 #pragma unroll
                 for (int k = 0; k < KC; k++)
-                    if (s_row[warp][k]) add_int8_x16(acc, v[k], s_g[warp][k], s_s[warp][k]);
+                    if (pk[k] >= 0) add_int8_x16(acc, v[k], gk[k], sk[k]);
                 store_bf16x16(dst + 2 * c, acc);
             }
         } else {
@@ -1121,130 +1115,6 @@ k_dispatch_int8_smooth_k(const uint4 *__restrict__ x, const int32_t *__restrict_
         }
         __syncthreads();                                   // sp, se, ssc and red are reused
     }
-}
-
-// The codes of q8x4 for four values whose fp32 products xs are given (the smoothing
-// dispatch), with inv = quant_inv(scale): y = fl(xs * inv) rounded half-to-even by the
-// 1.5 * 2^23 shift, as q8x8; when any y lies within 2^-15 of a half-integer, or 1/scale
-// overflows, the four take the IEEE quotient instead.
-__device__ __forceinline__ uint32_t q8x4_products(float a, float b, float c, float d, float scale, float inv)
-{
-    const float2 kShift = make_float2(12582912.0f, 12582912.0f), kNegShift = make_float2(-12582912.0f, -12582912.0f);
-    const float2 inv2 = make_float2(inv, inv);
-    const float2 y0 = mul2_rn(make_float2(a, b), inv2), y1 = mul2_rn(make_float2(c, d), inv2);
-    const float2 t0 = add2_rn(y0, kShift), t1 = add2_rn(y1, kShift);
-    const float2 r0 = add2_rn(t0, kNegShift), r1 = add2_rn(t1, kNegShift);
-    const float2 d0 = add2_rn(y0, make_float2(-r0.x, -r0.y)), d1 = add2_rn(y1, make_float2(-r1.x, -r1.y));
-    const float dmax = fmaxf(fmaxf(fabsf(d0.x), fabsf(d0.y)), fmaxf(fabsf(d1.x), fabsf(d1.y)));
-    if (inv < 0.0f || dmax >= 0.5f - 0x1p-15f) return q8x4(a, b, c, d, scale);
-    return __byte_perm(__byte_perm(__float_as_uint(t0.x), __float_as_uint(t0.y), 0x0040),
-                       __byte_perm(__float_as_uint(t1.x), __float_as_uint(t1.y), 0x0040), 0x5410);
-}
-
-// The smoothing dispatch with every smoothing row read once: a cluster of kCl CTAs per
-// token, CTA r of the cluster owning columns [r * H / kCl, (r + 1) * H / kCl), four per
-// thread (blockDim.x = H / (4 * kCl), a multiple of 32). For each of the token's K slots
-// a thread forms its four products fl(x * smooth[e_k]) and keeps them in registers
-// (4 * KC floats); the slot's amax is the maximum over the thread (registers), the warp
-// (redux.sync on the bit patterns, which order like the values since they are |.|), the
-// CTA (shared memory, one block barrier) and the cluster: every CTA writes its K maxima
-// into every CTA's shared memory and one cluster barrier later each CTA has all kCl of
-// them. Then scale = amax / 127 and the codes follow from the products still in
-// registers, stored as one 4-byte word per thread and slot. The slot list of the next
-// token is loaded into registers before the block barrier and written to shared memory
-// after it (every thread has then finished the previous token, which used that buffer);
-// every shared array is double-buffered by token parity, so one block barrier and one
-// cluster barrier per token suffice: buffer b is written again two tokens later, after
-// a barrier that every reader of b passes only after its reads.
-// All CTAs of a cluster take the same tokens (their trip counts are equal), so every
-// thread of the cluster reaches every cluster barrier. Needs x 8-byte and smooth 16-byte
-// aligned, recv 4-byte aligned, H % (128 * kCl) == 0.
-constexpr int kSmoothClMaxThreads = 512;
-
-template <int KC, int kCl>
-__global__ void __launch_bounds__(kSmoothClMaxThreads, 2)
-k_dispatch_int8_smooth_cl(const uint2 *__restrict__ x, const int32_t *__restrict__ ids, const int32_t *__restrict__ pos,
-                          int64_t T, int64_t H4, const float4 *__restrict__ smooth, int32_t n_experts, int64_t rows,
-                          uint32_t *__restrict__ recv, float *__restrict__ recv_scale)
-{
-    __shared__ int32_t s_p[2][KC], s_e[2][KC];
-    __shared__ float s_red[2][kSmoothClMaxThreads / 32][KC];
-    __shared__ float s_cl[2][kCl][KC];
-    const uint32_t cr = cluster_ctarank();
-    const int64_t cid = cluster_id_x(), ncl = cluster_count_x();
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-    const int64_t c = (int64_t)cr * blockDim.x + tid;      // this thread's 4-column chunk
-    // slot k's row and expert (threads k < KC): a slot without a valid expert is skipped
-    auto load_slot = [&](int64_t t, int32_t &p, int32_t &e) {
-        p = pos[t * KC + tid];
-        if (p < -1 || (int64_t)p >= rows) {
-            flag_error(MEP_DERR_ROW_RANGE);
-            p = -1;
-        }
-        e = ids[t * KC + tid];
-        if (e < 0 || e >= n_experts) {
-            flag_error(MEP_DERR_KEY_RANGE);
-            e = -1;
-            p = -1;
-        }
-    };
-    if (cid < T && tid < KC) {
-        int32_t p, e;
-        load_slot(cid, p, e);
-        s_p[0][tid] = p;
-        s_e[0][tid] = e;
-    }
-    __syncthreads();
-    int b = 0;
-    for (int64_t t = cid; t < T; t += ncl, b ^= 1) {
-        const uint2 xv = x[t * H4 + c];
-        const float2 x01 = make_float2(bf16lo(xv.x), bf16hi(xv.x)), x23 = make_float2(bf16lo(xv.y), bf16hi(xv.y));
-        float pr[KC][4];
-#pragma unroll
-        for (int k = 0; k < KC; k++) {
-            const int32_t e = s_e[b][k];
-            uint32_t m = 0u;
-            if (s_p[b][k] >= 0) {                           // uniform over the cluster
-                const float4 sv = smooth[(int64_t)e * H4 + c];
-                const float2 a = mul2_rn(x01, make_float2(sv.x, sv.y)), d = mul2_rn(x23, make_float2(sv.z, sv.w));
-                pr[k][0] = a.x;
-                pr[k][1] = a.y;
-                pr[k][2] = d.x;
-                pr[k][3] = d.y;
-                m = __float_as_uint(fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(d.x), fabsf(d.y))));
-            }
-            m = __reduce_max_sync(0xffffffffu, m);
-            if (lane == 0) s_red[b][warp][k] = __uint_as_float(m);
-        }
-        const bool more = t + ncl < T;
-        int32_t np = -1, ne = -1;
-        if (more && tid < KC) load_slot(t + ncl, np, ne);
-        __syncthreads();
-        if (tid < KC) {
-            float m = 0.0f;
-            for (int w = 0; w < nwarps; w++) m = fmaxf(m, s_red[b][w][tid]);
-#pragma unroll
-            for (int r = 0; r < kCl; r++) st_cluster_f32(cluster_map(&s_cl[b][cr][tid], (uint32_t)r), m);
-            if (more) {
-                s_p[b ^ 1][tid] = np;
-                s_e[b ^ 1][tid] = ne;
-            }
-        }
-        cluster_sync();
-#pragma unroll
-        for (int k = 0; k < KC; k++) {
-            const int32_t p = s_p[b][k];
-            if (p < 0) continue;
-            float amax = s_cl[b][0][k];
-#pragma unroll
-            for (int r = 1; r < kCl; r++) amax = fmaxf(amax, s_cl[b][r][k]);
-            const float scale = __fdiv_rn(amax, 127.0f), inv = quant_inv(scale);
-            recv[(int64_t)p * H4 + c] = q8x4_products(pr[k][0], pr[k][1], pr[k][2], pr[k][3], scale, inv);
-            if (cr == 0 && tid == k) recv_scale[p] = scale;
-        }
-    }
-    // no CTA leaves while a peer of its cluster may still write into its shared memory
-    cluster_sync();
 }
 
 // Element version for any H and alignment: two passes per slot over x and the scales.

@@ -33,13 +33,16 @@ def test_histogram_parity_ragged_and_skewed():
 
 
 # Plans of at most 16384 slots with few enough keys run as one CTA, the others as the
-# tiled four-kernel sort: the cases cover both, at and just past the boundary (ragged last
-# tile), and small plans whose keys are too many for the one-CTA path.
+# tiled four-kernel sort (tiles of 512, 1024 or 2048 slots by size): the cases cover each
+# path, at and just past the boundaries (ragged last tiles), and small plans whose keys
+# are too many for the one-CTA path.
 @pytest.mark.parametrize("R,E,S,K", [
     (2, 4, 2, 2), (3, 9, 37, 3), (4, 12, 1000, 3), (4, 16, 128, 2), (8, 64, 300, 8),
     (1, 5, 17, 1), (16, 4096, 32, 4), (8, 4096, 512, 8), (5, 5, 2048, 1),
     (4, 16, 1024, 4), (7, 7, 2340, 1), (2, 1024, 4096, 2), (3, 9, 1821, 3), (1, 2, 16385, 1),
     (64, 1536, 8, 8),
+    # ragged last tiles of the 1024- and 2048-slot tiles (more than 2^18 and 2^20 slots)
+    (7, 7, 37454, 1), (5, 10, 209916, 1),
 ])
 def test_plan_balanced_parity_random(R, E, S, K):
     rng = np.random.default_rng(R * 7919 + E * 31 + S)

@@ -1,8 +1,9 @@
 """GPU parity of the int8 dispatch with per-expert smoothing scales against the oracle
-(codes and scales bit for bit). K in {2, 4, 8} with H a multiple of 256 takes the
-cluster kernel (2, 4 or 8 CTAs per token), other K the per-slot kernel, other H the
-one-CTA kernels. The full int8 workload is compared whole, one rank partition at a time,
-and with all-ones scales against the plain per-token int8 dispatch."""
+(codes and scales bit for bit). K in {2, 4, 8} (with up to 64 columns per thread) takes
+the fused kernel (all K slots of a token in one CTA, two passes), other K the per-slot
+kernel, other H or alignments the scalar kernel. The full int8 workload is compared
+whole, one rank partition at a time, and with all-ones scales against the plain
+per-token int8 dispatch."""
 from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
@@ -39,9 +40,10 @@ def test_smooth_dispatch_matches_oracle(K, H):
 
 
 @pytest.mark.parametrize("K,H", [(2, 4096), (4, 7168), (8, 4096), (8, 12288), (8, 7168)])
-def test_smooth_dispatch_many_tokens_per_cluster(K, H):
-    """More tokens than clusters resident on the GPU, so every cluster walks many tokens
-    (the shared buffers alternate by token parity); dropped slots and whole buffers."""
+def test_smooth_dispatch_many_tokens_per_cta(K, H):
+    """More tokens than CTAs resident on the GPU, so every CTA walks many tokens (and
+    prefetches the next slot's smoothing row while computing one); dropped slots and
+    whole buffers."""
     rng = np.random.default_rng(K * 13 + H)
     T, E = 3001, 40
     x = (torch.randn((T, H), generator=torch.Generator().manual_seed(H + K)) * 3).to(torch.bfloat16)
@@ -150,9 +152,9 @@ def test_quantiser_at_and_next_to_half_integer_quotients(amax, K):
                 v = np.nextafter(v, np.float32(np.inf if j > 0 else -np.inf), dtype=np.float32)
             if abs(v) <= np.float32(amax):
                 vals.append(v)
-    # K = 1: the per-slot kernel (H a multiple of 8); K = 2: the cluster kernel (H a
-    # multiple of 256), the second slot on a second expert holding the values reversed
-    H = (len(vals) + 7) // 8 * 8 if K == 1 else (len(vals) + 255) // 256 * 256
+    # K = 1: the per-slot kernel; K = 2: the fused kernel, the second slot on a second
+    # expert holding the values reversed
+    H = (len(vals) + 7) // 8 * 8
     sm = np.zeros((K, H), np.float32)
     sm[0, :len(vals)] = vals
     if K == 2:
