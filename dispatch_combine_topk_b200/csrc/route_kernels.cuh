@@ -1018,9 +1018,9 @@ k_dispatch_int8_smooth(const uint4 *__restrict__ x, const int32_t *__restrict__ 
 
 // The same codes with the K slots of a token taken together (K fixed at KC): pass 1
 // forms, slot by slot, each thread's maximum of |fl(x * smooth[e_k])| and its warp
-// maximum (every smoothing row read once); one block barrier later the K scales follow
-// from the warps' maxima; pass 2 forms each product again (the smoothing rows a second
-// time, from L2) and stores the codes. Two block barriers per token instead of two per
+// maximum (every smoothing row read once; the warp maximum by redux.sync); one block
+// barrier later the K scales follow from the warps' maxima; pass 2 forms each product
+// again (the smoothing rows a second time, from L2) and stores the codes. Two block barriers per token instead of two per
 // slot. Both passes walk the slots in a loop that is not unrolled, which keeps the code
 // short and the registers at 64 (4 CTAs per SM).
 template <int KC, int kChunks>
@@ -1084,8 +1084,9 @@ k_dispatch_int8_smooth_k(const uint4 *__restrict__ x, const int32_t *__restrict_
                     }
                 }
             }
-#pragma unroll
-            for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+            // warp maximum of non-negative floats (fmaxf left out any NaN): their bits order
+            // like their values, so one integer reduction gives it
+            amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
             if (lane == 0) red[warp][k] = amax;
         }
         __syncthreads();
