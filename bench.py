@@ -116,19 +116,17 @@ def kernel_source_hash(name: str) -> str:
 _TRAFFIC_METRICS = "dram__bytes_read.sum + dram__bytes_write.sum"
 TRAFFIC = {
     ("k_dispatch_warp", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 998.22e6, "src": "2bdb2659ae3ccd32", "case_S": 1024, "case_mb": 998.22},
+        "bytes": 4 * 997.906e6, "src": "ecb53c46b3d954ca", "case_S": 1024, "case_mb": 997.906},
     ("k_combine_v8", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 1005.70e6, "src": "b8d0144407f8df74", "case_S": 1024, "case_mb": 1005.70},
+        "bytes": 4 * 1005.660e6, "src": "aa70b87f5f33b11a", "case_S": 1024, "case_mb": 1005.660},
     ("k_dispatch_int8_staged", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1115.86e6, "src": "cf5ee39cf4a3516f", "case_S": 512, "case_mb": 1115.86},
+        "bytes": 16 * 1114.875e6, "src": "597997762b516c3e", "case_S": 512, "case_mb": 1114.875},
     ("k_combine_int8_warp", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1117.18e6, "src": "d852eb58236fe244", "case_S": 512, "case_mb": 1117.18},
-    ("k_expand_warp", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 1793.81e6, "src": "a12dc9427177590d", "case_S": 1024, "case_mb": 1793.81},
+        "bytes": 16 * 1117.359e6, "src": "31ddea297a5f9077", "case_S": 512, "case_mb": 1117.359},
     ("k_dispatch_warp", "skew_r64_e512_s2048_k8_h4096"): {
-        "bytes": 4 * 2357.51e6, "src": "2bdb2659ae3ccd32", "case_S": 512, "case_mb": 2357.51},
+        "bytes": 4 * 2357.854e6, "src": "ecb53c46b3d954ca", "case_S": 512, "case_mb": 2357.854},
     ("k_combine_v8", "skew_r64_e512_s2048_k8_h4096"): {
-        "bytes": 4 * 2364.80e6, "src": "b8d0144407f8df74", "case_S": 512, "case_mb": 2364.80},
+        "bytes": 4 * 2364.469e6, "src": "aa70b87f5f33b11a", "case_S": 512, "case_mb": 2364.469},
 }
 
 
@@ -983,7 +981,7 @@ def main():
     ap.add_argument("--per-workload", default="tiny,r8,map,skew",
                     help="comma-separated workloads measured after the main one and reported under "
                          "per_workload (graph replays, no end-to-end leg); 'none' to skip")
-    ap.add_argument("--ref-div", type=int, default=8,
+    ap.add_argument("--ref-div", type=int, default=16,
                     help="--impl reference: the oracle routes S/ref_div tokens per rank per step")
     ap.add_argument("--cpu-div", type=int, default=1,
                     help="cpu_baseline: the oracle routes S/cpu_div tokens per rank once")

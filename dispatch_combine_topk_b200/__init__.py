@@ -103,12 +103,15 @@ def lib() -> ctypes.CDLL:
         L.mep_plan_rank_workspace_size.restype = ctypes.c_size_t
         L.mep_plan_rank.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.mep_plan_static_ws.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P]
+        L.mep_dispatch_ranks.argtypes = [P, P, i64, i32, i64, i32, P, P, i32, i64, P]
+        L.mep_combine_ranks.argtypes = [P, P, i32, i32, i64, P, P, i64, i32, i64, P, P]
         for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
                   "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8",
                   "mep_combine_add_rmsnorm", "mep_prefetch_plan", "mep_prefetch_weights",
                   "mep_grad_reduce", "mep_dispatch_int8_smooth", "mep_update_expert_ranks",
                   "mep_dedup_plan", "mep_expand", "mep_route_host", "mep_stream_synchronize_timeout",
-                  "mep_maxvio", "mep_plan_rank", "mep_plan_static_ws"]:
+                  "mep_maxvio", "mep_plan_rank", "mep_plan_static_ws", "mep_dispatch_ranks",
+                  "mep_combine_ranks"]:
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -287,6 +290,46 @@ def mep_plan_rank(ids: torch.Tensor, hist_all: torch.Tensor, R: int, E: int, S: 
                              _ptr(out.recv_off, torch.int32), _ptr(out.workspace), out.workspace.numel(),
                              _stream(stream))
     _ok(rc, "mep_plan_rank")
+    return out
+
+
+def rank_pointer_table(buffers, device=None) -> torch.Tensor:
+    """A device array of the ranks' buffer addresses (int64 [R]) for mep_dispatch_ranks /
+    mep_combine_ranks: one tensor per rank, on this device or (across GPUs) a peer
+    mapping of another GPU's buffer."""
+    dev = device or buffers[0].device
+    return torch.tensor([b.data_ptr() for b in buffers], dtype=torch.int64).to(dev)
+
+
+def mep_dispatch_ranks(x: torch.Tensor, pos: torch.Tensor, K: int, recv_table: torch.Tensor, rows_per_rank: int,
+                       quant: int = 0, scale_table: Optional[torch.Tensor] = None, stream=None):
+    """Dispatch into the ranks' own buffers (see include/mep.h): slot n's row goes to
+    rank pos[n] // rows_per_rank at local row pos[n] % rows_per_rank, through a device
+    table of buffer addresses (rank_pointer_table)."""
+    T, H = x.shape
+    _need(pos.numel() == T * K, "pos must hold T*K slots")
+    _need(recv_table.dtype == torch.int64 and recv_table.dim() == 1, "recv_table: int64 [R] addresses")
+    R = recv_table.numel()
+    _need(quant == 0 or (scale_table is not None and scale_table.numel() == R), "scale_table [R] needed for int8")
+    _ok(lib().mep_dispatch_ranks(_ptr(x, torch.bfloat16, "x"), _ptr(pos, torch.int32, "pos"), T, K, H, quant,
+                                 _ptr(recv_table, torch.int64, "recv_table"),
+                                 _ptr(scale_table, torch.int64, "scale_table"), R, rows_per_rank, _stream(stream)),
+        "mep_dispatch_ranks")
+
+
+def mep_combine_ranks(y_table: torch.Tensor, pos: torch.Tensor, gates: torch.Tensor, K: int, rows_per_rank: int,
+                      out: torch.Tensor, quant: int = 0, scale_table: Optional[torch.Tensor] = None, stream=None):
+    """Combine from the ranks' own buffers (see include/mep.h)."""
+    T, H = out.shape
+    _need(pos.numel() == T * K and gates.numel() == T * K, "pos and gates must hold T*K slots")
+    _need(y_table.dtype == torch.int64 and y_table.dim() == 1, "y_table: int64 [R] addresses")
+    R = y_table.numel()
+    _need(quant == 0 or (scale_table is not None and scale_table.numel() == R), "scale_table [R] needed for int8")
+    _ok(lib().mep_combine_ranks(_ptr(y_table, torch.int64, "y_table"), _ptr(scale_table, torch.int64, "scale_table"),
+                                quant, R, rows_per_rank, _ptr(pos, torch.int32, "pos"),
+                                _ptr(gates, torch.float32, "gates"), T, K, H, _ptr(out, torch.bfloat16, "out"),
+                                _stream(stream)),
+        "mep_combine_ranks")
     return out
 
 

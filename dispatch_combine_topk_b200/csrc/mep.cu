@@ -21,6 +21,7 @@
 #include "plan_kernels.cuh"
 #include "route_kernels.cuh"
 #include "dedup_kernels.cuh"
+#include "rank_kernels.cuh"
 
 namespace {
 
@@ -837,6 +838,68 @@ mep_status_t mep_expand(const void *src, const float *src_scale, int64_t src_row
     } else {
         mep::k_expand_bytes<<<token_grid(rows, 8), 256, 0, s>>>((const uint8_t *)src, ss, src_rows, gidx, rows,
                                                               row_bytes, (uint8_t *)dst, ds);
+    }
+    return launched();
+}
+
+// ------------------------------------------ (e): rows in the ranks' own buffers
+
+mep_status_t mep_dispatch_ranks(const uint16_t *x, const int32_t *pos, int64_t T, int32_t K, int64_t H,
+                                int32_t quant, void *const *recv_ptrs, float *const *scale_ptrs, int32_t R,
+                                int64_t rows_per_rank, mep_stream_t stream)
+{
+    if (quant != 0 && quant != 1) return MEP_ERR_DTYPE;
+    if (T > 0 && (!x || !pos || !recv_ptrs || (quant == 1 && !scale_ptrs))) return MEP_ERR_NULLPTR;
+    if (T < 0 || K < 1 || K > MEP_MAX_K || H < 8 || H % 8 != 0 || R < 1 || R > MEP_MAX_KEYS ||
+        rows_per_rank < 1 || T * K >= ((int64_t)1 << 31) || (int64_t)R * rows_per_rank >= ((int64_t)1 << 31))
+        return MEP_ERR_SHAPE;
+    if (T > 0 && (!aligned(x, 16) || !aligned(recv_ptrs, 8) || (quant == 1 && !aligned(scale_ptrs, 8))))
+        return MEP_ERR_VALUE;
+    if (T == 0) return MEP_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (quant == 0) {
+        const int64_t ctas = mep::ceil_div(T, 8);
+        const int64_t cap = (int64_t)sm_count() * 16;
+        mep::k_dispatch_ranks_warp<<<(int)(ctas < cap ? ctas : cap), 256, 0, s>>>(
+            (const uint4 *)x, pos, T, K, H / 8, (uint4 *const *)recv_ptrs, R, rows_per_rank);
+    } else {
+        mep::k_dispatch_ranks_int8<<<token_grid(T, 8), 256, 0, s>>>((const uint4 *)x, pos, T, K, H / 8,
+                                                                   (uint2 *const *)recv_ptrs, scale_ptrs, R,
+                                                                   rows_per_rank);
+    }
+    return launched();
+}
+
+mep_status_t mep_combine_ranks(const void *const *y_ptrs, const float *const *scale_ptrs, int32_t quant, int32_t R,
+                               int64_t rows_per_rank, const int32_t *pos, const float *gates, int64_t T, int32_t K,
+                               int64_t H, uint16_t *out, mep_stream_t stream)
+{
+    if (quant != 0 && quant != 1) return MEP_ERR_DTYPE;
+    if (T > 0 && (!y_ptrs || !pos || !gates || !out || (quant == 1 && !scale_ptrs))) return MEP_ERR_NULLPTR;
+    if (T < 0 || K < 1 || K > MEP_MAX_K || H < 8 || H % (quant == 1 ? 16 : 8) != 0 || R < 1 || R > MEP_MAX_KEYS ||
+        rows_per_rank < 1 || T * K >= ((int64_t)1 << 31) || (int64_t)R * rows_per_rank >= ((int64_t)1 << 31))
+        return MEP_ERR_SHAPE;
+    if (T > 0 && (!aligned(out, 16) || !aligned(y_ptrs, 8) || (quant == 1 && !aligned(scale_ptrs, 8))))
+        return MEP_ERR_VALUE;
+    if (T == 0) return MEP_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (quant == 0) {
+        using kern_t = void (*)(const uint4 *const *, const int32_t *, const float *, int64_t, int, int64_t, int32_t,
+                                int64_t, uint4 *);
+        kern_t kern = K == 8 ? mep::k_combine_ranks_v8<8>
+                    : K == 4 ? mep::k_combine_ranks_v8<4>
+                    : K == 2 ? mep::k_combine_ranks_v8<2> : mep::k_combine_ranks_v8<0>;
+        kern<<<resident_grid(kern, 256, mep::ceil_div(T, 8)), 256, 0, s>>>((const uint4 *const *)y_ptrs, pos, gates, T,
+                                                                          K, H / 8, R, rows_per_rank, (uint4 *)out);
+    } else {
+        using kern_t = void (*)(const uint4 *const *, const float *const *, const int32_t *, const float *, int64_t,
+                                int, int64_t, int32_t, int64_t, uint4 *);
+        kern_t kern = K == 8 ? mep::k_combine_ranks_int8<8>
+                    : K == 4 ? mep::k_combine_ranks_int8<4>
+                    : K == 2 ? mep::k_combine_ranks_int8<2> : mep::k_combine_ranks_int8<0>;
+        kern<<<resident_grid(kern, 128, mep::ceil_div(T, 4)), 128, 0, s>>>((const uint4 *const *)y_ptrs, scale_ptrs,
+                                                                          pos, gates, T, K, H / 16, R, rows_per_rank,
+                                                                          (uint4 *)out);
     }
     return launched();
 }

@@ -23,6 +23,7 @@
  *    mep_stream_synchronize_timeout waits for its `stream` with a time limit; and
  *    mep_route_host's copies are synchronous when its host buffers are pageable.
  *    No call synchronises the whole device. mep_histogram, mep_plan, mep_plan_rank,
+ *    mep_dispatch_ranks, mep_combine_ranks,
  *    mep_update_expert, mep_update_expert_ranks, mep_dedup_plan, mep_dispatch,
  *    mep_expand, mep_dispatch_int8_smooth, mep_dequantize, mep_combine,
  *    mep_combine_int8, mep_combine_add_rmsnorm, mep_prefetch_plan, mep_prefetch_weights
@@ -240,6 +241,41 @@ mep_status_t mep_plan_rank(const int32_t *ids, const int32_t *hist_all, int32_t 
                            int32_t S, int32_t K, int32_t rank, int32_t *pos, int32_t *send_count,
                            int32_t *send_off, int32_t *recv_count, int32_t *recv_off,
                            void *workspace, size_t workspace_bytes, mep_stream_t stream);
+
+/*
+ * (e) — dispatch and combine when every EP rank's receive buffer is its own allocation:
+ * on several GPUs, the other ranks' buffers as peer mappings (NVLink), so that the
+ * dispatch stores every token row straight into its final, expert-grouped row on the
+ * destination rank (MoonEP zero-copy dispatch: twodots.gr article on MoonEP, zero-copy
+ * paragraph) and the combine loads the expert outputs back from where they are. The
+ * global row p = pos[n] (from mep_plan or mep_plan_rank) lives on rank
+ * d = p / rows_per_rank at local row p mod rows_per_rank.
+ *   mep_dispatch_ranks:  recv_ptrs[d][local, :] = x[n / K, :]      (quant 0, bf16)
+ *                        or the int8 codes and scale of mep_dispatch quant 1, the scale
+ *                        at scale_ptrs[d][local]
+ *   mep_combine_ranks:   out[g, :] = the sum of mep_combine (quant 0) or mep_combine_int8
+ *                        (quant 1) over rows y_ptrs[d][local, :] (scales scale_ptrs[d][local])
+ * recv_ptrs / y_ptrs / scale_ptrs are DEVICE arrays of R pointers (8-byte aligned), each
+ * a rank's buffer [rows_per_rank, H] (bf16 or int8) or its scales [rows_per_rank] fp32;
+ * buffers 16-byte aligned (int8 dispatch: 8), scales 4-byte aligned. The calls only
+ * store to and load from these buffers with plain 16- or 8-byte accesses; they wait on
+ * nothing, so the caller orders them against the other ranks' use of the buffers
+ * (a barrier between the exchange and the experts, as for any all-to-all).
+ * x bf16 [T, H] 16-byte aligned; pos int32 [T*K]; gates fp32 [T*K]; out bf16 [T, H]
+ * 16-byte aligned.
+ * Errors: quant outside {0,1} (MEP_ERR_DTYPE); NULL pointer (MEP_ERR_NULLPTR); T < 0, K
+ * outside [1, MEP_MAX_K], H not a positive multiple of 8 (combine of int8 rows: of 16),
+ * R outside [1, MEP_MAX_KEYS], rows_per_rank < 1, T*K or R*rows_per_rank >= 2^31
+ * (MEP_ERR_SHAPE); x, out or the pointer arrays misaligned (MEP_ERR_VALUE). Data errors:
+ * a pos outside [-1, R*rows_per_rank), or a rank whose table entry is NULL or
+ * misaligned, skips the slot and sets MEP_DERR_ROW_RANGE.
+ */
+mep_status_t mep_dispatch_ranks(const uint16_t *x, const int32_t *pos, int64_t T, int32_t K, int64_t H,
+                                int32_t quant, void *const *recv_ptrs, float *const *scale_ptrs, int32_t R,
+                                int64_t rows_per_rank, mep_stream_t stream);
+mep_status_t mep_combine_ranks(const void *const *y_ptrs, const float *const *scale_ptrs, int32_t quant,
+                               int32_t R, int64_t rows_per_rank, const int32_t *pos, const float *gates,
+                               int64_t T, int32_t K, int64_t H, uint16_t *out, mep_stream_t stream);
 
 /*
  * a5 with int8 rows (quantised return path) — combine of per-row int8 codes with one

@@ -265,3 +265,21 @@ def test_plan_launch_count(L):
     assert L.mep_plan_launches(64, 1536, 8, 8) == 4           # too many keys for one CTA
     assert L.mep_plan_launches(32, 256, 8192, 8) == 4         # int8 workload
     assert L.mep_plan_launches(0, 16, 128, 2) == 0
+
+
+def test_rank_buffer_calls_argument_checks(L):
+    P = FAKE
+    A = ctypes.c_void_p(0x2000)                        # 8-byte aligned stand-ins, never read
+    assert L.mep_dispatch_ranks(P, P, 4, 2, 64, 2, A, None, 2, 8, None) == 2       # DTYPE
+    assert L.mep_dispatch_ranks(None, P, 4, 2, 64, 0, A, None, 2, 8, None) == 1    # NULLPTR
+    assert L.mep_dispatch_ranks(P, P, 4, 2, 64, 1, A, None, 2, 8, None) == 1       # int8 without scales
+    assert L.mep_dispatch_ranks(P, P, 4, 2, 60, 0, A, None, 2, 8, None) == 3       # H % 8
+    assert L.mep_dispatch_ranks(P, P, 4, 2, 64, 0, A, None, 0, 8, None) == 3       # R
+    assert L.mep_dispatch_ranks(P, P, 4, 2, 64, 0, A, None, 2, 0, None) == 3       # rows per rank
+    assert L.mep_dispatch_ranks(ctypes.c_void_p(0x1008), P, 4, 2, 64, 0, A, None, 2, 8, None) == 4  # x misaligned
+    assert L.mep_dispatch_ranks(P, P, 0, 2, 64, 0, A, None, 2, 8, None) == 0       # empty: no launch
+    assert L.mep_combine_ranks(A, None, 0, 2, 8, None, P, 4, 2, 64, P, None) == 1
+    assert L.mep_combine_ranks(A, None, 1, 2, 8, P, P, 4, 2, 64, P, None) == 1     # int8 without scales
+    assert L.mep_combine_ranks(A, A, 1, 2, 8, P, P, 4, 2, 72, P, None) == 3        # int8: H % 16
+    assert L.mep_combine_ranks(A, None, 0, 2, 8, P, P, 4, 2, 64, ctypes.c_void_p(0x1004), None) == 4
+    assert L.mep_combine_ranks(A, None, 0, 2, 8, P, P, 0, 2, 64, P, None) == 0
