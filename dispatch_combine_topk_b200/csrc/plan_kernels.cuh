@@ -401,13 +401,35 @@ k_plan_small(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, 
     const int64_t sub = ((N + kWarps - 1) / kWarps + 31) / 32 * 32;   // <= 32 * kSmallPlanPerLane
     const int64_t lo = (int64_t)warp * sub, hi = min(N, lo + sub);
     int32_t *mine = cnt + warp * n_keys;
-    // key + 1 (0 for a dropped slot; keys < 4096) in 16-bit halves, two per register
+    // Every load first (ids and keep flags, all in flight together), then the checks:
+    // key + 1 (0 for a dropped slot; keys < 4096) in 16-bit halves, two per register.
     uint32_t kp[kSmallPlanPerLane / 2];
+    {
+        int32_t raw[kSmallPlanPerLane];
+        uint32_t kept = ~0u;                          // bit j: slot j is not dropped by keep
 #pragma unroll
-    for (int j = 0; j < kSmallPlanPerLane; j += 2) {
-        const int32_t k0 = lo + 32 * j < hi ? slot_key(ids, keep, lo + 32 * j + lane, hi, n_keys) : -1;
-        const int32_t k1 = lo + 32 * (j + 1) < hi ? slot_key(ids, keep, lo + 32 * (j + 1) + lane, hi, n_keys) : -1;
-        kp[j / 2] = (uint32_t)(k0 + 1) | ((uint32_t)(k1 + 1) << 16);
+        for (int j = 0; j < kSmallPlanPerLane; j++) {
+            const int64_t n = lo + 32 * j + lane;
+            raw[j] = n < hi ? ids[n] : -1;
+            if (keep && n < hi && !keep[n]) kept &= ~(1u << j);
+        }
+#pragma unroll
+        for (int j = 0; j < kSmallPlanPerLane; j += 2) {
+            int32_t k2[2];
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int64_t n = lo + 32 * (j + h) + lane;
+                int32_t e = raw[j + h];
+                if (n >= hi || !((kept >> (j + h)) & 1u)) {
+                    e = -1;
+                } else if (e < 0 || e >= n_keys) {
+                    flag_error(MEP_DERR_KEY_RANGE);
+                    e = -1;
+                }
+                k2[h] = e;
+            }
+            kp[j / 2] = (uint32_t)(k2[0] + 1) | ((uint32_t)(k2[1] + 1) << 16);
+        }
     }
     auto key_at = [&](int j) -> int32_t { return (int32_t)((kp[j / 2] >> (16 * (j & 1))) & 0xffffu) - 1; };
 #pragma unroll
