@@ -22,16 +22,46 @@ import torch
 import torch.distributed as dist
 
 
+def _host_collectives(group) -> bool:
+    """True when the group's backend moves host tensors only (gloo)."""
+    return dist.get_backend(group) == "gloo"
+
+
 def gather_histograms(hist: torch.Tensor, group=None) -> torch.Tensor:
     """All-gather of the ranks' per-expert histograms: int32 [R, E], row r = rank r's
     ``hist``, on ``hist``'s device. Every rank of ``group`` must call it with a
-    histogram of the same length."""
+    histogram of the same length. Over gloo a device histogram goes through host memory."""
     if hist.dim() != 1 or hist.dtype != torch.int32:
         raise ValueError("hist must be a 1-D int32 tensor")
     world = dist.get_world_size(group)
-    parts = [torch.empty_like(hist) for _ in range(world)]
-    dist.all_gather(parts, hist.contiguous(), group=group)
-    return torch.stack(parts)
+    src = hist.contiguous()
+    if src.is_cuda and _host_collectives(group):
+        src = src.cpu()
+    parts = [torch.empty_like(src) for _ in range(world)]
+    dist.all_gather(parts, src, group=group)
+    return torch.stack(parts).to(hist.device)
+
+
+def share_buffers(buffers: dict, group=None) -> list:
+    """Every rank's receive buffers, mapped into this process: CUDA IPC handles of this
+    rank's tensors are all-gathered (as picklable objects over the process group) and the
+    other ranks' handles opened here. Returns one dict per rank, ``buffers`` itself for
+    this rank. The mapped tensors alias the other ranks' memory (on the same GPU, or on a
+    peer GPU through NVLink); each rank must keep its own buffers alive, and the ranks
+    must order their kernels on the buffers with a barrier, until every rank is done."""
+    from torch.multiprocessing.reductions import reduce_tensor
+
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    mine = {k: reduce_tensor(v) for k, v in buffers.items()}
+    every = [None] * world
+    dist.all_gather_object(every, mine, group=group)
+    out = []
+    for r, handles in enumerate(every):
+        if r == rank:
+            out.append(buffers)
+        else:
+            out.append({k: fn(*args) for k, (fn, args) in handles.items()})
+    return out
 
 
 def plan_rank(ids: torch.Tensor, E: int, S: int, K: int, group=None, stream=None,
