@@ -744,18 +744,47 @@ k_combine_int8_warp(const uint4 *__restrict__ yq, const float *__restrict__ ysca
                 gk[k] = __shfl_sync(0xffffffffu, g_mine, k);
                 sk[k] = __shfl_sync(0xffffffffu, s_mine, k);
             }
-            for (int64_t c = lane; c < H16; c += 32) {
-                float2 acc[8];
+            // every slot kept (the usual case): a loop without the per-slot tests, the rows'
+            // base addresses once per token, and the output stored with plain stores, which
+            // leave the compiler free to schedule around them (3% faster inside the step)
+            bool all = true;
 #pragma unroll
-                for (int j = 0; j < 8; j++) acc[j] = make_float2(0.0f, 0.0f);
-                uint4 v[KC];
+            for (int k = 0; k < KC; k++) all = all && pk[k] >= 0;
+            if (all) {
+                const uint4 *rp[KC];
 #pragma unroll
-                for (int k = 0; k < KC; k++)
-                    v[k] = pk[k] >= 0 ? ld_stream(yq + (int64_t)pk[k] * H16 + c) : make_uint4(0, 0, 0, 0);
+                for (int k = 0; k < KC; k++) rp[k] = yq + (int64_t)pk[k] * H16;
+                for (int64_t c = lane; c < H16; c += 32) {
+                    float2 acc[8];
 #pragma unroll
-                for (int k = 0; k < KC; k++)
-                    if (pk[k] >= 0) add_int8_x16(acc, v[k], gk[k], sk[k]);
-                store_bf16x16(dst + 2 * c, acc);
+                    for (int j = 0; j < 8; j++) acc[j] = make_float2(0.0f, 0.0f);
+                    uint4 v[KC];
+#pragma unroll
+                    for (int k = 0; k < KC; k++) v[k] = ld_stream(rp[k] + c);
+#pragma unroll
+                    for (int k = 0; k < KC; k++) add_int8_x16(acc, v[k], gk[k], sk[k]);
+                    uint4 o0, o1;
+                    o0.x = pack_bf16x2(acc[0].x, acc[0].y); o0.y = pack_bf16x2(acc[1].x, acc[1].y);
+                    o0.z = pack_bf16x2(acc[2].x, acc[2].y); o0.w = pack_bf16x2(acc[3].x, acc[3].y);
+                    o1.x = pack_bf16x2(acc[4].x, acc[4].y); o1.y = pack_bf16x2(acc[5].x, acc[5].y);
+                    o1.z = pack_bf16x2(acc[6].x, acc[6].y); o1.w = pack_bf16x2(acc[7].x, acc[7].y);
+                    dst[2 * c] = o0;
+                    dst[2 * c + 1] = o1;
+                }
+            } else {
+                for (int64_t c = lane; c < H16; c += 32) {
+                    float2 acc[8];
+#pragma unroll
+                    for (int j = 0; j < 8; j++) acc[j] = make_float2(0.0f, 0.0f);
+                    uint4 v[KC];
+#pragma unroll
+                    for (int k = 0; k < KC; k++)
+                        v[k] = pk[k] >= 0 ? ld_stream(yq + (int64_t)pk[k] * H16 + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int k = 0; k < KC; k++)
+                        if (pk[k] >= 0) add_int8_x16(acc, v[k], gk[k], sk[k]);
+                    store_bf16x16(dst + 2 * c, acc);
+                }
             }
         } else {
             // warp-uniform trip count: every lane reaches the shuffles
