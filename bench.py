@@ -120,9 +120,9 @@ TRAFFIC = {
     ("k_combine_v8", "r8_e64_s4096_k8_h7168"): {
         "bytes": 4 * 1005.660e6, "src": "aa70b87f5f33b11a", "case_S": 1024, "case_mb": 1005.660},
     ("k_dispatch_int8_staged", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1114.875e6, "src": "597997762b516c3e", "case_S": 512, "case_mb": 1114.875},
+        "bytes": 16 * 1115.672e6, "src": "597997762b516c3e", "case_S": 512, "case_mb": 1115.672},
     ("k_combine_int8_warp", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1117.359e6, "src": "31ddea297a5f9077", "case_S": 512, "case_mb": 1117.359},
+        "bytes": 16 * 1117.330e6, "src": "a2aec7cc7412bc6f", "case_S": 512, "case_mb": 1117.330},
     ("k_dispatch_warp", "skew_r64_e512_s2048_k8_h4096"): {
         "bytes": 4 * 2357.854e6, "src": "ecb53c46b3d954ca", "case_S": 512, "case_mb": 2357.854},
     ("k_combine_v8", "skew_r64_e512_s2048_k8_h4096"): {
