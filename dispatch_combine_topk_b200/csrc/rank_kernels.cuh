@@ -82,7 +82,7 @@ k_dispatch_ranks_warp(const uint4 *__restrict__ x, const int32_t *__restrict__ p
 // token: amax over the row, scale = amax / 127, codes by the IEEE quotient, 8 codes per
 // 8-byte store to each destination, the scale beside them. Requires H % 8 == 0, 16-byte
 // aligned x and 8-byte aligned buffers.
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 k_dispatch_ranks_int8(const uint4 *__restrict__ x, const int32_t *__restrict__ pos, int64_t T, int K, int64_t H8,
                       uint2 *const *__restrict__ recv, float *const *__restrict__ scales, int32_t R, int64_t rpr)
 {
@@ -133,7 +133,7 @@ k_dispatch_ranks_int8(const uint4 *__restrict__ x, const int32_t *__restrict__ p
 // fl(gate * y)), fp32, no FMA (the sum of k_combine_v8). One warp per token, 16-byte
 // chunks, all K loads of a chunk in flight. Requires H % 8 == 0, 16-byte alignment.
 template <int KC>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 3)
 k_combine_ranks_v8(const uint4 *const *__restrict__ y, const int32_t *__restrict__ pos,
                    const float *__restrict__ gates, int64_t T, int Krt, int64_t H8, int32_t R, int64_t rpr,
                    uint4 *__restrict__ out)

@@ -248,6 +248,24 @@ __device__ __forceinline__ uint2 q8x8_packed(const float (&x)[8], const float (&
                       __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410));
 }
 
+// q8x8_packed for four values: x (bf16 values as fp32) times the smoothing scales s, the
+// codes of the four products packed into one word (lowest column in the low byte).
+__device__ __forceinline__ uint32_t q8x4_packed(const float (&x)[4], const float4 &s, float scale, float inv)
+{
+    const float2 kShift = make_float2(12582912.0f, 12582912.0f), kNegShift = make_float2(-12582912.0f, -12582912.0f);
+    const float2 inv2 = make_float2(inv, inv);
+    const float2 v0 = mul2_rn(make_float2(x[0], x[1]), make_float2(s.x, s.y));
+    const float2 v1 = mul2_rn(make_float2(x[2], x[3]), make_float2(s.z, s.w));
+    const float2 y0 = mul2_rn(v0, inv2), y1 = mul2_rn(v1, inv2);
+    const float2 t0 = add2_rn(y0, kShift), t1 = add2_rn(y1, kShift);
+    const float2 r0 = add2_rn(t0, kNegShift), r1 = add2_rn(t1, kNegShift);
+    const float2 d0 = add2_rn(y0, make_float2(-r0.x, -r0.y)), d1 = add2_rn(y1, make_float2(-r1.x, -r1.y));
+    const float dmax = fmaxf(fmaxf(fabsf(d0.x), fabsf(d0.y)), fmaxf(fabsf(d1.x), fabsf(d1.y)));
+    if (inv < 0.0f || dmax >= 0.5f - 0x1p-15f) return q8x4(v0.x, v0.y, v1.x, v1.y, scale);
+    return __byte_perm(__byte_perm(__float_as_uint(t0.x), __float_as_uint(t0.y), 0x0040),
+                       __byte_perm(__float_as_uint(t1.x), __float_as_uint(t1.y), 0x0040), 0x5410);
+}
+
 // Per-token dynamic int8: one CTA per token, pass 1 reduces amax over the row, pass 2
 // re-reads the row (from L1/L2) and writes the K copies of the codes and the scale.
 // Needs H % 8 == 0 and 16-byte aligned x, 8-byte aligned recv.
@@ -856,9 +874,10 @@ __device__ __forceinline__ float block_sum(float v, float *red)
 // For every token: c = the combine output row (bf16, as k_combine_v8), x = fl(c + r)
 // with r the residual row, x_out = bf16(x), rstd = rsqrt_rn(fl(sum x^2 / H) + eps),
 // y_out = bf16(fl(fl(x * rstd) * gamma)). The fp32 row x is kept in shared memory
-// (H floats) between the reduction and the second pass.
+// (H floats) between the reduction and the second pass, column 8c + j of the row at
+// xs[j * H8 + c], so that the lanes of a warp (consecutive c) touch consecutive words.
 template <int KC>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 k_combine_add_rmsnorm_v8(const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
                          const float *__restrict__ gates, int64_t T, int Krt, int64_t H8, int64_t rows,
                          const uint4 *__restrict__ residual, const uint4 *__restrict__ gamma, float eps,
@@ -887,8 +906,8 @@ k_combine_add_rmsnorm_v8(const uint4 *__restrict__ y, const int32_t *__restrict_
                 const uint32_t cb = pack_bf16x2(acc[2 * j], acc[2 * j + 1]);   // the combine output
                 const float x0 = __fadd_rn(bf16lo(cb), bf16lo(rw[j]));
                 const float x1 = __fadd_rn(bf16hi(cb), bf16hi(rw[j]));
-                xs[8 * c + 2 * j] = x0;
-                xs[8 * c + 2 * j + 1] = x1;
+                xs[(2 * j) * H8 + c] = x0;
+                xs[(2 * j + 1) * H8 + c] = x1;
                 ss = fmaf(x0, x0, ss);
                 ss = fmaf(x1, x1, ss);
                 xo[j] = pack_bf16x2(x0, x1);
@@ -904,8 +923,8 @@ k_combine_add_rmsnorm_v8(const uint4 *__restrict__ y, const int32_t *__restrict_
             uint32_t yo[4];
 #pragma unroll
             for (int j = 0; j < 4; j++) {
-                const float y0 = __fmul_rn(__fmul_rn(xs[8 * c + 2 * j], rstd), bf16lo(gw[j]));
-                const float y1 = __fmul_rn(__fmul_rn(xs[8 * c + 2 * j + 1], rstd), bf16hi(gw[j]));
+                const float y0 = __fmul_rn(__fmul_rn(xs[(2 * j) * H8 + c], rstd), bf16lo(gw[j]));
+                const float y1 = __fmul_rn(__fmul_rn(xs[(2 * j + 1) * H8 + c], rstd), bf16hi(gw[j]));
                 yo[j] = pack_bf16x2(y0, y1);
             }
             st_v4(y_out + t * H8 + c, make_uint4(yo[0], yo[1], yo[2], yo[3]));
@@ -1049,19 +1068,24 @@ k_dispatch_int8_smooth(const uint4 *__restrict__ x, const int32_t *__restrict__ 
 // forms, slot by slot, each thread's maximum of |fl(x * smooth[e_k])| and its warp
 // maximum (every smoothing row read once; the warp maximum by redux.sync); one block
 // barrier later the K scales follow from the warps' maxima; pass 2 forms each product
-// again (the smoothing rows a second time, from L2) and stores the codes. Two block barriers per token instead of two per
-// slot. Both passes walk the slots in a loop that is not unrolled, which keeps the code
-// short and the registers at 64 (4 CTAs per SM).
-template <int KC, int kChunks>
+// again (the smoothing rows a second time, from L2) and stores the codes. Two block
+// barriers per token instead of two per slot. Both passes walk the slots in a loop that
+// is not unrolled, which keeps the code short and the registers at 64 (4 CTAs per SM).
+// A thread takes groups of 4 columns (g = tid + 256 i): its x, its smoothing scales and
+// its codes are then 8, 16 and 4 consecutive bytes, so every warp load and store of the
+// three is one contiguous span (the smoothing rows, read K times per token, are the
+// bulk of the traffic through L1).
+template <int KC, int kGroups>
 __global__ void __launch_bounds__(256)
-k_dispatch_int8_smooth_k(const uint4 *__restrict__ x, const int32_t *__restrict__ ids, const int32_t *__restrict__ pos,
-                         int64_t T, int64_t H8, const float4 *__restrict__ smooth, int32_t n_experts, int64_t rows,
-                         uint2 *__restrict__ recv, float *__restrict__ recv_scale)
+k_dispatch_int8_smooth_k(const uint2 *__restrict__ x, const int32_t *__restrict__ ids, const int32_t *__restrict__ pos,
+                         int64_t T, int64_t H4, const float4 *__restrict__ smooth, int32_t n_experts, int64_t rows,
+                         uint32_t *__restrict__ recv, float *__restrict__ recv_scale)
 {
     __shared__ int32_t sp[KC], se[KC];
     __shared__ float red[8][KC];                      // 256 threads = 8 warps
     __shared__ float ssc[KC];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h4 = (int)H4;                           // at most 256 * kGroups
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         if (threadIdx.x < KC) {
             int32_t p = pos[t * KC + threadIdx.x];
@@ -1077,18 +1101,17 @@ k_dispatch_int8_smooth_k(const uint4 *__restrict__ x, const int32_t *__restrict_
             sp[threadIdx.x] = p;
             se[threadIdx.x] = e;
         }
-        float xr[kChunks][8];
+        float xr[kGroups][4];
+        const uint2 *xrow = x + t * H4;
 #pragma unroll
-        for (int i = 0; i < kChunks; i++) {
-            const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
-            if (c < H8) {
-                const uint4 v = x[t * H8 + c];
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    xr[i][2 * j] = bf16lo(w[j]);
-                    xr[i][2 * j + 1] = bf16hi(w[j]);
-                }
+        for (int i = 0; i < kGroups; i++) {
+            const int g = threadIdx.x + i * 256;
+            if (g < h4) {
+                const uint2 v = xrow[g];
+                xr[i][0] = bf16lo(v.x);
+                xr[i][1] = bf16hi(v.x);
+                xr[i][2] = bf16lo(v.y);
+                xr[i][3] = bf16hi(v.y);
             }
         }
         __syncthreads();
@@ -1097,19 +1120,15 @@ k_dispatch_int8_smooth_k(const uint4 *__restrict__ x, const int32_t *__restrict_
             float amax = 0.0f;
             const int32_t e = se[k];
             if (sp[k] >= 0 && e >= 0) {
-                const float4 *srow = smooth + (int64_t)e * H8 * 2;
+                const float4 *srow = smooth + (int64_t)e * H4;
 #pragma unroll
-                for (int i = 0; i < kChunks; i++) {
-                    const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
-                    if (c < H8) {
-                        const float4 s0 = srow[2 * c], s1 = srow[2 * c + 1];
-                        const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-                        for (int j = 0; j < 4; j++) {
-                            const float2 v = mul2_rn(make_float2(xr[i][2 * j], xr[i][2 * j + 1]),
-                                                     make_float2(sv[2 * j], sv[2 * j + 1]));
-                            amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
-                        }
+                for (int i = 0; i < kGroups; i++) {
+                    const int g = threadIdx.x + i * 256;
+                    if (g < h4) {
+                        const float4 sv = srow[g];
+                        const float2 v0 = mul2_rn(make_float2(xr[i][0], xr[i][1]), make_float2(sv.x, sv.y));
+                        const float2 v1 = mul2_rn(make_float2(xr[i][2], xr[i][3]), make_float2(sv.z, sv.w));
+                        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v0.x), fabsf(v0.y)), fmaxf(fabsf(v1.x), fabsf(v1.y))));
                     }
                 }
             }
@@ -1132,15 +1151,12 @@ k_dispatch_int8_smooth_k(const uint4 *__restrict__ x, const int32_t *__restrict_
             const int32_t p = sp[k], e = se[k];
             if (p < 0 || e < 0) continue;
             const float scale = ssc[k], inv = quant_inv(scale);
-            const float4 *srow = smooth + (int64_t)e * H8 * 2;
+            const float4 *srow = smooth + (int64_t)e * H4;
+            uint32_t *dst = recv + (int64_t)p * H4;
 #pragma unroll
-            for (int i = 0; i < kChunks; i++) {
-                const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
-                if (c < H8) {
-                    const float4 s0 = srow[2 * c], s1 = srow[2 * c + 1];
-                    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-                    recv[(int64_t)p * H8 + c] = q8x8_packed(xr[i], sv, scale, inv);
-                }
+            for (int i = 0; i < kGroups; i++) {
+                const int g = threadIdx.x + i * 256;
+                if (g < h4) dst[g] = q8x4_packed(xr[i], srow[g], scale, inv);
             }
         }
         __syncthreads();                                   // sp, se, ssc and red are reused
