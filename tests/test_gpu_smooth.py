@@ -1,7 +1,8 @@
 """GPU parity of the int8 dispatch with per-expert smoothing scales against the oracle
-(codes and scales bit for bit). K in {2, 4, 8} (with up to 64 columns per thread) takes
-the fused kernel (all K slots of a token in one CTA, two passes), other K the per-slot
-kernel, other H or alignments the scalar kernel. The full int8 workload is compared
+(codes and scales bit for bit). K in {2, 4, 8} with H % 4 == 0 (up to 64 columns per
+thread, in groups of 4) takes the fused kernel (all K slots of a token in one CTA, two
+passes), other K the per-slot kernel (H % 8 == 0), other H or alignments the scalar
+kernel. The full int8 workload is compared
 whole, one rank partition at a time, and with all-ones scales against the plain
 per-token int8 dispatch."""
 from concurrent.futures import ThreadPoolExecutor
@@ -19,7 +20,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("K", [1, 2, 3, 4, 8])
-@pytest.mark.parametrize("H", [8, 64, 4096, 7168, 12288, 20000, 7])
+@pytest.mark.parametrize("H", [8, 12, 64, 4096, 4100, 7168, 12288, 16384, 16388, 20000, 7])
 def test_smooth_dispatch_matches_oracle(K, H):
     rng = np.random.default_rng(K * 7 + H)
     T, E = 23, 10
@@ -41,9 +42,8 @@ def test_smooth_dispatch_matches_oracle(K, H):
 
 @pytest.mark.parametrize("K,H", [(2, 4096), (4, 7168), (8, 4096), (8, 12288), (8, 7168)])
 def test_smooth_dispatch_many_tokens_per_cta(K, H):
-    """More tokens than CTAs resident on the GPU, so every CTA walks many tokens (and
-    prefetches the next slot's smoothing row while computing one); dropped slots and
-    whole buffers."""
+    """More tokens than CTAs resident on the GPU, so every CTA walks many tokens;
+    dropped slots and whole buffers."""
     rng = np.random.default_rng(K * 13 + H)
     T, E = 3001, 40
     x = (torch.randn((T, H), generator=torch.Generator().manual_seed(H + K)) * 3).to(torch.bfloat16)
@@ -58,6 +58,33 @@ def test_smooth_dispatch_many_tokens_per_cta(K, H):
                                  torch.from_numpy(pos).to(dev()), K, torch.from_numpy(sm).to(dev()), q, sc)
     q_ref, s_ref = oracle.dispatch_int8_smooth(bits(x), ids, pos, K, sm, rows)
     assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert mep.mep_get_error() == 0
+
+
+@pytest.mark.parametrize("x_off,q_off", [(4, 4), (4, 0), (0, 4), (1, 0), (0, 1)])
+def test_smooth_dispatch_offset_buffers(x_off, q_off):
+    """Token rows and receive rows that start off their usual alignment: an x 8 bytes and
+    a receive buffer 4 bytes off 16 still take the kernel of 4-column groups; 2-byte or
+    1-byte offsets take the scalar kernel. Same codes and scales either way."""
+    rng = np.random.default_rng(100 * x_off + q_off)
+    T, E, K, H = 37, 12, 8, 1028
+    x = (torch.randn((T, H), generator=torch.Generator().manual_seed(x_off)) * 2).to(torch.bfloat16)
+    ids = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
+    rows = T * K + 3
+    pos = rng.permutation(rows)[: T * K].astype(np.int32)
+    pos[rng.random(T * K) < 0.1] = -1
+    sm = (10.0 ** rng.uniform(-1, 1, (E, H))).astype(np.float32)
+    xb = torch.zeros(T * H + x_off, dtype=torch.bfloat16, device=dev())
+    xv = xb[x_off:].view(T, H)
+    xv.copy_(x.to(dev()))
+    qb = torch.zeros(rows * H + q_off, dtype=torch.int8, device=dev())
+    qv = qb[q_off:].view(rows, H)
+    sc = torch.zeros(rows, dtype=torch.float32, device=dev())
+    mep.mep_dispatch_int8_smooth(xv, torch.from_numpy(ids).to(dev()).view(-1), torch.from_numpy(pos).to(dev()), K,
+                                 torch.from_numpy(sm).to(dev()), qv, sc)
+    q_ref, s_ref = oracle.dispatch_int8_smooth(bits(x), ids, pos, K, sm, rows)
+    assert np.array_equal(qv.cpu().numpy(), q_ref)
     assert np.array_equal(sc.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
     assert mep.mep_get_error() == 0
 
