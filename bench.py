@@ -507,9 +507,9 @@ class Route:
         if step == "expand":
             return "k_expand_warp" if w.H % 16 == 0 or (not w.quant and w.H % 8 == 0) else "k_expand_bytes"
         if w.quant and self.smooth:
-            if w.H % 4 == 0 and w.K in (2, 4, 8) and w.H // 4 <= 16 * 256:
+            if w.H % 4 == 0 and w.H // 4 <= 16 * 256:
                 return "k_dispatch_int8_smooth_k"
-            return "k_dispatch_int8_smooth" if w.H % 8 == 0 else "k_dispatch_int8_smooth_scalar"
+            return "k_dispatch_int8_smooth_scalar"
         if w.quant:
             return "k_dispatch_int8_staged" if w.H % 16 == 0 else "k_dispatch_int8"
         return "k_dispatch_warp" if w.H % 8 == 0 else "k_dispatch_elem"

@@ -712,36 +712,19 @@ mep_status_t mep_dispatch_int8_smooth(const uint16_t *x, const int32_t *ids, con
         return MEP_ERR_SHAPE;
     if (T == 0) return MEP_OK;
     cudaStream_t s = (cudaStream_t)stream;
-    const int grid = token_grid(T, 8);
-    const int64_t H8 = H / 8, H4 = H / 4;
-    const bool vec = H % 8 == 0 && aligned(x, 16) && aligned(recv, 8) && aligned(smooth, 16);
+    const int64_t H4 = H / 4;
     const bool vec4 = H % 4 == 0 && aligned(x, 8) && aligned(recv, 4) && aligned(smooth, 16);
-    const int64_t per_thread = mep::ceil_div(H8, 256), groups = mep::ceil_div(H4, 256);
-    using smooth_k_t = void (*)(const uint2 *, const int32_t *, const int32_t *, int64_t, int64_t, const float4 *,
-                                int32_t, int64_t, uint32_t *, float *);
-    smooth_k_t fused = nullptr;
+    const int64_t groups = mep::ceil_div(H4, 256);
     if (vec4 && groups <= 16) {
-        const bool g8 = groups <= 8;
-        switch (K) {
-        case 2: fused = g8 ? mep::k_dispatch_int8_smooth_k<2, 8> : mep::k_dispatch_int8_smooth_k<2, 16>; break;
-        case 4: fused = g8 ? mep::k_dispatch_int8_smooth_k<4, 8> : mep::k_dispatch_int8_smooth_k<4, 16>; break;
-        case 8: fused = g8 ? mep::k_dispatch_int8_smooth_k<8, 8> : mep::k_dispatch_int8_smooth_k<8, 16>; break;
-        default: break;
-        }
-    }
-    if (fused) {
         // the K slots of a token together; the grid is what the GPU holds resident
-        fused<<<resident_grid(fused, 256, T), 256, 0, s>>>((const uint2 *)x, ids, pos, T, H4, (const float4 *)smooth,
+        using smooth_k_t = void (*)(const uint2 *, const int32_t *, const int32_t *, int64_t, int, int64_t,
+                                    const float4 *, int32_t, int64_t, uint32_t *, float *);
+        const smooth_k_t fused = groups <= 8 ? mep::k_dispatch_int8_smooth_k<8> : mep::k_dispatch_int8_smooth_k<16>;
+        fused<<<resident_grid(fused, 256, T), 256, 0, s>>>((const uint2 *)x, ids, pos, T, K, H4, (const float4 *)smooth,
                                                           n_experts, rows, (uint32_t *)recv, recv_scale);
-    } else if (vec && per_thread <= 4) {
-        mep::k_dispatch_int8_smooth<4><<<grid, 256, 0, s>>>((const uint4 *)x, ids, pos, T, K, H8, (const float4 *)smooth,
-                                                           n_experts, rows, (uint2 *)recv, recv_scale);
-    } else if (vec && per_thread <= 8) {
-        mep::k_dispatch_int8_smooth<8><<<grid, 256, 0, s>>>((const uint4 *)x, ids, pos, T, K, H8, (const float4 *)smooth,
-                                                           n_experts, rows, (uint2 *)recv, recv_scale);
     } else {
-        mep::k_dispatch_int8_smooth_scalar<<<grid, 256, 0, s>>>(x, ids, pos, T, K, H, smooth, n_experts, rows, recv,
-                                                               recv_scale);
+        mep::k_dispatch_int8_smooth_scalar<<<token_grid(T, 8), 256, 0, s>>>(x, ids, pos, T, K, H, smooth, n_experts,
+                                                                           rows, recv, recv_scale);
     }
     return launched();
 }

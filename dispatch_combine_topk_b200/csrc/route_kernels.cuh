@@ -178,9 +178,9 @@ __device__ __forceinline__ uint32_t q8x4(float a, float b, float c, float d, flo
     return q(a) | (q(b) << 8) | (q(c) << 16) | (q(d) << 24);
 }
 
-// 1 / scale for q8x8: 0 when scale is 0 (every value of such a row is 0), and -1 when
-// 1 / scale overflows (scale below about 2.9e-39, a subnormal): such rows take the IEEE
-// quotient.
+// 1 / scale for q8x4_packed: 0 when scale is 0 (every value of such a row is 0), and -1
+// when 1 / scale overflows (scale below about 2.9e-39, a subnormal): such rows take the
+// IEEE quotient.
 __device__ __forceinline__ float quant_inv(float scale)
 {
     if (scale == 0.0f) return 0.0f;
@@ -188,68 +188,21 @@ __device__ __forceinline__ float quant_inv(float scale)
     return isinf(inv) ? -1.0f : inv;
 }
 
-// The codes of q8x4 for eight values (two packed words), with inv = quant_inv(scale) and
-// the values of a row whose amax gave scale = fl(amax / 127) (the smoothing dispatches).
-// Each quotient is taken as y = fl(v * inv). |v / scale| < 127.0001 (scale is within one
-// rounding of amax / 127, also when it is subnormal with 1 / scale finite) and inv is
-// within 2^-24 of 1 / scale, so |y - v/scale| < 2^-16 and |y - fl(v/scale)| < 2^-15:
-// unless y lies within 2^-15 of a half-integer, y and the correctly rounded quotient round
-// to the same integer, which is in [-127, 127] without a clamp. y + 1.5 * 2^23 rounds y
-// half-to-even to an integer whose two's-complement low byte is the code. When any of
-// the eight lies that close to a half-integer (about 1 group in 2000), or the row's
-// 1 / scale overflows, all eight take the IEEE quotient of q8x4 instead.
-__device__ __forceinline__ uint2 q8x8(const float (&v)[8], float scale, float inv)
-{
-    constexpr float kShift = 12582912.0f;             // 1.5 * 2^23
-    constexpr float kNearHalf = 0.5f - 0x1p-15f;
-    uint32_t b[8];
-    bool exact = inv < 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; j++) {
-        const float y = __fmul_rn(v[j], inv);
-        const float t = __fadd_rn(y, kShift);
-        exact |= fabsf(__fsub_rn(y, __fsub_rn(t, kShift))) >= kNearHalf;
-        b[j] = __float_as_uint(t);
-    }
-    if (exact)
-        return make_uint2(q8x4(v[0], v[1], v[2], v[3], scale), q8x4(v[4], v[5], v[6], v[7], scale));
-    return make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410),
-                      __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410));
-}
-
-// q8x8 with the products and the rounding arithmetic on pairs of values (packed f32x2,
-// each half rounded on its own): xs = fl(x * s), y = fl(xs * inv), t = fl(y + 1.5*2^23),
-// r = t - 1.5*2^23, d = y - r. No product here feeds a sum whose rounding matters: had a
-// pair of them been fused, t would round the exact xs * inv, which is still within the
-// bound, and d only decides whether to take the IEEE quotient.
-__device__ __forceinline__ uint2 q8x8_packed(const float (&x)[8], const float (&s)[8], float scale, float inv)
-{
-    const float2 kShift = make_float2(12582912.0f, 12582912.0f), kNegShift = make_float2(-12582912.0f, -12582912.0f);
-    const float2 inv2 = make_float2(inv, inv);
-    float xs[8];
-    uint32_t b[8];
-    float dmax = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-        const float2 v = mul2_rn(make_float2(x[2 * j], x[2 * j + 1]), make_float2(s[2 * j], s[2 * j + 1]));
-        const float2 y = mul2_rn(v, inv2);
-        const float2 t = add2_rn(y, kShift);
-        const float2 r = add2_rn(t, kNegShift);
-        const float2 d = add2_rn(y, make_float2(-r.x, -r.y));
-        dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
-        xs[2 * j] = v.x;
-        xs[2 * j + 1] = v.y;
-        b[2 * j] = __float_as_uint(t.x);
-        b[2 * j + 1] = __float_as_uint(t.y);
-    }
-    if (inv < 0.0f || dmax >= 0.5f - 0x1p-15f)
-        return make_uint2(q8x4(xs[0], xs[1], xs[2], xs[3], scale), q8x4(xs[4], xs[5], xs[6], xs[7], scale));
-    return make_uint2(__byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410),
-                      __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410));
-}
-
-// q8x8_packed for four values: x (bf16 values as fp32) times the smoothing scales s, the
-// codes of the four products packed into one word (lowest column in the low byte).
+// The codes of q8x4 for the four products v = fl(x * s) of a row whose amax gave
+// scale = fl(amax / 127) (the smoothing dispatch), with inv = quant_inv(scale), packed
+// into one word (lowest column in the low byte). Each quotient is taken as
+// y = fl(v * inv). |v / scale| < 127.0001 (scale is within one rounding of amax / 127,
+// also when it is subnormal with 1 / scale finite) and inv is within 2^-24 of 1 / scale,
+// so |y - v/scale| < 2^-16 and |y - fl(v/scale)| < 2^-15: unless y lies within 2^-15 of
+// a half-integer, y and the correctly rounded quotient round to the same integer, which
+// is in [-127, 127] without a clamp. t = fl(y + 1.5 * 2^23) rounds y half-to-even to an
+// integer whose two's-complement low byte is the code; d = y - (t - 1.5 * 2^23) is its
+// distance to y. When any of the four lies that close to a half-integer (about 1 group
+// in 4000), or the row's 1 / scale overflows, all four take the IEEE quotient of q8x4.
+// The products and the rounding run on pairs (packed f32x2, each half rounded on its
+// own). No product feeds a sum whose rounding matters: had the compiler fused v * inv
+// into the sum t, t would round the exact product, which is within the same bound, and
+// d only decides whether to take the IEEE quotient.
 __device__ __forceinline__ uint32_t q8x4_packed(const float (&x)[4], const float4 &s, float scale, float inv)
 {
     const float2 kShift = make_float2(12582912.0f, 12582912.0f), kNegShift = make_float2(-12582912.0f, -12582912.0f);
@@ -994,78 +947,8 @@ __device__ __forceinline__ float block_max(float v, float *red)
     return red[32];
 }
 
-// One CTA per token; the token's row (up to kChunks 8-column chunks per thread) stays in
-// registers. For every kept slot: xs = fl(x * smooth[e]) with e the slot's expert, amax
-// over the row (block reduction), scale = amax / 127, codes round_half_even(xs / scale)
-// clamped to [-127, 127], stored 8 bytes per chunk with the slot's scale.
-template <int kChunks>
-__global__ void __launch_bounds__(256)
-k_dispatch_int8_smooth(const uint4 *__restrict__ x, const int32_t *__restrict__ ids, const int32_t *__restrict__ pos,
-                       int64_t T, int K, int64_t H8, const float4 *__restrict__ smooth, int32_t n_experts,
-                       int64_t rows, uint2 *__restrict__ recv, float *__restrict__ recv_scale)
-{
-    __shared__ int32_t sp[kMaxK];
-    __shared__ int32_t se[kMaxK];
-    __shared__ float red[33];
-    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-        load_token_rows(pos, t, K, rows, sp);
-        if (threadIdx.x < K) {
-            int32_t e = ids[t * K + threadIdx.x];
-            if (e < 0 || e >= n_experts) {
-                flag_error(MEP_DERR_KEY_RANGE);
-                e = -1;
-            }
-            se[threadIdx.x] = e;
-        }
-        float xr[kChunks][8];
-#pragma unroll
-        for (int i = 0; i < kChunks; i++) {
-            const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
-            if (c < H8) {
-                const uint4 v = x[t * H8 + c];
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    xr[i][2 * j] = bf16lo(w[j]);
-                    xr[i][2 * j + 1] = bf16hi(w[j]);
-                }
-            }
-        }
-        __syncthreads();
-        for (int k = 0; k < K; k++) {
-            const int32_t p = sp[k], e = se[k];
-            if (p < 0 || e < 0) continue;                 // uniform over the block
-            const float4 *srow = smooth + (int64_t)e * H8 * 2;
-            float xs[kChunks][8];
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < kChunks; i++) {
-                const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
-                if (c < H8) {
-                    const float4 s0 = srow[2 * c], s1 = srow[2 * c + 1];
-                    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-                    for (int j = 0; j < 8; j++) {
-                        xs[i][j] = __fmul_rn(xr[i][j], sv[j]);
-                        amax = fmaxf(amax, fabsf(xs[i][j]));
-                    }
-                }
-            }
-            amax = block_max(amax, red);
-            const float scale = __fdiv_rn(amax, 127.0f), inv = quant_inv(scale);
-            if (threadIdx.x == 0) recv_scale[p] = scale;
-#pragma unroll
-            for (int i = 0; i < kChunks; i++) {
-                const int64_t c = threadIdx.x + (int64_t)i * blockDim.x;
-                if (c < H8) recv[(int64_t)p * H8 + c] = q8x8(xs[i], scale, inv);
-            }
-            __syncthreads();                               // red is reused by the next slot
-        }
-    }
-}
-
-// The same codes with the K slots of a token taken together (K fixed at KC): pass 1
-// forms, slot by slot, each thread's maximum of |fl(x * smooth[e_k])| and its warp
+// Smooth-quantised int8 dispatch, the K slots of a token taken together (any K up to
+// kMaxK), one CTA of 256 threads per token, the token's row in registers: pass 1 forms, slot by slot, each thread's maximum of |fl(x * smooth[e_k])| and its warp
 // maximum (every smoothing row read once; the warp maximum by redux.sync); one block
 // barrier later the K scales follow from the warps' maxima; pass 2 forms each product
 // again (the smoothing rows a second time, from L2) and stores the codes. Two block
@@ -1075,25 +958,25 @@ k_dispatch_int8_smooth(const uint4 *__restrict__ x, const int32_t *__restrict__ 
 // its codes are then 8, 16 and 4 consecutive bytes, so every warp load and store of the
 // three is one contiguous span (the smoothing rows, read K times per token, are the
 // bulk of the traffic through L1).
-template <int KC, int kGroups>
+template <int kGroups>
 __global__ void __launch_bounds__(256)
 k_dispatch_int8_smooth_k(const uint2 *__restrict__ x, const int32_t *__restrict__ ids, const int32_t *__restrict__ pos,
-                         int64_t T, int64_t H4, const float4 *__restrict__ smooth, int32_t n_experts, int64_t rows,
+                         int64_t T, int K, int64_t H4, const float4 *__restrict__ smooth, int32_t n_experts, int64_t rows,
                          uint32_t *__restrict__ recv, float *__restrict__ recv_scale)
 {
-    __shared__ int32_t sp[KC], se[KC];
-    __shared__ float red[8][KC];                      // 256 threads = 8 warps
-    __shared__ float ssc[KC];
+    __shared__ int32_t sp[kMaxK], se[kMaxK];
+    __shared__ float red[8][kMaxK];                   // 256 threads = 8 warps
+    __shared__ float ssc[kMaxK];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h4 = (int)H4;                           // at most 256 * kGroups
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-        if (threadIdx.x < KC) {
-            int32_t p = pos[t * KC + threadIdx.x];
+        if (threadIdx.x < K) {
+            int32_t p = pos[t * K + threadIdx.x];
             if (p < -1 || (int64_t)p >= rows) {
                 flag_error(MEP_DERR_ROW_RANGE);
                 p = -1;
             }
-            int32_t e = ids[t * KC + threadIdx.x];
+            int32_t e = ids[t * K + threadIdx.x];
             if (e < 0 || e >= n_experts) {
                 flag_error(MEP_DERR_KEY_RANGE);
                 e = -1;
@@ -1116,7 +999,7 @@ k_dispatch_int8_smooth_k(const uint2 *__restrict__ x, const int32_t *__restrict_
         }
         __syncthreads();
 #pragma unroll 1
-        for (int k = 0; k < KC; k++) {
+        for (int k = 0; k < K; k++) {
             float amax = 0.0f;
             const int32_t e = se[k];
             if (sp[k] >= 0 && e >= 0) {
@@ -1138,7 +1021,7 @@ k_dispatch_int8_smooth_k(const uint2 *__restrict__ x, const int32_t *__restrict_
             if (lane == 0) red[warp][k] = amax;
         }
         __syncthreads();
-        if (threadIdx.x < KC) {
+        if (threadIdx.x < K) {
             float m = 0.0f;
             for (int w = 0; w < 8; w++) m = fmaxf(m, red[w][threadIdx.x]);
             const float scale = __fdiv_rn(m, 127.0f);
@@ -1147,7 +1030,7 @@ k_dispatch_int8_smooth_k(const uint2 *__restrict__ x, const int32_t *__restrict_
         }
         __syncthreads();
 #pragma unroll 1
-        for (int k = 0; k < KC; k++) {                    // one slot at a time: a short loop body
+        for (int k = 0; k < K; k++) {                     // one slot at a time: a short loop body
             const int32_t p = sp[k], e = se[k];
             if (p < 0 || e < 0) continue;
             const float scale = ssc[k], inv = quant_inv(scale);

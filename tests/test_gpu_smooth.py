@@ -1,8 +1,7 @@
 """GPU parity of the int8 dispatch with per-expert smoothing scales against the oracle
-(codes and scales bit for bit). K in {2, 4, 8} with H % 4 == 0 (up to 64 columns per
-thread, in groups of 4) takes the fused kernel (all K slots of a token in one CTA, two
-passes), other K the per-slot kernel (H % 8 == 0), other H or alignments the scalar
-kernel. The full int8 workload is compared
+(codes and scales bit for bit). H % 4 == 0 (up to 64 columns per thread, in groups of 4)
+takes the fused kernel (all K slots of a token in one CTA, two passes, any K), other H or
+alignments the scalar kernel. The full int8 workload is compared
 whole, one rank partition at a time, and with all-ones scales against the plain
 per-token int8 dispatch."""
 from concurrent.futures import ThreadPoolExecutor
@@ -179,8 +178,8 @@ def test_quantiser_at_and_next_to_half_integer_quotients(amax, K):
                 v = np.nextafter(v, np.float32(np.inf if j > 0 else -np.inf), dtype=np.float32)
             if abs(v) <= np.float32(amax):
                 vals.append(v)
-    # K = 1: the per-slot kernel; K = 2: the fused kernel, the second slot on a second
-    # expert holding the values reversed
+    # K = 1: one slot; K = 2: the second slot on a second expert holding the values
+    # reversed
     H = (len(vals) + 7) // 8 * 8
     sm = np.zeros((K, H), np.float32)
     sm[0, :len(vals)] = vals
