@@ -80,6 +80,7 @@ struct DeviceState {
     std::atomic<bool> ready{false};
     std::atomic<unsigned long long> ctx_id{0};
     int sm_count = 148;
+    bool cluster_plan = false;        // k_plan_cluster's cluster fits on the device
     void *plan_static_ws = nullptr;   // device address of g_plan_static_ws in ctx_id
 };
 DeviceState g_dev[kMaxDevices];
@@ -115,6 +116,24 @@ DeviceState &device_state(int dev)
     cudaFuncSetAttribute(mep::k_plan_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     cudaFuncSetAttribute(mep::k_source_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     cudaFuncSetAttribute(mep::k_plan_small, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallPlanSmemMax);
+    cudaFuncSetAttribute(mep::k_plan_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallPlanSmemMax);
+    {
+        // a cluster of CTAs with the largest shared memory the plan asks for
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(mep::kPlanClusterCTAs);
+        cfg.blockDim = dim3(mep::kSmallPlanThreads);
+        cfg.dynamicSmemBytes = kSmallPlanSmemMax;
+        cudaLaunchAttribute attr = {};
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = mep::kPlanClusterCTAs;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        st.cluster_plan = cudaOccupancyMaxActiveClusters(&clusters, mep::k_plan_cluster, &cfg) == cudaSuccess &&
+                          clusters >= 1;
+    }
     cudaFuncSetAttribute(mep::k_dispatch_int8_staged<4, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kBulkSmemMax);
     const int norm_smem = (int)(sizeof(float) * MEP_RMSNORM_MAX_H);
@@ -141,6 +160,14 @@ int sm_count()
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
     return device_state(dev).sm_count;
+}
+
+// Whether the current device can run k_plan_cluster's cluster.
+bool cluster_plan_ok()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+    return device_state(dev).cluster_plan;
 }
 
 mep_status_t launched()
@@ -347,7 +374,15 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
 
     cudaStream_t s = (cudaStream_t)stream;
     sm_count();
-    // small problems: the whole plan in one CTA (one launch instead of four)
+    // small problems: the whole plan in one launch instead of four, over a cluster of
+    // CTAs when it fits, else in one CTA
+    const size_t cluster_smem = sizeof(int32_t) * (size_t)(36 * (int64_t)n_keys + 34);
+    if (N <= mep::kClusterPlanMaxSlots && cluster_smem <= (size_t)kSmallPlanSmemMax && cluster_plan_ok()) {
+        mep::k_plan_cluster<<<mep::kPlanClusterCTAs, mep::kSmallPlanThreads, cluster_smem, s>>>(
+            ids, keep, N, n_keys, R, (int64_t)S * K, mode, keys_per_rank, pos, hist, rank_off, load, rep_count,
+            rep_key, rep_cu, (int32_t *)stats);
+        return launched();
+    }
     if (plan_is_small(N, n_keys)) {
         const size_t small_smem = sizeof(int32_t) * (size_t)(34 * (int64_t)n_keys + 34);
         mep::k_plan_small<<<1, mep::kSmallPlanThreads, small_smem, s>>>(ids, keep, N, n_keys, R, (int64_t)S * K, mode,

@@ -16,6 +16,8 @@
 // needs it.
 #pragma once
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 namespace mep {
@@ -475,6 +477,113 @@ k_plan_small(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, 
     }
     __syncthreads();
     plan_meta(tot, R, n_keys, SK, mode, keys_per_rank, rank_off_out, load_out, rep_count, rep_key, rep_cu, stats,
+              smem);
+}
+
+// The whole plan in one cluster of kPlanClusterCTAs CTAs of 1024 threads, for small
+// problems: k_plan_small's steps with the slots split over the cluster's CTAs (CTA c
+// takes the c-th eighth of the slots, in order), so each warp walks at most
+// kClusterPlanPerLane rounds instead of kSmallPlanPerLane. Each CTA counts its slots per
+// warp and key; after a cluster barrier every CTA reads the others' per-key totals
+// through distributed shared memory, forms hist and the totals of the CTAs before it,
+// and ranks its slots from there. CTA 0 then writes the replica tables (plan_meta).
+// Dynamic shared memory: cnt [32][n_keys], key_off [n_keys + 1], scratch [33], and
+// three [n_keys] arrays: this CTA's totals, hist, the earlier CTAs' totals.
+constexpr int kPlanClusterCTAs = 8;
+constexpr int kClusterPlanPerLane = 2;
+constexpr int64_t kClusterPlanMaxSlots = (int64_t)kPlanClusterCTAs * kSmallPlanThreads * kClusterPlanPerLane;
+
+__global__ void __cluster_dims__(kPlanClusterCTAs, 1, 1) __launch_bounds__(kSmallPlanThreads)
+k_plan_cluster(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, int64_t N, int32_t n_keys,
+               int32_t R, int64_t SK, int32_t mode, int32_t keys_per_rank, int32_t *__restrict__ pos,
+               int32_t *__restrict__ hist, int32_t *__restrict__ rank_off_out, int32_t *__restrict__ load_out,
+               int32_t *__restrict__ rep_count, int32_t *__restrict__ rep_key, int32_t *__restrict__ rep_cu,
+               int32_t *__restrict__ stats)
+{
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int crank = (int)cluster.block_rank();
+    extern __shared__ int32_t smem[];
+    constexpr int kWarps = kSmallPlanThreads / 32;
+    int32_t *cnt = smem;                              // [kWarps][n_keys]
+    int32_t *key_off = cnt + kWarps * n_keys;         // n_keys + 1
+    int32_t *scan_scratch = key_off + n_keys + 1;     // 33
+    int32_t *ctot = scan_scratch + 33;                // n_keys: this CTA's slots per key
+    int32_t *all = ctot + n_keys;                     // n_keys: hist (every CTA's slots)
+    int32_t *pre = all + n_keys;                      // n_keys: the slots of the CTAs before this one
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < kWarps * n_keys; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+    const int64_t per_cta = ((N + kPlanClusterCTAs - 1) / kPlanClusterCTAs + 31) / 32 * 32;
+    const int64_t c_lo = min(N, (int64_t)crank * per_cta), c_hi = min(N, c_lo + per_cta);
+    const int64_t sub = ((per_cta + kWarps - 1) / kWarps + 31) / 32 * 32;   // <= 32 * kClusterPlanPerLane
+    const int64_t lo = min(c_hi, c_lo + (int64_t)warp * sub), hi = min(c_hi, lo + sub);
+    int32_t *mine = cnt + warp * n_keys;
+    int32_t key[kClusterPlanPerLane];
+#pragma unroll
+    for (int j = 0; j < kClusterPlanPerLane; j++) {
+        const int64_t n = lo + 32 * j + lane;
+        int32_t e = n < hi ? ids[n] : -1;
+        if (n < hi && keep && !keep[n]) e = -1;
+        else if (n < hi && (e < 0 || e >= n_keys)) {
+            flag_error(MEP_DERR_KEY_RANGE);
+            e = -1;
+        }
+        key[j] = e;
+    }
+#pragma unroll
+    for (int j = 0; j < kClusterPlanPerLane; j++) {
+        if (lo + 32 * j >= hi) break;                 // uniform over the warp
+        const uint32_t peers = __match_any_sync(0xffffffffu, key[j]);
+        if (key[j] >= 0 && lane == __ffs(peers) - 1) mine[key[j]] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    // per key: exclusive prefix over warps (in place) and this CTA's total
+    for (int e = threadIdx.x; e < n_keys; e += blockDim.x) {
+        int32_t run = 0;
+        for (int w = 0; w < kWarps; w++) {
+            const int32_t v = cnt[w * n_keys + e];
+            cnt[w * n_keys + e] = run;
+            run += v;
+        }
+        ctot[e] = run;
+    }
+    cluster.sync();                                   // every CTA's totals are complete
+    for (int e = threadIdx.x; e < n_keys; e += blockDim.x) {
+        int32_t a = 0, b = 0;
+        for (int c = 0; c < kPlanClusterCTAs; c++) {
+            const int32_t v = cluster.map_shared_rank(ctot, c)[e];
+            a += v;
+            if (c < crank) b += v;
+        }
+        all[e] = a;
+        pre[e] = b;
+        if (crank == 0) hist[e] = a;
+    }
+    __syncthreads();
+    block_exclusive_scan(all, n_keys, key_off, scan_scratch);
+    for (int e = threadIdx.x; e < n_keys; e += blockDim.x) {
+        const int32_t b = key_off[e] + pre[e];
+        for (int w = 0; w < kWarps; w++) cnt[w * n_keys + e] += b;
+    }
+    __syncthreads();
+    const uint32_t lt = lanemask_lt();
+#pragma unroll
+    for (int j = 0; j < kClusterPlanPerLane; j++) {
+        if (lo + 32 * j >= hi) break;
+        const int64_t n = lo + 32 * j + lane;
+        const uint32_t peers = __match_any_sync(0xffffffffu, key[j]);
+        int32_t p = -1;
+        if (key[j] >= 0) p = mine[key[j]] + __popc(peers & lt);
+        __syncwarp();
+        if (key[j] >= 0 && lane == __ffs(peers) - 1) mine[key[j]] += __popc(peers);
+        __syncwarp();
+        if (n < hi) pos[n] = p;
+    }
+    cluster.sync();                                   // no CTA reads another's totals past here
+    if (crank != 0) return;
+    plan_meta(all, R, n_keys, SK, mode, keys_per_rank, rank_off_out, load_out, rep_count, rep_key, rep_cu, stats,
               smem);
 }
 

@@ -32,15 +32,20 @@ def test_histogram_parity_ragged_and_skewed():
     assert mep.mep_get_error() == 0
 
 
-# Plans of at most 16384 slots with few enough keys run as one CTA, the others as the
-# tiled four-kernel sort (tiles of 512, 1024 or 2048 slots by size): the cases cover each
-# path, at and just past the boundaries (ragged last tiles), and small plans whose keys
-# are too many for the one-CTA path.
+# Plans of at most 16384 slots run in one launch: over a cluster of 8 CTAs when at most
+# 1421 keys fit its shared memory, else in one CTA (up to 1504 keys); the others as the
+# tiled four-kernel sort (tiles of 512, 1024 or 2048 slots by size). The cases cover each
+# path, at and just past the boundaries (ragged last tiles and CTA shares), and small
+# plans whose keys are too many for either one-launch path.
 @pytest.mark.parametrize("R,E,S,K", [
     (2, 4, 2, 2), (3, 9, 37, 3), (4, 12, 1000, 3), (4, 16, 128, 2), (8, 64, 300, 8),
     (1, 5, 17, 1), (16, 4096, 32, 4), (8, 4096, 512, 8), (5, 5, 2048, 1),
     (4, 16, 1024, 4), (7, 7, 2340, 1), (2, 1024, 4096, 2), (3, 9, 1821, 3), (1, 2, 16385, 1),
     (64, 1536, 8, 8),
+    # the cluster at its key limit, the one-CTA plan past it, both at 16384 slots
+    (8, 1416, 256, 8), (8, 1480, 256, 8), (4, 1420, 1024, 4),
+    # CTA shares that end inside a warp's range, and CTAs left without slots
+    (1, 3, 8191, 2), (1, 3, 33, 1), (3, 6, 5, 7),
     # ragged last tiles of the 1024- and 2048-slot tiles (more than 2^18 and 2^20 slots)
     (7, 7, 37454, 1), (5, 10, 209916, 1),
 ])
