@@ -474,9 +474,9 @@ mep_status_t mep_update_expert(const int32_t *expert_ids, const int32_t *eplb_ta
     if (balance_mode == 0 && (world_size < 2 || world_size > 768)) return MEP_ERR_VALUE;
     if (balance_mode == 0 && (local_rank_id < 0 || local_rank_id >= world_size)) return MEP_ERR_VALUE;
     cudaStream_t s = (cudaStream_t)stream;
-    const int threads = 128;
-    int64_t g = (BS + threads - 1) / threads;
-    int cap = sm_count() * 4;
+    const int threads = 256;
+    int64_t g = (BS * K + threads - 1) / threads;
+    int cap = sm_count() * 8;
     mep::k_update_expert<<<(unsigned)(g < cap ? g : cap), threads, 0, s>>>(
         expert_ids, eplb_table, expert_scales, pruning_threshold, active_mask, BS, BS, local_rank_id, K,
         n_experts, F, world_size, balance_mode, balanced_expert_ids, balanced_active_mask);
@@ -501,10 +501,10 @@ mep_status_t mep_update_expert_ranks(const int32_t *expert_ids, const int32_t *e
     if (balance_mode == 0 && (world_size < 2 || world_size > 768)) return MEP_ERR_VALUE;
     if (BS * world_size * K >= ((int64_t)1 << 31)) return MEP_ERR_SHAPE;
     cudaStream_t s = (cudaStream_t)stream;
-    const int threads = 128;
+    const int threads = 256;
     const int64_t rows = BS * world_size;
-    int64_t g = (rows + threads - 1) / threads;
-    int cap = sm_count() * 4;
+    int64_t g = (rows * K + threads - 1) / threads;
+    int cap = sm_count() * 8;
     mep::k_update_expert<<<(unsigned)(g < cap ? g : cap), threads, 0, s>>>(
         expert_ids, eplb_table, expert_scales, pruning_threshold, active_mask, rows, BS, 0, K, n_experts, F,
         world_size, balance_mode, balanced_expert_ids, balanced_active_mask);

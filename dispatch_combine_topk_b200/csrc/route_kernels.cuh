@@ -15,9 +15,11 @@ constexpr int kMaxK = 32;
 
 // ------------------------------------------------------------------ mapping (a3)
 
-// One thread per token. Mapping of aclnnMoeUpdateExpert (gitcode ops-transformer doc,
-// 功能说明): instance column 1 for a single instance; otherwise local_rank_id /
-// ceil(world_size / count) + 1 (by rank) or (token mod count) + 1 (by token).
+// One thread per slot (token g, slot k): the three loads that depend on one another
+// (the id, the table row's count, the instance) are the only chain a thread waits on.
+// Mapping of aclnnMoeUpdateExpert (gitcode ops-transformer doc, 功能说明): instance
+// column 1 for a single instance; otherwise local_rank_id / ceil(world_size / count) + 1
+// (by rank) or (token mod count) + 1 (by token).
 // Pruning: v = sum_k fl(scale[k] * thr[k]) in fp32, ascending k, no FMA; a slot stays
 // active iff the token is active and !(scale[k] < v).
 // Rows are blocks of rows_per_rank tokens: row g belongs to rank rank0 + g / rows_per_rank
@@ -29,44 +31,45 @@ __global__ void k_update_expert(const int32_t *__restrict__ ids, const int32_t *
                                 int64_t mode, int32_t *__restrict__ out_ids,
                                 uint8_t *__restrict__ out_mask)
 {
-    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < rows;
-         g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t slots = rows * K;
+    for (int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; n < slots;
+         n += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t g = n / K;
+        const int32_t k = (int32_t)(n - g * K);
         const int64_t i = g % rows_per_rank;
         const int64_t local_rank = rank0 + g / rows_per_rank;
         uint8_t act = 1;
         if (active) {
             act = active[g] ? 1 : 0;
-            if (i > 0 && act && !active[g - 1]) flag_error(MEP_DERR_MASK);
+            if (k == 0 && i > 0 && act && !active[g - 1]) flag_error(MEP_DERR_MASK);
         }
-        for (int32_t k = 0; k < K; k++) {
-            const int32_t e = ids[g * K + k];
-            int32_t inst = -1;
-            if (e < 0 || e >= E) {
-                flag_error(MEP_DERR_KEY_RANGE);
-            } else {
-                const int32_t *row = table + (int64_t)e * F;
-                const int32_t c = row[0];
-                if (c < 1 || c > F - 1) {
-                    flag_error(MEP_DERR_TABLE);
-                } else {
-                    int64_t col;
-                    if (c == 1) col = 1;
-                    else if (mode == 0) col = local_rank / ((world_size + c - 1) / c) + 1;
-                    else col = (i % c) + 1;
-                    const int32_t v = row[col];   // col <= c <= F-1: inside the row
-                    if (v < 0 || v >= 1024) flag_error(MEP_DERR_TABLE);
-                    else inst = v;
-                }
-            }
-            out_ids[g * K + k] = inst;
-        }
-        if (scales) {
-            float v = 0.0f;
-            for (int32_t k = 0; k < K; k++) v = __fadd_rn(v, __fmul_rn(scales[g * K + k], thr[k]));
-            for (int32_t k = 0; k < K; k++)
-                out_mask[g * K + k] = (act && !(scales[g * K + k] < v)) ? 1 : 0;
+        const int32_t e = ids[n];
+        int32_t inst = -1;
+        if (e < 0 || e >= E) {
+            flag_error(MEP_DERR_KEY_RANGE);
         } else {
-            for (int32_t k = 0; k < K; k++) out_mask[g * K + k] = act;
+            const int32_t *row = table + (int64_t)e * F;
+            const int32_t c = row[0];
+            if (c < 1 || c > F - 1) {
+                flag_error(MEP_DERR_TABLE);
+            } else {
+                int64_t col;
+                if (c == 1) col = 1;
+                else if (mode == 0) col = local_rank / ((world_size + c - 1) / c) + 1;
+                else col = (i % c) + 1;
+                const int32_t v = row[col];   // col <= c <= F-1: inside the row
+                if (v < 0 || v >= 1024) flag_error(MEP_DERR_TABLE);
+                else inst = v;
+            }
+        }
+        out_ids[n] = inst;
+        if (scales) {
+            // the token's sum, formed alike by each of its K threads
+            float v = 0.0f;
+            for (int32_t j = 0; j < K; j++) v = __fadd_rn(v, __fmul_rn(scales[g * K + j], thr[j]));
+            out_mask[n] = (act && !(scales[n] < v)) ? 1 : 0;
+        } else {
+            out_mask[n] = act;
         }
     }
 }
