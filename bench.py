@@ -671,6 +671,56 @@ def e2e_route_host(mep, rt, w, dev, steps, pg):
                               "on three streams in turn")
 
 
+def link_rates(dev, nbytes: int = 1 << 30, reps: int = 5) -> dict:
+    """This box's pinned host<->device copy rates in GB/s: upload alone, download alone,
+    and each direction while both run on two streams (the end-to-end leg's bound)."""
+    h_in = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    h_out = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d_a = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    d_b = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    cur = torch.cuda.current_stream(dev)
+
+    def up():
+        s_up.wait_stream(cur)
+        with torch.cuda.stream(s_up):
+            d_a.copy_(h_in, non_blocking=True)
+        cur.wait_stream(s_up)
+
+    def down():
+        s_down.wait_stream(cur)
+        with torch.cuda.stream(s_down):
+            h_out.copy_(d_b, non_blocking=True)
+        cur.wait_stream(s_down)
+
+    def both():
+        s_up.wait_stream(cur)
+        s_down.wait_stream(cur)
+        with torch.cuda.stream(s_up):
+            d_a.copy_(h_in, non_blocking=True)
+        with torch.cuda.stream(s_down):
+            h_out.copy_(d_b, non_blocking=True)
+        cur.wait_stream(s_up)
+        cur.wait_stream(s_down)
+
+    def gbs(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        for _ in range(reps):
+            fn()
+        e1.record(cur)
+        torch.cuda.synchronize(dev)
+        return nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9
+
+    out = {"h2d_gbs": gbs(up), "d2h_gbs": gbs(down), "duplex_gbs_each": gbs(both), "bytes": nbytes}
+    del h_in, h_out, d_a, d_b
+    torch.cuda.empty_cache()
+    return out
+
+
 def e2e_pipeline(rt, w, dev, stream, steps, pg):
     """End to end through the binding's calls for the steps mep_route_host does not cover
     (the mapping workload, the fused epilogue, the deduplicated dispatch): every step
@@ -911,6 +961,12 @@ def run_gpu(args, w):
     else:
         e2e_ms, ok_e2e, h2d, d2h, how = e2e_pipeline(rt, w, dev, stream, e2e_steps, pg)
     torch.cuda.empty_cache()
+    link = None
+    if e2e_ms is not None:
+        # the copies alone bound the end-to-end step: the larger direction at the duplex rate
+        link = link_rates(dev)
+        link["bound_ms"] = max(h2d, d2h) / (link["duplex_gbs_each"] * 1e9) * 1e3
+        link["frac"] = link["bound_ms"] / e2e_ms
 
     line = None
     peak, peak_kind = load_peaks()
@@ -946,7 +1002,7 @@ def run_gpu(args, w):
             "cpu_baseline": cpu,
             "e2e": None if e2e_ms is None else {
                 "value": world * w.N / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "path": how},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "path": how, "link": link},
             "result_check": {"device": ok_device, "e2e": ok_e2e},
             "gpu_launches": tm["launches"],
             "clocks": tm["clocks"],
