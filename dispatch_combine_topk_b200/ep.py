@@ -11,8 +11,15 @@ its rows and its exchange counts on its own GPU (``mep_plan_rank``); all ranks s
 same gathered matrix, so their shares form exactly the plan of ``mep_plan`` over the
 ids of all ranks.
 
-This module is plumbing only (the histogram and the plan run in the library's
-kernels); its collectives go through ``torch.distributed`` (NCCL between GPUs).
+The exchange itself is one kernel per direction: every rank dispatches its own token
+rows straight into the receive buffers of all ranks (peer stores through a table of their
+addresses, ``mep_dispatch_ranks``), and combines its tokens by reading the expert outputs
+from all ranks' buffers (``mep_combine_ranks``). ``Exchange`` holds one rank's side:
+its buffer, shared with the group through CUDA IPC, and the address tables. The ranks
+meet only in host barriers between the phases; no kernel waits on another process.
+
+This module is plumbing only (the histogram, the plan and the exchange run in the
+library's kernels); its collectives go through ``torch.distributed`` (NCCL between GPUs).
 """
 from __future__ import annotations
 
@@ -96,3 +103,78 @@ def plan_rank(ids: torch.Tensor, E: int, S: int, K: int, group=None, stream=None
     else:
         hist_all = gather_histograms(hist, group)
     return plan(ids, hist_all, R, E, S, K, rank, out), hist_all
+
+
+class Exchange:
+    """One EP rank's side of the token exchange over a process group of R ranks, each
+    holding S tokens of K slots and an [S*K, H] receive buffer (bf16, or int8 codes with
+    fp32 scales for ``quant=1``).
+
+    Construction is collective: every rank allocates its buffer and maps every other
+    rank's (``share_buffers``). Per step:
+
+    - ``plan(ids)``: this rank's rows in the global plan (``plan_rank``);
+    - ``dispatch(x, rp)``: its token rows into every rank's buffer (peer stores);
+    - ``fence()``: waits for this rank's stream, then for every rank (host barrier), so
+      that the rows written by all ranks are in place before anyone reads them; call it
+      after ``dispatch``, after the experts have written their outputs into ``rows``,
+      and after ``combine`` before the next ``dispatch`` overwrites the buffers;
+    - ``combine(rp, gates, out)``: its tokens' gate-weighted sum read from every rank's
+      buffer.
+
+    ``close()`` (collective) ends the sharing: no rank frees its buffer while another
+    may still read it."""
+
+    def __init__(self, E: int, S: int, K: int, H: int, quant: int = 0, group=None, device=None, stream=None):
+        import dispatch_combine_topk_b200 as mep
+        self._mep = mep
+        self.group = group
+        self.R = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.E, self.S, self.K, self.H, self.quant = E, S, K, H, quant
+        self.rows_per_rank = S * K
+        self.device = device or torch.device("cuda", torch.cuda.current_device())
+        self.stream = stream
+        dt = torch.int8 if quant else torch.bfloat16
+        self.rows = torch.zeros((self.rows_per_rank, H), dtype=dt, device=self.device)
+        mine = {"rows": self.rows}
+        self.scale = None
+        if quant:
+            self.scale = torch.zeros(self.rows_per_rank, dtype=torch.float32, device=self.device)
+            mine["scale"] = self.scale
+        torch.cuda.synchronize(self.device)              # the buffers exist before they are shared
+        self._every = share_buffers(mine, group)
+        self.table = mep.rank_pointer_table([b["rows"] for b in self._every], self.device)
+        self.scale_table = (mep.rank_pointer_table([b["scale"] for b in self._every], self.device)
+                            if quant else None)
+
+    def plan(self, ids: torch.Tensor, out=None):
+        """This rank's rows in the global plan and its exchange counts (``plan_rank``).
+        Returns ``(RankPlanBuffers, hist_all)``."""
+        return plan_rank(ids, self.E, self.S, self.K, self.group, stream=self.stream, out=out)
+
+    def dispatch(self, x: torch.Tensor, rp) -> None:
+        """This rank's token rows x [S, H] into every rank's buffer, at the rows ``rp.pos``."""
+        self._mep.mep_dispatch_ranks(x, rp.pos, self.K, self.table, self.rows_per_rank, quant=self.quant,
+                                     scale_table=self.scale_table, stream=self.stream)
+
+    def fence(self) -> None:
+        """This rank's work on its stream done, then every rank's (host barrier)."""
+        if self.stream is not None:
+            self.stream.synchronize()
+        else:
+            torch.cuda.synchronize(self.device)
+        dist.barrier(group=self.group)
+
+    def combine(self, rp, gates: torch.Tensor, out: torch.Tensor) -> torch.Tensor:
+        """out [S, H] (bf16) = the gate-weighted sum of this rank's slots, read from the
+        buffers of the ranks they went to."""
+        self._mep.mep_combine_ranks(self.table, rp.pos, gates, self.K, self.rows_per_rank, out, quant=self.quant,
+                                    scale_table=self.scale_table, stream=self.stream)
+        return out
+
+    def close(self) -> None:
+        """Collective: every rank stops reading the others' buffers, then drops them."""
+        self.fence()
+        self._every = None
+        self.table = self.scale_table = None

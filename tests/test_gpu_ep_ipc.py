@@ -1,14 +1,14 @@
 """The expert-parallel exchange between processes: two processes, each one EP rank with
-its own tokens and its own receive buffer, on one GPU.
+its own tokens and its own receive buffer, on one GPU, through ep.Exchange.
 
-Each rank plans its own slots (ep.plan_rank: its histogram, the all-gather of the
-histograms over a gloo group, mep_plan_rank), maps the other rank's receive buffer into
-its process through CUDA IPC (ep.share_buffers), and dispatches its own token rows
-straight into both ranks' buffers through the table of their addresses
-(mep_dispatch_ranks). After a barrier every rank's buffer must equal the oracle's
-dispatch restricted to that rank's partition of the global plan, bit for bit, and each
-rank's combine over both buffers (mep_combine_ranks) must equal the oracle's combine of
-its tokens. No kernel waits on the other process: the processes meet only in host
+Each rank plans its own slots (its histogram, the all-gather of the histograms over a
+gloo group, mep_plan_rank), maps the other rank's receive buffer into its process
+through CUDA IPC, and dispatches its own token rows straight into both ranks' buffers
+through the table of their addresses (mep_dispatch_ranks). After a fence every rank's
+buffer must equal the oracle's dispatch restricted to that rank's partition of the
+global plan, bit for bit, and each rank's combine over both buffers (mep_combine_ranks)
+must equal the oracle's combine of its tokens. Two steps with different routings reuse
+the buffers. No kernel waits on the other process: the processes meet only in host
 barriers, with time limits."""
 import datetime
 import os
@@ -40,52 +40,51 @@ def _rank_main(rank, world, port, quant, q):
         torch.cuda.set_device(0)
         dev = torch.device("cuda", 0)
         w = synth.scaled(synth.get("tiny"), R=world, E=8 * world, S=384, K=4, H=512)
-        ids_all, gates_all = synth.router(w)                 # the whole batch, to check against
-        x_all = synth.hidden(w)
         SK = w.S * w.K
-        ids = torch.from_numpy(ids_all.reshape(world, SK)[rank].copy()).to(dev)
-        rp, hist_all = ep.plan_rank(ids, w.E, w.S, w.K)
-        # this rank's receive buffer, shared with the other ranks
-        dt = torch.int8 if quant else torch.bfloat16
-        mine = {"rows": torch.full((SK, w.H), 0x33 if quant else 0, dtype=dt, device=dev)}
-        if quant:
-            mine["scale"] = torch.zeros(SK, dtype=torch.float32, device=dev)
-        torch.cuda.synchronize()
-        every = ep.share_buffers(mine, None)
-        table = mep.rank_pointer_table([b["rows"] for b in every], dev)
-        stable = mep.rank_pointer_table([b["scale"] for b in every], dev) if quant else None
-        x = x_all[rank * w.S:(rank + 1) * w.S].to(dev)
-        mep.mep_dispatch_ranks(x, rp.pos, w.K, table, SK, quant=quant, scale_table=stable)
-        torch.cuda.synchronize()
-        dist.barrier()                                       # every rank's rows are in place
-        p = oracle.plan_balanced(ids_all, world, w.E, w.S, w.K)
-        assert np.array_equal(rp.pos.cpu().numpy(), p.pos[rank * SK:(rank + 1) * SK]), "rows of this rank's slots"
-        xb = bits(x_all)
-        inside = (p.pos >= rank * SK) & (p.pos < (rank + 1) * SK)
-        toks = np.unique(np.flatnonzero(inside) // w.K)
-        pos_r = np.where(inside, p.pos - rank * SK, -1).astype(np.int32).reshape(-1, w.K)[toks]
-        if quant:
-            q_ref, s_ref = oracle.dispatch_int8(xb[toks], pos_r, w.K, SK)
-            assert np.array_equal(mine["rows"].cpu().numpy(), q_ref), "codes in this rank's buffer"
-            assert np.array_equal(mine["scale"].cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
-        else:
-            assert np.array_equal(bits(mine["rows"]), oracle.dispatch(xb[toks], pos_r, w.K, SK)), "rows"
-        # the identity expert: combine this rank's tokens from both buffers
-        gates = torch.from_numpy(gates_all.reshape(world, SK)[rank].copy()).to(dev)
-        out = torch.empty((w.S, w.H), dtype=torch.bfloat16, device=dev)
-        mep.mep_combine_ranks(table, rp.pos, gates, w.K, SK, out, quant=quant, scale_table=stable)
-        torch.cuda.synchronize()
-        pos_l = np.arange(SK, dtype=np.int32)
-        xr = xb[rank * w.S:(rank + 1) * w.S]
-        g = gates_all.reshape(world, SK)[rank]
-        if quant:
-            qq, ss = oracle.dispatch_int8(xr, pos_l, w.K, SK)
-            ref = oracle.combine_int8(qq, ss, pos_l, g, w.K)
-        else:
-            ref = oracle.combine(oracle.dispatch(xr, pos_l, w.K, SK), pos_l, g, w.K)
-        assert np.array_equal(bits(out), ref), "combine"
+        ex = ep.Exchange(w.E, w.S, w.K, w.H, quant=quant, device=dev)
+        xb_all = None
+        for step in range(2):
+            ids_all, gates_all = synth.router(w)             # the whole batch, to check against
+            if step == 1:                                    # another routing on the same buffers
+                ids_all = np.ascontiguousarray(np.roll(ids_all.reshape(-1, w.K), 1, axis=1).reshape(ids_all.shape))
+                ids_all = ((ids_all + 3) % w.E).astype(np.int32)
+            x_all = synth.hidden(w)
+            xb_all = bits(x_all)
+            ids = torch.from_numpy(ids_all.reshape(world, SK)[rank].copy()).to(dev)
+            rp, hist_all = ex.plan(ids)
+            x = x_all[rank * w.S:(rank + 1) * w.S].to(dev)
+            ex.dispatch(x, rp)
+            ex.fence()                                       # every rank's rows are in place
+            p = oracle.plan_balanced(ids_all, world, w.E, w.S, w.K)
+            assert np.array_equal(rp.pos.cpu().numpy(), p.pos[rank * SK:(rank + 1) * SK]), "rows of this rank's slots"
+            inside = (p.pos >= rank * SK) & (p.pos < (rank + 1) * SK)
+            toks = np.unique(np.flatnonzero(inside) // w.K)
+            pos_r = np.where(inside, p.pos - rank * SK, -1).astype(np.int32).reshape(-1, w.K)[toks]
+            if quant:
+                q_ref, s_ref = oracle.dispatch_int8(xb_all[toks], pos_r, w.K, SK)
+                assert np.array_equal(ex.rows.cpu().numpy(), q_ref), "codes in this rank's buffer"
+                assert np.array_equal(ex.scale.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+            else:
+                assert np.array_equal(bits(ex.rows), oracle.dispatch(xb_all[toks], pos_r, w.K, SK)), "rows"
+            # the identity expert leaves the rows as they are; every rank's outputs are final
+            ex.fence()
+            gates = torch.from_numpy(gates_all.reshape(world, SK)[rank].copy()).to(dev)
+            out = torch.empty((w.S, w.H), dtype=torch.bfloat16, device=dev)
+            ex.combine(rp, gates, out)
+            torch.cuda.synchronize()
+            pos_l = np.arange(SK, dtype=np.int32)
+            xr = xb_all[rank * w.S:(rank + 1) * w.S]
+            g = gates_all.reshape(world, SK)[rank]
+            if quant:
+                qq, ss = oracle.dispatch_int8(xr, pos_l, w.K, SK)
+                ref = oracle.combine_int8(qq, ss, pos_l, g, w.K)
+            else:
+                ref = oracle.combine(oracle.dispatch(xr, pos_l, w.K, SK), pos_l, g, w.K)
+            assert np.array_equal(bits(out), ref), f"combine, step {step}"
+            assert hist_all.shape == (world, w.E)
+            ex.fence()                                       # nobody reads a buffer the next step writes
         assert mep.mep_get_error() == 0
-        assert hist_all.shape == (world, w.E)
+        ex.close()
         result["ok"] = True
     except Exception as e:                                   # reported to the parent
         result["error"] = repr(e)
