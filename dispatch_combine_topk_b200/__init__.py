@@ -189,7 +189,7 @@ def mep_plan_workspace_size(R: int, n_keys: int, S: int, K: int) -> int:
 
 
 def mep_plan_launches(R: int, n_keys: int, S: int, K: int) -> int:
-    """Kernels mep_plan launches for this shape (1: one CTA; 4: the tiled sort)."""
+    """Kernels mep_plan launches for this shape (1: one launch; 3: the tiled sort)."""
     return int(lib().mep_plan_launches(R, n_keys, S, K))
 
 

@@ -113,7 +113,7 @@ DeviceState &device_state(int dev)
     cudaFuncSetAttribute(mep::k_tile_count<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     cudaFuncSetAttribute(mep::k_tile_count<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     cudaFuncSetAttribute(mep::k_histogram, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-    cudaFuncSetAttribute(mep::k_plan_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    cudaFuncSetAttribute(mep::k_scan_cols_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     cudaFuncSetAttribute(mep::k_source_meta, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     cudaFuncSetAttribute(mep::k_plan_small, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallPlanSmemMax);
     cudaFuncSetAttribute(mep::k_plan_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallPlanSmemMax);
@@ -220,31 +220,51 @@ inline int elem_grid(int64_t total, int threads)
 inline int sort_rounds(int64_t N) { return N <= ((int64_t)1 << 18) ? 2 : (N <= ((int64_t)1 << 20) ? 4 : 8); }
 inline int64_t sort_tiles(int64_t N) { return mep::ceil_div(N, (int64_t)mep::kPlanWarps * 32 * sort_rounds(N)); }
 
+// The plan's replica-table arguments, for a counting sort that also writes them
+// (k_scan_cols_meta); arrived is one int of scratch.
+struct PlanMeta {
+    int32_t *arrived;
+    int32_t R;
+    int64_t SK;
+    int32_t mode, keys_per_rank;
+    int32_t *rank_off, *load, *rep_count, *rep_key, *rep_cu, *stats;
+};
+
+
 // Stable counting sort of N keys in [0, n_keys) (dropped: keep == 0 or out of range):
 // pos[n] = base[key] + (earlier slots of key), base = the exclusive prefix of the
 // histogram, or key_base when given. Writes the histogram to hist; tile_cnt holds
 // sort_tiles(N) * n_keys ints of scratch.
 template <int kRounds>
 void counting_sort_r(const int32_t *keys, const uint8_t *keep, int64_t N, int32_t n_keys, int32_t *tile_cnt,
-                     int32_t *hist, const int32_t *key_base, int32_t *pos, cudaStream_t s)
+                     int32_t *hist, const int32_t *key_base, int32_t *pos, cudaStream_t s, const PlanMeta *meta)
 {
     const int64_t tiles = mep::ceil_div(N, (int64_t)mep::sort_tile<kRounds>());
     const int threads = mep::kPlanWarps * 32;
     mep::k_tile_count<kRounds><<<(unsigned)tiles, threads, sizeof(int32_t) * n_keys, s>>>(keys, keep, N, n_keys,
-                                                                                         tile_cnt);
-    mep::k_scan_cols<<<(unsigned)mep::ceil_div(n_keys, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, n_keys, hist);
+                                                                                         tile_cnt, meta ? meta->arrived
+                                                                                                        : nullptr);
+    if (meta) {
+        const size_t meta_smem = sizeof(int32_t) * (size_t)(3 * n_keys + 2 + (meta->R + 1) + meta->R);
+        mep::k_scan_cols_meta<<<(unsigned)mep::ceil_div(n_keys, 32), 1024, meta_smem, s>>>(
+            tile_cnt, (int32_t)tiles, n_keys, hist, meta->arrived, meta->R, meta->SK, meta->mode, meta->keys_per_rank,
+            meta->rank_off, meta->load, meta->rep_count, meta->rep_key, meta->rep_cu, meta->stats);
+    } else {
+        mep::k_scan_cols<<<(unsigned)mep::ceil_div(n_keys, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, n_keys, hist);
+    }
     const size_t rank_smem = sizeof(int32_t) * ((size_t)mep::kPlanWarps * n_keys + n_keys + 1 + 33);
     mep::k_rank<kRounds><<<(unsigned)tiles, threads, rank_smem, s>>>(keys, keep, N, n_keys, tile_cnt, hist, key_base,
                                                                     pos);
 }
 
 void counting_sort(const int32_t *keys, const uint8_t *keep, int64_t N, int32_t n_keys, int32_t *tile_cnt,
-                   int32_t *hist, const int32_t *key_base, int32_t *pos, cudaStream_t s)
+                   int32_t *hist, const int32_t *key_base, int32_t *pos, cudaStream_t s,
+                   const PlanMeta *meta = nullptr)
 {
     switch (sort_rounds(N)) {
-    case 2: counting_sort_r<2>(keys, keep, N, n_keys, tile_cnt, hist, key_base, pos, s); break;
-    case 4: counting_sort_r<4>(keys, keep, N, n_keys, tile_cnt, hist, key_base, pos, s); break;
-    default: counting_sort_r<8>(keys, keep, N, n_keys, tile_cnt, hist, key_base, pos, s); break;
+    case 2: counting_sort_r<2>(keys, keep, N, n_keys, tile_cnt, hist, key_base, pos, s, meta); break;
+    case 4: counting_sort_r<4>(keys, keep, N, n_keys, tile_cnt, hist, key_base, pos, s, meta); break;
+    default: counting_sort_r<8>(keys, keep, N, n_keys, tile_cnt, hist, key_base, pos, s, meta); break;
     }
 }
 
@@ -311,7 +331,8 @@ size_t mep_plan_workspace_size(int32_t R, int32_t n_keys, int32_t S, int32_t K)
 {
     if (R < 1 || S < 1 || K < 1 || n_keys < 1) return 0;
     const int64_t N = (int64_t)R * S * K;
-    return align256(sizeof(int32_t) * (size_t)sort_tiles(N) * n_keys);
+    // the per-tile counts, then one int: the arrival counter of k_scan_cols_meta
+    return align256(sizeof(int32_t) * (size_t)sort_tiles(N) * n_keys) + 256;
 }
 
 }  // extern "C"
@@ -355,7 +376,7 @@ bool plan_is_small(int64_t N, int32_t n_keys)
 int32_t mep_plan_launches(int32_t R, int32_t n_keys, int32_t S, int32_t K)
 {
     if (R < 1 || S < 1 || K < 1 || n_keys < 1) return 0;
-    return plan_is_small((int64_t)R * S * K, n_keys) ? 1 : 4;
+    return plan_is_small((int64_t)R * S * K, n_keys) ? 1 : 3;
 }
 
 mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_t n_keys,
@@ -390,11 +411,21 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
                                                                        rep_count, rep_key, rep_cu, (int32_t *)stats);
         return launched();
     }
-    counting_sort(ids, keep, N, n_keys, (int32_t *)workspace, hist, nullptr, pos, s);
-    const size_t meta_smem = sizeof(int32_t) * (size_t)(2 * (n_keys + 1) + (R + 1) + R);
-    mep::k_plan_meta<<<1, 1024, meta_smem, s>>>(hist, R, n_keys, (int64_t)S * K, mode,
-                                                keys_per_rank, rank_off, load, rep_count, rep_key,
-                                                rep_cu, (int32_t *)stats);
+    // the sort, with the replica tables written by the last CTA of its scan
+    const int64_t N_tiles = sort_tiles(N);
+    PlanMeta meta;
+    meta.arrived = (int32_t *)((char *)workspace + align256(sizeof(int32_t) * (size_t)N_tiles * n_keys));
+    meta.R = R;
+    meta.SK = (int64_t)S * K;
+    meta.mode = mode;
+    meta.keys_per_rank = keys_per_rank;
+    meta.rank_off = rank_off;
+    meta.load = load;
+    meta.rep_count = rep_count;
+    meta.rep_key = rep_key;
+    meta.rep_cu = rep_cu;
+    meta.stats = (int32_t *)stats;
+    counting_sort(ids, keep, N, n_keys, (int32_t *)workspace, hist, nullptr, pos, s, &meta);
     return launched();
 }
 
@@ -433,11 +464,14 @@ mep_status_t mep_plan_rank(const int32_t *ids, const int32_t *hist_all, int32_t 
     const int threads = mep::kPlanWarps * 32;
     const int rounds = sort_rounds(N);
     if (rounds == 2)
-        mep::k_tile_count<2><<<(unsigned)tiles, threads, sizeof(int32_t) * E, s>>>(ids, nullptr, N, E, tile_cnt);
+        mep::k_tile_count<2><<<(unsigned)tiles, threads, sizeof(int32_t) * E, s>>>(ids, nullptr, N, E, tile_cnt,
+                                                                                 nullptr);
     else if (rounds == 4)
-        mep::k_tile_count<4><<<(unsigned)tiles, threads, sizeof(int32_t) * E, s>>>(ids, nullptr, N, E, tile_cnt);
+        mep::k_tile_count<4><<<(unsigned)tiles, threads, sizeof(int32_t) * E, s>>>(ids, nullptr, N, E, tile_cnt,
+                                                                                 nullptr);
     else
-        mep::k_tile_count<8><<<(unsigned)tiles, threads, sizeof(int32_t) * E, s>>>(ids, nullptr, N, E, tile_cnt);
+        mep::k_tile_count<8><<<(unsigned)tiles, threads, sizeof(int32_t) * E, s>>>(ids, nullptr, N, E, tile_cnt,
+                                                                                 nullptr);
     mep::k_scan_cols<<<(unsigned)mep::ceil_div(E, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, E, hist_local);
     const size_t meta_smem = sizeof(int32_t) * (size_t)(2 * E + 1 + 2 * R);
     mep::k_source_meta<<<1, 1024, meta_smem, s>>>(hist_all, hist_local, R, E, (int64_t)S * K, rank, key_base,

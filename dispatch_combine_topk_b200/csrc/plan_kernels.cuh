@@ -7,13 +7,14 @@
 //   row(n) = off[key] + #{m < n : key(m) == key(n)}.
 // The grouped plan over physical instance ids is the same sort with dropped slots
 // removed. Both are done in three passes over the ids (4 bytes per slot each):
-//   k_tile_count  per-tile key counts              (warp-aggregated with match.any)
-//   k_scan_cols   per-key prefix over tiles and hist, one CTA per 32 keys
-//   k_rank        per-slot stable rank inside its tile, written as the final row
-// and one single-CTA pass over the keys, k_plan_meta, that writes the per-rank replica
-// tables (cu_seqlens) and the summary counts. The exclusive prefix of hist over keys
-// (off) is small (at most 4096 keys) and is recomputed in shared memory by each CTA that
-// needs it.
+//   k_tile_count      per-tile key counts              (warp-aggregated with match.any)
+//   k_scan_cols_meta  per-key prefix over tiles and hist, one CTA per 32 keys; the CTA
+//                     that finishes last then writes the per-rank replica tables
+//                     (cu_seqlens) and the summary counts (plan_meta)
+//   k_rank            per-slot stable rank inside its tile, written as the final row
+// Small plans run as one launch (k_plan_cluster, k_plan_small). The exclusive prefix of
+// hist over keys (off) is small (at most 4096 keys) and is recomputed in shared memory
+// by each CTA that needs it.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -64,13 +65,15 @@ k_histogram(const int32_t *__restrict__ ids, int64_t N, int32_t n_keys, int32_t 
 }
 
 // tile_cnt[tile, key] = slots of `key` in tile `blockIdx.x` (tiles of sort_tile<kRounds>).
+// zero_word, when given, is set to 0 by CTA 0 (the arrival counter of k_scan_cols_meta).
 template <int kRounds>
 __global__ void __launch_bounds__(kPlanWarps * 32)
 k_tile_count(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, int64_t N,
-             int32_t n_keys, int32_t *__restrict__ tile_cnt)
+             int32_t n_keys, int32_t *__restrict__ tile_cnt, int32_t *__restrict__ zero_word)
 {
     constexpr int kTile = sort_tile<kRounds>();
     extern __shared__ int32_t sh[];
+    if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0;
     for (int i = threadIdx.x; i < n_keys; i += blockDim.x) sh[i] = 0;
     __syncthreads();
     const int lane = threadIdx.x & 31;
@@ -125,8 +128,8 @@ __device__ __forceinline__ void block_exclusive_scan(const int32_t *__restrict__
 
 // CTA c owns keys [32c, 32c + 32), one per lane; its 32 warps split the tiles. In place:
 // tile_cnt[t, key] <- sum_{t' < t} tile_cnt[t', key], and hist[key] = sum over tiles.
-__global__ void __launch_bounds__(1024)
-k_scan_cols(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys, int32_t *__restrict__ hist)
+__device__ __forceinline__ void scan_cols(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys,
+                                          int32_t *__restrict__ hist)
 {
     __shared__ int32_t part[32][33];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -161,6 +164,13 @@ k_scan_cols(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys, int
         }
     }
 }
+
+__global__ void __launch_bounds__(1024)
+k_scan_cols(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys, int32_t *__restrict__ hist)
+{
+    scan_cols(tile_cnt, n_tiles, n_keys, hist);
+}
+
 
 // pos[n] = off[key] + (slots of key in earlier tiles) + (earlier slots of key in this
 // tile), off = exclusive prefix of hist over keys, or key_base[key] when key_base is
@@ -358,16 +368,32 @@ __device__ __forceinline__ void plan_meta(const int32_t *__restrict__ hist, int3
     }
 }
 
-// Dynamic shared memory: as plan_meta.
+// k_scan_cols, then the replica tables in the CTA that finishes last: each CTA writes
+// its keys' hist entries, fences them and arrives once on *arrived; the CTA whose
+// arrival is the last copies hist into shared memory (through L2) and runs plan_meta.
+// One launch fewer than a separate replica-table kernel; nothing waits. *arrived must be 0
+// at launch (k_tile_count zeroes it).
+// Dynamic shared memory: plan_meta's (2 (n_keys + 1) + (R + 1) + R ints), then n_keys ints.
 __global__ void __launch_bounds__(1024)
-k_plan_meta(const int32_t *__restrict__ hist, int32_t R,
-            int32_t n_keys, int64_t SK, int32_t mode, int32_t keys_per_rank,
-            int32_t *__restrict__ rank_off_out, int32_t *__restrict__ load_out,
-            int32_t *__restrict__ rep_count, int32_t *__restrict__ rep_key,
-            int32_t *__restrict__ rep_cu, int32_t *__restrict__ stats)
+k_scan_cols_meta(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys, int32_t *__restrict__ hist,
+                 int32_t *__restrict__ arrived, int32_t R, int64_t SK, int32_t mode, int32_t keys_per_rank,
+                 int32_t *__restrict__ rank_off_out, int32_t *__restrict__ load_out,
+                 int32_t *__restrict__ rep_count, int32_t *__restrict__ rep_key, int32_t *__restrict__ rep_cu,
+                 int32_t *__restrict__ stats)
 {
     extern __shared__ int32_t smem[];
-    plan_meta(hist, R, n_keys, SK, mode, keys_per_rank, rank_off_out, load_out, rep_count, rep_key, rep_cu, stats,
+    __shared__ int32_t s_last;
+    scan_cols(tile_cnt, n_tiles, n_keys, hist);
+    __threadfence();                                  // this CTA's hist entries before its arrival
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(arrived, 1) == (int32_t)gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    int32_t *h = smem + 2 * (n_keys + 1) + (R + 1) + R;
+    for (int e = threadIdx.x; e < n_keys; e += blockDim.x) h[e] = __ldcg(hist + e);
+    __syncthreads();
+    plan_meta(h, R, n_keys, SK, mode, keys_per_rank, rank_off_out, load_out, rep_count, rep_key, rep_cu, stats,
               smem);
 }
 

@@ -156,9 +156,10 @@ mep_status_t mep_histogram(const int32_t *ids, int64_t n, int32_t n_keys, int32_
 /* Bytes of workspace mep_plan needs for N = R*S*K slots and n_keys keys. */
 size_t mep_plan_workspace_size(int32_t R, int32_t n_keys, int32_t S, int32_t K);
 
-/* Kernels mep_plan launches for this shape: 1 when the whole plan runs as one CTA (at
- * most 16384 slots and few enough keys for its shared memory), 4 otherwise (the tiled
- * sort); 0 for a shape below 1. For launch accounting; host only. */
+/* Kernels mep_plan launches for this shape: 1 when the whole plan runs in one launch
+ * (at most 16384 slots and few enough keys for shared memory: a cluster of CTAs, or one
+ * CTA), 3 otherwise (the tiled sort, whose scan also writes the replica tables); 0 for a
+ * shape below 1. For launch accounting; host only. */
 int32_t mep_plan_launches(int32_t R, int32_t n_keys, int32_t S, int32_t K);
 
 /*

@@ -255,15 +255,15 @@ def test_plan_rank_argument_checks(L):
 
 
 def test_plan_launch_count(L):
-    """Host-only query: one launch when the whole plan fits one CTA (at most 16384 slots
-    and few enough keys for its shared memory), four for the tiled sort."""
+    """Host-only query: one launch when the whole plan fits one launch (at most 16384
+    slots and few enough keys for shared memory), three for the tiled sort."""
     L.mep_plan_launches.argtypes = [ctypes.c_int32] * 4
     L.mep_plan_launches.restype = ctypes.c_int32
     assert L.mep_plan_launches(4, 16, 128, 2) == 1            # tiny
     assert L.mep_plan_launches(8, 272, 256, 8) == 1           # mapping workload: 16384 slots
-    assert L.mep_plan_launches(1, 2, 16385, 1) == 4           # one slot past the limit
-    assert L.mep_plan_launches(64, 1536, 8, 8) == 4           # too many keys for one CTA
-    assert L.mep_plan_launches(32, 256, 8192, 8) == 4         # int8 workload
+    assert L.mep_plan_launches(1, 2, 16385, 1) == 3           # one slot past the limit
+    assert L.mep_plan_launches(64, 1536, 8, 8) == 3           # too many keys for one launch
+    assert L.mep_plan_launches(32, 256, 8192, 8) == 3         # int8 workload
     assert L.mep_plan_launches(0, 16, 128, 2) == 0
 
 
