@@ -245,7 +245,7 @@ void counting_sort_r(const int32_t *keys, const uint8_t *keep, int64_t N, int32_
                                                                                          tile_cnt, meta ? meta->arrived
                                                                                                         : nullptr);
     if (meta) {
-        const size_t meta_smem = sizeof(int32_t) * (size_t)(3 * n_keys + 2 + (meta->R + 1) + meta->R);
+        const size_t meta_smem = sizeof(int32_t) * (size_t)(3 * n_keys + 2 + (meta->R + 1) + 2 * meta->R);
         mep::k_scan_cols_meta<<<(unsigned)mep::ceil_div(n_keys, 32), 1024, meta_smem, s>>>(
             tile_cnt, (int32_t)tiles, n_keys, hist, meta->arrived, meta->R, meta->SK, meta->mode, meta->keys_per_rank,
             meta->rank_off, meta->load, meta->rep_count, meta->rep_key, meta->rep_cu, meta->stats);

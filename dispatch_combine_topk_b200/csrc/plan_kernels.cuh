@@ -126,6 +126,68 @@ __device__ __forceinline__ void block_exclusive_scan(const int32_t *__restrict__
     __syncthreads();
 }
 
+// block_exclusive_scan of in[0..n) into out[0..n] and, in the same pass, of the flags
+// in[i] > 0 into nz[0..n] (nz[i] = how many of in[0..i) are positive). scratch holds 66
+// ints of shared memory. Ends with a block barrier.
+__device__ __forceinline__ void block_exclusive_scan2(const int32_t *__restrict__ in, int n, int32_t *out,
+                                                      int32_t *nz, int32_t *scratch)
+{
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+    const int per = (n + nt - 1) / nt;
+    const int lo = min(n, tid * per), hi = min(n, lo + per);
+    int32_t sum = 0, cnt = 0;
+    for (int i = lo; i < hi; i++) {
+        const int32_t v = in[i];
+        sum += v;
+        cnt += v > 0 ? 1 : 0;
+    }
+    int32_t inc = sum, incc = cnt;
+    for (int d = 1; d < 32; d <<= 1) {
+        const int32_t u = __shfl_up_sync(0xffffffffu, inc, d);
+        const int32_t uc = __shfl_up_sync(0xffffffffu, incc, d);
+        if (lane >= d) {
+            inc += u;
+            incc += uc;
+        }
+    }
+    if (lane == 31) {
+        scratch[warp] = inc;
+        scratch[33 + warp] = incc;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int32_t w = lane < nw ? scratch[lane] : 0, wc = lane < nw ? scratch[33 + lane] : 0;
+        int32_t wi = w, wci = wc;
+        for (int d = 1; d < 32; d <<= 1) {
+            const int32_t u = __shfl_up_sync(0xffffffffu, wi, d);
+            const int32_t uc = __shfl_up_sync(0xffffffffu, wci, d);
+            if (lane >= d) {
+                wi += u;
+                wci += uc;
+            }
+        }
+        scratch[lane] = wi - w;
+        scratch[33 + lane] = wci - wc;
+        if (lane == 31) {
+            scratch[32] = wi;
+            scratch[65] = wci;
+        }
+    }
+    __syncthreads();
+    int32_t run = scratch[warp] + inc - sum, runc = scratch[33 + warp] + incc - cnt;
+    for (int i = lo; i < hi; i++) {
+        out[i] = run;
+        nz[i] = runc;
+        run += in[i];
+        runc += in[i] > 0 ? 1 : 0;
+    }
+    if (tid == 0) {
+        out[n] = scratch[32];
+        nz[n] = scratch[65];
+    }
+    __syncthreads();
+}
+
 // CTA c owns keys [32c, 32c + 32), one per lane; its 32 warps split the tiles. In place:
 // tile_cnt[t, key] <- sum_{t' < t} tile_cnt[t', key], and hist[key] = sum over tiles.
 __device__ __forceinline__ void scan_cols(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys,
@@ -246,8 +308,8 @@ __device__ __forceinline__ int32_t upper_bound_sh(const int32_t *a, int32_t n, i
     return lo;
 }
 
-// Per-rank replica tables and the summary counts, by one CTA of 1024 threads.
-// smem: key_off (n_keys+1) + nz (n_keys+1) + rank_off (R+1) + e_lo (R) ints.
+// Per-rank replica tables and the summary counts, by one CTA (any multiple of 32 threads).
+// smem: key_off (n_keys+1) + nz (n_keys+1) + rank_off (R+1) + e_lo (R) + count (R) ints.
 __device__ __forceinline__ void plan_meta(const int32_t *__restrict__ hist, int32_t R,
                                           int32_t n_keys, int64_t SK, int32_t mode, int32_t keys_per_rank,
                                           int32_t *__restrict__ rank_off_out, int32_t *__restrict__ load_out,
@@ -259,44 +321,15 @@ __device__ __forceinline__ void plan_meta(const int32_t *__restrict__ hist, int3
     int32_t *nz = koff + (n_keys + 1);       // n_keys + 1: exclusive count of non-empty keys
     int32_t *roff = nz + (n_keys + 1);       // R + 1
     int32_t *elo = roff + (R + 1);           // R: first key on each rank
+    int32_t *rcnt = elo + R;                 // R: replicas on each rank
     __shared__ int32_t s_red[8];
-    __shared__ int32_t wsum[32];
-    __shared__ int32_t carry;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ int32_t scan_scratch[66];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     const int32_t cap = n_keys;
     const int32_t per_rank = (mode == 0) ? n_keys / R : keys_per_rank;
 
-    __shared__ int32_t scan_scratch[33];
-    block_exclusive_scan(hist, n_keys, koff, scan_scratch);
+    block_exclusive_scan2(hist, n_keys, koff, nz, scan_scratch);
     if (threadIdx.x < 8) s_red[threadIdx.x] = 0;
-    if (threadIdx.x == 0) carry = 0;
-    __syncthreads();
-    // nz = exclusive prefix count of keys with hist > 0
-    for (int e0 = 0; e0 <= n_keys; e0 += 1024) {
-        const int e = e0 + threadIdx.x;
-        int32_t v = (e < n_keys && koff[e + 1] > koff[e]) ? 1 : 0;
-        int32_t inc = v;
-        for (int d = 1; d < 32; d <<= 1) {
-            int32_t u = __shfl_up_sync(0xffffffffu, inc, d);
-            if (lane >= d) inc += u;
-        }
-        if (lane == 31) wsum[warp] = inc;
-        __syncthreads();
-        if (warp == 0) {
-            int32_t w = wsum[lane], wi = w;
-            for (int d = 1; d < 32; d <<= 1) {
-                int32_t u = __shfl_up_sync(0xffffffffu, wi, d);
-                if (lane >= d) wi += u;
-            }
-            wsum[lane] = wi - w;
-        }
-        __syncthreads();
-        const int32_t c = carry;
-        if (e <= n_keys) nz[e] = c + wsum[warp] + inc - v;
-        __syncthreads();
-        if (threadIdx.x == 1023) carry = c + wsum[31] + inc;
-        __syncthreads();
-    }
     // rank offsets
     for (int r = threadIdx.x; r <= R; r += blockDim.x) {
         int64_t ro = (mode == 0) ? (int64_t)r * SK : (int64_t)koff[min(n_keys, r * keys_per_rank)];
@@ -304,7 +337,7 @@ __device__ __forceinline__ void plan_meta(const int32_t *__restrict__ hist, int3
         rank_off_out[r] = (int32_t)ro;
     }
     __syncthreads();
-    // first key of each non-empty rank; replica counts; clear the tables
+    // first key of each non-empty rank; replica counts
     for (int r = threadIdx.x; r < R; r += blockDim.x) {
         int32_t cnt = 0, first = 0;
         if (roff[r + 1] > roff[r]) {
@@ -314,6 +347,7 @@ __device__ __forceinline__ void plan_meta(const int32_t *__restrict__ hist, int3
             atomicAdd(&s_red[6], 1);
         }
         elo[r] = first;
+        rcnt[r] = cnt;
         rep_count[r] = cnt;
         atomicMax(&s_red[1], roff[r + 1] - roff[r]);
         if (load_out) {
@@ -323,8 +357,6 @@ __device__ __forceinline__ void plan_meta(const int32_t *__restrict__ hist, int3
             load_out[r] = l;
         }
     }
-    for (int64_t i = threadIdx.x; i < (int64_t)R * cap; i += blockDim.x) rep_key[i] = -1;
-    for (int64_t i = threadIdx.x; i < (int64_t)R * (cap + 1); i += blockDim.x) rep_cu[i] = 0;
     __syncthreads();
     // one thread per key: write its replica entries on every rank it spans
     for (int e = threadIdx.x; e < n_keys; e += blockDim.x) {
@@ -353,9 +385,16 @@ __device__ __forceinline__ void plan_meta(const int32_t *__restrict__ hist, int3
         if (r1 > r0) atomicAdd(&s_red[2], r1 - r0);
         if (pf) atomicAdd(&s_red[3], pf);
     }
+    // the rest of every rank's rows (disjoint from the entries above): no key past its
+    // count, and the running row count ends at the rank's rows
+    for (int r = warp; r < R; r += nwarps) {
+        const int32_t c = rcnt[r];
+        for (int j = c + lane; j <= cap; j += 32) {
+            if (j < cap) rep_key[(int64_t)r * cap + j] = -1;
+            rep_cu[(int64_t)r * (cap + 1) + j] = j == c ? roff[r + 1] - roff[r] : 0;
+        }
+    }
     __syncthreads();
-    for (int r = threadIdx.x; r < R; r += blockDim.x)
-        rep_cu[(int64_t)r * (cap + 1) + rep_count[r]] = roff[r + 1] - roff[r];
     if (threadIdx.x == 0) {
         stats[0] = (mode == 0) ? s_red[0] : s_red[1];
         stats[1] = s_red[1];
@@ -373,7 +412,7 @@ __device__ __forceinline__ void plan_meta(const int32_t *__restrict__ hist, int3
 // arrival is the last copies hist into shared memory (through L2) and runs plan_meta.
 // One launch fewer than a separate replica-table kernel; nothing waits. *arrived must be 0
 // at launch (k_tile_count zeroes it).
-// Dynamic shared memory: plan_meta's (2 (n_keys + 1) + (R + 1) + R ints), then n_keys ints.
+// Dynamic shared memory: plan_meta's (2 (n_keys + 1) + (R + 1) + 2 R ints), then n_keys ints.
 __global__ void __launch_bounds__(1024)
 k_scan_cols_meta(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys, int32_t *__restrict__ hist,
                  int32_t *__restrict__ arrived, int32_t R, int64_t SK, int32_t mode, int32_t keys_per_rank,
@@ -390,7 +429,7 @@ k_scan_cols_meta(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    int32_t *h = smem + 2 * (n_keys + 1) + (R + 1) + R;
+    int32_t *h = smem + 2 * (n_keys + 1) + (R + 1) + 2 * R;
     for (int e = threadIdx.x; e < n_keys; e += blockDim.x) h[e] = __ldcg(hist + e);
     __syncthreads();
     plan_meta(h, R, n_keys, SK, mode, keys_per_rank, rank_off_out, load_out, rep_count, rep_key, rep_cu, stats,
