@@ -195,7 +195,9 @@ int32_t mep_plan_launches(int32_t R, int32_t n_keys, int32_t S, int32_t K);
  *                                 rank_off[r] (the grouped-GEMM offsets MoonEP's
  *                                 planner produces); 0 after rep_count[r]
  *   stats     mep_plan_stats_t [1]
- * Workspace: at least mep_plan_workspace_size(R, n_keys, S, K) bytes, 256-byte aligned.
+ * Workspace: at least mep_plan_workspace_size(R, n_keys, S, K) bytes, 256-byte aligned,
+ * caller-owned scratch (no contents needed on entry); calls in flight at the same time
+ * need workspaces of their own.
  * Errors: NULL pointer; R, S, K < 1, K > MEP_MAX_K, N >= 2^31, n_keys outside
  * [1, MEP_MAX_KEYS] (MEP_ERR_SHAPE); mode unknown, E % R != 0, keep given in
  * balanced mode, keys_per_rank * R != n_keys in grouped mode (MEP_ERR_VALUE);
