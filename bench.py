@@ -116,17 +116,17 @@ def kernel_source_hash(name: str) -> str:
 _TRAFFIC_METRICS = "dram__bytes_read.sum + dram__bytes_write.sum"
 TRAFFIC = {
     ("k_dispatch_warp", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 997.906e6, "src": "ecb53c46b3d954ca", "case_S": 1024, "case_mb": 997.906},
+        "bytes": 4 * 997.452e6, "src": "f2dc9831a61b7e83", "case_S": 1024, "case_mb": 997.452},
     ("k_combine_v8", "r8_e64_s4096_k8_h7168"): {
-        "bytes": 4 * 1005.660e6, "src": "aa70b87f5f33b11a", "case_S": 1024, "case_mb": 1005.660},
+        "bytes": 4 * 1005.611e6, "src": "75f948c1d2f4d491", "case_S": 1024, "case_mb": 1005.611},
     ("k_dispatch_int8_staged", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1115.672e6, "src": "597997762b516c3e", "case_S": 512, "case_mb": 1115.672},
+        "bytes": 16 * 1114.960e6, "src": "0158b32e901926e8", "case_S": 512, "case_mb": 1114.960},
     ("k_combine_int8_warp", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1117.330e6, "src": "a2aec7cc7412bc6f", "case_S": 512, "case_mb": 1117.330},
+        "bytes": 16 * 1117.223e6, "src": "528f2068b9109630", "case_S": 512, "case_mb": 1117.223},
     ("k_dispatch_warp", "skew_r64_e512_s2048_k8_h4096"): {
-        "bytes": 4 * 2357.854e6, "src": "ecb53c46b3d954ca", "case_S": 512, "case_mb": 2357.854},
+        "bytes": 4 * 2357.469e6, "src": "f2dc9831a61b7e83", "case_S": 512, "case_mb": 2357.469},
     ("k_combine_v8", "skew_r64_e512_s2048_k8_h4096"): {
-        "bytes": 4 * 2364.469e6, "src": "aa70b87f5f33b11a", "case_S": 512, "case_mb": 2364.469},
+        "bytes": 4 * 2364.012e6, "src": "75f948c1d2f4d491", "case_S": 512, "case_mb": 2364.012},
 }
 
 

@@ -81,6 +81,14 @@ __device__ __forceinline__ float2 mul2_rn(float2 a, float2 b)
     return d;
 }
 
+// Programmatic dependent launch (the host launches the routing step's kernels with the
+// programmatic-serialization attribute): pdl_wait() returns once the grid this one
+// depends on has finished and its memory is visible (at once when there is none), so a
+// kernel calls it before touching any memory the previous kernel may use;
+// pdl_launch_dependents() lets the next kernel's CTAs be scheduled while this one runs.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace mep

@@ -220,6 +220,25 @@ inline int elem_grid(int64_t total, int threads)
 inline int sort_rounds(int64_t N) { return N <= ((int64_t)1 << 18) ? 2 : (N <= ((int64_t)1 << 20) ? 4 : 8); }
 inline int64_t sort_tiles(int64_t N) { return mep::ceil_div(N, (int64_t)mep::kPlanWarps * 32 * sort_rounds(N)); }
 
+// Launch of a kernel of the routing step with programmatic stream serialization: it may
+// be scheduled before the previous kernel on the stream has finished and waits for it
+// itself (pdl_wait at its start); every kernel launched this way does so.
+template <typename... P, typename... A>
+void launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, ((P)args)...);
+}
+
 // The plan's replica-table arguments, for a counting sort that also writes them
 // (k_scan_cols_meta); arrived is one int of scratch.
 struct PlanMeta {
@@ -241,20 +260,20 @@ void counting_sort_r(const int32_t *keys, const uint8_t *keep, int64_t N, int32_
 {
     const int64_t tiles = mep::ceil_div(N, (int64_t)mep::sort_tile<kRounds>());
     const int threads = mep::kPlanWarps * 32;
-    mep::k_tile_count<kRounds><<<(unsigned)tiles, threads, sizeof(int32_t) * n_keys, s>>>(keys, keep, N, n_keys,
-                                                                                         tile_cnt, meta ? meta->arrived
-                                                                                                        : nullptr);
+    launch_pdl(mep::k_tile_count<kRounds>, dim3((unsigned)tiles), dim3(threads), sizeof(int32_t) * n_keys, s, keys, keep,
+               N, n_keys, tile_cnt, meta ? meta->arrived : nullptr);
     if (meta) {
         const size_t meta_smem = sizeof(int32_t) * (size_t)(3 * n_keys + 2 + (meta->R + 1) + 2 * meta->R);
-        mep::k_scan_cols_meta<<<(unsigned)mep::ceil_div(n_keys, 32), 1024, meta_smem, s>>>(
-            tile_cnt, (int32_t)tiles, n_keys, hist, meta->arrived, meta->R, meta->SK, meta->mode, meta->keys_per_rank,
-            meta->rank_off, meta->load, meta->rep_count, meta->rep_key, meta->rep_cu, meta->stats);
+        launch_pdl(mep::k_scan_cols_meta, dim3((unsigned)mep::ceil_div(n_keys, 32)), dim3(1024), meta_smem, s, tile_cnt,
+                   (int32_t)tiles, n_keys, hist, meta->arrived, meta->R, meta->SK, meta->mode, meta->keys_per_rank,
+                   meta->rank_off, meta->load, meta->rep_count, meta->rep_key, meta->rep_cu, meta->stats);
     } else {
-        mep::k_scan_cols<<<(unsigned)mep::ceil_div(n_keys, 32), 1024, 0, s>>>(tile_cnt, (int32_t)tiles, n_keys, hist);
+        launch_pdl(mep::k_scan_cols, dim3((unsigned)mep::ceil_div(n_keys, 32)), dim3(1024), 0, s, tile_cnt, (int32_t)tiles,
+                   n_keys, hist);
     }
     const size_t rank_smem = sizeof(int32_t) * ((size_t)mep::kPlanWarps * n_keys + n_keys + 1 + 33);
-    mep::k_rank<kRounds><<<(unsigned)tiles, threads, rank_smem, s>>>(keys, keep, N, n_keys, tile_cnt, hist, key_base,
-                                                                    pos);
+    launch_pdl(mep::k_rank<kRounds>, dim3((unsigned)tiles), dim3(threads), rank_smem, s, keys, keep, N, n_keys,
+               (const int32_t *)tile_cnt, (const int32_t *)hist, key_base, pos);
 }
 
 void counting_sort(const int32_t *keys, const uint8_t *keep, int64_t N, int32_t n_keys, int32_t *tile_cnt,
@@ -399,16 +418,16 @@ mep_status_t mep_plan(const int32_t *ids, const uint8_t *keep, int32_t R, int32_
     // CTAs when it fits, else in one CTA
     const size_t cluster_smem = sizeof(int32_t) * (size_t)(36 * (int64_t)n_keys + 34);
     if (N <= mep::kClusterPlanMaxSlots && cluster_smem <= (size_t)kSmallPlanSmemMax && cluster_plan_ok()) {
-        mep::k_plan_cluster<<<mep::kPlanClusterCTAs, mep::kSmallPlanThreads, cluster_smem, s>>>(
-            ids, keep, N, n_keys, R, (int64_t)S * K, mode, keys_per_rank, pos, hist, rank_off, load, rep_count,
-            rep_key, rep_cu, (int32_t *)stats);
+        launch_pdl(mep::k_plan_cluster, dim3(mep::kPlanClusterCTAs), dim3(mep::kSmallPlanThreads), cluster_smem, s, ids,
+                   keep, N, n_keys, R, (int64_t)S * K, mode, keys_per_rank, pos, hist, rank_off, load, rep_count,
+                   rep_key, rep_cu, (int32_t *)stats);
         return launched();
     }
     if (plan_is_small(N, n_keys)) {
         const size_t small_smem = sizeof(int32_t) * (size_t)(34 * (int64_t)n_keys + 34);
-        mep::k_plan_small<<<1, mep::kSmallPlanThreads, small_smem, s>>>(ids, keep, N, n_keys, R, (int64_t)S * K, mode,
-                                                                       keys_per_rank, pos, hist, rank_off, load,
-                                                                       rep_count, rep_key, rep_cu, (int32_t *)stats);
+        launch_pdl(mep::k_plan_small, dim3(1), dim3(mep::kSmallPlanThreads), small_smem, s, ids, keep, N, n_keys, R,
+                   (int64_t)S * K, mode, keys_per_rank, pos, hist, rank_off, load, rep_count, rep_key, rep_cu,
+                   (int32_t *)stats);
         return launched();
     }
     // the sort, with the replica tables written by the last CTA of its scan
@@ -562,8 +581,8 @@ mep_status_t mep_dispatch(const uint16_t *x, const int32_t *pos, int64_t T, int3
             // one warp per half token row, 8 warps per CTA, up to 64 CTAs per SM in waves
             const int64_t ctas = mep::ceil_div(2 * T, 8);
             const int64_t cap = (int64_t)sm_count() * 64;
-            mep::k_dispatch_warp<<<(int)(ctas < cap ? ctas : cap), 256, 0, s>>>((const uint4 *)x, pos, T, K, H / 8,
-                                                                              rows, (uint4 *)recv);
+            launch_pdl(mep::k_dispatch_warp, dim3((unsigned)(ctas < cap ? ctas : cap)), dim3(256), 0, s, (const uint4 *)x,
+                       pos, T, K, (int64_t)(H / 8), rows, (uint4 *)recv);
         } else {
             mep::k_dispatch_elem<<<grid, 256, 0, s>>>(x, pos, T, K, H, rows, (uint16_t *)recv);
         }
@@ -574,8 +593,8 @@ mep_status_t mep_dispatch(const uint16_t *x, const int32_t *pos, int64_t T, int3
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mep::k_dispatch_int8_staged<4, 128>, 128,
                                                           staged_smem);
             per_sm = per_sm < 1 ? 1 : (per_sm > 3 ? 3 : per_sm);
-            mep::k_dispatch_int8_staged<4, 128><<<token_grid(T, per_sm), 128, staged_smem, s>>>(
-                x, pos, T, K, H, rows, (int8_t *)recv, recv_scale);
+            launch_pdl(mep::k_dispatch_int8_staged<4, 128>, dim3((unsigned)token_grid(T, per_sm)), dim3(128), staged_smem, s,
+                       x, pos, T, (int)K, H, rows, (int8_t *)recv, recv_scale);
         } else if (H % 8 == 0 && aligned(x, 16) && aligned(recv, 8)) {
             mep::k_dispatch_int8<<<grid, 256, 0, s>>>((const uint4 *)x, pos, T, K, H / 8, rows,
                                                       (uint2 *)recv, recv_scale);
@@ -618,12 +637,12 @@ mep_status_t mep_combine(const uint16_t *y, int64_t rows, const int32_t *pos,
         uint4 *ov = (uint4 *)out;
         const int64_t H8 = H / 8;
         switch (K) {
-        case 1: mep::k_combine_v8<1><<<grid, 256, 0, s>>>(yv, pos, gates, T, K, H8, rows, ov); break;
-        case 2: mep::k_combine_v8<2><<<grid, 256, 0, s>>>(yv, pos, gates, T, K, H8, rows, ov); break;
-        case 4: mep::k_combine_v8<4><<<grid, 256, 0, s>>>(yv, pos, gates, T, K, H8, rows, ov); break;
-        case 6: mep::k_combine_v8<6><<<grid, 256, 0, s>>>(yv, pos, gates, T, K, H8, rows, ov); break;
-        case 8: mep::k_combine_v8<8><<<grid, 256, 0, s>>>(yv, pos, gates, T, K, H8, rows, ov); break;
-        default: mep::k_combine_v8<0><<<grid, 256, 0, s>>>(yv, pos, gates, T, K, H8, rows, ov); break;
+        case 1: launch_pdl(mep::k_combine_v8<1>, dim3(grid), dim3(256), 0, s, yv, pos, gates, T, (int)K, H8, rows, ov); break;
+        case 2: launch_pdl(mep::k_combine_v8<2>, dim3(grid), dim3(256), 0, s, yv, pos, gates, T, (int)K, H8, rows, ov); break;
+        case 4: launch_pdl(mep::k_combine_v8<4>, dim3(grid), dim3(256), 0, s, yv, pos, gates, T, (int)K, H8, rows, ov); break;
+        case 6: launch_pdl(mep::k_combine_v8<6>, dim3(grid), dim3(256), 0, s, yv, pos, gates, T, (int)K, H8, rows, ov); break;
+        case 8: launch_pdl(mep::k_combine_v8<8>, dim3(grid), dim3(256), 0, s, yv, pos, gates, T, (int)K, H8, rows, ov); break;
+        default: launch_pdl(mep::k_combine_v8<0>, dim3(grid), dim3(256), 0, s, yv, pos, gates, T, (int)K, H8, rows, ov); break;
         }
     } else {
         mep::k_combine_scalar<<<grid, 256, 0, s>>>(y, pos, gates, T, K, H, rows, out);
@@ -658,8 +677,8 @@ mep_status_t mep_combine_int8(const int8_t *yq, const float *y_scale, int64_t ro
         }
         // one warp per token, grid-stride: as many CTAs as can be resident at once
         const int tpb = mep::kCombineInt8Threads;
-        kern<<<resident_grid(kern, tpb, mep::ceil_div(T, tpb / 32)), tpb, 0, s>>>(yv, y_scale, pos, gates, T, K, H16,
-                                                                                   rows, ov);
+        launch_pdl(kern, dim3((unsigned)resident_grid(kern, tpb, mep::ceil_div(T, tpb / 32))), dim3(tpb), 0, s, yv, y_scale,
+                   pos, gates, T, (int)K, H16, rows, ov);
     } else if (H % 8 == 0 && aligned(yq, 8) && aligned(out, 16)) {
         const uint2 *yv = (const uint2 *)yq;
         uint4 *ov = (uint4 *)out;

@@ -73,6 +73,8 @@ k_tile_count(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, 
 {
     constexpr int kTile = sort_tile<kRounds>();
     extern __shared__ int32_t sh[];
+    pdl_wait();
+    pdl_launch_dependents();
     if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0;
     for (int i = threadIdx.x; i < n_keys; i += blockDim.x) sh[i] = 0;
     __syncthreads();
@@ -230,6 +232,8 @@ __device__ __forceinline__ void scan_cols(int32_t *__restrict__ tile_cnt, int32_
 __global__ void __launch_bounds__(1024)
 k_scan_cols(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys, int32_t *__restrict__ hist)
 {
+    pdl_wait();
+    pdl_launch_dependents();
     scan_cols(tile_cnt, n_tiles, n_keys, hist);
 }
 
@@ -251,6 +255,8 @@ k_rank(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, int64_
     int32_t *key_off = cnt + kPlanWarps * n_keys;
     int32_t *scan_scratch = key_off + n_keys + 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_launch_dependents();
     for (int i = threadIdx.x; i < kPlanWarps * n_keys; i += blockDim.x) cnt[i] = 0;
     if (key_base) {
         for (int i = threadIdx.x; i < n_keys; i += blockDim.x) key_off[i] = key_base[i];
@@ -422,6 +428,8 @@ k_scan_cols_meta(int32_t *__restrict__ tile_cnt, int32_t n_tiles, int32_t n_keys
 {
     extern __shared__ int32_t smem[];
     __shared__ int32_t s_last;
+    pdl_wait();
+    pdl_launch_dependents();
     scan_cols(tile_cnt, n_tiles, n_keys, hist);
     __threadfence();                                  // this CTA's hist entries before its arrival
     __syncthreads();
@@ -463,6 +471,8 @@ k_plan_small(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep, 
     int32_t *scan_scratch = key_off + n_keys + 1;     // 33
     int32_t *tot = scan_scratch + 33;                 // n_keys: hist, kept for plan_meta
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_launch_dependents();
     for (int i = threadIdx.x; i < kWarps * n_keys; i += blockDim.x) cnt[i] = 0;
     __syncthreads();
     const int64_t sub = ((N + kWarps - 1) / kWarps + 31) / 32 * 32;   // <= 32 * kSmallPlanPerLane
@@ -568,6 +578,8 @@ k_plan_cluster(const int32_t *__restrict__ ids, const uint8_t *__restrict__ keep
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     const int crank = (int)cluster.block_rank();
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ int32_t smem[];
     constexpr int kWarps = kSmallPlanThreads / 32;
     int32_t *cnt = smem;                              // [kWarps][n_keys]

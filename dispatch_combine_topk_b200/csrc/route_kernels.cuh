@@ -132,6 +132,8 @@ __global__ void __launch_bounds__(256)
 k_dispatch_warp(const uint4 *__restrict__ x, const int32_t *__restrict__ pos, int64_t T, int K, int64_t H8,
                 int64_t rows, uint4 *__restrict__ recv)
 {
+    pdl_wait();
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t per = (H8 + 1) / 2;
@@ -303,6 +305,8 @@ k_dispatch_int8_staged(const uint16_t *__restrict__ x, const int32_t *__restrict
         mbar_fence_init();
     }
     __syncthreads();
+    pdl_wait();                       // the barriers' set-up above touches only this CTA's memory
+    pdl_launch_dependents();
     const int64_t n = blockIdx.x < T ? (T - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
     auto token = [&](int64_t i) { return (int64_t)blockIdx.x + i * gridDim.x; };
     auto fetch = [&](int64_t i) {   // warp 0 only
@@ -514,6 +518,8 @@ k_combine_v8(const uint4 *__restrict__ y, const int32_t *__restrict__ pos,
     __shared__ int32_t sp[kMaxK];
     __shared__ float sg[kMaxK];
     const int K = kFixed ? KC : Krt;
+    pdl_wait();
+    pdl_launch_dependents();
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         load_token_rows(pos, t, K, rows, sp);
         if (threadIdx.x < K) sg[threadIdx.x] = gates[t * K + threadIdx.x];
@@ -696,6 +702,8 @@ k_combine_int8_warp(const uint4 *__restrict__ yq, const float *__restrict__ ysca
     const int K = kFixed ? KC : Krt;
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    pdl_wait();
+    pdl_launch_dependents();
     for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
         int32_t mine = -1;
         float g_mine = 0.0f, s_mine = 0.0f;
