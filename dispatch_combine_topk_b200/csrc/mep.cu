@@ -530,9 +530,9 @@ mep_status_t mep_update_expert(const int32_t *expert_ids, const int32_t *eplb_ta
     const int threads = 256;
     int64_t g = (BS * K + threads - 1) / threads;
     int cap = sm_count() * 8;
-    mep::k_update_expert<<<(unsigned)(g < cap ? g : cap), threads, 0, s>>>(
-        expert_ids, eplb_table, expert_scales, pruning_threshold, active_mask, BS, BS, local_rank_id, K,
-        n_experts, F, world_size, balance_mode, balanced_expert_ids, balanced_active_mask);
+    launch_pdl(mep::k_update_expert, dim3((unsigned)(g < cap ? g : cap)), dim3(threads), 0, s, expert_ids, eplb_table,
+               expert_scales, pruning_threshold, active_mask, BS, BS, local_rank_id, K, n_experts, F, world_size,
+               balance_mode, balanced_expert_ids, balanced_active_mask);
     return launched();
 }
 
@@ -558,9 +558,9 @@ mep_status_t mep_update_expert_ranks(const int32_t *expert_ids, const int32_t *e
     const int64_t rows = BS * world_size;
     int64_t g = (rows * K + threads - 1) / threads;
     int cap = sm_count() * 8;
-    mep::k_update_expert<<<(unsigned)(g < cap ? g : cap), threads, 0, s>>>(
-        expert_ids, eplb_table, expert_scales, pruning_threshold, active_mask, rows, BS, 0, K, n_experts, F,
-        world_size, balance_mode, balanced_expert_ids, balanced_active_mask);
+    launch_pdl(mep::k_update_expert, dim3((unsigned)(g < cap ? g : cap)), dim3(threads), 0, s, expert_ids, eplb_table,
+               expert_scales, pruning_threshold, active_mask, rows, BS, (int64_t)0, K, n_experts, F, world_size,
+               balance_mode, balanced_expert_ids, balanced_active_mask);
     return launched();
 }
 

@@ -31,6 +31,8 @@ __global__ void k_update_expert(const int32_t *__restrict__ ids, const int32_t *
                                 int64_t mode, int32_t *__restrict__ out_ids,
                                 uint8_t *__restrict__ out_mask)
 {
+    pdl_wait();
+    pdl_launch_dependents();
     const int64_t slots = rows * K;
     for (int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; n < slots;
          n += (int64_t)gridDim.x * blockDim.x) {
