@@ -18,11 +18,11 @@ from gpu_helpers import bits, dev, gpu_plan_balanced
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("K", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("K", [1, 2, 3, 4, 8, 16, 32])
 @pytest.mark.parametrize("H", [8, 12, 64, 4096, 4100, 7168, 12288, 16384, 16388, 20000, 7])
 def test_smooth_dispatch_matches_oracle(K, H):
     rng = np.random.default_rng(K * 7 + H)
-    T, E = 23, 10
+    T, E = 23, max(10, K + 3)
     x = (torch.randn((T, H), generator=torch.Generator().manual_seed(H)) * 4).to(torch.bfloat16)
     ids = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
     rows = T * K + 2
