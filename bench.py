@@ -878,6 +878,121 @@ def time_route(mep, rt, args, dev, stream, pg, steps):
     }
 
 
+class EPRoute:
+    """A balanced bf16 workload routed as R expert-parallel ranks, each with its own
+    tokens and its own receive buffer (a separate allocation on this GPU, reached through
+    a device table of the R buffers' addresses, as peer mappings would be across GPUs).
+    Plan: per source rank its histogram, then (the all-gather: every rank's row is
+    already on this GPU) its share of the plan (mep_plan_rank). Dispatch: every source
+    rank stores its rows into the ranks' buffers (mep_dispatch_ranks). Combine: every
+    rank sums its tokens from the buffers they went to (mep_combine_ranks). The identity
+    expert. The R ranks' calls of a phase run on R streams of their own, as R GPUs
+    would run them side by side, and the phase ends when all have."""
+
+    def __init__(self, mep, w, dev):
+        if w.quant or w.mapping:
+            raise ValueError("the expert-parallel layout is measured on the balanced bf16 workloads")
+        self.mep, self.w, self.dev = mep, w, dev
+        ids, gates = synth.router(w)
+        SK = w.S * w.K
+        self.ids = torch.from_numpy(ids).to(dev).view(w.R, SK)
+        self.gates = torch.from_numpy(gates).to(dev).view(w.R, SK)
+        self.x = synth.hidden(w).to(dev)
+        self.bufs = [torch.empty((SK, w.H), dtype=torch.bfloat16, device=dev) for _ in range(w.R)]
+        self.table = mep.rank_pointer_table(self.bufs, dev)
+        self.hist = torch.empty((w.R, w.E), dtype=torch.int32, device=dev)
+        self.rps = [mep.RankPlanBuffers.allocate(w.R, w.E, w.S, w.K, dev) for _ in range(w.R)]
+        self.out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
+        self.streams = [torch.cuda.Stream(dev) for _ in range(w.R)]
+
+    def _side_by_side(self, s, call):
+        """call(r, stream) for every rank on its own stream, after the work already on s;
+        s then waits for all of them."""
+        start = torch.cuda.Event()
+        start.record(s)
+        done = []
+        for r, st in enumerate(self.streams):
+            st.wait_event(start)
+            call(r, st)
+            e = torch.cuda.Event()
+            e.record(st)
+            done.append(e)
+        for e in done:
+            s.wait_event(e)
+
+    def phases(self):
+        return [("plan", self.plan), ("dispatch", self.dispatch), ("combine", self.combine)]
+
+    def plan(self, s):
+        w, mep = self.w, self.mep
+        self._side_by_side(s, lambda r, st: mep.mep_histogram(self.ids[r], w.E, self.hist[r], stream=st))
+        self._side_by_side(s, lambda r, st: mep.mep_plan_rank(self.ids[r], self.hist, w.R, w.E, w.S, w.K, r,
+                                                              self.rps[r], stream=st))
+        return w.R * 5           # a histogram, then k_tile_count, k_scan_cols, k_source_meta, k_rank
+
+    def dispatch(self, s):
+        w = self.w
+        self._side_by_side(s, lambda r, st: self.mep.mep_dispatch_ranks(
+            self.x[r * w.S:(r + 1) * w.S], self.rps[r].pos, w.K, self.table, w.S * w.K, stream=st))
+        return w.R
+
+    def combine(self, s):
+        w = self.w
+        self._side_by_side(s, lambda r, st: self.mep.mep_combine_ranks(
+            self.table, self.rps[r].pos, self.gates[r], w.K, w.S * w.K, self.out[r * w.S:(r + 1) * w.S], stream=st))
+        return w.R
+
+    def step(self, s, ev=None):
+        n = 0
+        for i, (_, run) in enumerate(self.phases()):
+            if ev is not None:
+                ev[i].record(s)
+            n += run(s)
+        if ev is not None:
+            ev[-1].record(s)
+        return n
+
+    def result_ok(self) -> bool:
+        """The identity expert with gates summing to 1 returns every token's row."""
+        return torch.equal(self.out.float(), self.x.float())
+
+    def kernel_name(self, step: str) -> str:
+        return {"plan": "k_rank", "dispatch": "k_dispatch_ranks_warp", "combine": "k_combine_ranks_v8"}[step]
+
+    def working_set_bytes(self) -> int:
+        return self.x.numel() * 2 * 2 + sum(b.numel() * 2 for b in self.bufs) + self.ids.numel() * 8
+
+    def bytes(self):
+        """Algorithmic bytes of the phases: the same rows move as on one buffer."""
+        w = self.w
+        row = 2 * w.H
+        return {"plan": 16 * w.N, "dispatch": w.T * row + w.N * row + 4 * w.N,
+                "combine": w.N * row + w.T * row + 8 * w.N}
+
+
+def per_workload_ep_entry(mep, name, args, dev, stream, pg, peak, peak_kind):
+    """The per_workload entry of a balanced bf16 workload in the expert-parallel layout
+    (EPRoute): R receive buffers of their own, reached through a table of addresses."""
+    w = synth.get(name)
+    rt = EPRoute(mep, w, dev)
+    steps = max(5, min(args.steps, 20))
+    tm = time_route(mep, rt, args, dev, stream, pg, steps)
+    roof, dc = roofline_of(rt, tm, peak, peak_kind)
+    entry = {
+        "workload": w.name + "_ep", "layout": "R receive buffers of their own through a device address table "
+        "(mep_plan_rank, mep_dispatch_ranks, mep_combine_ranks); the all-gather of the histograms is a no-op on "
+        "one GPU", "token_slots": w.N, "ms_per_step": tm["ms_step"],
+        "token_slots_per_s": w.N / (tm["ms_step"] * 1e-3), "step_ms": tm["step_ms"],
+        "breakdown_ms": tm["t_phase"], "dispatch_combine": dc,
+        "roofline": {k: roof[k] for k in ("kernel", "phase", "achieved", "frac", "algorithmic_bytes", "traffic")},
+        "launches_per_step": tm["launches"] // steps, "result_check": rt.result_ok(), "flush": tm["flush"],
+        "clocks": tm["clocks"],
+    }
+    del rt
+    torch.cuda.empty_cache()
+    return entry
+
+
 def roofline_of(rt, tm, peak, peak_kind):
     """The dominant HBM-bound phase (the slower of the moving phases) against the peak,
     with its algorithmic bytes; and the dispatch+combine rate over all moving phases."""
@@ -1017,6 +1132,10 @@ def run_gpu(args, w):
     others = [n for n in args.per_workload.split(",") if n] if args.per_workload != "none" else []
     per = {}
     for name in others:
+        if name.endswith("_ep"):
+            e = per_workload_ep_entry(mep, name[:-3], args, dev, stream, pg, peak, peak_kind)
+            per[e["workload"]] = e
+            continue
         if synth.get(name).name == w.name:
             continue
         e = per_workload_entry(mep, name, args, dev, stream, pg, peak, peak_kind)
@@ -1036,9 +1155,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="mep", choices=["mep", "reference"])
     ap.add_argument("--workload", default="int8")
-    ap.add_argument("--per-workload", default="tiny,r8,map,skew",
+    ap.add_argument("--per-workload", default="tiny,r8,map,skew,r8_ep",
                     help="comma-separated workloads measured after the main one and reported under "
-                         "per_workload (graph replays, no end-to-end leg); 'none' to skip")
+                         "per_workload (graph replays, no end-to-end leg); a name ending in _ep routes that "
+                         "balanced bf16 workload in the expert-parallel layout; 'none' to skip")
     ap.add_argument("--ref-div", type=int, default=16,
                     help="--impl reference: the oracle routes S/ref_div tokens per rank per step")
     ap.add_argument("--cpu-div", type=int, default=1,

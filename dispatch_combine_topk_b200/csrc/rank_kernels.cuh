@@ -153,6 +153,41 @@ k_combine_ranks_v8(const uint4 *const *__restrict__ y, const int32_t *__restrict
             if (b) mine = b + local * H8;
             g_mine = gates[t * K + lane];
         }
+        if constexpr (kFixed) {
+            // the slots' rows and gates once per token, in registers
+            const uint4 *rowp[KC];
+            float g[KC];
+#pragma unroll
+            for (int k = 0; k < KC; k++) {
+                rowp[k] = (const uint4 *)__shfl_sync(0xffffffffu, (unsigned long long)mine, k);
+                g[k] = __shfl_sync(0xffffffffu, g_mine, k);
+            }
+            for (int64_t c = lane; c < H8; c += 32) {
+                float acc[8];
+#pragma unroll
+                for (int j = 0; j < 8; j++) acc[j] = 0.0f;
+                uint4 v[KC];
+#pragma unroll
+                for (int k = 0; k < KC; k++) v[k] = rowp[k] ? ld_stream(rowp[k] + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int k = 0; k < KC; k++) {
+                    if (!rowp[k]) continue;
+                    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        acc[2 * j] = __fadd_rn(acc[2 * j], __fmul_rn(g[k], bf16lo(w[j])));
+                        acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], __fmul_rn(g[k], bf16hi(w[j])));
+                    }
+                }
+                uint4 o;
+                o.x = pack_bf16x2(acc[0], acc[1]);
+                o.y = pack_bf16x2(acc[2], acc[3]);
+                o.z = pack_bf16x2(acc[4], acc[5]);
+                o.w = pack_bf16x2(acc[6], acc[7]);
+                st_v4(out + t * H8 + c, o);
+            }
+            continue;
+        }
         for (int64_t base = 0; base < H8; base += 32) {
             const int64_t c = base + lane;
             float acc[8];
