@@ -879,7 +879,7 @@ def time_route(mep, rt, args, dev, stream, pg, steps):
 
 
 class EPRoute:
-    """A balanced bf16 workload routed as R expert-parallel ranks, each with its own
+    """A balanced workload (bf16, or int8 rows with scales) routed as R expert-parallel ranks, each with its own
     tokens and its own receive buffer (a separate allocation on this GPU, reached through
     a device table of the R buffers' addresses, as peer mappings would be across GPUs).
     Plan: per source rank its histogram, then (the all-gather: every rank's row is
@@ -890,16 +890,20 @@ class EPRoute:
     would run them side by side, and the phase ends when all have."""
 
     def __init__(self, mep, w, dev):
-        if w.quant or w.mapping:
-            raise ValueError("the expert-parallel layout is measured on the balanced bf16 workloads")
+        if w.mapping:
+            raise ValueError("the expert-parallel layout is measured on the balanced workloads")
         self.mep, self.w, self.dev = mep, w, dev
         ids, gates = synth.router(w)
         SK = w.S * w.K
         self.ids = torch.from_numpy(ids).to(dev).view(w.R, SK)
         self.gates = torch.from_numpy(gates).to(dev).view(w.R, SK)
         self.x = synth.hidden(w).to(dev)
-        self.bufs = [torch.empty((SK, w.H), dtype=torch.bfloat16, device=dev) for _ in range(w.R)]
+        dt = torch.int8 if w.quant else torch.bfloat16
+        self.bufs = [torch.empty((SK, w.H), dtype=dt, device=dev) for _ in range(w.R)]
         self.table = mep.rank_pointer_table(self.bufs, dev)
+        self.quant = 1 if w.quant else 0
+        self.scales = [torch.empty(SK, dtype=torch.float32, device=dev) for _ in range(w.R)] if w.quant else None
+        self.scale_table = mep.rank_pointer_table(self.scales, dev) if w.quant else None
         self.hist = torch.empty((w.R, w.E), dtype=torch.int32, device=dev)
         self.rps = [mep.RankPlanBuffers.allocate(w.R, w.E, w.S, w.K, dev) for _ in range(w.R)]
         self.out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=dev)
@@ -933,13 +937,15 @@ class EPRoute:
     def dispatch(self, s):
         w = self.w
         self._side_by_side(s, lambda r, st: self.mep.mep_dispatch_ranks(
-            self.x[r * w.S:(r + 1) * w.S], self.rps[r].pos, w.K, self.table, w.S * w.K, stream=st))
+            self.x[r * w.S:(r + 1) * w.S], self.rps[r].pos, w.K, self.table, w.S * w.K, quant=self.quant,
+            scale_table=self.scale_table, stream=st))
         return w.R
 
     def combine(self, s):
         w = self.w
         self._side_by_side(s, lambda r, st: self.mep.mep_combine_ranks(
-            self.table, self.rps[r].pos, self.gates[r], w.K, w.S * w.K, self.out[r * w.S:(r + 1) * w.S], stream=st))
+            self.table, self.rps[r].pos, self.gates[r], w.K, w.S * w.K, self.out[r * w.S:(r + 1) * w.S],
+            quant=self.quant, scale_table=self.scale_table, stream=st))
         return w.R
 
     def step(self, s, ev=None):
@@ -953,25 +959,43 @@ class EPRoute:
         return n
 
     def result_ok(self) -> bool:
-        """The identity expert with gates summing to 1 returns every token's row."""
-        return torch.equal(self.out.float(), self.x.float())
+        """The identity expert with gates summing to 1 returns every token's row (bf16);
+        on int8 rows, every token whose slots carry the same codes returns their
+        dequantised row (checked on the first slot's buffer row)."""
+        if not self.quant:
+            return torch.equal(self.out.float(), self.x.float())
+        w = self.w
+        pos0 = torch.stack([rp.pos.view(w.S, w.K)[:, 0] for rp in self.rps]).view(-1).long()
+        SK = w.S * w.K
+        rank, local = pos0 // SK, pos0 % SK
+        codes = torch.stack([self.bufs[int(r)][int(l)] for r, l in zip(rank[:64].tolist(), local[:64].tolist())])
+        scale = torch.stack([self.scales[int(r)][int(l)] for r, l in zip(rank[:64].tolist(), local[:64].tolist())])
+        ref = torch.empty((64, w.H), dtype=torch.bfloat16, device=self.dev)
+        self.mep.mep_dequantize(codes, scale, ref)
+        return torch.equal(self.out[:64].float(), ref.float())
 
     def kernel_name(self, step: str) -> str:
+        if self.quant:
+            return {"plan": "k_rank", "dispatch": "k_dispatch_ranks_int8", "combine": "k_combine_ranks_int8"}[step]
         return {"plan": "k_rank", "dispatch": "k_dispatch_ranks_warp", "combine": "k_combine_ranks_v8"}[step]
 
     def working_set_bytes(self) -> int:
-        return self.x.numel() * 2 * 2 + sum(b.numel() * 2 for b in self.bufs) + self.ids.numel() * 8
+        return (self.x.numel() * 2 * 2 + sum(b.numel() * b.element_size() for b in self.bufs) +
+                self.ids.numel() * 8)
 
     def bytes(self):
         """Algorithmic bytes of the phases: the same rows move as on one buffer."""
         w = self.w
         row = 2 * w.H
+        if self.quant:
+            return {"plan": 16 * w.N, "dispatch": w.T * row + w.N * w.H + 8 * w.N,
+                    "combine": w.N * w.H + 4 * w.N + w.T * row + 8 * w.N}
         return {"plan": 16 * w.N, "dispatch": w.T * row + w.N * row + 4 * w.N,
                 "combine": w.N * row + w.T * row + 8 * w.N}
 
 
 def per_workload_ep_entry(mep, name, args, dev, stream, pg, peak, peak_kind):
-    """The per_workload entry of a balanced bf16 workload in the expert-parallel layout
+    """The per_workload entry of a balanced workload in the expert-parallel layout
     (EPRoute): R receive buffers of their own, reached through a table of addresses."""
     w = synth.get(name)
     rt = EPRoute(mep, w, dev)
@@ -1155,10 +1179,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="mep", choices=["mep", "reference"])
     ap.add_argument("--workload", default="int8")
-    ap.add_argument("--per-workload", default="tiny,r8,map,skew,r8_ep",
+    ap.add_argument("--per-workload", default="tiny,r8,map,skew,r8_ep,int8_ep",
                     help="comma-separated workloads measured after the main one and reported under "
                          "per_workload (graph replays, no end-to-end leg); a name ending in _ep routes that "
-                         "balanced bf16 workload in the expert-parallel layout; 'none' to skip")
+                         "balanced workload in the expert-parallel layout; 'none' to skip")
     ap.add_argument("--ref-div", type=int, default=16,
                     help="--impl reference: the oracle routes S/ref_div tokens per rank per step")
     ap.add_argument("--cpu-div", type=int, default=1,

@@ -257,6 +257,30 @@ k_combine_ranks_int8(const uint4 *const *__restrict__ yq, const float *const *__
             g_mine = gates[t * K + lane];
         }
         uint4 *dst = out + t * 2 * H16;
+        if constexpr (kFixed) {
+            // the slots' rows, gates and scales once per token, in registers
+            const uint4 *rowp[KC];
+            float g[KC], sc[KC];
+#pragma unroll
+            for (int k = 0; k < KC; k++) {
+                rowp[k] = (const uint4 *)__shfl_sync(0xffffffffu, (unsigned long long)mine, k);
+                g[k] = __shfl_sync(0xffffffffu, g_mine, k);
+                sc[k] = __shfl_sync(0xffffffffu, s_mine, k);
+            }
+            for (int64_t c = lane; c < H16; c += 32) {
+                float2 acc[8];
+#pragma unroll
+                for (int j = 0; j < 8; j++) acc[j] = make_float2(0.0f, 0.0f);
+                uint4 v[KC];
+#pragma unroll
+                for (int k = 0; k < KC; k++) v[k] = rowp[k] ? ld_stream(rowp[k] + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int k = 0; k < KC; k++)
+                    if (rowp[k]) add_int8_x16(acc, v[k], g[k], sc[k]);
+                store_bf16x16(dst + 2 * c, acc);
+            }
+            continue;
+        }
         for (int64_t base = 0; base < H16; base += 32) {
             const int64_t c = base + lane;
             float2 acc[8];
