@@ -590,12 +590,9 @@ mep_status_t mep_dispatch(const uint16_t *x, const int32_t *pos, int64_t T, int3
     } else {
         const size_t staged_smem = (size_t)mep::kDispatchSmemHead + 4 * (size_t)H * 2 + 2 * (size_t)H;
         if (H % 16 == 0 && aligned(x, 16) && aligned(recv, 16) && staged_smem <= (size_t)kBulkSmemMax) {
-            int per_sm = 0;
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mep::k_dispatch_int8_staged<4, 128>, 128,
-                                                          staged_smem);
-            per_sm = per_sm < 1 ? 1 : (per_sm > 3 ? 3 : per_sm);
-            launch_pdl(mep::k_dispatch_int8_staged<4, 128>, dim3((unsigned)token_grid(T, per_sm)), dim3(128), staged_smem, s,
-                       x, pos, T, (int)K, H, rows, (int8_t *)recv, recv_scale);
+            // CTAs of kStagedChunk consecutive tokens, as many as the tokens need
+            launch_pdl(mep::k_dispatch_int8_staged<4, 128>, dim3((unsigned)mep::ceil_div(T, mep::kStagedChunk)),
+                       dim3(128), staged_smem, s, x, pos, T, (int)K, H, rows, (int8_t *)recv, recv_scale);
         } else if (H % 8 == 0 && aligned(x, 16) && aligned(recv, 8)) {
             mep::k_dispatch_int8<<<grid, 256, 0, s>>>((const uint4 *)x, pos, T, K, H / 8, rows,
                                                       (uint2 *)recv, recv_scale);

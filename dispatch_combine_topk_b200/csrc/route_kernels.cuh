@@ -276,11 +276,16 @@ k_dispatch_int8(const uint4 *__restrict__ x, const int32_t *__restrict__ pos, in
 // indices, a reduction buffer).
 constexpr int kDispatchSmemHead = 2048;
 
+// Tokens per CTA of k_dispatch_int8_staged: a grid of CTAs for kStagedChunk consecutive
+// tokens each, handed to SMs as they free up (2.6% faster than a resident grid striding
+// over the tokens; 8 and 32 tokens measured slower).
+constexpr int kStagedChunk = 16;
+
 // Per-token dynamic int8 staged through shared memory (the default int8 path).
 //
-// kThreads threads per CTA, several CTAs per SM, tokens strided over CTAs. Warp 0 keeps
-// a ring of kStages bf16 rows filled by bulk loads (mbarrier completion) ahead of the
-// token being quantised. For each token all threads reduce amax over the staged row,
+// kThreads threads per CTA, several CTAs per SM, kStagedChunk consecutive tokens per
+// CTA. Warp 0 keeps a ring of kStages bf16 rows filled by bulk loads (mbarrier
+// completion) ahead of the token being quantised. For each token all threads reduce amax over the staged row,
 // quantise it into one of two int8 row buffers, and lanes k < K of warp 0 bulk-store
 // the codes to the row of slot k and write the scale. The int8 buffer of token i is
 // reused at token i+2, after its stores have finished reading it.
@@ -309,8 +314,9 @@ k_dispatch_int8_staged(const uint16_t *__restrict__ x, const int32_t *__restrict
     __syncthreads();
     pdl_wait();                       // the barriers' set-up above touches only this CTA's memory
     pdl_launch_dependents();
-    const int64_t n = blockIdx.x < T ? (T - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-    auto token = [&](int64_t i) { return (int64_t)blockIdx.x + i * gridDim.x; };
+    const int64_t t_lo = (int64_t)blockIdx.x * kStagedChunk;
+    const int64_t n = t_lo < T ? (T - t_lo < kStagedChunk ? T - t_lo : kStagedChunk) : 0;
+    auto token = [&](int64_t i) { return t_lo + i; };
     auto fetch = [&](int64_t i) {   // warp 0 only
         const int s = (int)(i % kStages);
         const int64_t t = token(i);
