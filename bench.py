@@ -120,9 +120,9 @@ TRAFFIC = {
     ("k_combine_v8", "r8_e64_s4096_k8_h7168"): {
         "bytes": 4 * 1005.611e6, "src": "75f948c1d2f4d491", "case_S": 1024, "case_mb": 1005.611},
     ("k_dispatch_int8_staged", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1114.960e6, "src": "0158b32e901926e8", "case_S": 512, "case_mb": 1114.960},
+        "bytes": 16 * 1116.515e6, "src": "0909085f8f5d1cb1", "case_S": 512, "case_mb": 1116.515},
     ("k_combine_int8_warp", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1117.223e6, "src": "528f2068b9109630", "case_S": 512, "case_mb": 1117.223},
+        "bytes": 16 * 1117.508e6, "src": "528f2068b9109630", "case_S": 512, "case_mb": 1117.508},
     ("k_dispatch_warp", "skew_r64_e512_s2048_k8_h4096"): {
         "bytes": 4 * 2357.469e6, "src": "f2dc9831a61b7e83", "case_S": 512, "case_mb": 2357.469},
     ("k_combine_v8", "skew_r64_e512_s2048_k8_h4096"): {
