@@ -186,43 +186,43 @@ k_combine_ranks_v8(const uint4 *const *__restrict__ y, const int32_t *__restrict
                 o.w = pack_bf16x2(acc[6], acc[7]);
                 st_v4(out + t * H8 + c, o);
             }
-            continue;
-        }
-        for (int64_t base = 0; base < H8; base += 32) {
-            const int64_t c = base + lane;
-            float acc[8];
+        } else {
+            for (int64_t base = 0; base < H8; base += 32) {
+                const int64_t c = base + lane;
+                float acc[8];
 #pragma unroll
-            for (int j = 0; j < 8; j++) acc[j] = 0.0f;
+                for (int j = 0; j < 8; j++) acc[j] = 0.0f;
 #pragma unroll 1
-            for (int k0 = 0; k0 < K; k0 += kSlots) {
-                const uint4 *rowp[kSlots];
-                float g[kSlots];
-                uint4 v[kSlots];
+                for (int k0 = 0; k0 < K; k0 += kSlots) {
+                    const uint4 *rowp[kSlots];
+                    float g[kSlots];
+                    uint4 v[kSlots];
 #pragma unroll
-                for (int k = 0; k < kSlots; k++) {
-                    const bool in = k0 + k < K;
-                    rowp[k] = in ? (const uint4 *)__shfl_sync(0xffffffffu, (unsigned long long)mine, k0 + k) : nullptr;
-                    g[k] = in ? __shfl_sync(0xffffffffu, g_mine, k0 + k) : 0.0f;
-                    v[k] = (rowp[k] && c < H8) ? ld_stream(rowp[k] + c) : make_uint4(0, 0, 0, 0);
-                }
+                    for (int k = 0; k < kSlots; k++) {
+                        const bool in = k0 + k < K;
+                        rowp[k] = in ? (const uint4 *)__shfl_sync(0xffffffffu, (unsigned long long)mine, k0 + k) : nullptr;
+                        g[k] = in ? __shfl_sync(0xffffffffu, g_mine, k0 + k) : 0.0f;
+                        v[k] = (rowp[k] && c < H8) ? ld_stream(rowp[k] + c) : make_uint4(0, 0, 0, 0);
+                    }
 #pragma unroll
-                for (int k = 0; k < kSlots; k++) {
-                    if (!rowp[k]) continue;
-                    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+                    for (int k = 0; k < kSlots; k++) {
+                        if (!rowp[k]) continue;
+                        const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        acc[2 * j] = __fadd_rn(acc[2 * j], __fmul_rn(g[k], bf16lo(w[j])));
-                        acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], __fmul_rn(g[k], bf16hi(w[j])));
+                        for (int j = 0; j < 4; j++) {
+                            acc[2 * j] = __fadd_rn(acc[2 * j], __fmul_rn(g[k], bf16lo(w[j])));
+                            acc[2 * j + 1] = __fadd_rn(acc[2 * j + 1], __fmul_rn(g[k], bf16hi(w[j])));
+                        }
                     }
                 }
-            }
-            if (c < H8) {
-                uint4 o;
-                o.x = pack_bf16x2(acc[0], acc[1]);
-                o.y = pack_bf16x2(acc[2], acc[3]);
-                o.z = pack_bf16x2(acc[4], acc[5]);
-                o.w = pack_bf16x2(acc[6], acc[7]);
-                st_v4(out + t * H8 + c, o);
+                if (c < H8) {
+                    uint4 o;
+                    o.x = pack_bf16x2(acc[0], acc[1]);
+                    o.y = pack_bf16x2(acc[2], acc[3]);
+                    o.z = pack_bf16x2(acc[4], acc[5]);
+                    o.w = pack_bf16x2(acc[6], acc[7]);
+                    st_v4(out + t * H8 + c, o);
+                }
             }
         }
     }
@@ -279,31 +279,31 @@ k_combine_ranks_int8(const uint4 *const *__restrict__ yq, const float *const *__
                     if (rowp[k]) add_int8_x16(acc, v[k], g[k], sc[k]);
                 store_bf16x16(dst + 2 * c, acc);
             }
-            continue;
-        }
-        for (int64_t base = 0; base < H16; base += 32) {
-            const int64_t c = base + lane;
-            float2 acc[8];
+        } else {
+            for (int64_t base = 0; base < H16; base += 32) {
+                const int64_t c = base + lane;
+                float2 acc[8];
 #pragma unroll
-            for (int j = 0; j < 8; j++) acc[j] = make_float2(0.0f, 0.0f);
+                for (int j = 0; j < 8; j++) acc[j] = make_float2(0.0f, 0.0f);
 #pragma unroll 1
-            for (int k0 = 0; k0 < K; k0 += kSlots) {
-                const uint4 *rowp[kSlots];
-                float g[kSlots], sc[kSlots];
-                uint4 v[kSlots];
+                for (int k0 = 0; k0 < K; k0 += kSlots) {
+                    const uint4 *rowp[kSlots];
+                    float g[kSlots], sc[kSlots];
+                    uint4 v[kSlots];
 #pragma unroll
-                for (int k = 0; k < kSlots; k++) {
-                    const bool in = k0 + k < K;
-                    rowp[k] = in ? (const uint4 *)__shfl_sync(0xffffffffu, (unsigned long long)mine, k0 + k) : nullptr;
-                    g[k] = in ? __shfl_sync(0xffffffffu, g_mine, k0 + k) : 0.0f;
-                    sc[k] = in ? __shfl_sync(0xffffffffu, s_mine, k0 + k) : 0.0f;
-                    v[k] = (rowp[k] && c < H16) ? ld_stream(rowp[k] + c) : make_uint4(0, 0, 0, 0);
+                    for (int k = 0; k < kSlots; k++) {
+                        const bool in = k0 + k < K;
+                        rowp[k] = in ? (const uint4 *)__shfl_sync(0xffffffffu, (unsigned long long)mine, k0 + k) : nullptr;
+                        g[k] = in ? __shfl_sync(0xffffffffu, g_mine, k0 + k) : 0.0f;
+                        sc[k] = in ? __shfl_sync(0xffffffffu, s_mine, k0 + k) : 0.0f;
+                        v[k] = (rowp[k] && c < H16) ? ld_stream(rowp[k] + c) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int k = 0; k < kSlots; k++)
+                        if (rowp[k]) add_int8_x16(acc, v[k], g[k], sc[k]);
                 }
-#pragma unroll
-                for (int k = 0; k < kSlots; k++)
-                    if (rowp[k]) add_int8_x16(acc, v[k], g[k], sc[k]);
+                if (c < H16) store_bf16x16(dst + 2 * c, acc);
             }
-            if (c < H16) store_bf16x16(dst + 2 * c, acc);
         }
     }
 }
