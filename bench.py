@@ -392,6 +392,9 @@ class Route:
                     # per-expert smoothing scales, one per channel: exp(N(0, 0.25^2)), seeded
                     g = torch.Generator().manual_seed(w.seed * 1000 + 7)
                     self.smooth_scales = torch.exp(0.25 * torch.randn((w.E, w.H), generator=g)).to(dev)
+                    # scratch of the sorted slot list
+                    self.smooth_ws = torch.empty(max(1, mep.mep_dispatch_int8_smooth_workspace_size(w.T, w.K)),
+                                                 dtype=torch.uint8, device=dev)
             else:
                 self.recv = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=dev)
                 self.y = self.recv
@@ -432,8 +435,10 @@ class Route:
         if self.dedup:
             pos, recv, scale = self.db.dsend, self.sent, self.sent_scale
         if w.quant and self.smooth:
-            self.mep.mep_dispatch_int8_smooth(self.x, self.ids, pos, w.K, self.smooth_scales, recv, scale,
-                                              stream=s)
+            # the slots sorted by expert within chunks of tokens, then quantised along that list
+            self.mep.mep_dispatch_int8_smooth_grouped(self.x, self.ids, pos, w.K, self.smooth_scales, recv, scale,
+                                                      workspace=self.smooth_ws, stream=s)
+            return 2 if self.smooth_grouped() else 1
         elif w.quant:
             self.mep.mep_dispatch(self.x, pos, w.K, recv, scale, quant=1, stream=s)
         else:
@@ -493,6 +498,12 @@ class Route:
             return torch.equal(self.out.float(), y_first.float())
         return torch.equal(self.out.float(), self.x.float())
 
+    def smooth_grouped(self) -> bool:
+        """Whether mep_dispatch_int8_smooth_grouped sorts the slots on this workload's
+        shapes (two launches) rather than running the per-token kernel."""
+        w = self.w
+        return w.H % 4 == 0 and w.H <= 8192 and w.E <= 6000
+
     def kernel_name(self, step: str) -> str:
         """The library kernel that runs a step on this workload's shapes."""
         w = self.w
@@ -507,6 +518,8 @@ class Route:
         if step == "expand":
             return "k_expand_warp" if w.H % 16 == 0 or (not w.quant and w.H % 8 == 0) else "k_expand_bytes"
         if w.quant and self.smooth:
+            if self.smooth_grouped():
+                return "k_dispatch_int8_smooth_grouped"
             if w.H % 4 == 0 and w.H // 4 <= 16 * 256:
                 return "k_dispatch_int8_smooth_k"
             return "k_dispatch_int8_smooth_scalar"
@@ -1198,7 +1211,7 @@ def main():
                          "receiving side (mep_dedup_plan, mep_expand)")
     ap.add_argument("--smooth", type=int, default=0,
                     help="1 (int8 workload): per-expert smoothing scales before the int8 "
-                         "quantisation, codes and scale per slot (mep_dispatch_int8_smooth)")
+                         "quantisation, codes and scale per slot (mep_dispatch_int8_smooth_grouped)")
     ap.add_argument("--epilogue", default="none", choices=["none", "add_rmsnorm"],
                     help="add_rmsnorm: combine fused with residual add + RMSNorm")
     ap.add_argument("--ffn-dim", type=int, default=0,

@@ -92,6 +92,10 @@ def lib() -> ctypes.CDLL:
         L.mep_grad_reduce.argtypes = [P, P, P, i32, i32, i32, i64, P]
         L.mep_dispatch_int8_smooth.argtypes = [P, P, P, i64, i32, i64, P, i32, P, P, i64, P]
         L.mep_update_expert_ranks.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i64, P, P, P]
+        L.mep_dispatch_int8_smooth_workspace_size.argtypes = [i64, i32]
+        L.mep_dispatch_int8_smooth_workspace_size.restype = ctypes.c_size_t
+        L.mep_dispatch_int8_smooth_grouped.argtypes = [P, P, P, i64, i32, i64, P, i32, P, P, i64, P,
+                                                       ctypes.c_size_t, P]
         L.mep_dedup_workspace_size.argtypes = [i32, i32, i32]
         L.mep_dedup_workspace_size.restype = ctypes.c_size_t
         L.mep_dedup_plan.argtypes = [P, P, i32, i32, i32, P, P, P, P, P, P, ctypes.c_size_t, P]
@@ -108,7 +112,8 @@ def lib() -> ctypes.CDLL:
         for f in ["mep_get_error", "mep_histogram", "mep_plan", "mep_update_expert",
                   "mep_dispatch", "mep_dequantize", "mep_combine", "mep_combine_int8",
                   "mep_combine_add_rmsnorm", "mep_prefetch_plan", "mep_prefetch_weights",
-                  "mep_grad_reduce", "mep_dispatch_int8_smooth", "mep_update_expert_ranks",
+                  "mep_grad_reduce", "mep_dispatch_int8_smooth", "mep_dispatch_int8_smooth_grouped",
+                  "mep_update_expert_ranks",
                   "mep_dedup_plan", "mep_expand", "mep_route_host", "mep_stream_synchronize_timeout",
                   "mep_maxvio", "mep_plan_rank", "mep_plan_static_ws", "mep_dispatch_ranks",
                   "mep_combine_ranks"]:
@@ -587,6 +592,37 @@ def mep_dispatch_int8_smooth(x: torch.Tensor, ids: torch.Tensor, pos: torch.Tens
                                         _ptr(recv_scale, torch.float32, "recv_scale"), recv.shape[0],
                                         _stream(stream))
     _ok(rc, "mep_dispatch_int8_smooth")
+    return recv, recv_scale
+
+
+def mep_dispatch_int8_smooth_workspace_size(T: int, K: int) -> int:
+    """Bytes of scratch mep_dispatch_int8_smooth_grouped needs (the sorted slot list)."""
+    return int(lib().mep_dispatch_int8_smooth_workspace_size(T, K))
+
+
+def mep_dispatch_int8_smooth_grouped(x: torch.Tensor, ids: torch.Tensor, pos: torch.Tensor, K: int,
+                                     smooth: torch.Tensor, recv: torch.Tensor, recv_scale: torch.Tensor,
+                                     workspace: Optional[torch.Tensor] = None, stream=None):
+    """mep_dispatch_int8_smooth with the slots taken in expert order within chunks of
+    tokens (same codes and scales). ``workspace``: a uint8 device tensor of at least
+    mep_dispatch_int8_smooth_workspace_size(T, K) bytes; allocated here when None."""
+    T, H = x.shape
+    _need(ids.numel() == T * K and pos.numel() == T * K, "ids and pos must hold T*K slots")
+    _need(smooth.dim() == 2 and smooth.shape[1] == H, "smooth must be [experts, H]")
+    _need(recv.dim() == 2 and recv.shape[1] == H and _n(recv_scale) >= recv.shape[0],
+          "recv [rows, H] and recv_scale [rows] needed")
+    need = mep_dispatch_int8_smooth_workspace_size(T, K)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _need(workspace.numel() * workspace.element_size() >= need, "workspace too small")
+    rc = lib().mep_dispatch_int8_smooth_grouped(_ptr(x, torch.bfloat16, "x"), _ptr(ids, torch.int32, "ids"),
+                                                _ptr(pos, torch.int32, "pos"), T, K, H,
+                                                _ptr(smooth, torch.float32, "smooth"), smooth.shape[0],
+                                                _ptr(recv, torch.int8, "recv"),
+                                                _ptr(recv_scale, torch.float32, "recv_scale"), recv.shape[0],
+                                                _ptr(workspace, None, "workspace"),
+                                                workspace.numel() * workspace.element_size(), _stream(stream))
+    _ok(rc, "mep_dispatch_int8_smooth_grouped")
     return recv, recv_scale
 
 

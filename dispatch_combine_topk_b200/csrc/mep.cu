@@ -23,6 +23,7 @@
 #include "route_kernels.cuh"
 #include "dedup_kernels.cuh"
 #include "rank_kernels.cuh"
+#include "smooth_kernels.cuh"
 
 namespace {
 
@@ -816,6 +817,53 @@ mep_status_t mep_dispatch_int8_smooth(const uint16_t *x, const int32_t *ids, con
         mep::k_dispatch_int8_smooth_scalar<<<token_grid(T, 8), 256, 0, s>>>(x, ids, pos, T, K, H, smooth, n_experts,
                                                                            rows, recv, recv_scale);
     }
+    return launched();
+}
+
+size_t mep_dispatch_int8_smooth_workspace_size(int64_t T, int32_t K)
+{
+    if (T < 0 || K < 1 || K > MEP_MAX_K || T * K >= ((int64_t)1 << 31)) return 0;
+    return align256(sizeof(int32_t) * (size_t)(T * K));
+}
+
+mep_status_t mep_dispatch_int8_smooth_grouped(const uint16_t *x, const int32_t *ids, const int32_t *pos, int64_t T,
+                                              int32_t K, int64_t H, const float *smooth, int32_t n_experts,
+                                              int8_t *recv, float *recv_scale, int64_t rows, void *workspace,
+                                              size_t workspace_bytes, mep_stream_t stream)
+{
+    if (T > 0 && (!x || !ids || !pos || !smooth || (rows > 0 && (!recv || !recv_scale)))) return MEP_ERR_NULLPTR;
+    if (T < 0 || K < 1 || K > MEP_MAX_K || H < 1 || rows < 0 || n_experts < 1 || T * K >= ((int64_t)1 << 31))
+        return MEP_ERR_SHAPE;
+    const size_t need = mep_dispatch_int8_smooth_workspace_size(T, K);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return MEP_ERR_WORKSPACE;
+    if (T == 0) return MEP_OK;
+    const int64_t H4 = H / 4;
+    const bool vec4 = H % 4 == 0 && aligned(x, 8) && aligned(recv, 4) && aligned(smooth, 16);
+    if (!vec4 || H4 > 256 * mep::kSmoothMaxGroups || n_experts > mep::kSmoothOrderMaxExperts)   // per-token kernels
+        return mep_dispatch_int8_smooth(x, ids, pos, T, K, H, smooth, n_experts, recv, recv_scale, rows, stream);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t N = T * K;
+    int32_t *order = (int32_t *)workspace;
+    const int64_t chunk = std::max<int64_t>(1, mep::kSmoothChunkSlots / K);
+    launch_pdl(mep::k_smooth_order, dim3((unsigned)mep::ceil_div(T, chunk)), dim3(mep::kSmoothOrderThreads),
+               sizeof(int32_t) * (2 * (size_t)n_experts + 3), s, ids, pos, T, K, chunk, n_experts, rows, order);
+    // groups of 4 columns per thread: ceil(H / 4 / 256)
+    using grouped_t = void (*)(const uint2 *, const int32_t *, const int32_t *, const int32_t *, int64_t, int,
+                               int64_t, const float4 *, int32_t, int64_t, uint32_t *, float *);
+    static const grouped_t kern[2][mep::kSmoothMaxGroups] = {
+        {mep::k_dispatch_int8_smooth_grouped<1, false>, mep::k_dispatch_int8_smooth_grouped<2, false>,
+         mep::k_dispatch_int8_smooth_grouped<3, false>, mep::k_dispatch_int8_smooth_grouped<4, false>,
+         mep::k_dispatch_int8_smooth_grouped<5, false>, mep::k_dispatch_int8_smooth_grouped<6, false>,
+         mep::k_dispatch_int8_smooth_grouped<7, false>, mep::k_dispatch_int8_smooth_grouped<8, false>},
+        {mep::k_dispatch_int8_smooth_grouped<1, true>, mep::k_dispatch_int8_smooth_grouped<2, true>,
+         mep::k_dispatch_int8_smooth_grouped<3, true>, mep::k_dispatch_int8_smooth_grouped<4, true>,
+         mep::k_dispatch_int8_smooth_grouped<5, true>, mep::k_dispatch_int8_smooth_grouped<6, true>,
+         mep::k_dispatch_int8_smooth_grouped<7, true>, mep::k_dispatch_int8_smooth_grouped<8, true>}};
+    const int64_t groups = mep::ceil_div(H4, mep::kSmoothThreads);
+    const bool full = H4 == groups * mep::kSmoothThreads;
+    launch_pdl(kern[full][groups - 1], dim3((unsigned)mep::ceil_div(N, mep::kSmoothSlotsPerCTA)), dim3(mep::kSmoothThreads),
+               0, s, (const uint2 *)x, ids, pos, (const int32_t *)order, N, (int)K, H4, (const float4 *)smooth,
+               n_experts, rows, (uint32_t *)recv, recv_scale);
     return launched();
 }
 

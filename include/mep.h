@@ -25,7 +25,8 @@
  *    No call synchronises the whole device. mep_histogram, mep_plan, mep_plan_rank,
  *    mep_dispatch_ranks, mep_combine_ranks,
  *    mep_update_expert, mep_update_expert_ranks, mep_dedup_plan, mep_dispatch,
- *    mep_expand, mep_dispatch_int8_smooth, mep_dequantize, mep_combine,
+ *    mep_expand, mep_dispatch_int8_smooth, mep_dispatch_int8_smooth_grouped,
+ *    mep_dequantize, mep_combine,
  *    mep_combine_int8, mep_combine_add_rmsnorm, mep_prefetch_plan, mep_prefetch_weights
  *    and mep_grad_reduce can be captured into a CUDA graph and replayed on new inputs,
  *    once each has been called eagerly in the current context (the first call in a
@@ -317,6 +318,27 @@ mep_status_t mep_dispatch_int8_smooth(const uint16_t *x, const int32_t *ids, con
                                       int64_t T, int32_t K, int64_t H, const float *smooth,
                                       int32_t n_experts, int8_t *recv, float *recv_scale,
                                       int64_t rows, mep_stream_t stream);
+
+/*
+ * f1 smoothing, the same codes and scales as mep_dispatch_int8_smooth, with the slots
+ * taken in expert order: a first kernel sorts the slot indices by expert within chunks
+ * of about 2048 slots (the list goes into the workspace), a second quantises the slots
+ * along that list, so that each smoothing row is read once for a run of slots of its
+ * expert instead of twice per slot, while the chunk's token rows stay in L2.
+ * Arguments as mep_dispatch_int8_smooth, plus the caller-owned workspace (no contents
+ * needed on entry; calls in flight at the same time need workspaces of their own) of at
+ * least mep_dispatch_int8_smooth_workspace_size(T, K) bytes, 256-byte aligned (NULL
+ * allowed when that size is 0). Shapes the sorted path does not take (H % 4 != 0,
+ * unaligned x / recv / smooth, H > 8192, n_experts > 6000) run the kernels of
+ * mep_dispatch_int8_smooth instead, with the same results.
+ * Errors: those of mep_dispatch_int8_smooth; MEP_ERR_WORKSPACE.
+ */
+size_t mep_dispatch_int8_smooth_workspace_size(int64_t T, int32_t K);
+mep_status_t mep_dispatch_int8_smooth_grouped(const uint16_t *x, const int32_t *ids, const int32_t *pos,
+                                              int64_t T, int32_t K, int64_t H, const float *smooth,
+                                              int32_t n_experts, int8_t *recv, float *recv_scale,
+                                              int64_t rows, void *workspace, size_t workspace_bytes,
+                                              mep_stream_t stream);
 
 /* Largest hidden size of mep_combine_add_rmsnorm (one fp32 row in shared memory). */
 #define MEP_RMSNORM_MAX_H 49152

@@ -17,7 +17,8 @@ def test_every_named_kernel_is_found_and_hashed():
         "k_dispatch_warp", "k_dispatch_elem", "k_dispatch_int8_staged", "k_dispatch_int8",
         "k_combine_v8", "k_combine_scalar", "k_combine_int8_warp", "k_combine_int8_v8",
         "k_combine_int8_scalar", "k_combine_add_rmsnorm_v8", "k_combine_add_rmsnorm_scalar",
-        "k_dispatch_int8_smooth_k", "k_dispatch_int8_smooth_scalar",
+        "k_dispatch_int8_smooth_k", "k_dispatch_int8_smooth_scalar", "k_dispatch_int8_smooth_grouped",
+        "k_smooth_order",
         "k_expand_warp", "k_expand_bytes"}
     for n in names:
         assert n in funcs, n

@@ -149,6 +149,32 @@ def test_dispatch_combine_argument_checks(L):
     assert L.mep_selftest_bounded_wait(1 << 23, P, None) == 4
 
 
+def test_smooth_dispatch_grouped_argument_checks(L):
+    P = FAKE
+    c_size = ctypes.c_size_t
+    L.mep_dispatch_int8_smooth_workspace_size.argtypes = [ctypes.c_int64, ctypes.c_int32]
+    L.mep_dispatch_int8_smooth_workspace_size.restype = c_size
+    assert L.mep_dispatch_int8_smooth_workspace_size(1000, 8) == 32000
+    assert L.mep_dispatch_int8_smooth_workspace_size(3, 3) == 256          # 256-byte multiples
+    assert L.mep_dispatch_int8_smooth_workspace_size(0, 8) == 0
+    assert L.mep_dispatch_int8_smooth_workspace_size(-1, 8) == 0
+    assert L.mep_dispatch_int8_smooth_workspace_size(4, 0) == 0
+    i64, i32 = ctypes.c_int64, ctypes.c_int32
+    L.mep_dispatch_int8_smooth_grouped.argtypes = [ctypes.c_void_p] * 3 + [i64, i32, i64, ctypes.c_void_p, i32,
+                                                   ctypes.c_void_p, ctypes.c_void_p, i64, ctypes.c_void_p, c_size,
+                                                   ctypes.c_void_p]
+    W = ctypes.c_void_p(0x100000)                                          # 256-byte aligned, never read
+
+    def call(x=P, T=4, K=2, H=64, E=3, rows=8, ws=W, nbytes=256):
+        return L.mep_dispatch_int8_smooth_grouped(x, P, P, T, K, H, P, E, P, P, rows, ws, nbytes, None)
+    assert call(x=None) == 1                                               # NULLPTR
+    assert call(K=0) == 3 and call(K=33) == 3 and call(H=0) == 3 and call(E=0) == 3 and call(rows=-1) == 3
+    assert call(ws=None) == 5                                              # WORKSPACE: missing
+    assert call(nbytes=16) == 5                                            # too small
+    assert call(ws=ctypes.c_void_p(0x100010)) == 5                         # not 256-byte aligned
+    assert call(T=0, ws=None, nbytes=0) == 0                               # empty: no launch, no workspace
+
+
 def test_route_buffers_struct_layout_matches_the_header(tmp_path):
     """The binding's ctypes mirror of mep_route_buffers_t has the header's layout
     (size and field offsets as gcc lays the struct out)."""
