@@ -81,6 +81,27 @@ __device__ __forceinline__ float2 mul2_rn(float2 a, float2 b)
     return d;
 }
 
+__device__ __forceinline__ float2 sub2_rn(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n .reg .b64 pa, pb, pd;\n mov.b64 pa, {%2, %3};\n mov.b64 pb, {%4, %5};\n"
+        " sub.rn.f32x2 pd, pa, pb;\n mov.b64 {%0, %1}, pd;\n}\n"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// Two fused multiply-adds a * b + c, each rounded once (to nearest even).
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n .reg .b64 pa, pb, pc, pd;\n mov.b64 pa, {%2, %3};\n mov.b64 pb, {%4, %5};\n"
+        " mov.b64 pc, {%6, %7};\n fma.rn.f32x2 pd, pa, pb, pc;\n mov.b64 {%0, %1}, pd;\n}\n"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
 // Programmatic dependent launch (the host launches the routing step's kernels with the
 // programmatic-serialization attribute): pdl_wait() returns once the grid this one
 // depends on has finished and its memory is visible (at once when there is none), so a

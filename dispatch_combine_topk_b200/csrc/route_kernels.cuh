@@ -197,29 +197,30 @@ __device__ __forceinline__ float quant_inv(float scale)
 
 // The codes of q8x4 for the four products v = fl(x * s) of a row whose amax gave
 // scale = fl(amax / 127) (the smoothing dispatch), with inv = quant_inv(scale), packed
-// into one word (lowest column in the low byte). Each quotient is taken as
-// y = fl(v * inv). |v / scale| < 127.0001 (scale is within one rounding of amax / 127,
-// also when it is subnormal with 1 / scale finite) and inv is within 2^-24 of 1 / scale,
-// so |y - v/scale| < 2^-16 and |y - fl(v/scale)| < 2^-15: unless y lies within 2^-15 of
-// a half-integer, y and the correctly rounded quotient round to the same integer, which
-// is in [-127, 127] without a clamp. t = fl(y + 1.5 * 2^23) rounds y half-to-even to an
-// integer whose two's-complement low byte is the code; d = y - (t - 1.5 * 2^23) is its
-// distance to y. When any of the four lies that close to a half-integer (about 1 group
-// in 4000), or the row's 1 / scale overflows, all four take the IEEE quotient of q8x4.
-// The products and the rounding run on pairs (packed f32x2, each half rounded on its
-// own). No product feeds a sum whose rounding matters: had the compiler fused v * inv
-// into the sum t, t would round the exact product, which is within the same bound, and
-// d only decides whether to take the IEEE quotient.
+// into one word (lowest column in the low byte). The quotient is estimated by the exact
+// product z = v * inv inside a fused multiply-add: t = fl(z + 1.5 * 2^23) holds the
+// integer nearest z (half to even) in its low bits (for |z| < 2^22 the spacing of t is 1),
+// whose two's-complement low byte is the code; d = fl(z - (t - 1.5 * 2^23)) is the
+// distance of z to that integer (t - 1.5 * 2^23 is exact). inv is within 2^-24 of
+// 1 / scale (relative; a correctly rounded reciprocal of a scale whose reciprocal is
+// finite) and |v / scale| < 127.0001 (scale is within one rounding of amax / 127, also
+// when it is subnormal with 1 / scale finite), so
+// |z - v/scale| < 7.6e-6, and fl(v/scale) is within 3.9e-6 of v/scale: |z - fl(v/scale)|
+// < 2^-16. Unless z lies within 2^-15 of a half-integer, z and the correctly rounded
+// quotient therefore round to the same integer, which is in [-127, 127] without a
+// clamp. When any of the four lies that close (|d| >= 0.5 - 2^-15; about 1 group in
+// 4000), or the row's 1 / scale overflows, all four take the IEEE quotient of q8x4.
+// Each step runs on pairs (packed f32x2, each half rounded on its own); the products v
+// enter the fused steps as rounded values, as multiplicands.
 __device__ __forceinline__ uint32_t q8x4_packed(const float (&x)[4], const float4 &s, float scale, float inv)
 {
-    const float2 kShift = make_float2(12582912.0f, 12582912.0f), kNegShift = make_float2(-12582912.0f, -12582912.0f);
+    const float2 kShift = make_float2(12582912.0f, 12582912.0f);
     const float2 inv2 = make_float2(inv, inv);
     const float2 v0 = mul2_rn(make_float2(x[0], x[1]), make_float2(s.x, s.y));
     const float2 v1 = mul2_rn(make_float2(x[2], x[3]), make_float2(s.z, s.w));
-    const float2 y0 = mul2_rn(v0, inv2), y1 = mul2_rn(v1, inv2);
-    const float2 t0 = add2_rn(y0, kShift), t1 = add2_rn(y1, kShift);
-    const float2 r0 = add2_rn(t0, kNegShift), r1 = add2_rn(t1, kNegShift);
-    const float2 d0 = add2_rn(y0, make_float2(-r0.x, -r0.y)), d1 = add2_rn(y1, make_float2(-r1.x, -r1.y));
+    const float2 t0 = fma2_rn(v0, inv2, kShift), t1 = fma2_rn(v1, inv2, kShift);
+    const float2 n0 = sub2_rn(kShift, t0), n1 = sub2_rn(kShift, t1);      // minus the integers, exact
+    const float2 d0 = fma2_rn(v0, inv2, n0), d1 = fma2_rn(v1, inv2, n1);
     const float dmax = fmaxf(fmaxf(fabsf(d0.x), fabsf(d0.y)), fmaxf(fabsf(d1.x), fabsf(d1.y)));
     if (inv < 0.0f || dmax >= 0.5f - 0x1p-15f) return q8x4(v0.x, v0.y, v1.x, v1.y, scale);
     return __byte_perm(__byte_perm(__float_as_uint(t0.x), __float_as_uint(t0.y), 0x0040),
