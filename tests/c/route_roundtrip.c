@@ -3,7 +3,9 @@
  * balanced workload through the C ABI of include/mep.h, then the same round trip from
  * host memory in one mep_route_host call, checked against closed forms (every rank
  * receives exactly S*K rows; with gates summing to one, the identity expert gives every
- * token back). Prints "route_roundtrip ok" and exits 0 on success.
+ * token back). Then the int8 dispatch with all-ones smoothing scales, per token and
+ * sorted by expert (with its workspace query), against the plain per-token int8
+ * dispatch: the same codes and scales. Prints "route_roundtrip ok" and exits 0 on success.
  */
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -115,6 +117,42 @@ int main(void)
     CHECK(memcmp(out2, x, sizeof(uint16_t) * T * H) == 0);
     rb.quant = 5;
     CHECK(mep_route_host(&rb, ids, gates, x, out2, st) == MEP_ERR_DTYPE);
+    /* smoothing scales of one: the smoothed codes and scales are the plain int8 dispatch's */
+    {
+        float *ones = malloc(sizeof(float) * E * H), *d_sm, *d_sc0, *d_sc1, *d_sc2;
+        int8_t *d_q0, *d_q1, *d_q2;
+        void *d_sws;
+        for (int i = 0; i < E * H; i++) ones[i] = 1.0f;
+        const size_t sws = mep_dispatch_int8_smooth_workspace_size(T, K);
+        CHECK(sws >= sizeof(int32_t) * (size_t)N && sws % 256 == 0);
+        CHECK(cudaMalloc((void **)&d_sm, sizeof(float) * E * H) == cudaSuccess);
+        CHECK(cudaMalloc((void **)&d_q0, (size_t)N * H) == cudaSuccess);
+        CHECK(cudaMalloc((void **)&d_q1, (size_t)N * H) == cudaSuccess);
+        CHECK(cudaMalloc((void **)&d_q2, (size_t)N * H) == cudaSuccess);
+        CHECK(cudaMalloc((void **)&d_sc0, sizeof(float) * N) == cudaSuccess);
+        CHECK(cudaMalloc((void **)&d_sc1, sizeof(float) * N) == cudaSuccess);
+        CHECK(cudaMalloc((void **)&d_sc2, sizeof(float) * N) == cudaSuccess);
+        CHECK(cudaMalloc(&d_sws, sws) == cudaSuccess);
+        CHECK(cudaMemcpy(d_sm, ones, sizeof(float) * E * H, cudaMemcpyHostToDevice) == cudaSuccess);
+        CHECK(mep_dispatch(d_x, d_pos, T, K, H, 1, d_q0, d_sc0, N, st) == MEP_OK);
+        CHECK(mep_dispatch_int8_smooth(d_x, d_ids, d_pos, T, K, H, d_sm, E, d_q1, d_sc1, N, st) == MEP_OK);
+        CHECK(mep_dispatch_int8_smooth_grouped(d_x, d_ids, d_pos, T, K, H, d_sm, E, d_q2, d_sc2, N, NULL, sws, st) ==
+              MEP_ERR_WORKSPACE);
+        CHECK(mep_dispatch_int8_smooth_grouped(d_x, d_ids, d_pos, T, K, H, d_sm, E, d_q2, d_sc2, N, d_sws, sws, st) ==
+              MEP_OK);
+        CHECK(cudaStreamSynchronize(st) == cudaSuccess);
+        CHECK(mep_get_error(st, &derr, 1) == MEP_OK && derr == 0);
+        int8_t *q0 = malloc((size_t)N * H), *q1 = malloc((size_t)N * H), *q2 = malloc((size_t)N * H);
+        float *sc0 = malloc(sizeof(float) * N), *sc1 = malloc(sizeof(float) * N), *sc2 = malloc(sizeof(float) * N);
+        CHECK(cudaMemcpy(q0, d_q0, (size_t)N * H, cudaMemcpyDeviceToHost) == cudaSuccess);
+        CHECK(cudaMemcpy(q1, d_q1, (size_t)N * H, cudaMemcpyDeviceToHost) == cudaSuccess);
+        CHECK(cudaMemcpy(q2, d_q2, (size_t)N * H, cudaMemcpyDeviceToHost) == cudaSuccess);
+        CHECK(cudaMemcpy(sc0, d_sc0, sizeof(float) * N, cudaMemcpyDeviceToHost) == cudaSuccess);
+        CHECK(cudaMemcpy(sc1, d_sc1, sizeof(float) * N, cudaMemcpyDeviceToHost) == cudaSuccess);
+        CHECK(cudaMemcpy(sc2, d_sc2, sizeof(float) * N, cudaMemcpyDeviceToHost) == cudaSuccess);
+        CHECK(memcmp(q0, q1, (size_t)N * H) == 0 && memcmp(q0, q2, (size_t)N * H) == 0);
+        CHECK(memcmp(sc0, sc1, sizeof(float) * N) == 0 && memcmp(sc0, sc2, sizeof(float) * N) == 0);
+    }
     /* argument errors come back without touching the device */
     CHECK(mep_dispatch(d_x, d_pos, T, K, H, 7, d_recv, NULL, N, st) == MEP_ERR_DTYPE);
     CHECK(mep_plan(NULL, NULL, R, E, S, K, 0, 0, d_pos, d_hist, d_roff, NULL, d_rc, d_rk, d_rcu, d_stats, d_ws,
