@@ -102,6 +102,15 @@ __device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c)
     return d;
 }
 
+// The largest of three floats in one instruction (sm_100 three-input max.f32): for
+// inputs that are not NaN, fmaxf(fmaxf(a, b), c).
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Programmatic dependent launch (the host launches the routing step's kernels with the
 // programmatic-serialization attribute): pdl_wait() returns once the grid this one
 // depends on has finished and its memory is visible (at once when there is none), so a

@@ -221,7 +221,7 @@ __device__ __forceinline__ uint32_t q8x4_packed(const float (&x)[4], const float
     const float2 t0 = fma2_rn(v0, inv2, kShift), t1 = fma2_rn(v1, inv2, kShift);
     const float2 n0 = sub2_rn(kShift, t0), n1 = sub2_rn(kShift, t1);      // minus the integers, exact
     const float2 d0 = fma2_rn(v0, inv2, n0), d1 = fma2_rn(v1, inv2, n1);
-    const float dmax = fmaxf(fmaxf(fabsf(d0.x), fabsf(d0.y)), fmaxf(fabsf(d1.x), fabsf(d1.y)));
+    const float dmax = fmax3(fabsf(d0.x), fabsf(d0.y), fmaxf(fabsf(d1.x), fabsf(d1.y)));
     if (inv < 0.0f || dmax >= 0.5f - 0x1p-15f) return q8x4(v0.x, v0.y, v1.x, v1.y, scale);
     return __byte_perm(__byte_perm(__float_as_uint(t0.x), __float_as_uint(t0.y), 0x0040),
                        __byte_perm(__float_as_uint(t1.x), __float_as_uint(t1.y), 0x0040), 0x5410);
@@ -1031,11 +1031,11 @@ k_dispatch_int8_smooth_k(const uint2 *__restrict__ x, const int32_t *__restrict_
                         const float4 sv = srow[g];
                         const float2 v0 = mul2_rn(make_float2(xr[i][0], xr[i][1]), make_float2(sv.x, sv.y));
                         const float2 v1 = mul2_rn(make_float2(xr[i][2], xr[i][3]), make_float2(sv.z, sv.w));
-                        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v0.x), fabsf(v0.y)), fmaxf(fabsf(v1.x), fabsf(v1.y))));
+                        amax = fmax3(fmax3(amax, fabsf(v0.x), fabsf(v0.y)), fabsf(v1.x), fabsf(v1.y));
                     }
                 }
             }
-            // warp maximum of non-negative floats (fmaxf left out any NaN): their bits order
+            // warp maximum of non-negative floats (products of finite inputs): their bits order
             // like their values, so one integer reduction gives it
             amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
             if (lane == 0) red[warp][k] = amax;

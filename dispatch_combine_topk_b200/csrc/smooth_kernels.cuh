@@ -152,11 +152,11 @@ k_dispatch_int8_smooth_grouped(const uint2 *__restrict__ x, const int32_t *__res
                     const uint2 v = xr[i];
                     const float2 v0 = mul2_rn(make_float2(bf16lo(v.x), bf16hi(v.x)), make_float2(sv[i].x, sv[i].y));
                     const float2 v1 = mul2_rn(make_float2(bf16lo(v.y), bf16hi(v.y)), make_float2(sv[i].z, sv[i].w));
-                    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v0.x), fabsf(v0.y)), fmaxf(fabsf(v1.x), fabsf(v1.y))));
+                    amax = fmax3(fmax3(amax, fabsf(v0.x), fabsf(v0.y)), fabsf(v1.x), fabsf(v1.y));
                 }
             }
         }
-        // warp maximum of non-negative floats (fmaxf left out any NaN): their bits order
+        // warp maximum of non-negative floats (products of finite inputs): their bits order
         // like their values, so one integer reduction gives it
         amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
         if (lane == 0) red[j][warp] = amax;
