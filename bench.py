@@ -128,7 +128,7 @@ TRAFFIC = {
     ("k_combine_v8", "skew_r64_e512_s2048_k8_h4096"): {
         "bytes": 4 * 2364.012e6, "src": "75f948c1d2f4d491", "case_S": 512, "case_mb": 2364.012},
     ("k_dispatch_int8_smooth_grouped", "int8_r32_e256_s8192_k8_h7168"): {
-        "bytes": 16 * 1145.386e6, "src": "5ccc771bc28cc68e", "case_S": 512, "case_mb": 1145.386},
+        "bytes": 16 * 1151.300e6, "src": "77b03711df0d65be", "case_S": 512, "case_mb": 1151.300},
 }
 
 
