@@ -8,8 +8,9 @@ Default workload (the headline): R=32 simulated EP ranks, E=256 experts, S=8192 
 per rank, K=8, H=7168, with per-token dynamic int8 dispatch and the combine of the int8
 rows (N = 2,097,152 token-slots per step). Inputs (x 3.76 GB, receive buffer 15 GB) are
 larger than the 126 MB L2, so no flush is needed between steps. After it, the other four
-workloads (tiny, r8, map, skew) are measured the same way, more briefly, and reported
-in the same line under `per_workload`.
+workloads (tiny, r8, map, skew), r8 and int8 in the expert-parallel layout, and int8 with
+per-expert smoothing scales are measured the same way, more briefly, and reported in the
+same line under `per_workload`.
 
 Prints one JSON line (rank 0). `value` = token-slots of all ranks per second of the
 slowest rank's device time. With --gpus N > 1 (torchrun), every rank routes its own
@@ -1053,16 +1054,17 @@ def roofline_of(rt, tm, peak, peak_kind):
     return roof, dc
 
 
-def per_workload_entry(mep, name, args, dev, stream, pg, peak, peak_kind):
+def per_workload_entry(mep, name, args, dev, stream, pg, peak, peak_kind, smooth: bool = False):
     """A shorter measurement of another workload for the `per_workload` block: the same
-    timing method (graph replays, per-phase eager events), no end-to-end leg."""
+    timing method (graph replays, per-phase eager events), no end-to-end leg. With
+    `smooth` (the int8 workload), the dispatch applies per-expert smoothing scales."""
     w = synth.get(name)
-    rt = Route(mep, w, dev)
+    rt = Route(mep, w, dev, smooth=smooth)
     steps = max(5, min(args.steps, 20))
     tm = time_route(mep, rt, args, dev, stream, pg, steps)
     roof, dc = roofline_of(rt, tm, peak, peak_kind)
     entry = {
-        "workload": w.name, "token_slots": w.N, "ms_per_step": tm["ms_step"],
+        "workload": w.name + ("_smooth" if smooth else ""), "token_slots": w.N, "ms_per_step": tm["ms_step"],
         "token_slots_per_s": w.N / (tm["ms_step"] * 1e-3), "step_ms": tm["step_ms"],
         "breakdown_ms": tm["t_phase"], "dispatch_combine": dc,
         "roofline": {k: roof[k] for k in ("kernel", "phase", "achieved", "frac", "algorithmic_bytes", "traffic")},
@@ -1175,6 +1177,12 @@ def run_gpu(args, w):
             e = per_workload_ep_entry(mep, name[:-3], args, dev, stream, pg, peak, peak_kind)
             per[e["workload"]] = e
             continue
+        if name.endswith("_smooth"):
+            e = per_workload_entry(mep, name[:-7], args, dev, stream, pg, peak, peak_kind, smooth=True)
+            e["variant"] = ("per-expert smoothing scales before the int8 quantisation, codes and scale per slot "
+                            "(mep_dispatch_int8_smooth_grouped)")
+            per[e["workload"]] = e
+            continue
         if synth.get(name).name == w.name:
             continue
         e = per_workload_entry(mep, name, args, dev, stream, pg, peak, peak_kind)
@@ -1194,10 +1202,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="mep", choices=["mep", "reference"])
     ap.add_argument("--workload", default="int8")
-    ap.add_argument("--per-workload", default="tiny,r8,map,skew,r8_ep,int8_ep",
+    ap.add_argument("--per-workload", default="tiny,r8,map,skew,r8_ep,int8_ep,int8_smooth",
                     help="comma-separated workloads measured after the main one and reported under "
                          "per_workload (graph replays, no end-to-end leg); a name ending in _ep routes that "
-                         "balanced workload in the expert-parallel layout; 'none' to skip")
+                         "balanced workload in the expert-parallel layout, int8_smooth the int8 workload "
+                         "with per-expert smoothing scales; 'none' to skip")
     ap.add_argument("--ref-div", type=int, default=16,
                     help="--impl reference: the oracle routes S/ref_div tokens per rank per step")
     ap.add_argument("--cpu-div", type=int, default=1,
