@@ -3,7 +3,7 @@
 (per token: H % 4 == 0 with up to 64 columns per thread, in groups of 4, takes the fused
 kernel, all K slots of a token in one CTA; other H or alignments the scalar kernel) and
 mep_dispatch_int8_smooth_grouped (the slots sorted by expert within chunks of tokens,
-then quantised along that list, for H % 4 == 0 up to 32768 and aligned buffers; other
+then quantised along that list, for H % 4 == 0 up to 8192 and aligned buffers; other
 shapes fall back to the per-token kernels). The full int8 workload is compared whole,
 one rank partition at a time, and with all-ones scales against the plain per-token int8
 dispatch."""
